@@ -1,0 +1,353 @@
+#!/usr/bin/env python
+"""Benchmark of one S3R decode step on B200 (verified tokens/s, KV GB/s).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload I] [--impl ours|reference]
+
+A step is one whole round of the hot path on one batch: gamma sparse-draft
+calls (tail-page summary refresh + page scoring/top-B + split-KV attention),
+the drafter's token draws, dense causal verification of the gamma+1 rows, and
+exact speculative sampling. Inputs are seeded synthetic tensors shaped like
+the Qwen3-8B layer workload (16 sequences x 16384 tokens, 32q/8kv heads,
+head_dim 128, 64-token pages, B = 32 pages, gamma = 4, vocab 151936, bf16),
+resident in HBM before timing. Metric: verified (committed) tokens per second
+= sum over sequences of (accepted drafts + 1) / step time.
+
+Multi-GPU (torchrun, one rank per GPU): sequences are independent, so every
+rank runs its own full batch (weak scaling, no data-path collective); the
+step time is the max over ranks.
+
+--impl reference times the float64 CPU oracle on the host cores instead (a
+bounded sample of the same workload per step).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import signal
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, HERE)
+
+import numpy as np  # noqa: E402
+
+METRIC = "verified tokens/s per decode step on 1 B200; KV-read GB/s as % of HBM peak"
+UNIT = "tokens/s"
+
+
+def _peaks():
+    try:
+        with open(os.path.join(HERE, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------- CPU oracle
+def _oracle_seq_worker(args):
+    idx, seed, b = args
+    os.environ.setdefault("OMP_NUM_THREADS", "1")
+    from self_sparse_speculative_b200.workloads import Workload, spec
+    import oracle.reference_run as RR
+    wl = Workload(spec(idx), seed=seed)
+    t0 = time.perf_counter()
+    RR.oracle_attention_seq(wl, b)
+    s = RR.oracle_sampling_seq(wl, b)
+    return s["n_acc"] + 1, time.perf_counter() - t0
+
+
+def oracle_sample(idx, seed, seqs, workers):
+    """Run the oracle round on the listed sequences; returns (tokens, wall s, cores)."""
+    import multiprocessing as mp
+    jobs = [(idx, seed, b) for b in seqs]
+    t0 = time.perf_counter()
+    if workers > 1:
+        ctx = mp.get_context("spawn")
+        with ctx.Pool(workers) as pool:
+            res = pool.map(_oracle_seq_worker, jobs)
+    else:
+        res = [_oracle_seq_worker(j) for j in jobs]
+    wall = time.perf_counter() - t0
+    return sum(r[0] for r in res), wall, workers
+
+
+def cpu_cores():
+    return len(os.sched_getaffinity(0))
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.send_signal(signal.SIGTERM)
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(a):
+    import torch
+    import torch.distributed as dist
+    from self_sparse_speculative_b200.step import DecodeStep
+    from self_sparse_speculative_b200.workloads import Workload, spec
+    from self_sparse_speculative_b200 import s3r
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    ws = spec(a.workload)
+    wl = Workload(ws, seed=a.seed + rank)
+    st = DecodeStep(wl, device=f"cuda:{local}")
+    stream = torch.cuda.current_stream()
+    st.summaries(tail_only=False)
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    # ---- warm-up
+    for _ in range(a.warmup):
+        st.round()
+    barrier()
+
+    # ---- device-timed steps, with per-phase events on the launching stream
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(a.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for k in range(a.steps):
+        e = ev[k]
+        e[0].record(stream)
+        st.draw_draft_tokens()
+        e[1].record(stream)
+        for i in range(ws.gamma):
+            st.draft(i)
+        e[2].record(stream)
+        st.verify()
+        e[3].record(stream)
+        st.sample()
+        e[4].record(stream)
+    end.record(stream)
+    barrier()
+    clk = clocks.stop()
+    total_ms = start.elapsed_time(end)
+    t_draw = sum(e[0].elapsed_time(e[1]) for e in ev) / a.steps
+    t_draft = sum(e[1].elapsed_time(e[2]) for e in ev) / a.steps / ws.gamma
+    t_verify = sum(e[2].elapsed_time(e[3]) for e in ev) / a.steps
+    t_sample = sum(e[3].elapsed_time(e[4]) for e in ev) / a.steps
+    # inputs are the same every step, so every step commits the same tokens
+    n_acc_total = int(st.num_accepted.sum().item()) * a.steps
+    tokens = n_acc_total + ws.num_seqs * a.steps             # (n_acc + 1) per sequence per step
+    status = st.device_checks()
+    bad = {k: v for k, v in status.items() if v[0] != s3r.S3R_OK}
+    if bad:
+        raise RuntimeError(f"device checks failed: {bad}")
+
+    t = torch.tensor([total_ms, float(tokens)], dtype=torch.float64, device=f"cuda:{local}")
+    if world > 1:
+        tm = t[:1].clone()
+        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
+        tk = t[1:].clone()
+        dist.all_reduce(tk, op=dist.ReduceOp.SUM)
+        total_ms_max, tokens_all = float(tm.item()), float(tk.item())
+    else:
+        total_ms_max, tokens_all = total_ms, float(tokens)
+
+    # ---- end to end: host buffers, H2D of the step's inputs and D2H of the result
+    e2e = None
+    if not a.no_e2e:
+        host = {n: getattr(st, n).cpu().pin_memory() for n in
+                ("q_draft", "q_verify", "target_logits", "draft_logits", "u_draft", "u_accept", "u_sample")}
+        out_h = torch.empty_like(st.out_tokens, device="cpu").pin_memory()
+        nacc_h = torch.empty_like(st.num_accepted, device="cpu").pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in host.values())
+        d2h = out_h.numel() * 4 + nacc_h.numel() * 4
+        for _ in range(2):
+            for n, v in host.items():
+                getattr(st, n).copy_(v, non_blocking=True)
+            st.round()
+            out_h.copy_(st.out_tokens, non_blocking=True)
+            nacc_h.copy_(st.num_accepted, non_blocking=True)
+        barrier()
+        e_s = torch.cuda.Event(enable_timing=True)
+        e_e = torch.cuda.Event(enable_timing=True)
+        e2e_tokens = 0
+        e_s.record(stream)
+        for _ in range(a.steps):
+            for n, v in host.items():
+                getattr(st, n).copy_(v, non_blocking=True)
+            st.round()
+            out_h.copy_(st.out_tokens, non_blocking=True)
+            nacc_h.copy_(st.num_accepted, non_blocking=True)
+        e_e.record(stream)
+        barrier()
+        e2e_ms = e_s.elapsed_time(e_e)
+        e2e_tokens = (int(nacc_h.sum().item()) + ws.num_seqs) * a.steps
+        tt = torch.tensor([e2e_ms, float(e2e_tokens)], dtype=torch.float64, device=f"cuda:{local}")
+        if world > 1:
+            m = tt[:1].clone(); dist.all_reduce(m, op=dist.ReduceOp.MAX)
+            s_ = tt[1:].clone(); dist.all_reduce(s_, op=dist.ReduceOp.SUM)
+            e2e_ms, e2e_tokens = float(m.item()), float(s_.item())
+        e2e = {"value": e2e_tokens / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h)}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    nbytes = st.algorithmic_bytes()
+    peak, peak_kind = _peaks()
+    verify_gbs = nbytes["verify"] / (t_verify * 1e-3) / 1e9
+    draft_gbs = nbytes["draft_per_call"] / (t_draft * 1e-3) / 1e9
+    ms_per_step = total_ms_max / a.steps
+    value = tokens_all / (total_ms_max / 1e3)
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": a.steps,
+        "warmup": a.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "impl": "ours",
+        "config": {"workload": ws.name, "sequences_per_gpu": ws.num_seqs, "context": ws.context,
+                   "q_heads": ws.num_q_heads, "kv_heads": ws.num_kv_heads, "head_dim": ws.head_dim,
+                   "page": ws.page_size, "budget_pages": ws.budget_pages, "gamma": ws.gamma,
+                   "vocab": ws.vocab, "parallelism": f"replicas x{world} (sequence-sharded, no collective)",
+                   "l2": "not flushed: each step reads %.2f GB > 126 MB L2" % (nbytes["step"] / 1e9),
+                   "seed": a.seed},
+        "roofline": {"bound": "hbm", "kernel": "verify attention (s3r_verify_attn)",
+                     "achieved": round(verify_gbs, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(verify_gbs / peak, 4), "peak_kind": peak_kind,
+                     "traffic": None,
+                     "algorithmic_bytes_per_launch": nbytes["verify"]},
+        "phases_ms": {"draft_token_draws": round(t_draw, 4), "sparse_draft_per_call": round(t_draft, 4),
+                      "verify": round(t_verify, 4), "spec_sample": round(t_sample, 4)},
+        "kv_gbs": {"sparse_draft": round(draft_gbs, 1), "sparse_draft_frac_of_8tbs": round(draft_gbs / 8000, 4),
+                   "verify": round(verify_gbs, 1), "verify_frac_of_8tbs": round(verify_gbs / 8000, 4)},
+        "acceptance": {"mean_accepted_per_seq": round(n_acc_total / (ws.num_seqs * a.steps), 4),
+                       "committed_per_seq": round(tokens / (ws.num_seqs * a.steps), 4)},
+        "gpu_launches": (3 * ws.gamma + 5) * a.steps,
+        "clocks": clk,
+    }
+    if e2e:
+        line["e2e"] = {k: (round(v, 1) if isinstance(v, float) else v) for k, v in e2e.items()}
+    if not a.no_cpu_baseline and world == 1:
+        seqs = list(range(min(ws.num_seqs, a.cpu_seqs)))
+        workers = max(1, min(len(seqs), cpu_cores()))
+        tok, wall, cores = oracle_sample(a.workload, a.seed, seqs, workers)
+        line["cpu_baseline"] = {"value": round(tok / wall, 3), "unit": UNIT, "cores": cores, "kind": "oracle",
+                                "sample": f"float64 oracle round (summaries, {ws.gamma} sparse drafts, verify, "
+                                          f"sampling) of {len(seqs)} of {ws.num_seqs} sequences, one process "
+                                          f"per sequence, {wall:.1f} s wall"}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- reference arm
+def run_reference(a):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from self_sparse_speculative_b200.workloads import spec
+    ws = spec(a.workload)
+    workers = max(1, min(cpu_cores(), a.cpu_seqs))
+    seqs_per_step = min(ws.num_seqs, a.cpu_seqs)
+    for _ in range(a.warmup if a.warmup < 1 else 1):
+        oracle_sample(a.workload, a.seed, [0], 1)
+    toks, wall = 0, 0.0
+    for k in range(a.steps):
+        seqs = [(k * seqs_per_step + i) % ws.num_seqs for i in range(seqs_per_step)]
+        t, w, _ = oracle_sample(a.workload, a.seed, seqs, workers)
+        toks += t
+        wall += w
+    value = toks / wall
+    line = {"metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": 0, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": round(wall / a.steps * 1e3, 2), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": ws.name, "sequences_per_step": seqs_per_step},
+            "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": workers, "kind": "oracle",
+                             "sample": f"{seqs_per_step} of {ws.num_seqs} sequences per step, full float64 "
+                                       f"round per sequence"},
+            "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", type=int, default=1)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seqs", type=int, default=8, help="sequences in the CPU oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    a = ap.parse_args()
+    if a.impl == "ours":
+        a.warmup = max(3, a.warmup)     # at least 3 untimed warm-up steps
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_ours(a)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,223 @@
+/*
+ * s3r.h - C ABI of libs3r: one S3R decode step on NVIDIA B200 (sm_100a).
+ *
+ * S3R ("S3R: Fast and Faithful RL Rollouts via Self-Sparse Speculative
+ * Decoding", weekinpapers.com, Abstract) drafts tokens with sparse attention
+ * over the KV cache, then verifies them with full attention over the complete
+ * history and commits them by exact speculative sampling, with drafter and
+ * verifier sharing the same parameters and the same KV cache. This library
+ * implements the attention and sampling steps of one such round over a paged
+ * GQA KV cache:
+ *
+ *   s3r_page_summaries     per-page key min/max (Quest page metadata)
+ *   s3r_sparse_draft_attn  score pages, keep the top-B per KV head, attend
+ *   s3r_verify_attn        dense causal attention of the gamma+1 verify rows
+ *   s3r_spec_sample        accept/reject, residual or bonus draw
+ *   s3r_sample_tokens      the drafter's own draw x ~ softmax(logits / T)
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Every pointer argument is a caller-owned DEVICE pointer unless stated
+ *   otherwise. The library allocates and frees nothing and keeps no state
+ *   between calls; scratch space comes from the caller's workspace.
+ * - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *   stream). Work is enqueued asynchronously on it; outputs are ready when the
+ *   stream reaches that point.
+ * - Argument errors are detected on the host and returned synchronously
+ *   before anything is enqueued. A failed launch returns S3R_ERR_CUDA.
+ * - Data the host cannot see (context lengths, page ids, draft token ids) is
+ *   checked on the device: a bad value is skipped, never dereferenced, and
+ *   recorded in the workspace's status word; s3r_device_status() reports it.
+ *   A kernel wait that exceeds its time limit (about one second) is recorded
+ *   the same way and the kernel returns instead of hanging.
+ * - Shapes: S sequences, Hq query heads, Hkv KV heads, G = Hq / Hkv, head dim
+ *   D, page size P, context length L_b of sequence b, n_b = ceil(L_b / P)
+ *   pages, R = gamma + 1 verify rows.
+ * - Supported: D in {64, 128}; P in {16, 64}; dtype f32 or bf16 (KV cache,
+ *   queries and attention outputs share it); G <= 8; G * rows <= 128;
+ *   1 <= gamma <= 16; max_pages_per_seq <= 8192.
+ * - No exception crosses this ABI.
+ */
+#ifndef S3R_H_
+#define S3R_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  S3R_OK = 0,
+  S3R_ERR_INVALID_ARG = 1,   /* null pointer, bad size or inconsistent shape   */
+  S3R_ERR_UNSUPPORTED = 2,   /* valid but outside the supported shapes/dtypes  */
+  S3R_ERR_WORKSPACE = 3,     /* workspace null or smaller than required        */
+  S3R_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed           */
+  S3R_ERR_DEVICE_CHECK = 5   /* a device-side check failed (s3r_device_status) */
+} s3r_status;
+
+typedef enum { S3R_F32 = 0, S3R_BF16 = 1 } s3r_dtype;
+
+/* Bits of the device status word (s3r_device_status). */
+#define S3R_DEV_BAD_CONTEXT_LEN  0x1u  /* L_b < 1, L_b > max_pages*P, or L_b < rows (verify) */
+#define S3R_DEV_BAD_PAGE_ID      0x2u  /* block-table entry outside [0, num_pages_total)    */
+#define S3R_DEV_BAD_TOKEN_ID     0x4u  /* draft token outside [0, vocab)                    */
+#define S3R_DEV_WAIT_TIMEOUT     0x8u  /* an in-kernel wait ran past its limit              */
+
+/*
+ * A paged KV cache (PagedAttention's block tables, cited on the mlsanity.com
+ * page's reference list).
+ * k_cache, v_cache: [num_pages_total, Hkv, P, D] row-major in `dtype`; the
+ *   (page, head) tile of P*D values is contiguous. Base addresses must be
+ *   16-byte aligned.
+ * block_table: int32 [num_seqs, max_pages_per_seq]; entry i of row b is the
+ *   physical page holding tokens i*P .. i*P+P-1 of sequence b. Entries past
+ *   n_b are never read.
+ * context_lens: int32 [num_seqs], L_b >= 1. Cache slots of positions >= L_b
+ *   in a sequence's last page may hold anything (they are never used).
+ */
+typedef struct {
+  int32_t num_seqs;
+  int32_t num_q_heads;
+  int32_t num_kv_heads;
+  int32_t head_dim;
+  int32_t page_size;
+  int32_t max_pages_per_seq;
+  int32_t num_pages_total;
+  s3r_dtype dtype;
+  const void* k_cache;
+  const void* v_cache;
+  const int32_t* block_table;
+  const int32_t* context_lens;
+} s3r_paged_kv;
+
+/*
+ * Per-page key summaries (Quest: query-aware page sparsity, cited on the
+ * mlsanity.com page's reference list; S3R page, Abstract, "uses sparse
+ * attention to propose tokens").
+ *   kmin[p, h, d] = min over the valid tokens t of page p of K[p, h, t, d];
+ *   kmax likewise. Valid tokens of page i of sequence b: t < L_b - i*P.
+ * kmin, kmax: [num_pages_total, Hkv, D] in kv->dtype (min and max are exact).
+ * tail_only = 0 recomputes every page used by a sequence; tail_only = 1
+ * recomputes only each sequence's last page (the one a decode step appends
+ * to) and leaves every other entry untouched. Pages no sequence uses are never
+ * written.
+ */
+s3r_status s3r_page_summaries(const s3r_paged_kv* kv, int32_t tail_only,
+                              void* kmin, void* kmax, void* stream);
+
+/*
+ * Sparse draft attention (S3R page, Abstract: "uses sparse attention to
+ * propose tokens"; page choice after Quest).
+ * For each sequence b and KV head h:
+ *   score(p) = sum over the G query heads g of group h, sum over d, of
+ *              max(q[b,g,d] * kmin[p,h,d], q[b,g,d] * kmax[p,h,d])
+ *   (accumulated in float64, unscaled) for every page p < n_b; keep the
+ *   budget_pages highest scores, ties to the lower page index (all pages if
+ *   n_b <= budget_pages); then for every query head of the group
+ *   out = softmax(q k^T * scale) v over the valid tokens of the kept pages,
+ *   the query sitting at position L_b - 1.
+ * q: [S, Hq, D] in kv->dtype. out: [S, Hq, D] in kv->dtype.
+ * lse: float32 [S, Hq] natural-log log-sum-exp of the scaled scores, or NULL.
+ * selected: int32 [S, Hkv, budget_pages], the kept logical page indices in
+ *   ascending order, -1 after the first min(n_b, budget_pages) entries.
+ * kmin, kmax: as written by s3r_page_summaries for the current cache.
+ * workspace: at least s3r_attn_workspace_bytes(kv, 1, budget_pages) bytes.
+ */
+s3r_status s3r_sparse_draft_attn(const s3r_paged_kv* kv, const void* kmin, const void* kmax,
+                                 const void* q, int32_t budget_pages, float scale,
+                                 int32_t* selected, void* out, float* lse,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Dense verification attention (S3R page, Abstract: "full-attention
+ * verification"; "dense verification still requires the complete historical
+ * KV cache").
+ * Row r (0 <= r < rows) of sequence b sits at position L_b - rows + r and
+ * attends causally to every key at position <= its own:
+ *   out[b,r,hq] = softmax(q[b,r,hq] k^T * scale) v, keys of KV head hq / G.
+ * q, out: [S, rows, Hq, D] in kv->dtype; lse: float32 [S, rows, Hq] or NULL.
+ * Requires L_b >= rows (checked on the device).
+ * workspace: at least s3r_attn_workspace_bytes(kv, rows, 0) bytes.
+ */
+s3r_status s3r_verify_attn(const s3r_paged_kv* kv, const void* q, int32_t rows, float scale,
+                           void* out, float* lse,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Exact speculative sampling of one round (S3R page, Abstract: "exact
+ * speculative sampling", the committed responses "follow the dense-policy
+ * distribution"; rule of the speculative-sampling papers on the mlsanity.com
+ * reference list, restated on the ai.info SpecRoll page).
+ *   p_i = softmax(target_logits[b,i] / T), i = 0..gamma
+ *   q_i = softmax(draft_logits[b,i] / T),  i = 0..gamma-1
+ *   for i = 0..gamma-1: accept x_i = draft_tokens[b,i] iff
+ *       u_accept[b,i] < p_i(x_i) / q_i(x_i)          (q_i(x_i) = 0 rejects)
+ *   at the first rejection j: draw from max(p_j - q_j, 0) normalised (from
+ *   p_j if that is all zero); if all gamma are accepted: draw from p_gamma.
+ *   A draw from weights w with uniform u is the smallest k whose running sum
+ *   C(k) exceeds u * C(V-1) (the last positive-weight index if rounding
+ *   leaves none); it uses u_sample[b, j].
+ * target_logits: [S, gamma+1, V]; draft_logits: [S, gamma, V]; both in
+ *   logit_dtype. draft_tokens: int32 [S, gamma]. u_accept: float32 [S, gamma];
+ *   u_sample: float32 [S, gamma+1]; uniforms in [0, 1).
+ * out_tokens: int32 [S, gamma+1], the n_acc accepted drafts, the drawn token,
+ *   then -1. num_accepted: int32 [S] = n_acc.
+ * Row statistics accumulate in float64; decisions are taken in float64.
+ * workspace: at least s3r_sample_workspace_bytes(S, gamma, V) bytes.
+ */
+s3r_status s3r_spec_sample(const void* target_logits, const void* draft_logits,
+                           s3r_dtype logit_dtype, const int32_t* draft_tokens,
+                           const float* u_accept, const float* u_sample,
+                           int32_t num_seqs, int32_t gamma, int32_t vocab, float temperature,
+                           int32_t* out_tokens, int32_t* num_accepted,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * The drafter's own sampling step: tokens[r] = inverse-CDF draw from
+ * softmax(logits[r] / T) with uniform u[r] (same draw rule as above). In a
+ * round it draws each x_i ~ q_i from the draft logits.
+ * logits: [num_rows, V] in logit_dtype; u: float32 [num_rows];
+ * tokens: int32 [num_rows].
+ * workspace: at least s3r_sample_workspace_bytes(num_rows, 0, V) bytes.
+ */
+s3r_status s3r_sample_tokens(const void* logits, s3r_dtype logit_dtype, int32_t num_rows,
+                             int32_t vocab, float temperature, const float* u,
+                             int32_t* tokens, void* workspace, size_t workspace_bytes,
+                             void* stream);
+
+/* Workspace sizes. Return 0 for an invalid or unsupported request.
+ * Attention: rows = 1 and budget_pages > 0 for s3r_sparse_draft_attn;
+ * rows = gamma + 1 and budget_pages = 0 for s3r_verify_attn.
+ * Sampling: (num_seqs, gamma, vocab) for s3r_spec_sample;
+ * (num_rows, 0, vocab) for s3r_sample_tokens. */
+size_t s3r_attn_workspace_bytes(const s3r_paged_kv* kv, int32_t rows, int32_t budget_pages);
+size_t s3r_sample_workspace_bytes(int32_t num_seqs, int32_t gamma, int32_t vocab);
+
+/*
+ * Synchronises `stream`, then reads the status word that the most recent
+ * call using `workspace` left there: S3R_OK, or S3R_ERR_DEVICE_CHECK with the
+ * S3R_DEV_* bits in *bits (bits may be NULL). Every call clears the word when
+ * it starts. s3r_page_summaries has no workspace; its device checks use the
+ * status word at `status_word` if given via s3r_page_summaries_checked.
+ */
+s3r_status s3r_device_status(const void* workspace, uint32_t* bits, void* stream);
+
+/* As s3r_page_summaries, also recording device-check failures in the 4-byte
+ * device word status_word (which it clears first). */
+s3r_status s3r_page_summaries_checked(const s3r_paged_kv* kv, int32_t tail_only,
+                                      void* kmin, void* kmax, uint32_t* status_word,
+                                      void* stream);
+
+/* Human-readable name of a status code (static storage). */
+const char* s3r_status_str(s3r_status status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int32_t s3r_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* S3R_H_ */

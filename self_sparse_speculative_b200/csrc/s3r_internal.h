@@ -1,0 +1,97 @@
+// Host-side interface between the C ABI (s3r_api.cu) and the kernel files.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/s3r.h"
+
+namespace s3r {
+
+// Tokens per pipeline stage of the tensor-core attention kernel (one 64-token
+// page, or four 16-token pages).
+constexpr int kStageTokens = 64;
+// Upper bound on the pages one attention CTA processes (page list held in
+// shared memory).
+constexpr int kMaxSplitPages = 512;
+constexpr int kMaxPagesPerSeq = 8192;
+constexpr int kMaxGamma = 16;
+
+// Workspace header: word 0 is the device status word; the rest is reserved.
+constexpr size_t kWsHeader = 256;
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct AttnParams {
+  const void* q;
+  void* out;
+  float* lse;
+  const int32_t* block_table;
+  const int32_t* context_lens;
+  const int32_t* page_list;   // sparse: selected [S, Hkv, budget]; dense: nullptr
+  const void* k_cache;
+  const void* v_cache;
+  int32_t S, Hq, Hkv, G, D, P, R, rows;
+  int32_t max_pages, num_pages_total, budget;
+  int32_t nsplit, chunk_pages;   // grid splits per (seq, kv head) and pages per split
+  float scale_log2;              // scale * log2(e)
+  uint32_t* status;
+  uint32_t* tickets;             // [S * Hkv]
+  float* part_ml;                // [S * Hkv, nsplit, rows, 2]  (running max in log2 units, sum)
+  float* part_o;                 // [S * Hkv, nsplit, rows, D]  (unnormalised)
+};
+
+// Split plan shared by the workspace-size query and the launch.
+struct AttnPlan {
+  int32_t nsplit;
+  int32_t chunk_pages;
+  size_t ws_bytes;
+  size_t off_tickets, off_ml, off_o;
+};
+AttnPlan plan_attention(const s3r_paged_kv& kv, int32_t rows, int32_t budget_pages);
+
+cudaError_t launch_summaries(const s3r_paged_kv& kv, int tail_only, void* kmin, void* kmax,
+                             uint32_t* status, cudaStream_t st);
+cudaError_t launch_select(const s3r_paged_kv& kv, const void* kmin, const void* kmax,
+                          const void* q, int32_t budget, int32_t* selected, uint32_t* status,
+                          cudaStream_t st);
+cudaError_t launch_attention(const s3r_paged_kv& kv, const AttnParams& p, cudaStream_t st,
+                             s3r_status* api_status);
+
+struct SamplePlan {
+  int32_t nrows;        // rows with statistics (2*gamma+1 per sequence, or num_rows)
+  int32_t nseq;         // sequences (or rows for plain sampling)
+  int32_t c1, ch1;      // pass-1 chunks per row and elements per chunk
+  int32_t c2, ch2;      // pass-2 chunks per sequence and elements per chunk
+  size_t ws_bytes;
+  size_t off_tk_row, off_tk_seq1, off_tk_seq2, off_j, off_part1, off_stats, off_part2;
+  size_t memset_bytes;  // bytes from the start of the workspace cleared per call
+};
+SamplePlan plan_sampling(int32_t nseq, int32_t gamma, int32_t vocab);
+
+struct SampleParams {
+  const void* target;      // spec: [S, R, V]; plain: [N, V]
+  const void* draft;       // spec: [S, gamma, V]; plain: unused
+  const int32_t* draft_tokens;
+  const float* u_accept;
+  const float* u_sample;   // spec: [S, R]; plain: [N]
+  int32_t* out_tokens;     // spec: [S, R]; plain: [N]
+  int32_t* num_accepted;   // spec only
+  int32_t nseq, gamma, vocab;
+  float inv_temp;          // 1 / T
+  double inv_temp_d;
+  uint32_t* status;
+  uint32_t* tk_row;
+  uint32_t* tk_seq1;
+  uint32_t* tk_seq2;
+  int32_t* jsel;
+  void* part1;             // [nrows, c1] {float max, float pad, double sum}
+  double* stats;           // [nrows, 2] {max, Z}
+  double* part2;           // [nseq, c2]
+  int32_t c1, ch1, c2, ch2;
+};
+cudaError_t launch_sampling(const SampleParams& p, s3r_dtype dt, bool spec, cudaStream_t st);
+
+}  // namespace s3r

@@ -1,0 +1,183 @@
+"""ctypes binding of libs3r (include/s3r.h): argument marshalling only.
+
+Each function has the name of the C entry point it calls and takes torch
+tensors (device memory) or raw device addresses; every step of the computation
+runs in the library's CUDA kernels. A non-OK status raises S3RError. The
+library must have been built (``python -m self_sparse_speculative_b200.build``);
+if it is missing, importing this module raises ImportError - there is no
+fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libs3r.so")
+
+S3R_OK, S3R_ERR_INVALID_ARG, S3R_ERR_UNSUPPORTED, S3R_ERR_WORKSPACE, S3R_ERR_CUDA, S3R_ERR_DEVICE_CHECK = range(6)
+S3R_F32, S3R_BF16 = 0, 1
+S3R_DEV_BAD_CONTEXT_LEN, S3R_DEV_BAD_PAGE_ID, S3R_DEV_BAD_TOKEN_ID, S3R_DEV_WAIT_TIMEOUT = 0x1, 0x2, 0x4, 0x8
+
+EXPORTED = [
+    "s3r_page_summaries", "s3r_page_summaries_checked", "s3r_sparse_draft_attn", "s3r_verify_attn",
+    "s3r_spec_sample", "s3r_sample_tokens", "s3r_attn_workspace_bytes", "s3r_sample_workspace_bytes",
+    "s3r_device_status", "s3r_status_str", "s3r_version",
+]
+
+
+class S3RError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {status_str(status)}")
+
+
+class PagedKV(ctypes.Structure):
+    _fields_ = [
+        ("num_seqs", ctypes.c_int32), ("num_q_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32), ("page_size", ctypes.c_int32), ("max_pages_per_seq", ctypes.c_int32),
+        ("num_pages_total", ctypes.c_int32), ("dtype", ctypes.c_int32),
+        ("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p),
+        ("block_table", ctypes.c_void_p), ("context_lens", ctypes.c_void_p),
+    ]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libs3r.so is not built ({LIB_PATH}); run python -m self_sparse_speculative_b200.build")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, f32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+    kvp = ctypes.POINTER(PagedKV)
+    sig = {
+        "s3r_page_summaries": ([kvp, i32, vp, vp, vp], i32),
+        "s3r_page_summaries_checked": ([kvp, i32, vp, vp, vp, vp], i32),
+        "s3r_sparse_draft_attn": ([kvp, vp, vp, vp, i32, f32, vp, vp, vp, vp, sz, vp], i32),
+        "s3r_verify_attn": ([kvp, vp, i32, f32, vp, vp, vp, sz, vp], i32),
+        "s3r_spec_sample": ([vp, vp, i32, vp, vp, vp, i32, i32, i32, f32, vp, vp, vp, sz, vp], i32),
+        "s3r_sample_tokens": ([vp, i32, i32, i32, f32, vp, vp, vp, sz, vp], i32),
+        "s3r_attn_workspace_bytes": ([kvp, i32, i32], sz),
+        "s3r_sample_workspace_bytes": ([i32, i32, i32], sz),
+        "s3r_device_status": ([vp, ctypes.POINTER(ctypes.c_uint32), vp], i32),
+        "s3r_status_str": ([i32], ctypes.c_char_p),
+        "s3r_version": ([], i32),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = res
+    return lib
+
+
+_lib = _load()
+
+
+def lib():
+    return _lib
+
+
+def status_str(status: int) -> str:
+    return _lib.s3r_status_str(int(status)).decode()
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(fn, st):
+    if st != S3R_OK:
+        raise S3RError(fn, st)
+
+
+def dtype_code(dt) -> int:
+    import torch
+    if dt in (torch.bfloat16, "bf16", S3R_BF16):
+        return S3R_BF16
+    if dt in (torch.float32, "f32", S3R_F32):
+        return S3R_F32
+    raise ValueError(f"unsupported dtype {dt}")
+
+
+def paged_kv(k_cache, v_cache, block_table, context_lens, num_q_heads: int) -> PagedKV:
+    """Describe a cache [num_pages_total, Hkv, P, D] with its block table."""
+    n, h, p, d = k_cache.shape
+    return PagedKV(int(block_table.shape[0]), int(num_q_heads), int(h), int(d), int(p),
+                   int(block_table.shape[1]), int(n), dtype_code(k_cache.dtype),
+                   _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(context_lens))
+
+
+def s3r_attn_workspace_bytes(kv: PagedKV, rows: int, budget_pages: int) -> int:
+    return int(_lib.s3r_attn_workspace_bytes(ctypes.byref(kv), rows, budget_pages))
+
+
+def s3r_sample_workspace_bytes(num_seqs: int, gamma: int, vocab: int) -> int:
+    return int(_lib.s3r_sample_workspace_bytes(num_seqs, gamma, vocab))
+
+
+def s3r_page_summaries(kv: PagedKV, tail_only: int, kmin, kmax, stream=None, status_word=None):
+    if status_word is None:
+        st = _lib.s3r_page_summaries(ctypes.byref(kv), int(tail_only), _ptr(kmin), _ptr(kmax), _stream(stream))
+    else:
+        st = _lib.s3r_page_summaries_checked(ctypes.byref(kv), int(tail_only), _ptr(kmin), _ptr(kmax),
+                                             _ptr(status_word), _stream(stream))
+    _check("s3r_page_summaries", st)
+
+
+def s3r_sparse_draft_attn(kv: PagedKV, kmin, kmax, q, budget_pages: int, scale: float, selected, out,
+                          lse, workspace, workspace_bytes=None, stream=None):
+    wb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    st = _lib.s3r_sparse_draft_attn(ctypes.byref(kv), _ptr(kmin), _ptr(kmax), _ptr(q), int(budget_pages),
+                                    float(scale), _ptr(selected), _ptr(out), _ptr(lse), _ptr(workspace), wb,
+                                    _stream(stream))
+    _check("s3r_sparse_draft_attn", st)
+
+
+def s3r_verify_attn(kv: PagedKV, q, rows: int, scale: float, out, lse, workspace, workspace_bytes=None,
+                    stream=None):
+    wb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    st = _lib.s3r_verify_attn(ctypes.byref(kv), _ptr(q), int(rows), float(scale), _ptr(out), _ptr(lse),
+                              _ptr(workspace), wb, _stream(stream))
+    _check("s3r_verify_attn", st)
+
+
+def s3r_spec_sample(target_logits, draft_logits, logit_dtype, draft_tokens, u_accept, u_sample,
+                    num_seqs: int, gamma: int, vocab: int, temperature: float, out_tokens, num_accepted,
+                    workspace, workspace_bytes=None, stream=None):
+    wb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    st = _lib.s3r_spec_sample(_ptr(target_logits), _ptr(draft_logits), dtype_code(logit_dtype),
+                              _ptr(draft_tokens), _ptr(u_accept), _ptr(u_sample), int(num_seqs), int(gamma),
+                              int(vocab), float(temperature), _ptr(out_tokens), _ptr(num_accepted),
+                              _ptr(workspace), wb, _stream(stream))
+    _check("s3r_spec_sample", st)
+
+
+def s3r_sample_tokens(logits, logit_dtype, num_rows: int, vocab: int, temperature: float, u, tokens,
+                      workspace, workspace_bytes=None, stream=None):
+    wb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    st = _lib.s3r_sample_tokens(_ptr(logits), dtype_code(logit_dtype), int(num_rows), int(vocab),
+                                float(temperature), _ptr(u), _ptr(tokens), _ptr(workspace), wb,
+                                _stream(stream))
+    _check("s3r_sample_tokens", st)
+
+
+def s3r_device_status(workspace, stream=None):
+    """(status, bits) of the most recent call that used `workspace` (synchronises)."""
+    bits = ctypes.c_uint32(0)
+    st = _lib.s3r_device_status(_ptr(workspace), ctypes.byref(bits), _stream(stream))
+    return int(st), int(bits.value)
+
+
+def s3r_version() -> int:
+    return int(_lib.s3r_version())

@@ -149,16 +149,20 @@ class Workload:
     in host memory at once.
     """
 
-    def __init__(self, ws: WorkloadSpec, seed: int = 0):
+    def __init__(self, ws: WorkloadSpec, seed: int = 0, context_lens=None):
         self.spec = ws
         self.seed = seed
         S, P = ws.num_seqs, ws.page_size
-        if ws.context:
+        if context_lens is not None:
+            lens = np.asarray(context_lens, dtype=np.int64)
+            assert lens.shape == (S,)
+        elif ws.context:
             lens = np.full(S, ws.context, dtype=np.int64)
         else:
             u = self._rng(_S_LENS).uniform(ws.ragged_lo, ws.ragged_hi, size=S)
             lens = (np.floor(u / P) * P).astype(np.int64)
-        lens = np.maximum(lens, ws.rows)
+        if context_lens is None:
+            lens = np.maximum(lens, ws.rows)
         self.context_lens = lens.astype(np.int32)
         self.pages_per_seq = ((lens + P - 1) // P).astype(np.int64)
         self.max_pages_per_seq = int(self.pages_per_seq.max())

@@ -1,0 +1,147 @@
+"""GPU vs float64 oracle on small workloads that the oracle finishes in
+seconds: several tiles, several splits, ragged and partial pages, both the
+M=64 and M=128 tensor-core tiles, head_dim 64/128, page 16/64, fp32 and bf16.
+Every GPU result comes from the C ABI (libs3r.so)."""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+from self_sparse_speculative_b200 import s3r                      # noqa: E402
+from self_sparse_speculative_b200.step import DecodeStep          # noqa: E402
+from self_sparse_speculative_b200.workloads import Workload, custom_spec, spec, to_float64  # noqa: E402
+
+import oracle.reference_run as RR                                  # noqa: E402
+
+CASES = {
+    # the tiny fp32 workload itself
+    "tiny-fp32": (spec(0), None),
+    # bf16, D128, P64, G4, R5 -> 20 packed rows (M=64 tile); a sequence with
+    # fewer pages than the budget, a partial tail page, several splits
+    "bf16-d128-p64": (custom_spec(1, num_seqs=3, num_q_heads=8, num_kv_heads=2, budget_pages=4, vocab=1000),
+                      [130, 64, 1007 + 1024]),
+    # G8 x R9 = 72 packed rows -> M=128 tile
+    "bf16-g8-r9": (custom_spec(1, num_seqs=2, num_q_heads=16, num_kv_heads=2, gamma=8, budget_pages=3,
+                               vocab=2048), [300, 777]),
+    # D64 with 16-token pages (four pages per 64-token stage)
+    "bf16-d64-p16": (custom_spec(1, num_seqs=3, num_q_heads=8, num_kv_heads=2, head_dim=64, page_size=16,
+                                 gamma=3, budget_pages=6, vocab=999), [500, 33, 16 * 40 + 5]),
+    # fp32 with D128, P64 and fp32 logits
+    "f32-d128-p64": (custom_spec(0, num_seqs=2, num_q_heads=6, num_kv_heads=2, head_dim=128, page_size=64,
+                                 budget_pages=2, vocab=777), [200, 4 * 64 + 1]),
+    # shortest legal history: L = R for verify
+    "bf16-min-len": (custom_spec(1, num_seqs=2, num_q_heads=4, num_kv_heads=1, gamma=2, budget_pages=1,
+                                 vocab=512), [3, 70]),
+}
+
+
+def _run(name):
+    s, lens = CASES[name]
+    wl = Workload(s, seed=1, context_lens=lens)
+    st = DecodeStep(wl)
+    st.summaries(tail_only=False)
+    st.round()
+    torch.cuda.synchronize()
+    return wl, st
+
+
+@pytest.fixture(scope="module", params=list(CASES))
+def case(request):
+    return request.param, _run(request.param)
+
+
+def test_device_status_clean(case):
+    name, (wl, st) = case
+    for ws_name, (status, bits) in st.device_checks().items():
+        assert status == s3r.S3R_OK, f"{name} {ws_name}: device status bits {bits:#x}"
+
+
+def test_summaries_bit_exact(case):
+    name, (wl, st) = case
+    dt = wl.spec.kv_dtype
+    kmin = st.kmin.float().cpu().numpy().astype(np.float64)
+    kmax = st.kmax.float().cpu().numpy().astype(np.float64)
+    for b in range(wl.spec.num_seqs):
+        ref = RR.oracle_attention_seq(wl, b, draft_steps=[])
+        assert np.array_equal(kmin[ref["phys"]], ref["kmin"]), f"{name} seq {b} kmin"
+        assert np.array_equal(kmax[ref["phys"]], ref["kmax"]), f"{name} seq {b} kmax"
+
+
+def test_selection_and_attention(case):
+    name, (wl, st) = case
+    ws = wl.spec
+    dt = ws.kv_dtype
+    tally = RR.Tally()
+    sel = st.selected.cpu().numpy()
+    dout = st.draft_out.float().cpu().numpy()
+    dlse = st.draft_lse.cpu().numpy()
+    vout = st.verify_out.float().cpu().numpy()
+    vlse = st.verify_lse.cpu().numpy()
+    for b in range(ws.num_seqs):
+        ref = RR.oracle_attention_seq(wl, b)
+        for i, d in ref["draft"].items():
+            ok = RR.compare_selection(f"{name} seq {b} draft {i}", sel[i, b], d["selected"], d["gaps"], tally)
+            n_b = int(wl.pages_per_seq[b])
+            assert np.all(sel[i, b][:, min(n_b, ws.budget_pages):] == -1)
+            if all(ok):
+                RR.assert_close(f"{name} seq {b} draft {i} out", dout[i, b], d["out"], dt)
+                RR.assert_close(f"{name} seq {b} draft {i} lse", dlse[i, b], d["lse"], dt)
+        RR.assert_close(f"{name} seq {b} verify out", vout[b], ref["verify_out"], dt)
+        RR.assert_close(f"{name} seq {b} verify lse", vlse[b], ref["verify_lse"], dt)
+    assert tally.near_ties <= max(0, int(1e-4 * tally.decisions)), tally.notes
+
+
+def test_sampling_round(case):
+    """Draft draws, accept/reject and the drawn token of the GPU round."""
+    name, (wl, st) = case
+    tally = RR.Tally()
+    x = st.draft_tokens.cpu().numpy()
+    out = st.out_tokens.cpu().numpy()
+    nacc = st.num_accepted.cpu().numpy()
+    for b in range(wl.spec.num_seqs):
+        ref = RR.oracle_sampling_seq(wl, b)
+        RR.compare_sampling(f"{name} seq {b}", x[b], out[b], nacc[b], ref, tally)
+    assert tally.near_ties <= max(0, int(1e-4 * tally.decisions)), tally.notes
+
+
+def test_spec_sample_with_oracle_drafts(case):
+    """s3r_spec_sample fed the oracle's own draft tokens."""
+    name, (wl, st) = case
+    ws = wl.spec
+    refs = [RR.oracle_sampling_seq(wl, b) for b in range(ws.num_seqs)]
+    xo = torch.from_numpy(np.stack([r["x"] for r in refs]).astype(np.int32)).cuda()
+    st.draft_tokens.copy_(xo)
+    st.sample()
+    torch.cuda.synchronize()
+    out = st.out_tokens.cpu().numpy()
+    nacc = st.num_accepted.cpu().numpy()
+    tally = RR.Tally()
+    for b, r in enumerate(refs):
+        # the draws are the oracle's, so only accept decisions and the draw count
+        r2 = dict(r, x_margin=np.full_like(r["x_margin"], 1.0))
+        RR.compare_sampling(f"{name} seq {b}", r["x"], out[b], nacc[b], r2, tally)
+    assert tally.near_ties <= max(0, int(1e-4 * tally.decisions)), tally.notes
+
+
+def test_tail_only_summaries_touch_only_tail_pages(case):
+    name, (wl, st) = case
+    st.kmin.zero_()
+    st.kmax.zero_()
+    st.summaries(tail_only=True)
+    torch.cuda.synchronize()
+    kmin = st.kmin.float().cpu().numpy().astype(np.float64)
+    tails = set()
+    for b in range(wl.spec.num_seqs):
+        n = int(wl.pages_per_seq[b])
+        tails.add(int(wl.block_table[b, n - 1]))
+        ref = RR.oracle_attention_seq(wl, b, draft_steps=[])
+        assert np.array_equal(kmin[ref["phys"][n - 1]], ref["kmin"][n - 1])
+    others = [p for p in range(wl.num_pages_total) if p not in tails]
+    assert np.all(kmin[others] == 0.0)
+    st.summaries(tail_only=False)
+    torch.cuda.synchronize()
