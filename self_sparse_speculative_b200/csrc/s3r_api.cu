@@ -41,6 +41,7 @@ s3r_status check_attn(const s3r_paged_kv* kv, int32_t rows, int32_t budget, bool
   const int G = kv->num_q_heads / kv->num_kv_heads;
   if ((int64_t)G * rows > 128) return S3R_ERR_UNSUPPORTED;
   if (!sparse && rows > kMaxGamma + 1) return S3R_ERR_UNSUPPORTED;
+  if (kv->num_seqs > kMaxSeqs) return S3R_ERR_UNSUPPORTED;
   return S3R_OK;
 }
 

@@ -29,79 +29,13 @@
 #include <cmath>
 #include <cstring>
 
+#include "s3r_attn_common.cuh"
 #include "s3r_device.cuh"
 #include "s3r_internal.h"
 
 namespace s3r {
 namespace {
 
-constexpr int kTcThreads = 192;     // 4 softmax warps + producer + MMA
-constexpr int kStages = 2;
-constexpr float kRescaleTau = 8.0f; // log2 units
-constexpr float kLn2 = 0.6931471805599453f;
-
-// ------------------------------------------------------------------ combine
-template <typename OutT>
-__device__ __forceinline__ void store_out4(OutT* dst, float a, float b, float c, float d);
-template <>
-__device__ __forceinline__ void store_out4<__nv_bfloat16>(__nv_bfloat16* dst, float a, float b, float c, float d) {
-  uint2 v = make_uint2(pack_bf16x2(a, b), pack_bf16x2(c, d));
-  *reinterpret_cast<uint2*>(dst) = v;
-}
-template <>
-__device__ __forceinline__ void store_out4<float>(float* dst, float a, float b, float c, float d) {
-  *reinterpret_cast<float4*>(dst) = make_float4(a, b, c, d);
-}
-
-__device__ __forceinline__ size_t out_row_offset(const AttnParams& p, int b, int h, int i) {
-  const int r = i / p.G, g = i - (i / p.G) * p.G;
-  return ((size_t)(b * p.R + r) * p.Hq + (size_t)h * p.G + g);
-}
-
-// Merge the nsplit_u partial states of unit (b, h) into the final output.
-// Runs on `nthreads` consecutive threads starting at thread 0.
-template <typename OutT>
-__device__ void combine_unit(const AttnParams& p, int b, int h, int nsplit_u, int nthreads) {
-  const int unit = b * p.Hkv + h;
-  const int D4 = p.D / 4;
-  for (int idx = threadIdx.x; idx < p.rows * D4; idx += nthreads) {
-    const int i = idx / D4, d4 = idx - (idx / D4) * D4;
-    float M = -INFINITY;
-    for (int s = 0; s < nsplit_u; ++s) {
-      const float m = __ldcg(p.part_ml + (((size_t)unit * p.nsplit + s) * p.rows + i) * 2);
-      M = fmaxf(M, m);
-    }
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    float Ls = 0.f;
-    if (M != -INFINITY) {
-      for (int s = 0; s < nsplit_u; ++s) {
-        const size_t pi = ((size_t)unit * p.nsplit + s) * p.rows + i;
-        const float m = __ldcg(p.part_ml + pi * 2), l = __ldcg(p.part_ml + pi * 2 + 1);
-        if (m == -INFINITY || l == 0.f) continue;
-        const float w = exp2f(m - M);
-        Ls += l * w;
-        const float4 o = __ldcg(reinterpret_cast<const float4*>(p.part_o + pi * p.D) + d4);
-        acc.x += w * o.x; acc.y += w * o.y; acc.z += w * o.z; acc.w += w * o.w;
-      }
-    }
-    const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
-    const size_t orow = out_row_offset(p, b, h, i);
-    store_out4<OutT>(static_cast<OutT*>(p.out) + orow * p.D + d4 * 4, acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-    if (d4 == 0 && p.lse) p.lse[orow] = Ls > 0.f ? (M + log2f(Ls)) * kLn2 : -INFINITY;
-  }
-}
-
-// Outputs of a unit whose context length is invalid: zeros and lse = -inf.
-template <typename OutT>
-__device__ void write_empty_unit(const AttnParams& p, int b, int h, int nthreads) {
-  const int D4 = p.D / 4;
-  for (int idx = threadIdx.x; idx < p.rows * D4; idx += nthreads) {
-    const int i = idx / D4, d4 = idx - (idx / D4) * D4;
-    const size_t orow = out_row_offset(p, b, h, i);
-    store_out4<OutT>(static_cast<OutT*>(p.out) + orow * p.D + d4 * 4, 0.f, 0.f, 0.f, 0.f);
-    if (d4 == 0 && p.lse) p.lse[orow] = -INFINITY;
-  }
-}
 
 // Geometry of one CTA's share of a unit.
 struct SplitGeom {
@@ -140,344 +74,6 @@ __device__ __forceinline__ void resolve_page(const AttnParams& p, int b, int h, 
   *phys_out = phys;
 }
 
-// ================================================================== tcgen05 kernel
-template <int M, int D>
-struct TcLayout {
-  static constexpr int kHalves = D / 64;
-  static constexpr uint32_t kQBytes = M * D * 2;
-  static constexpr uint32_t kPBytes = M * 128;                // 64 tokens x bf16
-  static constexpr uint32_t kTileBytes = kStageTokens * D * 2; // K or V of one stage
-  static constexpr uint32_t kOffP = kQBytes;
-  static constexpr uint32_t kOffKV = kOffP + 2 * kPBytes;
-  static constexpr uint32_t kDynBytes = kOffKV + kStages * 2 * kTileBytes;
-  static constexpr uint32_t kTmemCols = 256;                   // S0 | S1 | O
-};
-
-template <int M, int D>
-__global__ void __launch_bounds__(kTcThreads, 1)
-attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-               const AttnParams p) {
-  using Lay = TcLayout<M, D>;
-  extern __shared__ __align__(1024) uint8_t dyn_raw[];
-  uint8_t* dyn = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ __align__(8) uint64_t s_bar[2 * kStages + 7];
-  __shared__ uint32_t s_tmem;
-  __shared__ int s_abort;
-  __shared__ int s_ticket;
-  __shared__ int32_t s_lp[kMaxSplitPages];
-  __shared__ int32_t s_phys[kMaxSplitPages];
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const SplitGeom g = split_geom(p, b, split);
-  if (g.bad_len) {
-    if (split == 0) {
-      if (tid == 0) flag_status(p.status, S3R_DEV_BAD_CONTEXT_LEN);
-      write_empty_unit<__nv_bfloat16>(p, b, h, kTcThreads);
-    }
-    return;
-  }
-  if (split >= g.nsplit_u) return;
-  const int ppt = kStageTokens / p.P;                 // pages per stage
-  const int nstages = (g.npg + ppt - 1) / ppt;
-
-  const uint32_t bar_full = smem_addr(&s_bar[0]);
-  const uint32_t bar_empty = smem_addr(&s_bar[kStages]);
-  const uint32_t bar_sfull = smem_addr(&s_bar[2 * kStages]);      // 2
-  const uint32_t bar_pfull = smem_addr(&s_bar[2 * kStages + 2]);  // 2
-  const uint32_t bar_odone = smem_addr(&s_bar[2 * kStages + 4]);
-  const uint32_t bar_td = smem_addr(&s_bar[2 * kStages + 5]);
-  auto bar = [](uint32_t base, int i) { return base + 8u * i; };
-
-  uint8_t* sQ = dyn;
-  uint8_t* sP = dyn + Lay::kOffP;
-  uint8_t* sKV = dyn + Lay::kOffKV;
-  const uint32_t aQ = smem_addr(sQ), aP = smem_addr(sP), aKV = smem_addr(sKV);
-
-  // ---- setup
-  if (warp == 5) {
-    tmem_alloc(smem_addr(&s_tmem), Lay::kTmemCols);
-    tmem_relinquish();
-  }
-  if (tid == 0) {
-    for (int i = 0; i < kStages; ++i) { mbar_init(bar(bar_full, i), 1); mbar_init(bar(bar_empty, i), 1); }
-    for (int i = 0; i < 2; ++i) { mbar_init(bar(bar_sfull, i), 1); mbar_init(bar(bar_pfull, i), 128); }
-    mbar_init(bar_odone, 1);
-    mbar_init(bar_td, 1);
-    s_abort = 0;
-    fence_barrier_init();
-  }
-  if (warp == 4 && lane == 0) { prefetch_tensormap(&tmK); prefetch_tensormap(&tmV); }
-  for (int k = tid; k < g.npg; k += kTcThreads) resolve_page(p, b, h, g, k, &s_lp[k], &s_phys[k]);
-  if (tid < 128) {
-    // Q rows -> tile rows, bf16, K-major 128-byte swizzle; padding rows zero
-    const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(p.q);
-    constexpr int kChunks = D / 8;                   // 16-byte chunks per row
-    for (int idx = tid; idx < M * kChunks; idx += 128) {
-      const int slot = idx / kChunks, c16 = idx - (idx / kChunks) * kChunks;
-      const int i = (M == 64) ? 4 * (slot & 15) + (slot >> 4) : 4 * (slot & 31) + (slot >> 5);
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (i < p.rows) v = *reinterpret_cast<const uint4*>(q + out_row_offset(p, b, h, i) * D + c16 * 8);
-      const int half = c16 >> 3, c = c16 & 7;
-      *reinterpret_cast<uint4*>(sQ + half * (M * 128) + slot * 128 + ((c ^ (slot & 7)) << 4)) = v;
-    }
-    for (int idx = tid; idx < (int)(2 * Lay::kPBytes / 16); idx += 128)
-      reinterpret_cast<uint4*>(sP)[idx] = make_uint4(0u, 0u, 0u, 0u);
-    fence_proxy_async_smem();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = s_tmem;
-  const uint32_t tS = tmem, tO = tmem + 128;
-
-  if (warp == 4) {
-    // ================= TMA producer
-    if (lane == 0) {
-      const uint64_t pol = l2_policy_evict_first();
-      int issued = 0;
-      for (int j = 0; j < nstages; ++j) {
-        const int st = j % kStages;
-        if (!mbar_wait(bar(bar_empty, st), ((j / kStages) & 1) ^ 1, &s_abort, p.status)) break;
-        int nreal = 0;
-        for (int pp = 0; pp < ppt; ++pp) {
-          const int k = j * ppt + pp;
-          if (k < g.npg && s_phys[k] >= 0) ++nreal;
-        }
-        mbar_arrive_expect_tx(bar(bar_full, st), (uint32_t)nreal * Lay::kHalves * 2u * (uint32_t)p.P * 128u);
-        const uint32_t dK = aKV + st * 2 * Lay::kTileBytes, dV = dK + Lay::kTileBytes;
-        for (int pp = 0; pp < ppt; ++pp) {
-          const int k = j * ppt + pp;
-          if (k >= g.npg || s_phys[k] < 0) continue;
-          const int z = s_phys[k] * p.Hkv + h;
-          for (int hh = 0; hh < Lay::kHalves; ++hh) {
-            const uint32_t off = hh * (kStageTokens * 128) + pp * (p.P * 128);
-            tma_load_3d(dK + off, &tmK, bar(bar_full, st), hh * 64, 0, z, pol);
-            tma_load_3d(dV + off, &tmV, bar(bar_full, st), hh * 64, 0, z, pol);
-          }
-        }
-        issued = j + 1;
-      }
-      for (int j = max(0, issued - kStages); j < issued; ++j)
-        mbar_wait_drain(bar(bar_full, j % kStages), (j / kStages) & 1, p.status);
-    }
-  } else if (warp == 5) {
-    // ================= MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idQK = idesc_bf16_f32(M, kStageTokens, false, false);
-      constexpr uint32_t idPV = idesc_bf16_f32(M, D, false, true);
-      for (int j = 0; j <= nstages; ++j) {
-        if (j < nstages) {
-          const int st = j % kStages;
-          if (!mbar_wait(bar(bar_full, st), (j / kStages) & 1, &s_abort, p.status)) break;
-          tc_fence_after();
-          const uint32_t kb = aKV + st * 2 * Lay::kTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const int hh = kk >> 2, sub = kk & 3;
-            const uint64_t a = smem_desc_sw128(aQ + hh * (M * 128) + sub * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(kb + hh * (kStageTokens * 128) + sub * 32, 16, 1024);
-            umma_f16(tS + (j & 1) * kStageTokens, a, bd, idQK, kk > 0 ? 1u : 0u);
-          }
-          umma_commit(bar(bar_sfull, j & 1));
-        }
-        if (j >= 1) {
-          const int jp = j - 1, stp = jp % kStages;
-          if (!mbar_wait(bar(bar_pfull, jp & 1), (jp >> 1) & 1, &s_abort, p.status)) break;
-          tc_fence_after();
-          const uint32_t vb = aKV + stp * 2 * Lay::kTileBytes + Lay::kTileBytes;
-          const uint32_t pb = aP + (jp & 1) * Lay::kPBytes;
-#pragma unroll
-          for (int kk = 0; kk < kStageTokens / 16; ++kk) {
-            const uint64_t a = smem_desc_sw128(pb + kk * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(vb + kk * (16 * 128), kStageTokens * 128, 1024);
-            umma_f16(tO, a, bd, idPV, (jp > 0 || kk > 0) ? 1u : 0u);
-          }
-          umma_commit(bar(bar_empty, stp));
-          umma_commit(bar_odone);
-        }
-      }
-      umma_commit(bar_td);
-    }
-  } else {
-    // ================= softmax warps (tid 0..127)
-    const int q4 = warp;
-    const int slot = (M == 64) ? (lane < 16 ? 16 * q4 + lane : -1) : 32 * q4 + lane;
-    const int i = 4 * lane + q4;                       // packed row of this thread's slot
-    const bool valid_row = slot >= 0 && i < p.rows;
-    const int r = valid_row ? i / p.G : 0;
-    const int qpos = g.L - p.R + r;                    // this row's position
-    const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
-    float m_run = -INFINITY, l_run = 0.f;
-    bool ok = true;
-    for (int j = 0; j < nstages; ++j) {
-      const int sb = j & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(bar_sfull, sb), (j >> 1) & 1, &s_abort, p.status))) { ok = false; break; }
-      tc_fence_after();
-      float s[kStageTokens];
-      tmem_ld32(tS + lane_base + sb * kStageTokens, s);
-      tmem_ld32(tS + lane_base + sb * kStageTokens + 32, s + 32);
-      tmem_wait_ld();
-
-      // token validity of this stage: positions lp*P + t must be < L, and
-      // <= the row position (causal); pages may be missing at the end
-      const int k0 = j * ppt;
-      bool any_invalid = false;      // some token of the stage must be zeroed in V
-      bool need_mask = false;        // some column is masked for some row
-      for (int pp = 0; pp < ppt; ++pp) {
-        const int k = k0 + pp;
-        if (k >= g.npg || s_phys[k] < 0) { any_invalid = true; continue; }
-        const int last_pos = s_lp[k] * p.P + p.P - 1;
-        if (last_pos >= g.L) any_invalid = true;
-        if (last_pos > g.L - p.R) need_mask = true;
-      }
-      need_mask |= any_invalid;
-      float mx = -INFINITY;
-      if (need_mask) {
-#pragma unroll
-        for (int c = 0; c < kStageTokens; ++c) {
-          const int k = k0 + c / p.P;
-          bool v = false;
-          if (k < g.npg && s_phys[k] >= 0) {
-            const int pos = s_lp[k] * p.P + (c % p.P);
-            v = pos < g.L && pos <= qpos;
-          }
-          s[c] = v ? s[c] * p.scale_log2 : -INFINITY;
-          mx = fmaxf(mx, s[c]);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < kStageTokens; ++c) { s[c] *= p.scale_log2; mx = fmaxf(mx, s[c]); }
-      }
-      // lazy running-max update
-      float alpha = 1.f;
-      bool rescale = false;
-      if (valid_row) {
-        if (m_run == -INFINITY) {
-          m_run = mx;                                   // O rows are still zero
-        } else if (mx > m_run + kRescaleTau) {
-          alpha = ex2(m_run - mx);
-          m_run = mx;
-          l_run *= alpha;
-          rescale = true;
-        }
-      }
-      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-      // P = 2^(s - m), rounded to bf16; l sums the rounded values
-      uint32_t pk[kStageTokens / 2];
-      float lsum = 0.f;
-#pragma unroll
-      for (int c = 0; c < kStageTokens; c += 2) {
-        const float e0 = ex2(s[c] - m_use), e1 = ex2(s[c + 1] - m_use);
-        pk[c / 2] = pack_bf16x2(e0, e1);
-        const __nv_bfloat162 rb = *reinterpret_cast<__nv_bfloat162*>(&pk[c / 2]);
-        lsum += __low2float(rb) + __high2float(rb);
-      }
-      if (valid_row) l_run += lsum;
-
-      // PV(j-1) must be complete before O is rescaled or P[sb] is rewritten
-      if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(bar_odone, (j - 1) & 1, &s_abort, p.status))) { ok = false; break; }
-      tc_fence_after();
-      if (__any_sync(0xffffffffu, rescale)) {
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          float o[32];
-          tmem_ld32(tO + lane_base + c0, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int c = 0; c < 32; ++c) o[c] *= alpha;
-          tmem_st32(tO + lane_base + c0, o);
-        }
-        tmem_wait_st();
-      }
-      if (any_invalid) {
-        // zero the V rows of tokens that do not exist (beyond L, missing
-        // pages) so that 0 * garbage cannot reach O
-        if (!__all_sync(0xffffffffu, mbar_wait(bar(bar_full, j % kStages), (j / kStages) & 1, &s_abort, p.status))) { ok = false; break; }
-        uint8_t* sV = sKV + (j % kStages) * 2 * Lay::kTileBytes + Lay::kTileBytes;
-        for (int idx = tid; idx < kStageTokens * Lay::kHalves * 8; idx += 128) {
-          const int t = idx / (Lay::kHalves * 8);
-          const int rem = idx - t * (Lay::kHalves * 8);
-          const int hh = rem >> 3, c = rem & 7;
-          const int k = k0 + t / p.P;
-          bool v = false;
-          if (k < g.npg && s_phys[k] >= 0) v = s_lp[k] * p.P + (t % p.P) < g.L;
-          if (!v) *reinterpret_cast<uint4*>(sV + hh * (kStageTokens * 128) + t * 128 + c * 16) = make_uint4(0u, 0u, 0u, 0u);
-        }
-      }
-      if (valid_row) {
-        uint8_t* prow = sP + sb * Lay::kPBytes + slot * 128;
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<uint4*>(prow + ((c ^ (slot & 7)) << 4)) =
-              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(bar(bar_pfull, sb));
-    }
-    // ---- epilogue
-    if (ok && nstages > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar_odone, (nstages - 1) & 1, &s_abort, p.status));
-    tc_fence_after();
-    const bool single = (g.nsplit_u == 1);
-    const int unit = b * p.Hkv + h;
-    const size_t pi = ((size_t)unit * p.nsplit + split) * p.rows + (valid_row ? i : 0);
-    const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
-    for (int c0 = 0; c0 < D; c0 += 32) {
-      float o[32];
-      tmem_ld32(tO + lane_base + c0, o);
-      tmem_wait_ld();
-      if (!valid_row) continue;
-      if (!ok || nstages == 0) {
-#pragma unroll
-        for (int c = 0; c < 32; ++c) o[c] = 0.f;
-      }
-      if (single) {
-        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) + out_row_offset(p, b, h, i) * D + c0;
-#pragma unroll
-        for (int c = 0; c < 32; c += 8)
-          *reinterpret_cast<uint4*>(dst + c) =
-              make_uint4(pack_bf16x2(o[c] * inv_l, o[c + 1] * inv_l), pack_bf16x2(o[c + 2] * inv_l, o[c + 3] * inv_l),
-                         pack_bf16x2(o[c + 4] * inv_l, o[c + 5] * inv_l), pack_bf16x2(o[c + 6] * inv_l, o[c + 7] * inv_l));
-      } else {
-        float* dst = p.part_o + pi * D + c0;
-#pragma unroll
-        for (int c = 0; c < 32; c += 4) *reinterpret_cast<float4*>(dst + c) = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
-      }
-    }
-    if (valid_row) {
-      if (!ok) { m_run = -INFINITY; l_run = 0.f; }
-      if (single) {
-        if (p.lse) p.lse[out_row_offset(p, b, h, i)] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
-      } else {
-        p.part_ml[pi * 2] = l_run > 0.f ? m_run : -INFINITY;
-        p.part_ml[pi * 2 + 1] = l_run;
-      }
-    }
-    if (!single) {
-      __threadfence();
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      if (tid == 0) s_ticket = atomicAdd(p.tickets + unit, 1u);
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      if (s_ticket == g.nsplit_u - 1) {
-        __threadfence();
-        combine_unit<__nv_bfloat16>(p, b, h, g.nsplit_u, 128);
-        if (tid == 0) p.tickets[unit] = 0u;
-      }
-    }
-  }
-
-  // ---- teardown: every role is done; wait for the MMAs, free TMEM
-  __syncwarp();
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 5) {
-    tc_fence_after();
-    if (lane == 0) mbar_wait_drain(bar_td, 0, p.status);
-    __syncwarp();
-    tmem_dealloc(tmem, Lay::kTmemCols);
-  }
-}
-
 // ================================================================== fp32 kernel
 constexpr int kF32Threads = 128;
 constexpr int kF32Tok = 16;
@@ -492,7 +88,7 @@ __global__ void __launch_bounds__(kF32Threads) attn_f32_kernel(const AttnParams 
   if (g.bad_len) {
     if (split == 0) {
       if (tid == 0) flag_status(p.status, S3R_DEV_BAD_CONTEXT_LEN);
-      write_empty_unit<float>(p, b, h, kF32Threads);
+      write_empty_unit<float>(p, b, h, tid, kF32Threads);
     }
     return;
   }
@@ -615,7 +211,7 @@ __global__ void __launch_bounds__(kF32Threads) attn_f32_kernel(const AttnParams 
     __syncthreads();
     if (s_ticket == g.nsplit_u - 1) {
       __threadfence();
-      combine_unit<float>(p, b, h, g.nsplit_u, kF32Threads);
+      combine_partials<float>(p, b, h, unit * p.nsplit, g.nsplit_u, kF32Threads);
       if (tid == 0) p.tickets[unit] = 0u;
     }
   }
@@ -638,6 +234,8 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
+}  // namespace
+
 // 3-D map over a [pages * Hkv, P, D] bf16 cache, box = 64 channels x P tokens x 1.
 bool make_cache_map(CUtensorMap* map, const void* base, const s3r_paged_kv& kv) {
   EncodeTiledFn enc = get_encode_fn();
@@ -653,20 +251,14 @@ bool make_cache_map(CUtensorMap* map, const void* base, const s3r_paged_kv& kv) 
   return r == CUDA_SUCCESS;
 }
 
-template <int M, int D>
-cudaError_t launch_tc(const s3r_paged_kv& kv, const AttnParams& p, cudaStream_t st, s3r_status* api) {
-  CUtensorMap mk, mv;
-  if (!make_cache_map(&mk, kv.k_cache, kv) || !make_cache_map(&mv, kv.v_cache, kv)) {
-    *api = S3R_ERR_CUDA;
-    return cudaErrorInvalidValue;
-  }
-  const size_t smem = TcLayout<M, D>::kDynBytes + 1024;
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<M, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  dim3 grid(p.nsplit, p.Hkv, p.S);
-  attn_tc_kernel<M, D><<<grid, kTcThreads, smem, st>>>(mk, mv, p);
-  return cudaGetLastError();
+int device_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) return 148;
+  return n;
 }
+
+namespace {
 
 template <int D>
 cudaError_t launch_f32(const AttnParams& p, cudaStream_t st) {
@@ -703,13 +295,18 @@ AttnPlan plan_attention(const s3r_paged_kv& kv, int32_t rows, int32_t budget_pag
   pl.chunk_pages = chunk_stages * ppt;
   pl.nsplit = (max_list + pl.chunk_pages - 1) / pl.chunk_pages;
   if (pl.nsplit < 1) pl.nsplit = 1;
+  // partial-result slots: fp32 path (unit, split); tensor-core path one slot
+  // per (unit, CTA sharing it), at most units + grid
+  const size_t slots_f32 = (size_t)units * pl.nsplit;
+  const size_t slots_tc = (size_t)units + kMaxPersistentCtas;
+  const size_t slots = kv.dtype == S3R_F32 ? slots_f32 : slots_tc;
   size_t off = kWsHeader;
   pl.off_tickets = off;
   off = align_up(off + sizeof(uint32_t) * units, 256);
   pl.off_ml = off;
-  off = align_up(off + sizeof(float) * 2 * (size_t)units * pl.nsplit * prow, 256);
+  off = align_up(off + sizeof(float) * 2 * slots * prow, 256);
   pl.off_o = off;
-  off = align_up(off + sizeof(float) * (size_t)units * pl.nsplit * prow * kv.head_dim, 256);
+  off = align_up(off + sizeof(float) * slots * prow * kv.head_dim, 256);
   pl.ws_bytes = off;
   return pl;
 }
@@ -719,9 +316,7 @@ cudaError_t launch_attention(const s3r_paged_kv& kv, const AttnParams& p, cudaSt
   if (kv.dtype == S3R_F32) {
     return kv.head_dim == 64 ? launch_f32<64>(p, st) : launch_f32<128>(p, st);
   }
-  const bool small = p.rows <= 64;
-  if (kv.head_dim == 64) return small ? launch_tc<64, 64>(kv, p, st, api) : launch_tc<128, 64>(kv, p, st, api);
-  return small ? launch_tc<64, 128>(kv, p, st, api) : launch_tc<128, 128>(kv, p, st, api);
+  return launch_attention_tc(kv, p, st, api);
 }
 
 }  // namespace s3r

@@ -13,11 +13,16 @@ namespace s3r {
 // Tokens per pipeline stage of the tensor-core attention kernel (one 64-token
 // page, or four 16-token pages).
 constexpr int kStageTokens = 64;
-// Upper bound on the pages one attention CTA processes (page list held in
-// shared memory).
+// Upper bound on the pages one fp32 attention CTA processes.
 constexpr int kMaxSplitPages = 512;
 constexpr int kMaxPagesPerSeq = 8192;
 constexpr int kMaxGamma = 16;
+// Sequences per call (the tensor-core attention keeps a per-sequence prefix
+// of page counts in shared memory).
+constexpr int kMaxSeqs = 1024;
+// Upper bound on the persistent attention grid (one CTA per SM); sizes the
+// partial-result slots of the workspace.
+constexpr int kMaxPersistentCtas = 160;
 
 // Workspace header: word 0 is the device status word; the rest is reserved.
 constexpr size_t kWsHeader = 256;
@@ -35,12 +40,12 @@ struct AttnParams {
   const void* v_cache;
   int32_t S, Hq, Hkv, G, D, P, R, rows;
   int32_t max_pages, num_pages_total, budget;
-  int32_t nsplit, chunk_pages;   // grid splits per (seq, kv head) and pages per split
+  int32_t nsplit, chunk_pages;   // fp32 path: grid splits per (seq, kv head) and pages per split
   float scale_log2;              // scale * log2(e)
   uint32_t* status;
   uint32_t* tickets;             // [S * Hkv]
-  float* part_ml;                // [S * Hkv, nsplit, rows, 2]  (running max in log2 units, sum)
-  float* part_o;                 // [S * Hkv, nsplit, rows, D]  (unnormalised)
+  float* part_ml;                // [slots, rows, 2]  (running max in log2 units, sum)
+  float* part_o;                 // [slots, rows, D]  (unnormalised)
 };
 
 // Split plan shared by the workspace-size query and the launch.
@@ -59,6 +64,10 @@ cudaError_t launch_select(const s3r_paged_kv& kv, const void* kmin, const void* 
                           cudaStream_t st);
 cudaError_t launch_attention(const s3r_paged_kv& kv, const AttnParams& p, cudaStream_t st,
                              s3r_status* api_status);
+cudaError_t launch_attention_tc(const s3r_paged_kv& kv, const AttnParams& p, cudaStream_t st,
+                                s3r_status* api_status);
+bool make_cache_map(CUtensorMap* map, const void* base, const s3r_paged_kv& kv);
+int device_sm_count();
 
 struct SamplePlan {
   int32_t nrows;        // rows with statistics (2*gamma+1 per sequence, or num_rows)

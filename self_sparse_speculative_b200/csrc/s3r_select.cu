@@ -2,16 +2,19 @@
 // the mlsanity.com page's reference list; S3R page, Abstract, "uses sparse
 // attention to propose tokens").
 //
-// One CTA per (sequence, KV head):
-//   1. score every page p < n_b with the float64 bound
+// One thread-block cluster of CL CTAs per (sequence, KV head):
+//   1. every CTA scores its share of the pages p < n_b with the float64 bound
 //        s(p) = sum_g sum_d max(q[g,d] * kmin[p,d], q[g,d] * kmax[p,d])
-//      over the G query heads of the group, one warp per page (bf16 products
-//      are exact in float32; fp32 products are taken in float64);
-//   2. radix-select the budget-th largest score on order-preserving 64-bit
-//      keys (8 passes of 8 bits: shared-memory histogram, one-warp scan of
-//      the 256 bins);
-//   3. keep the keys above it plus the lowest-index pages equal to it, and
-//      write them in ascending page order with a block-wide prefix sum.
+//      over the G query heads of the group (one warp per page, four pages in
+//      flight per warp; bf16 products are exact in float32, fp32 products are
+//      taken in float64) and stores the page's order-preserving 64-bit key
+//      into the shared memory of the cluster's first CTA (distributed shared
+//      memory);
+//   2. that CTA radix-selects the budget-th largest key (8-bit digits from the
+//      top: shared-memory histogram, one-warp scan of the 256 bins), stopping
+//      as soon as the boundary bin holds exactly the keys still needed;
+//   3. it keeps the keys above the boundary plus the lowest-index pages on it,
+//      and writes them in ascending page order with block-wide prefix sums.
 #include <cuda_bf16.h>
 
 #include "s3r_device.cuh"
@@ -69,32 +72,80 @@ struct SelParams {
   uint32_t* status;
 };
 
-template <typename T>
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void st_cluster_u64(uint32_t local_addr, uint32_t rank, unsigned long long v) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
+  asm volatile("st.shared::cluster.u64 [%0], %1;" :: "r"(remote), "l"(v) : "memory");
+}
+
+// channels [lane*CPL, lane*CPL+CPL) of one summary row, as floats
+template <typename T, int CPL>
+__device__ __forceinline__ void load_row(const T* row, int lane, float* v) {
+  if constexpr (sizeof(T) == 2) {
+    if constexpr (CPL == 4) {
+      const uint2 u = __ldg(reinterpret_cast<const uint2*>(row) + lane);
+      v[0] = __uint_as_float(u.x << 16); v[1] = __uint_as_float(u.x & 0xFFFF0000u);
+      v[2] = __uint_as_float(u.y << 16); v[3] = __uint_as_float(u.y & 0xFFFF0000u);
+    } else {
+      const uint32_t u = __ldg(reinterpret_cast<const uint32_t*>(row) + lane);
+      v[0] = __uint_as_float(u << 16); v[1] = __uint_as_float(u & 0xFFFF0000u);
+    }
+  } else {
+    if constexpr (CPL == 4) {
+      const float4 u = __ldg(reinterpret_cast<const float4*>(row) + lane);
+      v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
+    } else {
+      const float2 u = __ldg(reinterpret_cast<const float2*>(row) + lane);
+      v[0] = u.x; v[1] = u.y;
+    }
+  }
+}
+
+constexpr int kUnroll = 4;     // pages in flight per warp
+
+template <typename T, int CPL>
 __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelParams p) {
-  extern __shared__ unsigned long long s_keys[];          // [n_b]
+  extern __shared__ unsigned long long s_keys[];          // [n_b], filled in the first CTA
   __shared__ float s_q[8 * 128];                          // [G, D] (bf16 path)
   __shared__ double s_qd[8 * 128];                        // [G, D] (fp32 path)
   __shared__ unsigned int s_hist[256];
   __shared__ unsigned long long s_prefix;
-  __shared__ int s_k;
+  __shared__ int s_k, s_done, s_shift;
   __shared__ int s_warp[kSelWarps];
 
-  const int h = blockIdx.x, b = blockIdx.y;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const uint32_t rank = cluster_rank();
+  const int ncta = gridDim.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int32_t* out = p.selected + ((size_t)b * p.Hkv + h) * p.budget;
+  // every decision before the cluster barriers is uniform over the cluster
   const int L = p.context_lens[b];
   if (L < 1 || L > p.max_pages * p.P) {
-    if (tid == 0) flag_status(p.status, S3R_DEV_BAD_CONTEXT_LEN);
-    for (int k = tid; k < p.budget; k += kSelThreads) out[k] = -1;
+    if (rank == 0) {
+      if (tid == 0) flag_status(p.status, S3R_DEV_BAD_CONTEXT_LEN);
+      for (int k = tid; k < p.budget; k += kSelThreads) out[k] = -1;
+    }
     return;
   }
   const int n_b = (L + p.P - 1) / p.P;
   if (n_b <= p.budget) {
-    for (int k = tid; k < p.budget; k += kSelThreads) out[k] = k < n_b ? k : -1;
+    if (rank == 0)
+      for (int k = tid; k < p.budget; k += kSelThreads) out[k] = k < n_b ? k : -1;
     return;
   }
+  cluster_sync_all();                                     // every CTA of the cluster is running
 
-  // ---- 1. scores
+  // ---- 1. scores of pages [beg, end)
+  const int per = (n_b + ncta - 1) / ncta;
+  const int beg = min(n_b, (int)rank * per), end = min(n_b, beg + per);
   const T* qp = static_cast<const T*>(p.q) + ((size_t)b * p.Hq + (size_t)h * p.G) * p.D;
   for (int i = tid; i < p.G * p.D; i += kSelThreads) {
     if constexpr (sizeof(T) == 2) s_q[i] = load_elem(qp, i);
@@ -103,38 +154,57 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelParams p) 
   __syncthreads();
   const T* kmn = static_cast<const T*>(p.kmin);
   const T* kmx = static_cast<const T*>(p.kmax);
-  for (int pg = warp; pg < n_b; pg += kSelWarps) {
-    const int phys = p.block_table[(size_t)b * p.max_pages + pg];
-    double acc = 0.0;
-    const bool ok = phys >= 0 && phys < p.num_pages_total;
-    if (ok) {
-      const size_t base = ((size_t)phys * p.Hkv + h) * p.D;
-      for (int d = lane; d < p.D; d += 32) {
-        const float lo = load_elem(kmn, base + d), hi = load_elem(kmx, base + d);
-        for (int g = 0; g < p.G; ++g) {
-          if constexpr (sizeof(T) == 2) {
-            const float qv = s_q[g * p.D + d];
-            acc += static_cast<double>(fmaxf(qv * lo, qv * hi));    // bf16 x bf16 is exact in fp32
-          } else {
-            const double qv = s_qd[g * p.D + d];
-            acc += fmax(qv * static_cast<double>(lo), qv * static_cast<double>(hi));
-          }
-        }
+  const uint32_t keys_addr = smem_addr(s_keys);
+  for (int pg0 = beg + warp * kUnroll; pg0 < end; pg0 += kSelWarps * kUnroll) {
+    int phys_l = -1;
+    if (lane < kUnroll && pg0 + lane < end) phys_l = p.block_table[(size_t)b * p.max_pages + pg0 + lane];
+    float lo[kUnroll][CPL], hi[kUnroll][CPL];
+    bool ok[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int phys = __shfl_sync(0xffffffffu, phys_l, u);
+      ok[u] = pg0 + u < end && phys >= 0 && phys < p.num_pages_total;
+      if (ok[u]) {
+        const size_t base = ((size_t)phys * p.Hkv + h) * p.D;
+        load_row<T, CPL>(kmn + base, lane, lo[u]);
+        load_row<T, CPL>(kmx + base, lane, hi[u]);
       }
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) {
-      if (!ok) flag_status(p.status, S3R_DEV_BAD_PAGE_ID);
-      s_keys[pg] = ok ? order_key(acc) : 0ull;              // a bad page sorts last
+    for (int u = 0; u < kUnroll; ++u) {
+      if (pg0 + u >= end) continue;                     // warp-uniform
+      double acc = 0.0;
+      if (ok[u]) {
+        for (int g = 0; g < p.G; ++g) {
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) {
+            const int d = lane * CPL + c;
+            if constexpr (sizeof(T) == 2) {
+              const float qv = s_q[g * p.D + d];
+              acc += static_cast<double>(fmaxf(qv * lo[u][c], qv * hi[u][c]));   // exact products
+            } else {
+              const double qv = s_qd[g * p.D + d];
+              acc += fmax(qv * static_cast<double>(lo[u][c]), qv * static_cast<double>(hi[u][c]));
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (lane == 0) {
+        if (!ok[u]) flag_status(p.status, S3R_DEV_BAD_PAGE_ID);
+        st_cluster_u64(keys_addr + 8u * (uint32_t)(pg0 + u), 0u, ok[u] ? order_key(acc) : 0ull);
+      }
     }
   }
-  if (tid == 0) { s_prefix = 0ull; s_k = p.budget; }
-  __syncthreads();
+  cluster_sync_all();                                     // all keys are in the first CTA
+  if (rank != 0) return;
 
   // ---- 2. radix select of the budget-th largest key
+  if (tid == 0) { s_prefix = 0ull; s_k = p.budget; s_done = 0; s_shift = 0; }
+  __syncthreads();
   for (int shift = 56; shift >= 0; shift -= 8) {
-    s_hist[tid] = 0u;                                        // kSelThreads == 256 bins
+    s_hist[tid] = 0u;                                      // kSelThreads == 256 bins
     __syncthreads();
     const unsigned long long prefix = s_prefix;
     for (int pg = tid; pg < n_b; pg += kSelThreads) {
@@ -152,19 +222,19 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelParams p) 
       unsigned int incl = sum;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        unsigned int y = __shfl_up_sync(0xffffffffu, incl, o);
+        const unsigned int y = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += y;
       }
       const int k = s_k;
       const unsigned int excl = incl - sum;
-      const bool here = excl < (unsigned)k && incl >= (unsigned)k;
-      if (here) {
+      if (excl < (unsigned)k && incl >= (unsigned)k) {
         unsigned int run = excl;
         for (int i = 0; i < 8; ++i) {
           if (run + c[i] >= (unsigned)k) {
             const unsigned long long digit = 255u - 8u * lane - i;
             s_prefix = prefix | (digit << shift);
             s_k = k - (int)run;
+            if (c[i] == (unsigned)(k - (int)run)) { s_done = 1; s_shift = shift; }   // the whole bin is kept
             break;
           }
           run += c[i];
@@ -172,22 +242,24 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelParams p) 
       }
     }
     __syncthreads();
+    if (s_done) break;
   }
-  const unsigned long long thr = s_prefix;
+  const int sh = s_shift;
+  const unsigned long long thr = s_prefix >> sh;
   const int need_eq = s_k;
 
-  // ---- 3. compaction in ascending page order
-  const int per = (n_b + kSelThreads - 1) / kSelThreads;
-  const int beg = min(n_b, tid * per), end = min(n_b, beg + per);
+  // ---- 3. compaction in ascending page order (keys compared above the stop digit)
+  const int per2 = (n_b + kSelThreads - 1) / kSelThreads;
+  const int b0 = min(n_b, tid * per2), b1 = min(n_b, b0 + per2);
   int n_eq = 0;
-  for (int pg = beg; pg < end; ++pg) n_eq += (s_keys[pg] == thr);
+  for (int pg = b0; pg < b1; ++pg) n_eq += ((s_keys[pg] >> sh) == thr);
   int tot;
-  int eq_before = block_exclusive_scan(n_eq, &tot, s_warp);
+  const int eq_before = block_exclusive_scan(n_eq, &tot, s_warp);
   int n_sel = 0;
   {
     int e = eq_before;
-    for (int pg = beg; pg < end; ++pg) {
-      const unsigned long long key = s_keys[pg];
+    for (int pg = b0; pg < b1; ++pg) {
+      const unsigned long long key = s_keys[pg] >> sh;
       if (key > thr) ++n_sel;
       else if (key == thr) { if (e < need_eq) ++n_sel; ++e; }
     }
@@ -195,14 +267,33 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelParams p) 
   int pos = block_exclusive_scan(n_sel, &tot, s_warp);
   {
     int e = eq_before;
-    for (int pg = beg; pg < end; ++pg) {
-      const unsigned long long key = s_keys[pg];
+    for (int pg = b0; pg < b1; ++pg) {
+      const unsigned long long key = s_keys[pg] >> sh;
       bool take = false;
       if (key > thr) take = true;
       else if (key == thr) { take = e < need_eq; ++e; }
       if (take && pos < p.budget) out[pos++] = pg;
     }
   }
+}
+
+template <typename T, int CPL>
+cudaError_t launch_typed(const SelParams& p, int cl, size_t smem, cudaStream_t st) {
+  cudaError_t e = cudaFuncSetAttribute(select_kernel<T, CPL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cl, p.Hkv, p.S);
+  cfg.blockDim = dim3(kSelThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cl;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, select_kernel<T, CPL>, p);
 }
 
 }  // namespace
@@ -228,17 +319,15 @@ cudaError_t launch_select(const s3r_paged_kv& kv, const void* kmin, const void* 
   p.budget = budget;
   p.status = status;
   const size_t smem = (size_t)kv.max_pages_per_seq * sizeof(unsigned long long);
-  dim3 grid(kv.num_kv_heads, kv.num_seqs);
+  // cluster size: about 64 pages per CTA, at most the portable 8
+  int cl = (kv.max_pages_per_seq + 63) / 64;
+  if (cl < 1) cl = 1;
+  if (cl > 8) cl = 8;
+  const bool bf = kv.dtype == S3R_BF16;
   cudaError_t e;
-  if (kv.dtype == S3R_BF16) {
-    e = cudaFuncSetAttribute(select_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    select_kernel<__nv_bfloat16><<<grid, kSelThreads, smem, st>>>(p);
-  } else {
-    e = cudaFuncSetAttribute(select_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    select_kernel<float><<<grid, kSelThreads, smem, st>>>(p);
-  }
+  if (kv.head_dim == 128) e = bf ? launch_typed<__nv_bfloat16, 4>(p, cl, smem, st) : launch_typed<float, 4>(p, cl, smem, st);
+  else e = bf ? launch_typed<__nv_bfloat16, 2>(p, cl, smem, st) : launch_typed<float, 2>(p, cl, smem, st);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -3,9 +3,8 @@
 // Long-Context LLM Inference" on the mlsanity.com page's reference list).
 //
 // HBM-bound scan: every (page, kv head) tile of P x D keys is read once with
-// 16-byte read-only loads and reduced over tokens in registers; each thread
-// owns one 16-byte channel group of one head, so a warp reads whole 256-byte
-// key rows. Writes are 2 * D values per (page, head).
+// 16-byte read-only loads; a warp reads whole key rows. Writes are 2 * D
+// values per (page, head).
 #include <cuda_bf16.h>
 
 #include "s3r_device.cuh"
@@ -14,10 +13,7 @@
 namespace s3r {
 namespace {
 
-constexpr int kSumThreads = 128;
-constexpr int kPagesPerCta = 4;
-
-struct Vec16 { uint4 v; };
+constexpr int kSumThreads = 256;
 
 __device__ __forceinline__ uint4 ldg_nc16(const void* p) {
   uint4 r;
@@ -69,58 +65,59 @@ struct SumParams {
   uint32_t* status;
 };
 
+// One CTA per (KV head, page index i, sequence): the P x D tile is split over
+// the CTA as (token group, 16-byte channel chunk); every thread reduces its
+// few tokens with independent loads, then token groups are merged in shared
+// memory. The whole tile is in flight at once, so a tail-page refresh costs
+// about one memory latency.
 template <typename T>
 __global__ void __launch_bounds__(kSumThreads) summaries_kernel(const SumParams p) {
-  const int b = blockIdx.y;
+  __shared__ uint4 s_min[kSumThreads];
+  __shared__ uint4 s_max[kSumThreads];
+  const int h = blockIdx.x, b = blockIdx.z;
   const int L = p.context_lens[b];
   if (L < 1 || L > p.max_pages * p.P) {
-    if (blockIdx.x == 0 && threadIdx.x == 0) flag_status(p.status, S3R_DEV_BAD_CONTEXT_LEN);
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) flag_status(p.status, S3R_DEV_BAD_CONTEXT_LEN);
     return;
   }
   const int n_b = (L + p.P - 1) / p.P;
-  int first, last;
-  if (p.tail_only) {
-    first = n_b - 1;
-    last = n_b;
-  } else {
-    first = blockIdx.x * kPagesPerCta;
-    last = min(n_b, first + kPagesPerCta);
+  const int i = p.tail_only ? n_b - 1 : (int)blockIdx.y;
+  if (i >= n_b) return;
+  const int phys = p.block_table[(size_t)b * p.max_pages + i];
+  if (phys < 0 || phys >= p.num_pages_total) {
+    if (threadIdx.x == 0) flag_status(p.status, S3R_DEV_BAD_PAGE_ID);
+    return;
   }
+  const int valid = min(p.P, L - i * p.P);
   constexpr int VEC = 16 / sizeof(T);
-  const int vecs_per_row = p.D / VEC;
-  const int items = p.Hkv * vecs_per_row;
-  const T* kc = static_cast<const T*>(p.k_cache);
-  for (int i = first; i < last; ++i) {
-    const int phys = p.block_table[(size_t)b * p.max_pages + i];
-    if (phys < 0 || phys >= p.num_pages_total) {
-      if (threadIdx.x == 0) flag_status(p.status, S3R_DEV_BAD_PAGE_ID);
-      continue;
+  const int chunks = p.D / VEC;                       // 16-byte chunks per key row
+  const int groups = kSumThreads / chunks;            // token groups
+  const int c = threadIdx.x % chunks, grp = threadIdx.x / chunks;
+  const T* base = static_cast<const T*>(p.k_cache) + ((size_t)(phys * p.Hkv + h) * p.P) * p.D + c * VEC;
+  uint4 mn = MinMax<T>::lo(), mx = MinMax<T>::hi();
+  constexpr int kMaxPer = 8;   // >= 8 token groups x 8 tokens covers P <= 64
+  uint4 v[kMaxPer];
+#pragma unroll
+  for (int k = 0; k < kMaxPer; ++k) {
+    const int t = grp + k * groups;
+    if (t < valid) v[k] = ldg_nc16(base + (size_t)t * p.D);
+  }
+#pragma unroll
+  for (int k = 0; k < kMaxPer; ++k) {
+    const int t = grp + k * groups;
+    if (t < valid) { vmin<T>(mn, v[k]); vmax<T>(mx, v[k]); }
+  }
+  s_min[threadIdx.x] = mn;
+  s_max[threadIdx.x] = mx;
+  __syncthreads();
+  if (threadIdx.x < chunks) {
+    for (int gi = 1; gi < groups; ++gi) {
+      vmin<T>(mn, s_min[gi * chunks + c]);
+      vmax<T>(mx, s_max[gi * chunks + c]);
     }
-    const int valid = min(p.P, L - i * p.P);
-    for (int it = threadIdx.x; it < items; it += blockDim.x) {
-      const int hh = it / vecs_per_row;
-      const int c = it - hh * vecs_per_row;
-      const T* base = kc + ((size_t)(phys * p.Hkv + hh) * p.P) * p.D + c * VEC;
-      uint4 mn = MinMax<T>::lo(), mx = MinMax<T>::hi();
-      int t = 0;
-      for (; t + 4 <= valid; t += 4) {
-        uint4 v0 = ldg_nc16(base + (size_t)(t + 0) * p.D);
-        uint4 v1 = ldg_nc16(base + (size_t)(t + 1) * p.D);
-        uint4 v2 = ldg_nc16(base + (size_t)(t + 2) * p.D);
-        uint4 v3 = ldg_nc16(base + (size_t)(t + 3) * p.D);
-        vmin<T>(mn, v0); vmax<T>(mx, v0);
-        vmin<T>(mn, v1); vmax<T>(mx, v1);
-        vmin<T>(mn, v2); vmax<T>(mx, v2);
-        vmin<T>(mn, v3); vmax<T>(mx, v3);
-      }
-      for (; t < valid; ++t) {
-        uint4 v = ldg_nc16(base + (size_t)t * p.D);
-        vmin<T>(mn, v); vmax<T>(mx, v);
-      }
-      const size_t o = ((size_t)phys * p.Hkv + hh) * p.D + c * VEC;
-      *reinterpret_cast<uint4*>(static_cast<T*>(p.kmin) + o) = mn;
-      *reinterpret_cast<uint4*>(static_cast<T*>(p.kmax) + o) = mx;
-    }
+    const size_t o = ((size_t)phys * p.Hkv + h) * p.D + c * VEC;
+    *reinterpret_cast<uint4*>(static_cast<T*>(p.kmin) + o) = mn;
+    *reinterpret_cast<uint4*>(static_cast<T*>(p.kmax) + o) = mx;
   }
 }
 
@@ -141,7 +138,7 @@ cudaError_t launch_summaries(const s3r_paged_kv& kv, int tail_only, void* kmin, 
   p.num_pages_total = kv.num_pages_total;
   p.tail_only = tail_only;
   p.status = status;
-  dim3 grid(tail_only ? 1 : (kv.max_pages_per_seq + kPagesPerCta - 1) / kPagesPerCta, kv.num_seqs);
+  dim3 grid(kv.num_kv_heads, tail_only ? 1 : kv.max_pages_per_seq, kv.num_seqs);
   if (kv.dtype == S3R_BF16)
     summaries_kernel<__nv_bfloat16><<<grid, kSumThreads, 0, st>>>(p);
   else
