@@ -17,18 +17,19 @@
 // of one MMA tile (M = 64, or 128 above 64 rows), so every 64-token K/V tile
 // read from HBM feeds one dense contraction:
 //   S = Q K^T (M x 64, K = D) and O += P V (M x D, K = 64), fp32 in TMEM.
-// Warp roles (192 threads):
-//   warps 0-3  softmax + epilogue; thread t of warp q owns TMEM lane 32q+t
-//              (= one packed row);
-//   warp 4     producer: resolves page ids ahead of use, loads each segment's
-//              Q into a double buffer, streams K/V tiles by TMA (3-D tensor
-//              map, 128-byte swizzle) into an NS-stage ring;
-//   warp 5     MMA issuer (one thread) and TMEM owner.
-// TMEM: S double buffer (2 x 64 columns) and O double buffer (2 x D
-// columns), so QK(j+1) overlaps softmax(j) and one segment's epilogue
-// overlaps the next segment's first pages. The running max is rescaled lazily
-// (only when it grows by more than 2^8); O and l always share one reference,
-// so the result is exact.
+// Warp roles (320 threads):
+//   warps 0-7  two softmax warpgroups working on alternate stages (ping-pong),
+//              each with its own S, P and O buffers; warpgroup 0 also merges
+//              the two partial states and writes each segment's output;
+//   warp 8     producer: resolves page ids ahead of use, loads each segment's
+//              Q into a double buffer, prefetches K/V tiles 8 stages ahead
+//              into L2 and streams them by TMA (3-D tensor map, 128-byte
+//              swizzle) into an NS-stage ring;
+//   warp 9     MMA issuer (one thread, QK two stages ahead of PV) and TMEM
+//              owner.
+// TMEM: S[2] (64 columns each) and O[2] (D columns each), one per stream.
+// The running max is rescaled lazily (only when it grows by more than 2^8);
+// O and l always share one reference, so the result is exact.
 #include <cuda_bf16.h>
 
 #include <cmath>
@@ -40,7 +41,9 @@
 namespace s3r {
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;               // 2 softmax warpgroups + producer + MMA
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
 constexpr float kRescaleTau = 8.0f;      // log2 units
 constexpr int kSmemBudget = 232448 - 8192;
 
@@ -92,15 +95,47 @@ __device__ __forceinline__ Seg locate(const AttnParams& p, const int* s_prefix, 
   return s;
 }
 
-// Logical and physical page of flattened position x (-1 when out of range).
+// Logical page and unit (b * Hkv + h) of flattened position x (-1 when out of range).
 __device__ __forceinline__ void page_of(const AttnParams& p, const int* s_prefix, int x, int hi, int W,
-                                        int* lp_out, int* b_out) {
+                                        int* lp_out, int* u_out) {
   *lp_out = -1;
-  *b_out = 0;
+  *u_out = 0;
   if (x >= hi) return;
   const Seg s = locate(p, s_prefix, x, hi, W);
-  *b_out = s.b;
+  *u_out = s.unit;
   *lp_out = p.page_list ? p.page_list[((size_t)s.b * p.Hkv + s.h) * p.budget + s.k0] : s.k0;
+}
+
+// Walk over the stages of a CTA's range, segment by segment.
+struct Cursor {
+  int x, s, j, nst, g;    // segment start, segment index, stage in segment, stages in segment, global stage
+  bool valid;
+  Seg sg;
+};
+__device__ __forceinline__ Cursor cursor_begin(const AttnParams& p, const int* s_prefix, int lo, int hi, int W,
+                                               int ppt) {
+  Cursor c;
+  c.x = lo; c.s = 0; c.j = 0; c.g = 0; c.nst = 0;
+  c.valid = lo < hi;
+  if (c.valid) {
+    c.sg = locate(p, s_prefix, lo, hi, W);
+    c.nst = (c.sg.npg + ppt - 1) / ppt;
+  }
+  return c;
+}
+__device__ __forceinline__ void cursor_next(const AttnParams& p, const int* s_prefix, int hi, int W, int ppt,
+                                            Cursor& c) {
+  ++c.g;
+  if (++c.j >= c.nst) {
+    c.x = c.sg.end;
+    ++c.s;
+    c.j = 0;
+    c.valid = c.x < hi;
+    if (c.valid) {
+      c.sg = locate(p, s_prefix, c.x, hi, W);
+      c.nst = (c.sg.npg + ppt - 1) / ppt;
+    }
+  }
 }
 
 template <int M, int D>
@@ -111,12 +146,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
   constexpr int NS = L::kNS;
   extern __shared__ __align__(1024) uint8_t dyn_raw[];
   uint8_t* dyn = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ __align__(8) uint64_t s_bar[2 * NS + 16];   // 2*NS + 15 used
+  __shared__ __align__(8) uint64_t s_bar[2 * NS + 14];
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   __shared__ int s_ticket;
   __shared__ int s_prefix[kMaxSeqs + 1];
   __shared__ int s_stage_lp[NS][4];
+  __shared__ float s_ml[2][2][128];                      // [segment parity][m, l][row] of stream 1
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -158,13 +194,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
   const uint32_t bar0 = smem_addr(&s_bar[0]);
   auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
   const int B_FULL = 0, B_EMPTY = NS, B_SFULL = 2 * NS, B_PFULL = 2 * NS + 2, B_ODONE = 2 * NS + 4,
-            B_OFULL = 2 * NS + 6, B_OEMPTY = 2 * NS + 8, B_QFULL = 2 * NS + 10, B_QEMPTY = 2 * NS + 12,
-            B_TD = 2 * NS + 14;
+            B_OFULL = 2 * NS + 6, B_OEMPTY = 2 * NS + 8, B_QFULL = 2 * NS + 9, B_QEMPTY = 2 * NS + 11,
+            B_TD = 2 * NS + 13;
   uint8_t* sP = dyn + L::kOffP;
   uint8_t* sKV = dyn + L::kOffKV;
   const uint32_t aQ = smem_addr(dyn), aP = smem_addr(sP), aKV = smem_addr(sKV);
 
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(smem_addr(&s_tmem), L::kTmemCols);
     tmem_relinquish();
   }
@@ -173,18 +209,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     for (int i = 0; i < 2; ++i) {
       mbar_init(BAR(B_SFULL + i), 1);
       mbar_init(BAR(B_PFULL + i), 128);
+      mbar_init(BAR(B_ODONE + i), 1);
       mbar_init(BAR(B_OFULL + i), 1);
-      mbar_init(BAR(B_OEMPTY + i), 128);
       mbar_init(BAR(B_QFULL + i), 32);
       mbar_init(BAR(B_QEMPTY + i), 1);
     }
-    mbar_init(BAR(B_ODONE), 1);
-    mbar_init(BAR(B_ODONE + 1), 1);
+    mbar_init(BAR(B_OEMPTY), 128);
     mbar_init(BAR(B_TD), 1);
     s_abort = 0;
     fence_barrier_init();
   }
-  if (warp == 4 && lane == 0) { prefetch_tensormap(&tmK); prefetch_tensormap(&tmV); }
+  if (warp == kProducerWarp && lane == 0) { prefetch_tensormap(&tmK); prefetch_tensormap(&tmV); }
   // zero both Q buffers (padding rows stay zero) and both P buffers
   for (int i = tid; i < (int)((2 * L::kQBytes + 2 * L::kPBytes) / 16); i += kThreads)
     reinterpret_cast<uint4*>(dyn)[i] = make_uint4(0u, 0u, 0u, 0u);
@@ -194,30 +229,30 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
   tc_fence_after();
   const uint32_t tmem = s_tmem;
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // ======================================================= producer warp
     const uint64_t pol = l2_policy_evict_first();
     // page-id windows of 32 flattened positions: lane k of a window holds
     // position wbase + k. w0 = in use, w1 = phys loads in flight, w2 = lp
     // loads in flight.
-    int w0_lp, w0_ph, w1_lp, w1_ph, w1_b, w2_lp, w2_b;
+    int w0_lp, w0_ph, w0_u, w1_lp, w1_ph, w1_u, w2_lp, w2_u;
     // issue the block-table load of a page (checked against the sequence
     // length first; the loaded id is range-checked where it is used)
-    auto phys_load = [&](int lp, int b) {
+    auto phys_load = [&](int lp, int u) {
       if (lp < 0) return -1;
+      const int b = u / p.Hkv;
       const int n_b = (p.context_lens[b] + p.P - 1) / p.P;
       if (lp >= n_b) { flag_status(p.status, S3R_DEV_BAD_PAGE_ID); return -1; }
       return p.block_table[(size_t)b * p.max_pages + lp];
     };
     int wbase = lo;
-    {
-      int b0;
-      page_of(p, s_prefix, wbase + lane, hi, W, &w0_lp, &b0);
-      w0_ph = phys_load(w0_lp, b0);
-      page_of(p, s_prefix, wbase + 32 + lane, hi, W, &w1_lp, &w1_b);
-      w1_ph = phys_load(w1_lp, w1_b);
-      page_of(p, s_prefix, wbase + 64 + lane, hi, W, &w2_lp, &w2_b);
-    }
+    page_of(p, s_prefix, wbase + lane, hi, W, &w0_lp, &w0_u);
+    w0_ph = phys_load(w0_lp, w0_u);
+    page_of(p, s_prefix, wbase + 32 + lane, hi, W, &w1_lp, &w1_u);
+    w1_ph = phys_load(w1_lp, w1_u);
+    page_of(p, s_prefix, wbase + 64 + lane, hi, W, &w2_lp, &w2_u);
+    // L2 prefetch distance in flattened positions (8 stages ahead, <= 32)
+    const int pfd = 8 * ppt;
     int g = 0;
     bool ok = true;
     int s = 0;
@@ -248,16 +283,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
           break;
         }
         // page ids of this stage: positions x + j*ppt + pp (pp < ppt)
-        int my_lp = -1, my_ph = -1;
+        int my_lp = -1, my_ph = -1, pf_z = -1;
         for (int pp = 0; pp < ppt; ++pp) {
           const int xp = x + j * ppt + pp;
           const bool in = (j * ppt + pp) < sg.npg;
           while (xp >= wbase + 32) {                   // advance the windows (warp-uniform)
             wbase += 32;
-            w0_lp = w1_lp; w0_ph = w1_ph;
-            w1_lp = w2_lp; w1_b = w2_b;
-            w1_ph = phys_load(w1_lp, w1_b);
-            page_of(p, s_prefix, wbase + 64 + lane, hi, W, &w2_lp, &w2_b);
+            w0_lp = w1_lp; w0_ph = w1_ph; w0_u = w1_u;
+            w1_lp = w2_lp; w1_u = w2_u;
+            w1_ph = phys_load(w1_lp, w1_u);
+            page_of(p, s_prefix, wbase + 64 + lane, hi, W, &w2_lp, &w2_u);
           }
           const int src = xp - wbase;
           const int lp = __shfl_sync(0xffffffffu, w0_lp, src & 31);
@@ -267,6 +302,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
             ph = -1;
           }
           if (lane == pp && in) { my_lp = lp; my_ph = ph; }
+          // the page pfd positions ahead, into L2 (whatever unit it belongs to)
+          const int s2 = src + pfd;
+          const int lp2 = __shfl_sync(0xffffffffu, s2 < 32 ? w0_lp : w1_lp, s2 & 31);
+          const int ph2 = __shfl_sync(0xffffffffu, s2 < 32 ? w0_ph : w1_ph, s2 & 31);
+          const int u2 = __shfl_sync(0xffffffffu, s2 < 32 ? w0_u : w1_u, s2 & 31);
+          if (lane == pp && xp + pfd < hi && lp2 >= 0 && ph2 >= 0 && ph2 < p.num_pages_total)
+            pf_z = ph2 * p.Hkv + (u2 % p.Hkv);
+        }
+        if (pf_z >= 0) {
+#pragma unroll
+          for (int hh = 0; hh < L::kHalves; ++hh) {
+            tma_prefetch_3d(&tmK, hh * 64, 0, pf_z);
+            tma_prefetch_3d(&tmV, hh * 64, 0, pf_z);
+          }
         }
         if (lane < 4) s_stage_lp[st][lane] = (lane < ppt && my_ph >= 0) ? my_lp : -1;
         const unsigned real = __ballot_sync(0xffffffffu, my_ph >= 0);
@@ -290,72 +339,84 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     // drain: wait until every issued copy has landed
     if (lane == 0)
       for (int k = max(0, g - NS); k < g; ++k) mbar_wait_drain(BAR(B_FULL + k % NS), (k / NS) & 1, p.status);
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ======================================================= MMA issuer
+    // QK runs two stages ahead of PV: after PV(g) (softmax(g) done, so S[g&1]
+    // is free) comes QK(g+2); the two softmax warpgroups then overlap.
     if (lane == 0) {
       constexpr uint32_t idQK = idesc_bf16_f32(M, kStageTokens, false, false);
       constexpr uint32_t idPV = idesc_bf16_f32(M, D, false, true);
-      // previous stage (for its PV)
-      int pv_g = -1, pv_s = 0, pv_j = 0;
-      bool pv_last = false;
-      int g = 0, s = 0;
+      Cursor qc = cursor_begin(p, s_prefix, lo, hi, W, ppt);
+      Cursor pc = qc;
+      int oe_seg = 0;                                    // segments whose O buffers are known free
       bool ok = true;
-      auto issue_pv = [&]() -> bool {
-        if (pv_j == 0 && !mbar_wait(BAR(B_OEMPTY + (pv_s & 1)), ((pv_s >> 1) & 1) ^ 1, &s_abort, p.status))
-          return false;
-        if (!mbar_wait(BAR(B_PFULL + (pv_g & 1)), (pv_g >> 1) & 1, &s_abort, p.status)) return false;
+      // Descriptor bases; advancing along K inside a 128-byte swizzle row is
+      // a 32-byte (2-unit) step of the start address, a 64-column half of
+      // Q/K is M*128 / 64*128 bytes further, a 16-token step of V is 2048 bytes.
+      const uint64_t dQ0 = smem_desc_sw128(aQ, 16, 1024);
+      const uint64_t dK0 = smem_desc_sw128(aKV, 16, 1024);
+      const uint64_t dV0 = smem_desc_sw128(aKV + L::kTileBytes, kStageTokens * 128, 1024);
+      const uint64_t dP0 = smem_desc_sw128(aP, 16, 1024);
+      constexpr uint64_t kQBuf = L::kQBytes >> 4, kQHalf = (M * 128) >> 4;
+      constexpr uint64_t kStage = (2 * L::kTileBytes) >> 4, kKHalf = (kStageTokens * 128) >> 4;
+      constexpr uint64_t kPBuf = L::kPBytes >> 4, kVStep = (16 * 128) >> 4;
+      auto issue_qk = [&]() -> bool {
+        if (qc.j == 0 && !mbar_wait(BAR(B_QFULL + (qc.s & 1)), (qc.s >> 1) & 1, &s_abort, p.status)) return false;
+        const int st = qc.g % NS;
+        if (!mbar_wait(BAR(B_FULL + st), (qc.g / NS) & 1, &s_abort, p.status)) return false;
         tc_fence_after();
-        const int stp = pv_g % NS;
-        const uint32_t vb = aKV + stp * 2 * L::kTileBytes + L::kTileBytes;
-        const uint32_t pb = aP + (pv_g & 1) * L::kPBytes;
-        const uint32_t tO = tmem + L::kColO + (pv_s & 1) * D;
+        const uint64_t qd = dQ0 + (uint64_t)(qc.s & 1) * kQBuf;
+        const uint64_t kd = dK0 + (uint64_t)st * kStage;
+        const uint32_t dS = tmem + L::kColS + (qc.g & 1) * kStageTokens;
 #pragma unroll
-        for (int kk = 0; kk < kStageTokens / 16; ++kk) {
-          const uint64_t a = smem_desc_sw128(pb + kk * 32, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(vb + kk * (16 * 128), kStageTokens * 128, 1024);
-          umma_f16(tO, a, bd, idPV, (pv_j > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t off = (uint64_t)(kk & 3) * 2;
+          umma_f16(dS, qd + (kk >> 2) * kQHalf + off, kd + (kk >> 2) * kKHalf + off, idQK, kk > 0 ? 1u : 0u);
         }
-        umma_commit(BAR(B_EMPTY + stp));
-        umma_commit(BAR(B_ODONE + (pv_g & 1)));
-        if (pv_last) umma_commit(BAR(B_OFULL + (pv_s & 1)));
+        umma_commit(BAR(B_SFULL + (qc.g & 1)));
+        if (qc.j == qc.nst - 1) umma_commit(BAR(B_QEMPTY + (qc.s & 1)));
+        cursor_next(p, s_prefix, hi, W, ppt, qc);
         return true;
       };
-      for (int x = lo; x < hi && ok; ++s) {
-        const Seg sg = locate(p, s_prefix, x, hi, W);
-        const int nst = (sg.npg + ppt - 1) / ppt;
-        if (!mbar_wait(BAR(B_QFULL + (s & 1)), (s >> 1) & 1, &s_abort, p.status)) { ok = false; break; }
-        const uint32_t qb = aQ + (s & 1) * L::kQBytes;
-        for (int j = 0; j < nst; ++j, ++g) {
-          const int st = g % NS;
-          if (!mbar_wait(BAR(B_FULL + st), (g / NS) & 1, &s_abort, p.status)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t kb = aKV + st * 2 * L::kTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const int hh = kk >> 2, sub = kk & 3;
-            const uint64_t a = smem_desc_sw128(qb + hh * (M * 128) + sub * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(kb + hh * (kStageTokens * 128) + sub * 32, 16, 1024);
-            umma_f16(tmem + L::kColS + (g & 1) * kStageTokens, a, bd, idQK, kk > 0 ? 1u : 0u);
-          }
-          umma_commit(BAR(B_SFULL + (g & 1)));
-          if (j == nst - 1) umma_commit(BAR(B_QEMPTY + (s & 1)));
-          if (pv_g >= 0 && !issue_pv()) { ok = false; break; }
-          pv_g = g; pv_s = s; pv_j = j; pv_last = (j == nst - 1);
+      for (int k = 0; k < 2 && qc.valid && ok; ++k) ok = issue_qk();
+      while (ok && pc.valid) {
+        const int k = pc.g & 1;
+        if (pc.j <= 1 && pc.s > oe_seg) {                // first PV of a stream in a new segment
+          if (!mbar_wait(BAR(B_OEMPTY), (pc.s - 1) & 1, &s_abort, p.status)) { ok = false; break; }
+          oe_seg = pc.s;
         }
-        x = sg.end;
+        if (!mbar_wait(BAR(B_PFULL + k), (pc.g >> 1) & 1, &s_abort, p.status)) { ok = false; break; }
+        tc_fence_after();
+        const int st = pc.g % NS;
+        const uint64_t vd = dV0 + (uint64_t)st * kStage;
+        const uint64_t pd = dP0 + (uint64_t)k * kPBuf;
+        const uint32_t tO = tmem + L::kColO + k * D;
+        const uint32_t acc0 = pc.j >= 2 ? 1u : 0u;
+#pragma unroll
+        for (int kk = 0; kk < kStageTokens / 16; ++kk)
+          umma_f16(tO, pd + (uint64_t)kk * 2, vd + (uint64_t)kk * kVStep, idPV, kk > 0 ? 1u : acc0);
+        umma_commit(BAR(B_EMPTY + st));
+        umma_commit(BAR(B_ODONE + k));
+        if (pc.j >= pc.nst - 2) umma_commit(BAR(B_OFULL + k));   // stream k's last PV of the segment
+        cursor_next(p, s_prefix, hi, W, ppt, pc);
+        if (qc.valid && !issue_qk()) { ok = false; break; }
       }
-      if (ok && pv_g >= 0) issue_pv();
       umma_commit(BAR(B_TD));
     }
   } else {
-    // ======================================================= softmax warps
-    // Epilogue view (32x32b TMEM loads): thread t of warp q reads TMEM lane
-    // 32q+t, which holds packed row `i` below. Stage view: for M = 64 the
-    // 16x256b loads give thread t rows ra = 16q + t/4 and rb = ra + 8, columns
+    // ======================================================= softmax warpgroups
+    // Warpgroup w (warps 4w..4w+3) takes the stages g with g % 2 == w, with
+    // its own S, P and O buffers and its own running (max, sum) per row; the
+    // two partial states of a segment are merged by warpgroup 0 in the
+    // epilogue. Epilogue view (32x32b TMEM loads): thread t of warp q reads
+    // TMEM lane 32q+t = packed row `i`. Stage view: for M = 64 the 16x256b
+    // loads give thread t rows ra = 16q + t/4 and rb = ra + 8, columns
     // 8k + 2(t%4) + {0,1}: every lane holds live data and a row's 64 columns
     // are spread over 4 threads (quad reductions by shuffles); for M = 128
     // each thread takes its own row's 64 columns.
-    const int q4 = warp;
+    const int wg = warp >> 2;
+    const int q4 = warp & 3;
+    const int wtid = tid & 127;                          // thread index inside the warpgroup
     const int slot = (M == 64) ? (lane < 16 ? 16 * q4 + lane : M) : 32 * q4 + lane;
     const int i = slot;                                  // packed row (epilogue view)
     const bool row_ok = i < p.rows;
@@ -364,17 +425,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     const int ra = 16 * q4 + (lane >> 2), rb = ra + 8;   // M = 64 stage view
     const bool ok_a = ra < p.rows, ok_b = rb < p.rows;
     const int cq = 2 * (lane & 3);
+    const uint32_t tO_mine = tmem + lane_base + L::kColO + wg * D;
     int g = 0, s = 0;
+    int ofull_cnt[2] = {0, 0};
     bool ok = true;
     for (int x = lo; x < hi && ok; ++s) {
       const Seg sg = locate(p, s_prefix, x, hi, W);
       const int nst = (sg.npg + ppt - 1) / ppt;
+      const int g0 = g;
       const int Lb = p.context_lens[sg.b];
       const int qpos = Lb - p.R + (row_ok ? i / p.G : 0);
       const int qpos_a = Lb - p.R + (ok_a ? ra / p.G : 0), qpos_b = Lb - p.R + (ok_b ? rb / p.G : 0);
       float m_run = -INFINITY, l_run = 0.f;            // M = 128 view (and epilogue)
       float m_a = -INFINITY, l_a = 0.f, m_b = -INFINITY, l_b = 0.f;   // M = 64 stage view
       for (int j = 0; j < nst; ++j, ++g) {
+        if ((g & 1) != wg) continue;
         const int st = g % NS, sb = g & 1;
         if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_SFULL + sb), (g >> 1) & 1, &s_abort, p.status) &&
                                          mbar_wait(BAR(B_FULL + st), (g / NS) & 1, &s_abort, p.status))) {
@@ -498,43 +563,35 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
             if (row_ok) l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
           }
         }
-        // P[sb] was last read by PV(g-2); a rescale of O also needs PV(g-1).
-        // ODONE[b] completes once per PV of a stage with (g & 1) == b.
-        {
-          bool w = true;
-          if (g >= 2) w = mbar_wait(BAR(B_ODONE + sb), ((g - 2) >> 1) & 1, &s_abort, p.status);
-          const bool need_prev = __any_sync(0xffffffffu, rescale) && j > 0;
-          if (w && need_prev) w = mbar_wait(BAR(B_ODONE + (sb ^ 1)), ((g - 1) >> 1) & 1, &s_abort, p.status);
-          if (!__all_sync(0xffffffffu, w)) {
-            ok = false;
-            break;
-          }
+        // P[sb] and O[sb] were last used by this stream's PV(g-2)
+        if (g >= 2 && !__all_sync(0xffffffffu, mbar_wait(BAR(B_ODONE + sb), ((g - 2) >> 1) & 1, &s_abort, p.status))) {
+          ok = false;
+          break;
         }
         if (warp_busy) {
           tc_fence_after();
           if (__any_sync(0xffffffffu, rescale)) {
-            const uint32_t tO = tmem + lane_base + L::kColO + (s & 1) * D;
             if constexpr (M == 64) {
 #pragma unroll
               for (int c0 = 0; c0 < D; c0 += 64) {
                 float o[32];
-                tmem_ld16x256b_x8(tO + c0, o);
+                tmem_ld16x256b_x8(tO_mine + c0, o);
                 tmem_wait_ld();
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                   o[4 * k] *= alpha_a; o[4 * k + 1] *= alpha_a;
                   o[4 * k + 2] *= alpha_b; o[4 * k + 3] *= alpha_b;
                 }
-                tmem_st16x256b_x8(tO + c0, o);
+                tmem_st16x256b_x8(tO_mine + c0, o);
               }
             } else {
               for (int c0 = 0; c0 < D; c0 += 32) {
                 float o[32];
-                tmem_ld32(tO + c0, o);
+                tmem_ld32(tO_mine + c0, o);
                 tmem_wait_ld();
 #pragma unroll
                 for (int c = 0; c < 32; ++c) o[c] *= alpha;
-                tmem_st32(tO + c0, o);
+                tmem_st32(tO_mine + c0, o);
               }
             }
             tmem_wait_st();
@@ -558,7 +615,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
           // zero the V rows of tokens that do not exist (beyond L, missing
           // pages) so that 0 * garbage cannot reach O
           uint8_t* sV = sKV + st * 2 * L::kTileBytes + L::kTileBytes;
-          for (int idx = tid; idx < kStageTokens * L::kHalves * 8; idx += 128) {
+          for (int idx = wtid; idx < kStageTokens * L::kHalves * 8; idx += 128) {
             const int t = idx / (L::kHalves * 8);
             const int rem = idx - t * (L::kHalves * 8);
             if (col_pos(t) < 0)
@@ -570,6 +627,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
         tc_fence_before();
         mbar_arrive(BAR(B_PFULL + sb));
       }
+      if (!ok) break;
       if constexpr (M == 64) {
         // stage view -> epilogue view: total l over the quad, then row 16q + t
         // (t < 16) takes its values from quad 4(t % 8), row a for t < 8, b above
@@ -583,24 +641,48 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
         l_run = (lane & 8) ? lb : la;
         m_run = (lane & 8) ? mvb : mva;
       }
-      if (!ok) break;
-      // ---- segment epilogue
-      if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_OFULL + (s & 1)), (s >> 1) & 1, &s_abort, p.status))) {
+      // ---- segment epilogue: warpgroup 1 hands its (max, sum) to warpgroup 0
+      const bool has0 = nst >= 2 || (g0 & 1) == 0, has1 = nst >= 2 || (g0 & 1) == 1;
+      if (wg == 1 && row_ok) {
+        s_ml[s & 1][0][i] = m_run;
+        s_ml[s & 1][1][i] = l_run;
+      }
+      asm volatile("bar.sync 2, 256;" ::: "memory");
+      if (wg == 1) { x = sg.end; continue; }
+      bool w = true;
+      if (has0) w = mbar_wait(BAR(B_OFULL + 0), ofull_cnt[0] & 1, &s_abort, p.status);
+      if (w && has1) w = mbar_wait(BAR(B_OFULL + 1), ofull_cnt[1] & 1, &s_abort, p.status);
+      ofull_cnt[0] += has0;
+      ofull_cnt[1] += has1;
+      if (!__all_sync(0xffffffffu, w)) {
         ok = false;
         break;
       }
       tc_fence_after();
+      float m0 = has0 ? m_run : -INFINITY, l0 = has0 ? l_run : 0.f;
+      float m1 = -INFINITY, l1 = 0.f;
+      if (has1 && row_ok) { m1 = s_ml[s & 1][0][i]; l1 = s_ml[s & 1][1][i]; }
+      const float mm = fmaxf(m0, m1);
+      const float w0 = (m0 == -INFINITY || l0 == 0.f) ? 0.f : ex2(m0 - mm);
+      const float w1 = (m1 == -INFINITY || l1 == 0.f) ? 0.f : ex2(m1 - mm);
+      const float lt = l0 * w0 + l1 * w1;
       const bool single = sg.nseg == 1;
-      const int slot_idx = sg.first_cta + sg.unit + (blockIdx.x - sg.first_cta);
+      const int slot_idx = sg.unit + blockIdx.x;           // partial slot of (unit, this CTA)
       const size_t pi = (size_t)slot_idx * p.rows + (row_ok ? i : 0);
-      const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+      const float inv_l = lt > 0.f ? 1.f / lt : 0.f;
       if (warp_busy) {
-        const uint32_t tO = tmem + lane_base + L::kColO + (s & 1) * D;
+        const uint32_t tO0 = tmem + lane_base + L::kColO, tO1 = tO0 + D;
         for (int c0 = 0; c0 < D; c0 += 32) {
-          float o[32];
-          tmem_ld32(tO + c0, o);
+          float o[32], o1[32];
+          if (has0) { tmem_ld32(tO0 + c0, o); } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] = 0.f;
+          }
+          if (has1) tmem_ld32(tO1 + c0, o1);
           tmem_wait_ld();
           if (!row_ok) continue;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = o[c] * w0 + (has1 ? o1[c] * w1 : 0.f);
           if (single) {
             __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) + out_row_offset(p, sg.b, sg.h, i) * D + c0;
 #pragma unroll
@@ -616,24 +698,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
         }
       }
       tc_fence_before();
-      mbar_arrive(BAR(B_OEMPTY + (s & 1)));
+      mbar_arrive(BAR(B_OEMPTY));
       if (row_ok) {
         if (single) {
-          if (p.lse) p.lse[out_row_offset(p, sg.b, sg.h, i)] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
+          if (p.lse) p.lse[out_row_offset(p, sg.b, sg.h, i)] = lt > 0.f ? (mm + log2f(lt)) * kLn2 : -INFINITY;
         } else {
-          p.part_ml[pi * 2] = l_run > 0.f ? m_run : -INFINITY;
-          p.part_ml[pi * 2 + 1] = l_run;
+          p.part_ml[pi * 2] = lt > 0.f ? mm : -INFINITY;
+          p.part_ml[pi * 2 + 1] = lt;
         }
       }
       if (!single) {
         __threadfence();
         asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (tid == 0) s_ticket = atomicAdd(p.tickets + sg.unit, 1u);
+        if (wtid == 0) s_ticket = atomicAdd(p.tickets + sg.unit, 1u);
         asm volatile("bar.sync 1, 128;" ::: "memory");
         if (s_ticket == sg.nseg - 1) {
           __threadfence();
           combine_partials<__nv_bfloat16>(p, sg.b, sg.h, sg.first_cta + sg.unit, sg.nseg, 128);
-          if (tid == 0) p.tickets[sg.unit] = 0u;
+          if (wtid == 0) p.tickets[sg.unit] = 0u;
         }
       }
       x = sg.end;
@@ -644,7 +726,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
   __syncwarp();
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     if (lane == 0) mbar_wait_drain(BAR(B_TD), 0, p.status);
     __syncwarp();

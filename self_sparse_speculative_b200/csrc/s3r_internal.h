@@ -6,7 +6,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
-#include "../../include/s3r.h"
+#include "s3r.h"
 
 namespace s3r {
 
