@@ -19,7 +19,8 @@
  * --------------------------------
  * - Every pointer argument is a caller-owned DEVICE pointer unless stated
  *   otherwise. The library allocates and frees nothing and keeps no state
- *   between calls; scratch space comes from the caller's workspace.
+ *   between calls; scratch space comes from the caller's workspace (the one
+ *   exception, s3r_spec_sample_noalloc, uses a static array of its own).
  * - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *   stream). Work is enqueued asynchronously on it; outputs are ready when the
  *   stream reaches that point.
@@ -186,6 +187,35 @@ s3r_status s3r_sample_tokens(const void* logits, s3r_dtype logit_dtype, int32_t 
                              int32_t vocab, float temperature, const float* u,
                              int32_t* tokens, void* workspace, size_t workspace_bytes,
                              void* stream);
+
+/*
+ * s3r_spec_sample without a workspace argument, for callers that cannot
+ * allocate device memory themselves (a plug-in inside a host framework whose
+ * device memory belongs to the framework's pooling allocator, code that must
+ * not allocate while a stream is being captured, and the like). This entry
+ * point has no counterpart on the S3R pages: it only changes where the
+ * scratch memory comes from. Same arguments and results as s3r_spec_sample.
+ * - Scratch: a 4 MiB device array owned by the library (a file-scope
+ *   __device__ variable), held on every GPU that loads the library until the
+ *   process exits. Shapes whose scratch need exceeds it
+ *   (s3r_sample_workspace_bytes(num_seqs, gamma, vocab) > 4 MiB) return
+ *   S3R_ERR_UNSUPPORTED before anything is enqueued.
+ * - The first call on a device looks up the array's device address for that
+ *   device (with the device current); make that first call before any
+ *   stream capture.
+ * - The function allocates nothing (no cudaMalloc, cudaFree or allocating
+ *   library routine); it clears the part of the array that must start at
+ *   zero with cudaMemsetAsync on `stream`.
+ * - Every call shares the one array and leaves its contents behind: calls
+ *   that can overlap on the GPU (other streams, other host threads) race and
+ *   must be serialised by the caller. Device-check results land in the
+ *   shared array and cannot be read back; use s3r_spec_sample to get them.
+ */
+s3r_status s3r_spec_sample_noalloc(const void* target_logits, const void* draft_logits,
+                                   s3r_dtype logit_dtype, const int32_t* draft_tokens,
+                                   const float* u_accept, const float* u_sample,
+                                   int32_t num_seqs, int32_t gamma, int32_t vocab, float temperature,
+                                   int32_t* out_tokens, int32_t* num_accepted, void* stream);
 
 /* Workspace sizes. Return 0 for an invalid or unsupported request.
  * Attention: rows = 1 and budget_pages > 0 for s3r_sparse_draft_attn;

@@ -1,0 +1,98 @@
+// Speculative sampling without a caller-provided workspace.
+//
+// Some callers cannot hand the library scratch memory: a caller that runs
+// inside a host framework whose device memory is owned by its own pooling
+// allocator (so a bare cudaMalloc would fragment or exceed the pool's
+// budget), a plug-in that is never given an allocator handle, or code that
+// must not allocate while a stream is being captured into a CUDA graph. For
+// them this file gives s3r_spec_sample a variant whose scratch lives in a
+// statically sized device array that the library itself owns; the caller
+// still passes every input and output buffer.
+//
+// The array is a file-scope __device__ variable, so every GPU that loads the
+// library holds kStaticScratchBytes of it until the process exits. Its
+// device address is looked up once per device (cudaGetSymbolAddress) on the
+// first call made with that device current; the host-side symbol itself is
+// only a stand-in and is never passed to a kernel.
+#include <atomic>
+#include <cmath>
+#include <cstring>
+
+#include "s3r_internal.h"
+
+#define S3R_EXPORT extern "C" __attribute__((visibility("default")))
+
+using namespace s3r;
+
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(4) << 20;      // 4 MiB
+constexpr int kMaxDevices = 64;
+
+__device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+std::atomic<void*> g_scratch_addr[kMaxDevices];
+
+// Device address of the scratch array on the current device (nullptr on error).
+void* scratch_on_current_device(s3r_status* st) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) { *st = S3R_ERR_CUDA; return nullptr; }
+  if (dev < 0 || dev >= kMaxDevices) { *st = S3R_ERR_UNSUPPORTED; return nullptr; }
+  void* p = g_scratch_addr[dev].load(std::memory_order_acquire);
+  if (!p) {
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) { *st = S3R_ERR_CUDA; return nullptr; }
+    g_scratch_addr[dev].store(p, std::memory_order_release);
+  }
+  *st = S3R_OK;
+  return p;
+}
+
+}  // namespace
+
+S3R_EXPORT s3r_status s3r_spec_sample_noalloc(const void* target_logits, const void* draft_logits,
+                                              s3r_dtype logit_dtype, const int32_t* draft_tokens,
+                                              const float* u_accept, const float* u_sample, int32_t num_seqs,
+                                              int32_t gamma, int32_t vocab, float temperature,
+                                              int32_t* out_tokens, int32_t* num_accepted, void* stream) {
+  if (!target_logits || !draft_logits || !draft_tokens || !u_accept || !u_sample || !out_tokens || !num_accepted)
+    return S3R_ERR_INVALID_ARG;
+  if (logit_dtype != S3R_F32 && logit_dtype != S3R_BF16) return S3R_ERR_INVALID_ARG;
+  if (num_seqs < 1 || vocab < 1 || gamma < 1) return S3R_ERR_INVALID_ARG;
+  if (!(temperature > 0.0f) || !std::isfinite(temperature)) return S3R_ERR_INVALID_ARG;
+  if (gamma > kMaxGamma) return S3R_ERR_UNSUPPORTED;
+  const SamplePlan pl = plan_sampling(num_seqs, gamma, vocab);
+  if (pl.ws_bytes > kStaticScratchBytes) return S3R_ERR_UNSUPPORTED;     // batch too large for the array
+  s3r_status s;
+  uint8_t* w = static_cast<uint8_t*>(scratch_on_current_device(&s));
+  if (!w) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // tickets and the status word must start at zero on every call
+  if (cudaMemsetAsync(w, 0, pl.memset_bytes, st) != cudaSuccess) return S3R_ERR_CUDA;
+  SampleParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.target = target_logits;
+  p.draft = draft_logits;
+  p.draft_tokens = draft_tokens;
+  p.u_accept = u_accept;
+  p.u_sample = u_sample;
+  p.out_tokens = out_tokens;
+  p.num_accepted = num_accepted;
+  p.nseq = num_seqs;
+  p.gamma = gamma;
+  p.vocab = vocab;
+  p.inv_temp = 1.0f / temperature;
+  p.inv_temp_d = 1.0 / static_cast<double>(temperature);
+  p.status = reinterpret_cast<uint32_t*>(w);
+  p.tk_row = reinterpret_cast<uint32_t*>(w + pl.off_tk_row);
+  p.tk_seq1 = reinterpret_cast<uint32_t*>(w + pl.off_tk_seq1);
+  p.tk_seq2 = reinterpret_cast<uint32_t*>(w + pl.off_tk_seq2);
+  p.jsel = reinterpret_cast<int32_t*>(w + pl.off_j);
+  p.part1 = w + pl.off_part1;
+  p.stats = reinterpret_cast<double*>(w + pl.off_stats);
+  p.part2 = reinterpret_cast<double*>(w + pl.off_part2);
+  p.c1 = pl.c1;
+  p.ch1 = pl.ch1;
+  p.c2 = pl.c2;
+  p.ch2 = pl.ch2;
+  return launch_sampling(p, logit_dtype, true, st) == cudaSuccess ? S3R_OK : S3R_ERR_CUDA;
+}

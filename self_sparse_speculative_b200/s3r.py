@@ -21,7 +21,7 @@ S3R_DEV_BAD_CONTEXT_LEN, S3R_DEV_BAD_PAGE_ID, S3R_DEV_BAD_TOKEN_ID, S3R_DEV_WAIT
 
 EXPORTED = [
     "s3r_page_summaries", "s3r_page_summaries_checked", "s3r_sparse_draft_attn", "s3r_verify_attn",
-    "s3r_spec_sample", "s3r_sample_tokens", "s3r_attn_workspace_bytes", "s3r_sample_workspace_bytes",
+    "s3r_spec_sample", "s3r_spec_sample_noalloc", "s3r_sample_tokens", "s3r_attn_workspace_bytes", "s3r_sample_workspace_bytes",
     "s3r_device_status", "s3r_status_str", "s3r_version",
 ]
 
@@ -54,6 +54,7 @@ def _load():
         "s3r_sparse_draft_attn": ([kvp, vp, vp, vp, i32, f32, vp, vp, vp, vp, sz, vp], i32),
         "s3r_verify_attn": ([kvp, vp, i32, f32, vp, vp, vp, sz, vp], i32),
         "s3r_spec_sample": ([vp, vp, i32, vp, vp, vp, i32, i32, i32, f32, vp, vp, vp, sz, vp], i32),
+        "s3r_spec_sample_noalloc": ([vp, vp, i32, vp, vp, vp, i32, i32, i32, f32, vp, vp, vp], i32),
         "s3r_sample_tokens": ([vp, i32, i32, i32, f32, vp, vp, vp, sz, vp], i32),
         "s3r_attn_workspace_bytes": ([kvp, i32, i32], sz),
         "s3r_sample_workspace_bytes": ([i32, i32, i32], sz),
@@ -161,6 +162,18 @@ def s3r_spec_sample(target_logits, draft_logits, logit_dtype, draft_tokens, u_ac
                               int(vocab), float(temperature), _ptr(out_tokens), _ptr(num_accepted),
                               _ptr(workspace), wb, _stream(stream))
     _check("s3r_spec_sample", st)
+
+
+def s3r_spec_sample_noalloc(target_logits, draft_logits, logit_dtype, draft_tokens, u_accept, u_sample,
+                            num_seqs: int, gamma: int, vocab: int, temperature: float, out_tokens,
+                            num_accepted, stream=None):
+    """s3r_spec_sample with the library's own static device scratch instead of a workspace
+    (for callers that cannot allocate device memory; calls must not overlap on the GPU)."""
+    st = _lib.s3r_spec_sample_noalloc(_ptr(target_logits), _ptr(draft_logits), dtype_code(logit_dtype),
+                                      _ptr(draft_tokens), _ptr(u_accept), _ptr(u_sample), int(num_seqs),
+                                      int(gamma), int(vocab), float(temperature), _ptr(out_tokens),
+                                      _ptr(num_accepted), _stream(stream))
+    _check("s3r_spec_sample_noalloc", st)
 
 
 def s3r_sample_tokens(logits, logit_dtype, num_rows: int, vocab: int, temperature: float, u, tokens,
