@@ -171,24 +171,12 @@ SampleParams make_sample_params(const SamplePlan& pl, void* ws, int32_t nseq, in
                                 float temperature) {
   SampleParams p;
   std::memset(&p, 0, sizeof(p));
-  uint8_t* w = static_cast<uint8_t*>(ws);
   p.nseq = nseq;
   p.gamma = gamma;
   p.vocab = vocab;
   p.inv_temp = 1.0f / temperature;
   p.inv_temp_d = 1.0 / static_cast<double>(temperature);
-  p.status = reinterpret_cast<uint32_t*>(w);
-  p.tk_row = reinterpret_cast<uint32_t*>(w + pl.off_tk_row);
-  p.tk_seq1 = reinterpret_cast<uint32_t*>(w + pl.off_tk_seq1);
-  p.tk_seq2 = reinterpret_cast<uint32_t*>(w + pl.off_tk_seq2);
-  p.jsel = reinterpret_cast<int32_t*>(w + pl.off_j);
-  p.part1 = w + pl.off_part1;
-  p.stats = reinterpret_cast<double*>(w + pl.off_stats);
-  p.part2 = reinterpret_cast<double*>(w + pl.off_part2);
-  p.c1 = pl.c1;
-  p.ch1 = pl.ch1;
-  p.c2 = pl.c2;
-  p.ch2 = pl.ch2;
+  bind_sample_workspace(&p, pl, ws);
   return p;
 }
 }  // namespace

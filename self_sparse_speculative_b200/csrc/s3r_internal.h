@@ -75,7 +75,8 @@ struct SamplePlan {
   int32_t c1, ch1;      // pass-1 chunks per row and elements per chunk
   int32_t c2, ch2;      // pass-2 chunks per sequence and elements per chunk
   size_t ws_bytes;
-  size_t off_tk_row, off_tk_seq1, off_tk_seq2, off_j, off_part1, off_stats, off_part2;
+  size_t off_tk_row, off_tk_seq1, off_tk_seq2, off_tk_seq3, off_j;
+  size_t off_part1, off_stats, off_znorm, off_zpart, off_wpart;
   size_t memset_bytes;  // bytes from the start of the workspace cleared per call
 };
 SamplePlan plan_sampling(int32_t nseq, int32_t gamma, int32_t vocab);
@@ -95,12 +96,17 @@ struct SampleParams {
   uint32_t* tk_row;
   uint32_t* tk_seq1;
   uint32_t* tk_seq2;
+  uint32_t* tk_seq3;
   int32_t* jsel;
   void* part1;             // [nrows, c1] {float max, float pad, double sum}
-  double* stats;           // [nrows, 2] {max, Z}
-  double* part2;           // [nseq, c2]
+  double* stats;           // [nrows, 2] {max, Z}   (Z from float32 exponentials)
+  double* znorm;           // [nseq, 2] exact float64 Z of the residual's two rows
+  double* zpart;           // [nseq, c2, 2] chunk partials of znorm
+  double* wpart;           // [nseq, c2, 8] per-warp partial sums of the draw weights
   int32_t c1, ch1, c2, ch2;
 };
+// Fill the workspace pointers and sizes of `p` from a plan and a workspace base.
+void bind_sample_workspace(SampleParams* p, const SamplePlan& pl, void* ws);
 cudaError_t launch_sampling(const SampleParams& p, s3r_dtype dt, bool spec, cudaStream_t st);
 
 }  // namespace s3r

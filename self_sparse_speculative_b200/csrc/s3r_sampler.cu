@@ -7,16 +7,20 @@
 // at the first rejection j draw from norm(max(p_j - q_j, 0)); if all gamma
 // drafts pass, draw a bonus token from p_gamma.
 //
-// Pass 1 (grid: vocab chunks x rows): every CTA holds its chunk of one
-// logits row in registers (one HBM read), reduces its max, then sums
-// exp((x - max)/T) in float64. The last CTA of a row (atomic ticket) merges
-// the chunk partials into the row's (max, Z) in float64; the last row of a
-// sequence to finish takes the accept/reject decisions in float64.
-// Pass 2 (grid: vocab chunks x sequences): every CTA sums its chunk of the
-// residual (or bonus) weights in float64; the last CTA of a sequence locates
-// the chunk holding u * total and scans it for the drawn token.
-// The drafter's own draw (s3r_sample_tokens) is the same two passes in
-// "plain" mode: one row per draw, weights softmax(logits / T).
+// Pass 1 (grid: vocab chunks x rows): every CTA holds its chunk of one logits
+// row in registers (one HBM read), reduces its max, then sums exp((x - max)/T)
+// with float32 exponentials into float64. The last CTA of a row (atomic
+// ticket) merges the chunk partials into the row's (max, Z); the last row of
+// a sequence takes the gamma accept/reject tests (one lane each) in float64.
+// Pass 2a (residual sequences only): the exact float64 normalisers of the
+// two rows the residual is drawn from (float64 exponentials).
+// Pass 2b (grid: vocab chunks x sequences): float64 draw weights, summed per
+// warp segment; the last CTA of a sequence finds the chunk, then the warp
+// segment holding u * total, and one warp scans it for the drawn token. Every
+// draw is decided in float64 on both sides, so it is exact up to the order of
+// the float64 sums.
+// The drafter's own draw (s3r_sample_tokens) is pass 1 + pass 2b in "plain"
+// mode: one row per draw, weights exp((x - max)/T).
 #include <cuda_bf16.h>
 
 #include <cmath>
@@ -30,6 +34,7 @@ namespace {
 constexpr int kSmpThreads = 256;
 constexpr int kSmpWarps = kSmpThreads / 32;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kWarpSegs = kSmpWarps;         // pass-2 chunk = 8 contiguous warp segments
 
 struct Part1 {
   float m;
@@ -68,9 +73,18 @@ __device__ __forceinline__ uint4 ldg_stream16(const void* p) {
   return r;
 }
 
-__device__ float block_max(float v, float* s_red) {
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max_f(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ float block_max(float v, float* s_red) {
+  v = warp_max_f(v);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (lane == 0) s_red[warp] = v;
   __syncthreads();
@@ -78,37 +92,6 @@ __device__ float block_max(float v, float* s_red) {
   for (int w = 1; w < kSmpWarps; ++w) r = fmaxf(r, s_red[w]);
   __syncthreads();
   return r;
-}
-__device__ double block_sum(double v, double* s_red) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (lane == 0) s_red[warp] = v;
-  __syncthreads();
-  double r = 0.0;
-  for (int w = 0; w < kSmpWarps; ++w) r += s_red[w];
-  __syncthreads();
-  return r;
-}
-// Exclusive prefix sum of doubles over the CTA; *total gets the sum.
-__device__ double block_exclusive_scan_d(double v, double* total, double* s_red) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  double x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const double y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) s_red[warp] = x;
-  __syncthreads();
-  double before = 0.0, tot = 0.0;
-  for (int w = 0; w < kSmpWarps; ++w) {
-    if (w < warp) before += s_red[w];
-    tot += s_red[w];
-  }
-  __syncthreads();
-  *total = tot;
-  return before + x - v;
 }
 
 // Row pointers of the spec layout: rows 0..R-1 target, R..2*gamma draft.
@@ -121,34 +104,40 @@ __device__ __forceinline__ const T* row_ptr(const SampleParams& p, bool spec, in
   return static_cast<const T*>(p.draft) + ((size_t)b * p.gamma + (rr - R)) * p.vocab;
 }
 
-// accept/reject decisions of sequence b (one thread)
+// Accept/reject tests of sequence b, one lane per draft position (warp 0).
 template <typename T>
 __device__ void decide(const SampleParams& p, int b) {
+  const int lane = threadIdx.x & 31;
   const int per = 2 * p.gamma + 1, R = p.gamma + 1;
-  int j = p.gamma;
-  for (int i = 0; i < p.gamma; ++i) {
-    const int x = p.draft_tokens[(size_t)b * p.gamma + i];
+  bool acc = true;
+  int x = 0;
+  if (lane < p.gamma) {
+    x = p.draft_tokens[(size_t)b * p.gamma + lane];
     double ratio = 0.0;
     if (x >= 0 && x < p.vocab) {
       // statistics written by other CTAs of this grid: read through L2
-      const double* st = p.stats + 2 * ((size_t)b * per + i);
-      const double* sd = p.stats + 2 * ((size_t)b * per + R + i);
-      const double lt = LogitIO<T>::at(static_cast<const T*>(p.target) + ((size_t)b * R + i) * p.vocab, x);
-      const double ld = LogitIO<T>::at(static_cast<const T*>(p.draft) + ((size_t)b * p.gamma + i) * p.vocab, x);
+      const double* st = p.stats + 2 * ((size_t)b * per + lane);
+      const double* sd = p.stats + 2 * ((size_t)b * per + R + lane);
+      const double lt = LogitIO<T>::at(static_cast<const T*>(p.target) + ((size_t)b * R + lane) * p.vocab, x);
+      const double ld = LogitIO<T>::at(static_cast<const T*>(p.draft) + ((size_t)b * p.gamma + lane) * p.vocab, x);
       const double px = exp((lt - __ldcg(st)) * p.inv_temp_d) / __ldcg(st + 1);
       const double qx = exp((ld - __ldcg(sd)) * p.inv_temp_d) / __ldcg(sd + 1);
       ratio = qx > 0.0 ? px / qx : 0.0;
     } else {
       flag_status(p.status, S3R_DEV_BAD_TOKEN_ID);
     }
-    if (!(static_cast<double>(p.u_accept[(size_t)b * p.gamma + i]) < ratio)) { j = i; break; }
+    acc = static_cast<double>(p.u_accept[(size_t)b * p.gamma + lane]) < ratio;
   }
-  for (int i = 0; i < R; ++i) {
+  const unsigned rej = __ballot_sync(0xffffffffu, !acc) & ((1u << p.gamma) - 1u);
+  const int j = rej ? __ffs(rej) - 1 : p.gamma;         // first rejected position
+  for (int i = lane; i < R; i += 32) {
     if (i < j) p.out_tokens[(size_t)b * R + i] = p.draft_tokens[(size_t)b * p.gamma + i];
     else if (i > j) p.out_tokens[(size_t)b * R + i] = -1;
   }
-  p.num_accepted[b] = j;
-  p.jsel[b] = j;
+  if (lane == 0) {
+    p.num_accepted[b] = j;
+    p.jsel[b] = j;
+  }
 }
 
 // ---------------------------------------------------------------- pass 1
@@ -159,12 +148,11 @@ __global__ void __launch_bounds__(kSmpThreads) rowstats_kernel(const SampleParam
   __shared__ int s_last;
   using IO = LogitIO<T>;
   constexpr int E = IO::kPerVec * IO::kVecs;     // elements per thread
-  const int row = blockIdx.y, c = blockIdx.x, tid = threadIdx.x;
+  const int row = blockIdx.y, c = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const T* src = row_ptr<T>(p, SPEC, row);
   const int beg = c * p.ch1;
   const int end = min(p.vocab, beg + p.ch1);
   float x[E];
-  float mx = -INFINITY;
   if constexpr (VEC) {
 #pragma unroll
     for (int k = 0; k < IO::kVecs; ++k) {
@@ -183,15 +171,20 @@ __global__ void __launch_bounds__(kSmpThreads) rowstats_kernel(const SampleParam
       x[k] = e < end ? IO::at(src, e) : -INFINITY;
     }
   }
+  float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-  for (int k = 0; k < E; ++k) mx = fmaxf(mx, x[k]);
-  const float M = block_max(mx, s_redf);
+  for (int k = 0; k < E; ++k) mx[k & 3] = fmaxf(mx[k & 3], x[k]);
+  const float M = block_max(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), s_redf);
   const float k2 = kLog2e * p.inv_temp;
-  double s = 0.0;
+  double s4[4] = {0.0, 0.0, 0.0, 0.0};
 #pragma unroll
-  for (int k = 0; k < E; ++k) s += static_cast<double>(ex2((x[k] - M) * k2));
-  const double S = block_sum(s, s_redd);
+  for (int k = 0; k < E; ++k) s4[k & 3] += static_cast<double>(ex2((x[k] - M) * k2));
+  double s = warp_sum_d((s4[0] + s4[1]) + (s4[2] + s4[3]));
+  if (lane == 0) s_redd[warp] = s;
+  __syncthreads();
   if (tid == 0) {
+    double S = 0.0;
+    for (int w = 0; w < kSmpWarps; ++w) S += s_redd[w];
     Part1* part = static_cast<Part1*>(p.part1) + (size_t)row * p.c1 + c;
     part->m = M;
     part->s = S;
@@ -199,184 +192,307 @@ __global__ void __launch_bounds__(kSmpThreads) rowstats_kernel(const SampleParam
     s_last = (atomicAdd(p.tk_row + row, 1u) == (unsigned)(p.c1 - 1));
   }
   __syncthreads();
-  if (!s_last) return;
-  // last CTA of the row: merge chunk partials in float64
-  if (tid == 0) {
-    __threadfence();
-    const Part1* part = static_cast<const Part1*>(p.part1) + (size_t)row * p.c1;
-    float Mr = -INFINITY;
-    for (int i = 0; i < p.c1; ++i) Mr = fmaxf(Mr, __ldcg(&part[i].m));
-    double Z = 0.0;
-    for (int i = 0; i < p.c1; ++i) {
-      const float mi = __ldcg(&part[i].m);
-      if (mi == -INFINITY) continue;
+  if (!s_last || warp != 0) return;
+  // last CTA of the row: merge chunk partials in float64 (warp 0)
+  __threadfence();
+  const Part1* part = static_cast<const Part1*>(p.part1) + (size_t)row * p.c1;
+  float Mr = -INFINITY;
+  for (int i = lane; i < p.c1; i += 32) Mr = fmaxf(Mr, __ldcg(&part[i].m));
+  Mr = warp_max_f(Mr);
+  double Z = 0.0;
+  for (int i = lane; i < p.c1; i += 32) {
+    const float mi = __ldcg(&part[i].m);
+    if (mi != -INFINITY)
       Z += __ldcg(&part[i].s) * exp((static_cast<double>(mi) - static_cast<double>(Mr)) * p.inv_temp_d);
-    }
+  }
+  Z = warp_sum_d(Z);
+  if (lane == 0) {
     p.stats[2 * (size_t)row] = Mr;
     p.stats[2 * (size_t)row + 1] = Z;
     p.tk_row[row] = 0u;
-    if constexpr (SPEC) {
-      const int per = 2 * p.gamma + 1;
-      const int b = row / per;
+  }
+  if constexpr (SPEC) {
+    const int per = 2 * p.gamma + 1;
+    const int b = row / per;
+    int last = 0;
+    if (lane == 0) {
       __threadfence();
-      if (atomicAdd(p.tk_seq1 + b, 1u) == (unsigned)(per - 1)) {
-        __threadfence();
-        p.tk_seq1[b] = 0u;
-        decide<T>(p, b);
-      }
+      last = atomicAdd(p.tk_seq1 + b, 1u) == (unsigned)(per - 1);
+    }
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (last) {
+      __threadfence();
+      if (lane == 0) p.tk_seq1[b] = 0u;
+      decide<T>(p, b);
     }
   }
 }
 
 // ---------------------------------------------------------------- pass 2
+// The rows and normalisers a draw uses.
 struct DrawRows {
-  const void* prow;   // weights' p row
-  const void* qrow;   // residual: q row, else null
-  double Mp, Zp, Mq, Zq;
+  const void* prow;      // p row (target j, target gamma, or the plain row)
+  const void* qrow;      // residual: draft row j, else null
+  double Mp, Mq;         // row maxima (shifts)
+  double iZp, iZq;       // residual: exact 1/Z of the two rows; else 1
 };
 
-template <typename T>
-__device__ __forceinline__ double weight(const DrawRows& w, int e, double invT) {
-  const double pe = exp((static_cast<double>(LogitIO<T>::at(static_cast<const T*>(w.prow), e)) - w.Mp) * invT) / w.Zp;
-  if (!w.qrow) return pe;
-  const double qe = exp((static_cast<double>(LogitIO<T>::at(static_cast<const T*>(w.qrow), e)) - w.Mq) * invT) / w.Zq;
-  return pe > qe ? pe - qe : 0.0;
-}
-
 template <typename T, bool SPEC>
-__device__ DrawRows draw_rows(const SampleParams& p, int s, int j) {
+__device__ DrawRows draw_rows(const SampleParams& p, int s, int j, bool exact_z) {
   DrawRows w;
+  w.iZp = 1.0;
+  w.iZq = 1.0;
+  w.qrow = nullptr;
+  w.Mq = 0.0;
   if (!SPEC) {
     w.prow = static_cast<const T*>(p.target) + (size_t)s * p.vocab;
-    w.qrow = nullptr;
     w.Mp = p.stats[2 * (size_t)s];
-    w.Zp = p.stats[2 * (size_t)s + 1];
-    w.Mq = 0.0; w.Zq = 1.0;
     return w;
   }
   const int per = 2 * p.gamma + 1, R = p.gamma + 1;
   w.prow = static_cast<const T*>(p.target) + ((size_t)s * R + j) * p.vocab;
   w.Mp = p.stats[2 * ((size_t)s * per + j)];
-  w.Zp = p.stats[2 * ((size_t)s * per + j) + 1];
   if (j < p.gamma) {
     w.qrow = static_cast<const T*>(p.draft) + ((size_t)s * p.gamma + j) * p.vocab;
     w.Mq = p.stats[2 * ((size_t)s * per + R + j)];
-    w.Zq = p.stats[2 * ((size_t)s * per + R + j) + 1];
-  } else {
-    w.qrow = nullptr;
-    w.Mq = 0.0; w.Zq = 1.0;
+    if (exact_z) {
+      w.iZp = 1.0 / __ldcg(p.znorm + 2 * (size_t)s);
+      w.iZq = 1.0 / __ldcg(p.znorm + 2 * (size_t)s + 1);
+    }
   }
   return w;
 }
 
-// Sum of weights over [beg, end) by the whole CTA.
-template <typename T>
-__device__ double chunk_sum(const DrawRows& w, int beg, int end, double invT, double* s_red) {
-  double acc = 0.0;
-  for (int e = beg + threadIdx.x; e < end; e += kSmpThreads) acc += weight<T>(w, e, invT);
-  return block_sum(acc, s_red);
-}
-
-// Smallest k in [beg, end) with base + sum_{e in [beg, k]} w(e) > thr, by
-// contiguous per-thread segments and a block scan; -1 if none.
-template <typename T>
-__device__ int chunk_search(const DrawRows& w, int beg, int end, double base, double thr, double invT,
-                            double* s_red, int* s_int) {
-  const int n = end - beg;
-  const int per = (n + kSmpThreads - 1) / kSmpThreads;
-  const int sb = beg + min(n, (int)threadIdx.x * per), se = min(end, sb + per);
-  double loc = 0.0;
-  for (int e = sb; e < se; ++e) loc += weight<T>(w, e, invT);
-  double tot;
-  const double before = block_exclusive_scan_d(loc, &tot, s_red);
-  if (threadIdx.x == 0) { s_int[0] = 0x7FFFFFFF; s_int[1] = -1; }
-  __syncthreads();
-  double run = base + before;
-  int found = -1, last_pos = -1;
-  for (int e = sb; e < se; ++e) {
-    const double we = weight<T>(w, e, invT);
-    run += we;
-    if (we > 0.0) last_pos = e;
-    if (found < 0 && run > thr) found = e;
+// float64 draw weights of n consecutive elements starting at e
+template <typename T, bool VEC>
+__device__ __forceinline__ void load_vals(const T* row, int e, int n, float* v) {
+  using IO = LogitIO<T>;
+  if constexpr (VEC) {
+    IO::unpack(ldg_stream16(row + e), v);
+  } else {
+    for (int t = 0; t < IO::kPerVec; ++t) v[t] = t < n ? IO::at(row, e + t) : 0.f;
   }
-  if (found >= 0) atomicMin(&s_int[0], found);
-  if (last_pos >= 0) atomicMax(&s_int[1], last_pos);
-  __syncthreads();
-  const int k = s_int[0] != 0x7FFFFFFF ? s_int[0] : -1;
-  const int lp = s_int[1];
-  __syncthreads();
-  return k >= 0 ? k : (lp >= 0 ? -2 - lp : -1);   // -2-lp encodes "none, last positive lp"
 }
 
-template <typename T, bool SPEC>
-__global__ void __launch_bounds__(kSmpThreads) draw_kernel(const SampleParams p) {
-  __shared__ double s_redd[kSmpWarps];
-  __shared__ int s_int[2];
+template <typename T, bool VEC>
+__device__ __forceinline__ void weights(const DrawRows& w, int e, int n, double invT, double* out) {
+  using IO = LogitIO<T>;
+  float a[IO::kPerVec], b[IO::kPerVec];
+  load_vals<T, VEC>(static_cast<const T*>(w.prow), e, n, a);
+  if (w.qrow) load_vals<T, VEC>(static_cast<const T*>(w.qrow), e, n, b);
+#pragma unroll
+  for (int t = 0; t < IO::kPerVec; ++t) {
+    double wt = 0.0;
+    if (t < n) {
+      const double pe = exp((static_cast<double>(a[t]) - w.Mp) * invT) * w.iZp;
+      if (w.qrow) {
+        const double qe = exp((static_cast<double>(b[t]) - w.Mq) * invT) * w.iZq;
+        wt = pe > qe ? pe - qe : 0.0;
+      } else {
+        wt = pe;
+      }
+    }
+    out[t] = wt;
+  }
+}
+
+// Pass 2a: exact float64 normalisers of the residual's two rows.
+template <typename T, bool VEC>
+__global__ void __launch_bounds__(kSmpThreads) znorm_kernel(const SampleParams p) {
+  __shared__ double s_red[2][kSmpWarps];
   __shared__ int s_last;
-  __shared__ int s_chunk;
-  __shared__ double s_base, s_thr;
-  const int s = blockIdx.y, c = blockIdx.x, tid = threadIdx.x;
-  const int j = SPEC ? p.jsel[s] : 0;
-  DrawRows w = draw_rows<T, SPEC>(p, s, j);
+  using IO = LogitIO<T>;
+  const int s = blockIdx.y, c = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int j = p.jsel[s];
+  if (j >= p.gamma) return;                              // bonus draw: no residual (uniform per sequence)
+  DrawRows w = draw_rows<T, true>(p, s, j, false);
   const int beg = c * p.ch2, end = min(p.vocab, beg + p.ch2);
-  const double S = chunk_sum<T>(w, beg, end, p.inv_temp_d, s_redd);
+  double zt = 0.0, zd = 0.0;
+  for (int e = beg + tid * IO::kPerVec; e < end; e += kSmpThreads * IO::kPerVec) {
+    const int n = min(IO::kPerVec, end - e);
+    float a[IO::kPerVec], b[IO::kPerVec];
+    load_vals<T, VEC>(static_cast<const T*>(w.prow), e, n, a);
+    load_vals<T, VEC>(static_cast<const T*>(w.qrow), e, n, b);
+#pragma unroll
+    for (int t = 0; t < IO::kPerVec; ++t) {
+      if (t < n) {
+        zt += exp((static_cast<double>(a[t]) - w.Mp) * p.inv_temp_d);
+        zd += exp((static_cast<double>(b[t]) - w.Mq) * p.inv_temp_d);
+      }
+    }
+  }
+  zt = warp_sum_d(zt);
+  zd = warp_sum_d(zd);
+  if (lane == 0) { s_red[0][warp] = zt; s_red[1][warp] = zd; }
+  __syncthreads();
   if (tid == 0) {
-    p.part2[(size_t)s * p.c2 + c] = S;
+    double a = 0.0, b = 0.0;
+    for (int i = 0; i < kSmpWarps; ++i) { a += s_red[0][i]; b += s_red[1][i]; }
+    p.zpart[2 * ((size_t)s * p.c2 + c)] = a;
+    p.zpart[2 * ((size_t)s * p.c2 + c) + 1] = b;
     __threadfence();
-    s_last = (atomicAdd(p.tk_seq2 + s, 1u) == (unsigned)(p.c2 - 1));
+    s_last = atomicAdd(p.tk_seq3 + s, 1u) == (unsigned)(p.c2 - 1);
   }
   __syncthreads();
-  if (!s_last) return;
+  if (!s_last || warp != 0) return;
+  __threadfence();
+  double a = 0.0, b = 0.0;
+  for (int i = lane; i < p.c2; i += 32) {
+    a += __ldcg(p.zpart + 2 * ((size_t)s * p.c2 + i));
+    b += __ldcg(p.zpart + 2 * ((size_t)s * p.c2 + i) + 1);
+  }
+  a = warp_sum_d(a);
+  b = warp_sum_d(b);
+  if (lane == 0) {
+    p.znorm[2 * (size_t)s] = a;
+    p.znorm[2 * (size_t)s + 1] = b;
+    p.tk_seq3[s] = 0u;
+  }
+}
+
+// One warp scans [beg, end) from running sum `base` for the first k whose
+// running sum exceeds thr. Returns k, or -1 - (last index with weight > 0).
+template <typename T, bool VEC>
+__device__ int warp_scan_find(const DrawRows& w, int beg, int end, double base, double thr, double invT) {
+  using IO = LogitIO<T>;
+  constexpr int PV = IO::kPerVec;
+  const int lane = threadIdx.x & 31;
+  int last_pos = -1;
+  double run = base;
+  for (int e0 = beg; e0 < end; e0 += 32 * PV) {
+    const int e = e0 + lane * PV;
+    double wv[PV];
+    const int n = max(0, min(PV, end - e));
+    if (n > 0) weights<T, VEC>(w, e, n, invT, wv);
+    else
+#pragma unroll
+      for (int t = 0; t < PV; ++t) wv[t] = 0.0;
+    double loc = 0.0;
+#pragma unroll
+    for (int t = 0; t < PV; ++t) loc += wv[t];
+    double incl = loc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const double y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const double before = run + incl - loc;
+    int hit = -1, lp = -1;
+    double r = before;
+#pragma unroll
+    for (int t = 0; t < PV; ++t) {
+      r += wv[t];
+      if (wv[t] > 0.0) lp = e + t;
+      if (hit < 0 && r > thr) hit = e + t;
+    }
+    const unsigned m = __ballot_sync(0xffffffffu, hit >= 0);
+    if (m) return __shfl_sync(0xffffffffu, hit, __ffs(m) - 1);
+    const unsigned mp = __ballot_sync(0xffffffffu, lp >= 0);
+    if (mp) last_pos = __shfl_sync(0xffffffffu, lp, 31 - __clz(mp));
+    run = __shfl_sync(0xffffffffu, run + incl, 31);
+  }
+  return -1 - last_pos;
+}
+
+// Pass 2b: the draw.
+template <typename T, bool SPEC, bool VEC>
+__global__ void __launch_bounds__(kSmpThreads) draw_kernel(const SampleParams p) {
+  __shared__ double s_w[kSmpWarps];
+  __shared__ int s_last;
+  using IO = LogitIO<T>;
+  constexpr int PV = IO::kPerVec;
+  const int s = blockIdx.y, c = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int j = SPEC ? p.jsel[s] : 0;
+  const DrawRows w = draw_rows<T, SPEC>(p, s, j, true);
+  const int cbeg = c * p.ch2, cend = min(p.vocab, cbeg + p.ch2);
+  const int seg = p.ch2 / kWarpSegs;                     // elements per warp segment
+  const int sbeg = min(cend, cbeg + warp * seg), send = min(cend, sbeg + seg);
+  double acc = 0.0;
+  for (int e = sbeg + lane * PV; e < send; e += 32 * PV) {
+    double wv[PV];
+    weights<T, VEC>(w, e, min(PV, send - e), p.inv_temp_d, wv);
+#pragma unroll
+    for (int t = 0; t < PV; ++t) acc += wv[t];
+  }
+  acc = warp_sum_d(acc);
+  if (lane == 0) {
+    p.wpart[((size_t)s * p.c2 + c) * kWarpSegs + warp] = acc;
+    s_w[warp] = acc;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    s_last = atomicAdd(p.tk_seq2 + s, 1u) == (unsigned)(p.c2 - 1);
+  }
+  __syncthreads();
+  if (!s_last || warp != 0) return;
   __threadfence();
   const int R = p.gamma + 1;
   const double u = SPEC ? static_cast<double>(p.u_sample[(size_t)s * R + j]) : static_cast<double>(p.u_sample[s]);
-  // totals of the chunk sums; an all-zero residual falls back to p_j
-  if (tid == 0) {
-    double tot = 0.0;
-    for (int i = 0; i < p.c2; ++i) tot += __ldcg(p.part2 + (size_t)s * p.c2 + i);
-    s_base = tot;
-  }
-  __syncthreads();
-  if (SPEC && s_base <= 0.0 && w.qrow) {
-    w.qrow = nullptr;                                     // empty residual: draw from p_j
-    for (int i = 0; i < p.c2; ++i) {
-      const int b2 = i * p.ch2, e2 = min(p.vocab, b2 + p.ch2);
-      const double cs = chunk_sum<T>(w, b2, e2, p.inv_temp_d, s_redd);
-      if (tid == 0) p.part2[(size_t)s * p.c2 + i] = cs;
-    }
-    __syncthreads();
-  }
-  if (tid == 0) {
-    double tot = 0.0;
-    for (int i = 0; i < p.c2; ++i) tot += __ldcg(p.part2 + (size_t)s * p.c2 + i);
+  const double* wp = p.wpart + (size_t)s * p.c2 * kWarpSegs;
+  const int nseg = p.c2 * kWarpSegs;
+  // total of all segments, then the first segment whose running sum passes thr
+  double tot = 0.0;
+  for (int i = lane; i < nseg; i += 32) tot += __ldcg(wp + i);
+  tot = warp_sum_d(tot);
+  int k = -1;
+  if (tot > 0.0) {
     const double thr = u * tot;
     double run = 0.0;
-    int cstar = -1, lastpos = -1;
-    double base = 0.0;
-    for (int i = 0; i < p.c2; ++i) {
-      const double ci = __ldcg(p.part2 + (size_t)s * p.c2 + i);
-      if (ci > 0.0) { lastpos = i; }
-      if (cstar < 0 && run + ci > thr) { cstar = i; base = run; }
-      run += ci;
+    int sel = -1, lastpos = -1;
+    double sel_base = 0.0;
+    for (int i0 = 0; i0 < nseg && sel < 0; i0 += 32) {
+      const int i = i0 + lane;
+      const double v = i < nseg ? __ldcg(wp + i) : 0.0;
+      double incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const double y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const unsigned m = __ballot_sync(0xffffffffu, run + incl > thr && v > 0.0);
+      if (m) {
+        const int src = __ffs(m) - 1;
+        sel = i0 + src;
+        sel_base = __shfl_sync(0xffffffffu, run + incl - v, src);
+      }
+      const unsigned mp = __ballot_sync(0xffffffffu, v > 0.0);
+      if (mp) lastpos = i0 + 31 - __clz(mp);
+      run = __shfl_sync(0xffffffffu, run + incl, 31);
     }
-    if (cstar < 0) {            // rounding left no crossing: last chunk with weight
-      cstar = lastpos < 0 ? 0 : lastpos;
-      base = 0.0;
-      for (int i = 0; i < cstar; ++i) base += __ldcg(p.part2 + (size_t)s * p.c2 + i);
+    if (sel < 0) {                                       // rounding left no crossing: last segment with weight
+      sel = lastpos;
+      sel_base = 0.0;
+      for (int i = lane; i < sel; i += 32) sel_base += __ldcg(wp + i);
+      sel_base = warp_sum_d(sel_base);
     }
-    s_chunk = cstar;
-    s_base = base;
-    s_thr = thr;
-    p.tk_seq2[s] = 0u;
+    if (sel >= 0) {
+      const int cc = sel / kWarpSegs, ww = sel - cc * kWarpSegs;
+      const int b0 = min(p.vocab, cc * p.ch2 + ww * seg), b1 = min(min(p.vocab, cc * p.ch2 + p.ch2), b0 + seg);
+      k = warp_scan_find<T, VEC>(w, b0, b1, sel_base, thr, p.inv_temp_d);
+      if (k < 0) k = -1 - k;                            // last positive weight of the segment
+    }
+  } else if (SPEC && w.qrow) {
+    // all-zero residual (p_j == q_j after rounding): draw from p_j instead
+    DrawRows wb = w;
+    wb.qrow = nullptr;
+    wb.iZp = 1.0;
+    double total = 0.0;
+    for (int e = lane * PV; e < p.vocab; e += 32 * PV) {
+      double wv[PV];
+      weights<T, VEC>(wb, e, min(PV, p.vocab - e), p.inv_temp_d, wv);
+#pragma unroll
+      for (int t = 0; t < PV; ++t) total += wv[t];
+    }
+    total = warp_sum_d(total);
+    k = warp_scan_find<T, VEC>(wb, 0, p.vocab, 0.0, u * total, p.inv_temp_d);
+    if (k < 0) k = -1 - k;
   }
-  __syncthreads();
-  const int cb = s_chunk * p.ch2, ce = min(p.vocab, cb + p.ch2);
-  int k = chunk_search<T>(w, cb, ce, s_base, s_thr, p.inv_temp_d, s_redd, s_int);
-  if (tid == 0) {
-    if (k <= -2) k = -2 - k;          // no crossing inside: last positive weight
-    if (k < 0) k = cb;                // no weight at all (cannot happen for a distribution)
+  if (lane == 0) {
+    if (k < 0) k = 0;
     if (SPEC) p.out_tokens[(size_t)s * R + j] = k;
     else p.out_tokens[s] = k;
+    p.tk_seq2[s] = 0u;
   }
 }
 
@@ -387,13 +503,19 @@ cudaError_t launch_typed(const SampleParams& p, cudaStream_t st) {
   const bool vec = (((size_t)p.vocab * sizeof(T)) % 16 == 0) &&
                    (reinterpret_cast<uintptr_t>(p.target) % 16 == 0) &&
                    (!SPEC || reinterpret_cast<uintptr_t>(p.draft) % 16 == 0);
-  dim3 g1(p.c1, nrows);
+  dim3 g1(p.c1, nrows), g2(p.c2, p.nseq);
   if (vec) rowstats_kernel<T, SPEC, true><<<g1, kSmpThreads, 0, st>>>(p);
   else rowstats_kernel<T, SPEC, false><<<g1, kSmpThreads, 0, st>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  dim3 g2(p.c2, p.nseq);
-  draw_kernel<T, SPEC><<<g2, kSmpThreads, 0, st>>>(p);
+  if (SPEC) {
+    if (vec) znorm_kernel<T, true><<<g2, kSmpThreads, 0, st>>>(p);
+    else znorm_kernel<T, false><<<g2, kSmpThreads, 0, st>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (vec) draw_kernel<T, SPEC, true><<<g2, kSmpThreads, 0, st>>>(p);
+  else draw_kernel<T, SPEC, false><<<g2, kSmpThreads, 0, st>>>(p);
   return cudaGetLastError();
 }
 
@@ -416,12 +538,13 @@ SamplePlan plan_sampling(int32_t nseq, int32_t gamma, int32_t vocab) {
   pl.ch1 = (int)align_up((size_t)((vocab + c1 - 1) / c1), 8);
   if (pl.ch1 > max_per_cta) pl.ch1 = max_per_cta;
   pl.c1 = (vocab + pl.ch1 - 1) / pl.ch1;
-  // pass 2: about 4 CTAs per SM, at least 1024 elements per CTA
+  // pass 2: about 4 CTAs per SM, at least 2048 elements per CTA; a chunk is
+  // 8 warp segments whose length is a multiple of 32 lanes x 8 elements
   int c2 = (target + nseq - 1) / nseq;
-  const int cap2 = (vocab + 1023) / 1024;
+  const int cap2 = (vocab + 2047) / 2048;
   if (c2 > cap2) c2 = cap2;
   if (c2 < 1) c2 = 1;
-  pl.ch2 = (int)align_up((size_t)((vocab + c2 - 1) / c2), 8);
+  pl.ch2 = (int)align_up((size_t)((vocab + c2 - 1) / c2), (size_t)kWarpSegs * 32 * 8);
   pl.c2 = (vocab + pl.ch2 - 1) / pl.ch2;
   size_t off = kWsHeader;
   pl.off_tk_row = off;
@@ -430,6 +553,8 @@ SamplePlan plan_sampling(int32_t nseq, int32_t gamma, int32_t vocab) {
   off = align_up(off + sizeof(uint32_t) * nseq, 16);
   pl.off_tk_seq2 = off;
   off = align_up(off + sizeof(uint32_t) * nseq, 16);
+  pl.off_tk_seq3 = off;
+  off = align_up(off + sizeof(uint32_t) * nseq, 16);
   pl.memset_bytes = off;
   pl.off_j = off;
   off = align_up(off + sizeof(int32_t) * nseq, 256);
@@ -437,10 +562,33 @@ SamplePlan plan_sampling(int32_t nseq, int32_t gamma, int32_t vocab) {
   off = align_up(off + sizeof(Part1) * (size_t)pl.nrows * pl.c1, 256);
   pl.off_stats = off;
   off = align_up(off + sizeof(double) * 2 * (size_t)pl.nrows, 256);
-  pl.off_part2 = off;
-  off = align_up(off + sizeof(double) * (size_t)nseq * pl.c2, 256);
+  pl.off_znorm = off;
+  off = align_up(off + sizeof(double) * 2 * (size_t)nseq, 256);
+  pl.off_zpart = off;
+  off = align_up(off + sizeof(double) * 2 * (size_t)nseq * pl.c2, 256);
+  pl.off_wpart = off;
+  off = align_up(off + sizeof(double) * kWarpSegs * (size_t)nseq * pl.c2, 256);
   pl.ws_bytes = off;
   return pl;
+}
+
+void bind_sample_workspace(SampleParams* p, const SamplePlan& pl, void* ws) {
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  p->status = reinterpret_cast<uint32_t*>(w);
+  p->tk_row = reinterpret_cast<uint32_t*>(w + pl.off_tk_row);
+  p->tk_seq1 = reinterpret_cast<uint32_t*>(w + pl.off_tk_seq1);
+  p->tk_seq2 = reinterpret_cast<uint32_t*>(w + pl.off_tk_seq2);
+  p->tk_seq3 = reinterpret_cast<uint32_t*>(w + pl.off_tk_seq3);
+  p->jsel = reinterpret_cast<int32_t*>(w + pl.off_j);
+  p->part1 = w + pl.off_part1;
+  p->stats = reinterpret_cast<double*>(w + pl.off_stats);
+  p->znorm = reinterpret_cast<double*>(w + pl.off_znorm);
+  p->zpart = reinterpret_cast<double*>(w + pl.off_zpart);
+  p->wpart = reinterpret_cast<double*>(w + pl.off_wpart);
+  p->c1 = pl.c1;
+  p->ch1 = pl.ch1;
+  p->c2 = pl.c2;
+  p->ch2 = pl.ch2;
 }
 
 cudaError_t launch_sampling(const SampleParams& p, s3r_dtype dt, bool spec, cudaStream_t st) {

@@ -1,0 +1,80 @@
+"""Full-size parity: every workload at its stated size, run exactly as the
+benchmark runs it (DecodeStep.round through the C ABI), checked against the
+float64 oracle on sampled sequences (attention, summaries, page selection)
+and on every sequence (draft draws, accept/reject, drawn token)."""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+from self_sparse_speculative_b200 import s3r                         # noqa: E402
+from self_sparse_speculative_b200.step import DecodeStep             # noqa: E402
+from self_sparse_speculative_b200.workloads import Workload, spec    # noqa: E402
+
+import oracle.reference_run as RR                                     # noqa: E402
+
+TALLY = RR.Tally()
+
+
+def _sample_seqs(wl):
+    S = wl.spec.num_seqs
+    lens = wl.context_lens
+    pick = {0, S - 1, int(np.argmax(lens)), int(np.argmin(lens))}
+    return sorted(pick)[:4]
+
+
+@pytest.fixture(scope="module", params=[0, 1, 2, 3, 4])
+def full_run(request):
+    wl = Workload(spec(request.param), seed=0)
+    st = DecodeStep(wl)
+    st.summaries(tail_only=False)
+    st.round()
+    torch.cuda.synchronize()
+    yield wl, st
+    del st
+    torch.cuda.empty_cache()
+
+
+def test_full_device_status(full_run):
+    wl, st = full_run
+    for name, (status, bits) in st.device_checks().items():
+        assert status == s3r.S3R_OK, (wl.spec.name, name, bits)
+
+
+def test_full_attention_sampled_sequences(full_run):
+    wl, st = full_run
+    ws = wl.spec
+    dt = ws.kv_dtype
+    sel = st.selected.cpu().numpy()
+    kmin = st.kmin.float().cpu().numpy()
+    kmax = st.kmax.float().cpu().numpy()
+    for b in _sample_seqs(wl):
+        ref = RR.oracle_attention_seq(wl, b)
+        name = f"{ws.name.split(':')[0]} seq {b}"
+        assert np.array_equal(kmin[ref["phys"]].astype(np.float64), ref["kmin"]), name
+        assert np.array_equal(kmax[ref["phys"]].astype(np.float64), ref["kmax"]), name
+        for i, d in ref["draft"].items():
+            ok = RR.compare_selection(f"{name} draft {i}", sel[i, b], d["selected"], d["gaps"], TALLY)
+            if all(ok):
+                RR.assert_close(f"{name} draft {i} out", st.draft_out[i, b].float().cpu().numpy(), d["out"], dt)
+                RR.assert_close(f"{name} draft {i} lse", st.draft_lse[i, b].cpu().numpy(), d["lse"], dt)
+        RR.assert_close(f"{name} verify out", st.verify_out[b].float().cpu().numpy(), ref["verify_out"], dt)
+        RR.assert_close(f"{name} verify lse", st.verify_lse[b].cpu().numpy(), ref["verify_lse"], dt)
+    # near-ties (left out of the exact comparison) stay under 1e-4 of all decisions so far
+    assert TALLY.near_ties <= 1e-4 * TALLY.decisions, TALLY.notes
+
+
+def test_full_sampling_every_sequence(full_run):
+    wl, st = full_run
+    x = st.draft_tokens.cpu().numpy()
+    out = st.out_tokens.cpu().numpy()
+    nacc = st.num_accepted.cpu().numpy()
+    for b in range(wl.spec.num_seqs):
+        ref = RR.oracle_sampling_seq(wl, b)
+        RR.compare_sampling(f"{wl.spec.name.split(':')[0]} seq {b}", x[b], out[b], nacc[b], ref, TALLY)
+    assert TALLY.near_ties <= 1e-4 * TALLY.decisions, TALLY.notes

@@ -34,6 +34,9 @@ CASES = {
     # fp32 with D128, P64 and fp32 logits
     "f32-d128-p64": (custom_spec(0, num_seqs=2, num_q_heads=6, num_kv_heads=2, head_dim=128, page_size=64,
                                  budget_pages=2, vocab=777), [200, 4 * 64 + 1]),
+    # the largest packed tile: G8 x R16 = 128 rows
+    "bf16-g8-r16": (custom_spec(1, num_seqs=2, num_q_heads=16, num_kv_heads=2, gamma=15, budget_pages=2,
+                                vocab=1536), [200, 64 * 5]),
     # shortest legal history: L = R for verify
     "bf16-min-len": (custom_spec(1, num_seqs=2, num_q_heads=4, num_kv_heads=1, gamma=2, budget_pages=1,
                                  vocab=512), [3, 70]),
@@ -145,3 +148,55 @@ def test_tail_only_summaries_touch_only_tail_pages(case):
     assert np.all(kmin[others] == 0.0)
     st.summaries(tail_only=False)
     torch.cuda.synchronize()
+
+
+def test_q_equals_p_accepts_every_draft_on_gpu():
+    """Identical draft and target logits: every draft is accepted, the bonus
+    token is drawn from p_gamma (the degenerate case of the accept rule)."""
+    ws = custom_spec(1, num_seqs=6, gamma=5, vocab=4096)
+    wl = Workload(ws, seed=5)
+    t, _ = wl.logits()
+    tl = torch.from_numpy(t.view(np.int16)).view(torch.bfloat16).cuda()
+    dl = tl[:, :ws.gamma].contiguous()
+    S, g, V = ws.num_seqs, ws.gamma, ws.vocab
+    x = torch.empty((S, g), dtype=torch.int32, device="cuda")
+    wt = torch.zeros(s3r.s3r_sample_workspace_bytes(S * g, 0, V), dtype=torch.uint8, device="cuda")
+    s3r.s3r_sample_tokens(dl, "bf16", S * g, V, 1.0, torch.from_numpy(wl.u_draft).cuda(), x, wt)
+    out = torch.empty((S, g + 1), dtype=torch.int32, device="cuda")
+    n = torch.empty((S,), dtype=torch.int32, device="cuda")
+    w = torch.zeros(s3r.s3r_sample_workspace_bytes(S, g, V), dtype=torch.uint8, device="cuda")
+    s3r.s3r_spec_sample(tl, dl, "bf16", x, torch.from_numpy(wl.u_accept).cuda(), torch.from_numpy(wl.u_sample).cuda(),
+                        S, g, V, 1.0, out, n, w)
+    torch.cuda.synchronize()
+    assert torch.all(n == g)
+    assert torch.equal(out[:, :g], x)
+    assert int(out[:, g].min()) >= 0
+
+
+def test_device_checks_flag_bad_inputs_without_faulting():
+    """A bad context length and a bad page id are recorded in the status word;
+    the kernels skip them and the context stays usable."""
+    ws = custom_spec(1, num_seqs=3, num_q_heads=8, num_kv_heads=2, budget_pages=2, vocab=512)
+    wl = Workload(ws, seed=2, context_lens=[300, 200, 130])
+    st = DecodeStep(wl)
+    st.summaries()
+    torch.cuda.synchronize()
+    # sequence 1: length 0 (unusable); sequence 2: a block-table entry out of range
+    st.context_lens[1] = 0
+    st.block_table[2, 1] = wl.num_pages_total + 5
+    st.verify()
+    status, bits = s3r.s3r_device_status(st.ws_verify)
+    assert status == s3r.S3R_ERR_DEVICE_CHECK
+    assert bits & s3r.S3R_DEV_BAD_CONTEXT_LEN and bits & s3r.S3R_DEV_BAD_PAGE_ID
+    out = st.verify_out.float().cpu().numpy()
+    lse = st.verify_lse.cpu().numpy()
+    assert np.all(out[1] == 0.0) and np.all(np.isneginf(lse[1]))
+    assert np.all(np.isfinite(out[0])) and np.all(np.isfinite(out[2]))
+    # sequence 0 is untouched by the bad entries of the others
+    ref = RR.oracle_attention_seq(wl, 0, draft_steps=[])
+    RR.assert_close("seq 0 verify", out[0], ref["verify_out"], "bf16")
+    # the next call on the same workspace starts clean
+    st.context_lens[1] = 200
+    st.block_table[2, 1] = int(wl.block_table[2, 1])
+    st.verify()
+    assert s3r.s3r_device_status(st.ws_verify) == (s3r.S3R_OK, 0)
