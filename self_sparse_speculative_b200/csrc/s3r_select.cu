@@ -5,9 +5,9 @@
 // One thread-block cluster of CL CTAs per (sequence, KV head):
 //   1. every CTA scores its share of the pages p < n_b with the float64 bound
 //        s(p) = sum_g sum_d max(q[g,d] * kmin[p,d], q[g,d] * kmax[p,d])
-//      over the G query heads of the group (one warp per page, four pages in
+//      over the G query heads of the group (one warp per page, eight pages in
 //      flight per warp; bf16 products are exact in float32, fp32 products are
-//      taken in float64) and stores the page's order-preserving 64-bit key
+//      taken in float64) and copies the pages' order-preserving 64-bit keys
 //      into the shared memory of the cluster's first CTA (distributed shared
 //      memory);
 //   2. that CTA radix-selects the budget-th largest key (8-bit digits from the
@@ -75,6 +75,12 @@ struct SelParams {
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+}
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
@@ -109,7 +115,7 @@ __device__ __forceinline__ void load_row(const T* row, int lane, float* v) {
   }
 }
 
-constexpr int kUnroll = 4;     // pages in flight per warp
+constexpr int kUnroll = 8;     // pages in flight per warp
 
 template <typename T, int CPL>
 __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelParams p) {
@@ -141,9 +147,11 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelParams p) 
       for (int k = tid; k < p.budget; k += kSelThreads) out[k] = k < n_b ? k : -1;
     return;
   }
-  cluster_sync_all();                                     // every CTA of the cluster is running
+  // announce this CTA to the cluster now; wait for the others only before
+  // touching the first CTA's shared memory
+  cluster_arrive();
 
-  // ---- 1. scores of pages [beg, end)
+  // ---- 1. scores of pages [beg, end) into this CTA's own key array
   const int per = (n_b + ncta - 1) / ncta;
   const int beg = min(n_b, (int)rank * per), end = min(n_b, beg + per);
   const T* qp = static_cast<const T*>(p.q) + ((size_t)b * p.Hq + (size_t)h * p.G) * p.D;
@@ -154,7 +162,6 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelParams p) 
   __syncthreads();
   const T* kmn = static_cast<const T*>(p.kmin);
   const T* kmx = static_cast<const T*>(p.kmax);
-  const uint32_t keys_addr = smem_addr(s_keys);
   for (int pg0 = beg + warp * kUnroll; pg0 < end; pg0 += kSelWarps * kUnroll) {
     int phys_l = -1;
     if (lane < kUnroll && pg0 + lane < end) phys_l = p.block_table[(size_t)b * p.max_pages + pg0 + lane];
@@ -193,9 +200,16 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelParams p) 
       for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
       if (lane == 0) {
         if (!ok[u]) flag_status(p.status, S3R_DEV_BAD_PAGE_ID);
-        st_cluster_u64(keys_addr + 8u * (uint32_t)(pg0 + u), 0u, ok[u] ? order_key(acc) : 0ull);
+        s_keys[pg0 + u] = ok[u] ? order_key(acc) : 0ull;
       }
     }
+  }
+  __syncthreads();
+  // ---- copy this CTA's keys into the first CTA (distributed shared memory)
+  cluster_wait();                                         // every CTA of the cluster is running
+  if (rank != 0) {
+    const uint32_t keys_addr = smem_addr(s_keys);
+    for (int pg = beg + tid; pg < end; pg += kSelThreads) st_cluster_u64(keys_addr + 8u * (uint32_t)pg, 0u, s_keys[pg]);
   }
   cluster_sync_all();                                     // all keys are in the first CTA
   if (rank != 0) return;
@@ -319,10 +333,11 @@ cudaError_t launch_select(const s3r_paged_kv& kv, const void* kmin, const void* 
   p.budget = budget;
   p.status = status;
   const size_t smem = (size_t)kv.max_pages_per_seq * sizeof(unsigned long long);
-  // cluster size: about 64 pages per CTA, at most the portable 8
+  // cluster size: about 64 pages per CTA (one 8-page load round per warp),
+  // at most 4 CTAs (larger clusters cannot all be co-scheduled)
   int cl = (kv.max_pages_per_seq + 63) / 64;
   if (cl < 1) cl = 1;
-  if (cl > 8) cl = 8;
+  if (cl > 4) cl = 4;
   const bool bf = kv.dtype == S3R_BF16;
   cudaError_t e;
   if (kv.head_dim == 128) e = bf ? launch_typed<__nv_bfloat16, 4>(p, cl, smem, st) : launch_typed<float, 4>(p, cl, smem, st);
