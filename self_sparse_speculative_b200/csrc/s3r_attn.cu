@@ -316,7 +316,8 @@ cudaError_t launch_attention(const s3r_paged_kv& kv, const AttnParams& p, cudaSt
   if (kv.dtype == S3R_F32) {
     return kv.head_dim == 64 ? launch_f32<64>(p, st) : launch_f32<128>(p, st);
   }
-  return launch_attention_tc(kv, p, st, api);
+  // up to 64 packed rows: token-major tiles; more: rows-major M = 128 tiles
+  return p.rows <= 64 ? launch_attention_tok(kv, p, st, api) : launch_attention_tc(kv, p, st, api);
 }
 
 }  // namespace s3r

@@ -35,6 +35,7 @@
 #include <cmath>
 
 #include "s3r_attn_common.cuh"
+#include "s3r_attn_sched.cuh"
 #include "s3r_device.cuh"
 #include "s3r_internal.h"
 
@@ -62,81 +63,6 @@ struct Lay {
   static constexpr uint32_t kTmemCols = (kColO + 2 * D) <= 256 ? 256 : 512;
   static_assert(kNS >= 2, "pipeline needs two stages");
 };
-
-// One maximal piece of a (sequence, KV head) unit inside a CTA's range.
-struct Seg {
-  int b, h;        // sequence, KV head
-  int k0, npg;     // first page-list index and number of pages
-  int end;         // flattened position after the segment
-  int unit;        // b * Hkv + h
-  int first_cta;   // first CTA whose range holds part of the unit
-  int nseg;        // number of CTAs sharing the unit
-};
-
-// s_prefix[b] = sum over sequences before b of Hkv * pages(b)
-__device__ __forceinline__ Seg locate(const AttnParams& p, const int* s_prefix, int x, int hi, int W) {
-  int lo_b = 0, hi_b = p.S - 1;
-  while (lo_b < hi_b) {                      // first b with prefix[b+1] > x
-    const int mid = (lo_b + hi_b) >> 1;
-    if (s_prefix[mid + 1] > x) hi_b = mid; else lo_b = mid + 1;
-  }
-  Seg s;
-  s.b = lo_b;
-  const int pages = (s_prefix[lo_b + 1] - s_prefix[lo_b]) / p.Hkv;
-  const int o = x - s_prefix[lo_b];
-  s.h = o / pages;
-  s.k0 = o - s.h * pages;
-  const int ustart = s_prefix[lo_b] + s.h * pages, uend = ustart + pages;
-  s.end = min(hi, uend);
-  s.npg = s.end - x;
-  s.unit = s.b * p.Hkv + s.h;
-  s.first_cta = ustart / W;
-  s.nseg = (uend - 1) / W - s.first_cta + 1;
-  return s;
-}
-
-// Logical page and unit (b * Hkv + h) of flattened position x (-1 when out of range).
-__device__ __forceinline__ void page_of(const AttnParams& p, const int* s_prefix, int x, int hi, int W,
-                                        int* lp_out, int* u_out) {
-  *lp_out = -1;
-  *u_out = 0;
-  if (x >= hi) return;
-  const Seg s = locate(p, s_prefix, x, hi, W);
-  *u_out = s.unit;
-  *lp_out = p.page_list ? p.page_list[((size_t)s.b * p.Hkv + s.h) * p.budget + s.k0] : s.k0;
-}
-
-// Walk over the stages of a CTA's range, segment by segment.
-struct Cursor {
-  int x, s, j, nst, g;    // segment start, segment index, stage in segment, stages in segment, global stage
-  bool valid;
-  Seg sg;
-};
-__device__ __forceinline__ Cursor cursor_begin(const AttnParams& p, const int* s_prefix, int lo, int hi, int W,
-                                               int ppt) {
-  Cursor c;
-  c.x = lo; c.s = 0; c.j = 0; c.g = 0; c.nst = 0;
-  c.valid = lo < hi;
-  if (c.valid) {
-    c.sg = locate(p, s_prefix, lo, hi, W);
-    c.nst = (c.sg.npg + ppt - 1) / ppt;
-  }
-  return c;
-}
-__device__ __forceinline__ void cursor_next(const AttnParams& p, const int* s_prefix, int hi, int W, int ppt,
-                                            Cursor& c) {
-  ++c.g;
-  if (++c.j >= c.nst) {
-    c.x = c.sg.end;
-    ++c.s;
-    c.j = 0;
-    c.valid = c.x < hi;
-    if (c.valid) {
-      c.sg = locate(p, s_prefix, c.x, hi, W);
-      c.nst = (c.sg.npg + ppt - 1) / ppt;
-    }
-  }
-}
 
 template <int M, int D>
 __global__ void __launch_bounds__(kThreads, 1)

@@ -1,0 +1,596 @@
+// Token-major persistent tcgen05 attention for up to 64 packed query rows
+// per (sequence, KV head): the S3R sparse draft step (G rows) and the dense
+// verify step (G x (gamma + 1) rows) ("S3R: Fast and Faithful RL Rollouts
+// via Self-Sparse Speculative Decoding", weekinpapers.com, Abstract: sparse
+// attention over selected pages proposes, full attention over the complete
+// KV history verifies, both over one shared paged cache).
+//
+// Decode attention has few query rows and many keys, so the contraction is
+// laid out with the keys in the MMA's M dimension: every 128-token stage of
+// K/V read from HBM feeds
+//   S^T = K Q^T   (M = 128 tokens, N = rows rounded up to 16, K = D)
+//   O^T += V^T P^T (M = D, N, K = 128 tokens),
+// both fp32 in TMEM: 16 MMA instructions per 128 tokens at D = 128, where a
+// rows-major M = 64 tile needs 24 and wastes most of its rows. The softmax
+// thread t owns token t of the stage (TMEM lane t of S^T) and all N rows of
+// it, so the per-row sums stay in registers, P^T is written one token per
+// thread, and the row maximum needs a cross-thread reduction only when some
+// score exceeds the row's reference by more than 2^8 (the reference is lazy:
+// O^T columns and the sums always share it, so the result is exact).
+//
+// Work partition (stream-K): the flattened (sequence, KV head, page) list is
+// split into one contiguous range per CTA (s3r_attn_sched.cuh); a unit split
+// over several CTAs is merged by log-sum-exp in the epilogue of the last CTA
+// to finish (atomic ticket, no waiting).
+//
+// Warp roles (192 threads): warps 0-3 softmax and epilogue (thread = token);
+// warp 4 producer (page ids, L2 prefetch of K/V 4 stages ahead, TMA into an
+// NS-stage ring); warp 5 MMA issuer (QK two stages ahead of PV) and TMEM
+// owner. The softmax warps also stage each segment's Q (fetched into
+// registers one segment ahead).
+#include <cuda_bf16.h>
+
+#include <cmath>
+
+#include "s3r_attn_common.cuh"
+#include "s3r_attn_sched.cuh"
+#include "s3r_device.cuh"
+#include "s3r_internal.h"
+
+namespace s3r {
+namespace {
+
+constexpr int kTokThreads = 192;
+constexpr int kTokProducer = 4;
+constexpr int kTokMma = 5;
+constexpr int kTok = 128;                    // tokens per stage (MMA M of S^T)
+constexpr float kTau = 8.0f;                 // lazy reference slack, log2 units
+constexpr float kNuInit = 1e30f;             // -(reference) before the first score of a segment
+constexpr int kTokSmemBudget = 232448 - 8192;
+
+template <int N, int D>
+struct TokLay {
+  static constexpr int kHalves = D / 64;
+  static constexpr uint32_t kQBytes = N * D * 2;           // [d half][N rows][128 B]
+  static constexpr uint32_t kPBytes = N * kTok * 2;        // [token half][N rows][128 B]
+  static constexpr uint32_t kTileBytes = kTok * D * 2;     // K or V of one stage: [d half][128 tokens][128 B]
+  static constexpr int kNSraw = (kTokSmemBudget - (int)kQBytes - (int)kPBytes) / (2 * (int)kTileBytes);
+  static constexpr int kNS = kNSraw > 6 ? 6 : kNSraw;
+  static constexpr uint32_t kOffP = kQBytes;
+  static constexpr uint32_t kOffKV = kOffP + kPBytes;
+  static constexpr uint32_t kDynBytes = kOffKV + kNS * 2 * kTileBytes;
+  static constexpr uint32_t kColS = 0, kColO = 2 * N;      // S^T[2], O^T
+  static constexpr int kQChunks = N * D / 8 / 128;         // 16-byte Q chunks per softmax thread
+  static_assert(kNS >= 2, "pipeline needs two stages");
+  static_assert(3 * N <= 256, "TMEM columns");
+};
+
+// Reduce N per-thread values per row over the warp: afterwards lane l holds
+// the result for row l of v[0..C) (C = 32), or row l % 16 (C = 16).
+template <int C, bool kMax>
+__device__ __forceinline__ float warp_rows_reduce(float* v, int lane) {
+#pragma unroll
+  for (int w = C / 2; w >= 1; w >>= 1) {
+    const bool up = (lane & w) != 0;
+#pragma unroll
+    for (int k = 0; k < w; ++k) {
+      const float send = up ? v[k] : v[k + w];
+      const float keep = up ? v[k + w] : v[k];
+      const float got = __shfl_xor_sync(0xffffffffu, send, w);
+      v[k] = kMax ? fmaxf(keep, got) : keep + got;
+    }
+  }
+  float r = v[0];
+  if constexpr (C == 16) {
+    const float o = __shfl_xor_sync(0xffffffffu, r, 16);
+    r = kMax ? fmaxf(r, o) : r + o;
+  }
+  return r;
+}
+
+// Row-wise reduction over the 128 softmax threads into red[row] (N rows).
+template <int N, bool kMax>
+__device__ __forceinline__ void wg_rows_reduce(float* v, float (*s_red)[64], float* out, int q4, int lane,
+                                               int tid) {
+#pragma unroll
+  for (int c0 = 0; c0 < N; c0 += 32) {
+    if (N - c0 >= 32) {
+      const float r = warp_rows_reduce<32, kMax>(v + c0, lane);
+      s_red[q4][c0 + lane] = r;
+    } else {
+      const float r = warp_rows_reduce<16, kMax>(v + c0, lane);
+      if (lane < 16) s_red[q4][c0 + lane] = r;
+    }
+  }
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+  if (tid < N) {
+    const float a = s_red[0][tid], b = s_red[1][tid], c = s_red[2][tid], d = s_red[3][tid];
+    out[tid] = kMax ? fmaxf(fmaxf(a, b), fmaxf(c, d)) : (a + b) + (c + d);
+  }
+}
+
+// Number of the 128 softmax threads whose predicate is true (named barrier 1).
+__device__ __forceinline__ int wg_count(bool pred) {
+  int r;
+  asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.popc.u32 %0, 1, 128, p;\n\t}"
+               : "=r"(r) : "r"((int)pred) : "memory");
+  return r;
+}
+
+template <int N, int D>
+__global__ void __launch_bounds__(kTokThreads, 1)
+attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                const AttnParams p) {
+  using L = TokLay<N, D>;
+  constexpr int NS = L::kNS;
+  extern __shared__ __align__(1024) uint8_t dyn_raw[];
+  uint8_t* dyn = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t s_bar[2 * NS + 6];
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+  __shared__ int s_ticket;
+  __shared__ int s_prefix[kMaxSeqs + 1];
+  __shared__ int s_stage_lp[NS][8];
+  __shared__ int s_roff[64];                    // output row of packed row r relative to (b, h)
+  __shared__ float s_red[4][64];
+  __shared__ float s_mx[64];                    // stage maximum per row (raw score)
+  __shared__ __align__(16) float s_nu[64];      // -(reference) per row, log2 units
+  __shared__ __align__(16) float s_alpha[64];   // rescale factor / 1 / l per row
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  // ---- per-sequence prefix of unit pages (warp 0), range of this CTA
+  if (warp == 0) {
+    const int per = (p.S + 31) / 32;
+    const int b0 = min(p.S, lane * per), b1 = min(p.S, b0 + per);
+    int sum = 0;
+    for (int b = b0; b < b1; ++b) sum += unit_pages(p, p.context_lens[b]) * p.Hkv;
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int run = incl - sum;
+    for (int b = b0; b < b1; ++b) {
+      s_prefix[b] = run;
+      run += unit_pages(p, p.context_lens[b]) * p.Hkv;
+    }
+    if (lane == 31) s_prefix[p.S] = incl;
+  }
+  if (tid < 64) s_roff[tid] = (tid / p.G) * p.Hq + (tid % p.G);
+  __syncthreads();
+  if (blockIdx.x == 0) {
+    // unusable lengths: flag them, give their rows zero output and lse -inf
+    for (int b = 0; b < p.S; ++b) {
+      if (!bad_context(p, p.context_lens[b])) continue;
+      if (tid == 0) flag_status(p.status, S3R_DEV_BAD_CONTEXT_LEN);
+      for (int h = 0; h < p.Hkv; ++h) write_empty_unit<__nv_bfloat16>(p, b, h, tid, kTokThreads);
+    }
+  }
+  const int total = s_prefix[p.S];
+  const int W = (total + gridDim.x - 1) / gridDim.x;
+  const int lo = blockIdx.x * W, hi = min(total, lo + W);
+  if (lo >= hi) return;                                 // uniform over the CTA
+  const int ppt = kTok / p.P;                           // pages per stage
+
+  const uint32_t bar0 = smem_addr(&s_bar[0]);
+  auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+  const int B_FULL = 0, B_EMPTY = NS, B_SFULL = 2 * NS, B_PFULL = 2 * NS + 2, B_ODONE = 2 * NS + 3,
+            B_QFULL = 2 * NS + 4, B_TD = 2 * NS + 5;
+  uint8_t* sQ = dyn;
+  uint8_t* sP = dyn + L::kOffP;
+  uint8_t* sKV = dyn + L::kOffKV;
+  const uint32_t aQ = smem_addr(sQ), aP = smem_addr(sP), aKV = smem_addr(sKV);
+
+  if (warp == kTokMma) {
+    tmem_alloc(smem_addr(&s_tmem), 256);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    for (int i = 0; i < NS; ++i) { mbar_init(BAR(B_FULL + i), 1); mbar_init(BAR(B_EMPTY + i), 1); }
+    mbar_init(BAR(B_SFULL), 1);
+    mbar_init(BAR(B_SFULL + 1), 1);
+    mbar_init(BAR(B_PFULL), 128);
+    mbar_init(BAR(B_ODONE), 1);
+    mbar_init(BAR(B_QFULL), 128);
+    mbar_init(BAR(B_TD), 1);
+    s_abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == kTokProducer && lane == 0) { prefetch_tensormap(&tmK); prefetch_tensormap(&tmV); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+
+  if (warp == kTokProducer) {
+    // ======================================================= producer warp
+    const uint64_t pol = l2_policy_evict_first();
+    // page-id windows of 32 flattened positions: lane k of a window holds
+    // position wbase + k. w0 = in use, w1 = phys loads in flight, w2 = lp
+    // loads in flight.
+    int w0_lp, w0_ph, w0_u, w1_lp, w1_ph, w1_u, w2_lp, w2_u;
+    auto phys_load = [&](int lp, int u) {
+      if (lp < 0) return -1;
+      const int b = u / p.Hkv;
+      const int n_b = (p.context_lens[b] + p.P - 1) / p.P;
+      if (lp >= n_b) { flag_status(p.status, S3R_DEV_BAD_PAGE_ID); return -1; }
+      return p.block_table[(size_t)b * p.max_pages + lp];
+    };
+    int wbase = lo;
+    page_of(p, s_prefix, wbase + lane, hi, W, &w0_lp, &w0_u);
+    w0_ph = phys_load(w0_lp, w0_u);
+    page_of(p, s_prefix, wbase + 32 + lane, hi, W, &w1_lp, &w1_u);
+    w1_ph = phys_load(w1_lp, w1_u);
+    page_of(p, s_prefix, wbase + 64 + lane, hi, W, &w2_lp, &w2_u);
+    const int pfd = 4 * ppt;                           // L2 prefetch distance (4 stages, <= 32 positions)
+    int g = 0;
+    bool ok = true;
+    for (int x = lo; x < hi && ok;) {
+      const Seg sg = locate(p, s_prefix, x, hi, W);
+      const int nst = (sg.npg + ppt - 1) / ppt;
+      for (int j = 0; j < nst; ++j, ++g) {
+        const int st = g % NS;
+        if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_EMPTY + st), ((g / NS) & 1) ^ 1, &s_abort, p.status))) {
+          ok = false;
+          break;
+        }
+        int my_lp = -1, my_ph = -1, pf_z = -1;
+        for (int pp = 0; pp < ppt; ++pp) {
+          const int xp = x + j * ppt + pp;
+          const bool in = (j * ppt + pp) < sg.npg;
+          while (xp >= wbase + 32) {                   // advance the windows (warp-uniform)
+            wbase += 32;
+            w0_lp = w1_lp; w0_ph = w1_ph; w0_u = w1_u;
+            w1_lp = w2_lp; w1_u = w2_u;
+            w1_ph = phys_load(w1_lp, w1_u);
+            page_of(p, s_prefix, wbase + 64 + lane, hi, W, &w2_lp, &w2_u);
+          }
+          const int src = xp - wbase;
+          const int lp = __shfl_sync(0xffffffffu, w0_lp, src & 31);
+          int ph = __shfl_sync(0xffffffffu, w0_ph, src & 31);
+          if (in && lp >= 0 && (ph < 0 || ph >= p.num_pages_total)) {
+            if (lane == 0) flag_status(p.status, S3R_DEV_BAD_PAGE_ID);
+            ph = -1;
+          }
+          if (lane == pp && in) { my_lp = lp; my_ph = ph; }
+          const int s2 = src + pfd;                    // < 64: inside windows w0, w1
+          const int lp2 = __shfl_sync(0xffffffffu, s2 < 32 ? w0_lp : w1_lp, s2 & 31);
+          const int ph2 = __shfl_sync(0xffffffffu, s2 < 32 ? w0_ph : w1_ph, s2 & 31);
+          const int u2 = __shfl_sync(0xffffffffu, s2 < 32 ? w0_u : w1_u, s2 & 31);
+          if (lane == pp && xp + pfd < hi && lp2 >= 0 && ph2 >= 0 && ph2 < p.num_pages_total)
+            pf_z = ph2 * p.Hkv + (u2 % p.Hkv);
+        }
+        if (pf_z >= 0) {
+#pragma unroll
+          for (int hh = 0; hh < L::kHalves; ++hh) {
+            tma_prefetch_3d(&tmK, hh * 64, 0, pf_z);
+            tma_prefetch_3d(&tmV, hh * 64, 0, pf_z);
+          }
+        }
+        if (lane < 8) s_stage_lp[st][lane] = (lane < ppt && my_ph >= 0) ? my_lp : -1;
+        const unsigned real = __ballot_sync(0xffffffffu, my_ph >= 0);
+        __syncwarp();
+        if (lane == 0)
+          mbar_arrive_expect_tx(BAR(B_FULL + st), (uint32_t)__popc(real) * L::kHalves * 2u * (uint32_t)p.P * 128u);
+        __syncwarp();
+        if (my_ph >= 0) {
+          const uint32_t dK = aKV + st * 2 * L::kTileBytes, dV = dK + L::kTileBytes;
+          const int z = my_ph * p.Hkv + sg.h;
+#pragma unroll
+          for (int hh = 0; hh < L::kHalves; ++hh) {
+            const uint32_t off = hh * (kTok * 128) + lane * (p.P * 128);
+            tma_load_3d(dK + off, &tmK, BAR(B_FULL + st), hh * 64, 0, z, pol);
+            tma_load_3d(dV + off, &tmV, BAR(B_FULL + st), hh * 64, 0, z, pol);
+          }
+        }
+      }
+      x = sg.end;
+    }
+    // drain: wait until every issued copy has landed
+    if (lane == 0)
+      for (int k = max(0, g - NS); k < g; ++k) mbar_wait_drain(BAR(B_FULL + k % NS), (k / NS) & 1, p.status);
+  } else if (warp == kTokMma) {
+    // ======================================================= MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idQK = idesc_bf16_f32(kTok, N, false, false);
+      constexpr uint32_t idPV = idesc_bf16_f32(D, N, true, false);
+      Cursor qc = cursor_begin(p, s_prefix, lo, hi, W, ppt);
+      Cursor pc = qc;
+      bool ok = true;
+      // K (A of S^T) and Q (B): K-major, 128-byte rows, 8-row groups 1024 B
+      // apart; a K16 step is 32 bytes inside the swizzle row, the next 64
+      // columns are one half-tile further. V^T (A of O^T) is M-major: the
+      // two 64-dim halves one 128-token half-tile apart, 16 tokens = 2048 B.
+      // P^T (B of O^T): K-major, 64-token halves N * 128 bytes apart.
+      const uint64_t dQ0 = smem_desc_sw128(aQ, 16, 1024);
+      const uint64_t dK0 = smem_desc_sw128(aKV, 16, 1024);
+      const uint64_t dV0 = smem_desc_sw128(aKV + L::kTileBytes, kTok * 128, 1024);
+      const uint64_t dP0 = smem_desc_sw128(aP, 16, 1024);
+      constexpr uint64_t kQHalf = (N * 128) >> 4, kPHalf = (N * 128) >> 4;
+      constexpr uint64_t kStage = (2 * L::kTileBytes) >> 4, kKHalf = (kTok * 128) >> 4, kVStep = (16 * 128) >> 4;
+      auto issue_qk = [&]() -> bool {
+        if (qc.j == 0 && !mbar_wait(BAR(B_QFULL), qc.s & 1, &s_abort, p.status)) return false;
+        const int st = qc.g % NS;
+        if (!mbar_wait(BAR(B_FULL + st), (qc.g / NS) & 1, &s_abort, p.status)) return false;
+        tc_fence_after();
+        const uint64_t kd = dK0 + (uint64_t)st * kStage;
+        const uint32_t dS = tmem + L::kColS + (qc.g & 1) * N;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t off = (uint64_t)(kk & 3) * 2;
+          umma_f16(dS, kd + (kk >> 2) * kKHalf + off, dQ0 + (kk >> 2) * kQHalf + off, idQK, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(BAR(B_SFULL + (qc.g & 1)));
+        cursor_next(p, s_prefix, hi, W, ppt, qc);
+        return true;
+      };
+      for (int k = 0; k < 2 && qc.valid && ok; ++k) ok = issue_qk();
+      while (ok && pc.valid) {
+        if (!mbar_wait(BAR(B_PFULL), pc.g & 1, &s_abort, p.status)) { ok = false; break; }
+        tc_fence_after();
+        const int st = pc.g % NS;
+        const uint64_t vd = dV0 + (uint64_t)st * kStage;
+        const uint32_t tO = tmem + L::kColO;
+        const uint32_t acc0 = pc.j > 0 ? 1u : 0u;
+#pragma unroll
+        for (int kk = 0; kk < kTok / 16; ++kk)
+          umma_f16(tO, vd + (uint64_t)kk * kVStep, dP0 + (kk >> 2) * kPHalf + (uint64_t)(kk & 3) * 2, idPV,
+                   kk > 0 ? 1u : acc0);
+        umma_commit(BAR(B_EMPTY + st));
+        umma_commit(BAR(B_ODONE));
+        cursor_next(p, s_prefix, hi, W, ppt, pc);
+        if (qc.valid && !issue_qk()) { ok = false; break; }
+      }
+      umma_commit(BAR(B_TD));
+    }
+  } else {
+    // ======================================================= softmax warps
+    // Thread t: token t of each stage (TMEM lane t of S^T), and TMEM lane t
+    // of O^T in the epilogue (dimension t for D = 128; for D = 64 the M = 64
+    // accumulator puts dimension 16q + l in lane 32q + l, l < 16).
+    const int q4 = warp;
+    const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
+    const int d_mine = (D == 128) ? tid : (lane < 16 ? 16 * q4 + lane : -1);
+    const int log2P = __ffs(p.P) - 1;
+    const float c = p.scale_log2;
+    constexpr int kQC = L::kQChunks;
+    constexpr int kDc = D / 8;                          // 16-byte chunks per Q row
+    uint4 qr[kQC];
+    auto q_fetch = [&](const Seg& s) {
+      const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(p.q);
+      const size_t base = (size_t)(s.b * p.R) * p.Hq + (size_t)s.h * p.G;
+#pragma unroll
+      for (int k = 0; k < kQC; ++k) {
+        const int ch = tid + 128 * k, r = ch / kDc, c16 = ch - (ch / kDc) * kDc;
+        qr[k] = r < p.rows ? __ldg(reinterpret_cast<const uint4*>(q + (base + s_roff[r]) * D + c16 * 8))
+                           : make_uint4(0u, 0u, 0u, 0u);
+      }
+    };
+    auto q_store = [&]() {
+#pragma unroll
+      for (int k = 0; k < kQC; ++k) {
+        const int ch = tid + 128 * k, r = ch / kDc, c16 = ch - (ch / kDc) * kDc;
+        *reinterpret_cast<uint4*>(sQ + (c16 >> 3) * (N * 128) + r * 128 + (((c16 & 7) ^ (r & 7)) << 4)) = qr[k];
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(BAR(B_QFULL));
+    };
+    Seg sg = locate(p, s_prefix, lo, hi, W);
+    q_fetch(sg);
+    q_store();
+    int g = 0;
+    bool ok = true;
+    for (int x = lo; x < hi;) {
+      const bool has_next = sg.end < hi;
+      Seg nx = sg;
+      if (has_next) {
+        nx = locate(p, s_prefix, sg.end, hi, W);
+        q_fetch(nx);                                   // lands while this segment runs
+      }
+      const int nst = (sg.npg + ppt - 1) / ppt;
+      const int Lb = p.context_lens[sg.b];
+      if (tid < N) s_nu[tid] = kNuInit;
+      float l[N];
+#pragma unroll
+      for (int r = 0; r < N; ++r) l[r] = 0.f;
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      bool abort_all = false;
+      for (int j = 0; j < nst; ++j, ++g) {
+        const int st = g % NS, sb = g & 1;
+        ok &= mbar_wait(BAR(B_SFULL + sb), (g >> 1) & 1, &s_abort, p.status) &&
+              mbar_wait(BAR(B_FULL + st), (g / NS) & 1, &s_abort, p.status);
+        tc_fence_after();
+        // this thread's token: position, existence, causal mask of the rows
+        const int lp = s_stage_lp[st][tid >> log2P];
+        const int pos = lp * p.P + (tid & (p.P - 1));
+        const bool valid = lp >= 0 && pos < Lb;
+        const int excess = pos - (Lb - p.R);
+        const int nm = !valid ? N : (excess > 0 ? min(N, p.G * excess) : 0);
+        float s[N];
+        auto load_s = [&]() {
+          tmem_ld_cols<N>(tmem + lane_base + L::kColS + sb * N, s);
+          tmem_wait_ld();
+          if (nm > 0) {
+#pragma unroll
+            for (int r = 0; r < N; ++r)
+              if (r < nm) s[r] = -INFINITY;
+          }
+        };
+        load_s();
+        float ymax = -INFINITY;
+#pragma unroll
+        for (int r = 0; r < N; r += 4) {
+          const float4 v = *reinterpret_cast<const float4*>(&s_nu[r]);
+          ymax = fmaxf(fmaxf(ymax, fmaf(s[r], c, v.x)), fmaf(s[r + 1], c, v.y));
+          ymax = fmaxf(fmaxf(ymax, fmaf(s[r + 2], c, v.z)), fmaf(s[r + 3], c, v.w));
+        }
+        // one barrier per stage: stop together, or raise the references together
+        const int cnt = wg_count(!ok || ymax > kTau);
+        bool rescale_o = false;
+        if (cnt > 0) {
+          if (wg_count(!ok) > 0) { abort_all = true; break; }
+          // stage maximum per row (S^T is intact until PFULL), then reload
+          wg_rows_reduce<N, true>(s, s_red, s_mx, q4, lane, tid);
+          if (tid < N) {
+            const float m_old = -s_nu[tid];
+            const float m_new = fmaxf(m_old, s_mx[tid] * c);
+            s_alpha[tid] = ex2(m_old - m_new);
+            s_nu[tid] = -m_new;
+          }
+          asm volatile("bar.sync 1, 128;" ::: "memory");
+#pragma unroll
+          for (int r = 0; r < N; r += 4) {
+            const float4 a = *reinterpret_cast<const float4*>(&s_alpha[r]);
+            l[r] *= a.x; l[r + 1] *= a.y; l[r + 2] *= a.z; l[r + 3] *= a.w;
+          }
+          load_s();
+          rescale_o = j > 0;
+        }
+        // s <- P = 2^(s c - m_ref), row sums
+#pragma unroll
+        for (int r = 0; r < N; r += 4) {
+          const float4 v = *reinterpret_cast<const float4*>(&s_nu[r]);
+          s[r] = ex2(fmaf(s[r], c, v.x));
+          s[r + 1] = ex2(fmaf(s[r + 1], c, v.y));
+          s[r + 2] = ex2(fmaf(s[r + 2], c, v.z));
+          s[r + 3] = ex2(fmaf(s[r + 3], c, v.w));
+          l[r] += s[r]; l[r + 1] += s[r + 1]; l[r + 2] += s[r + 2]; l[r + 3] += s[r + 3];
+        }
+        // P and O^T were last used by PV(g - 1)
+        if (g > 0) ok &= mbar_wait(BAR(B_ODONE), (g - 1) & 1, &s_abort, p.status);
+        tc_fence_after();
+        if (rescale_o) {
+          float o[N];
+          tmem_ld_cols<N>(tmem + lane_base + L::kColO, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int r = 0; r < N; ++r) o[r] *= s_alpha[r];
+          tmem_st_cols<N>(tmem + lane_base + L::kColO, o);
+          tmem_wait_st();
+        }
+        {
+          const int half = tid >> 6, tt = tid & 63;
+          uint8_t* pb = sP + half * (N * 128) + (tt & 7) * 2;
+          const int ck = tt >> 3;
+#pragma unroll
+          for (int r = 0; r < N; ++r)
+            *reinterpret_cast<__nv_bfloat16*>(pb + r * 128 + ((ck ^ (r & 7)) << 4)) = __float2bfloat16_rn(s[r]);
+        }
+        if (!valid) {
+          // a token that does not exist (beyond L, or a missing page): zero
+          // its V row so that 0 * stale data cannot reach O
+          uint8_t* sV = sKV + st * 2 * L::kTileBytes + L::kTileBytes + tid * 128;
+#pragma unroll
+          for (int hh = 0; hh < L::kHalves; ++hh)
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              *reinterpret_cast<uint4*>(sV + hh * (kTok * 128) + k * 16) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(BAR(B_PFULL));
+      }
+      if (abort_all) break;
+      // ---- the last QK of this segment is done: stage the next segment's Q
+      if (has_next) q_store();
+      // ---- segment epilogue: row sums, then O^T / l
+      wg_rows_reduce<N, false>(l, s_red, s_alpha, q4, lane, tid);
+      const bool single = sg.nseg == 1;
+      const int slot_idx = sg.unit + blockIdx.x;          // partial slot of (unit, this CTA)
+      const size_t rowbase = (size_t)(sg.b * p.R) * p.Hq + (size_t)sg.h * p.G;
+      if (tid < p.rows) {
+        const float lt = s_alpha[tid], m = -s_nu[tid];
+        if (single) {
+          if (p.lse) p.lse[rowbase + s_roff[tid]] = lt > 0.f ? (m + log2f(lt)) * kLn2 : -INFINITY;
+        } else {
+          const size_t pi = (size_t)slot_idx * p.rows + tid;
+          p.part_ml[pi * 2] = lt > 0.f ? m : -INFINITY;
+          p.part_ml[pi * 2 + 1] = lt;
+        }
+        s_alpha[tid] = lt > 0.f ? 1.f / lt : 0.f;
+      }
+      ok &= mbar_wait(BAR(B_ODONE), (g - 1) & 1, &s_abort, p.status);     // PV of the last stage
+      tc_fence_after();
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      {
+        float o[N];
+        tmem_ld_cols<N>(tmem + lane_base + L::kColO, o);
+        tmem_wait_ld();
+        if (d_mine >= 0) {
+          if (single) {
+            __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) + rowbase * D + d_mine;
+#pragma unroll
+            for (int r = 0; r < N; ++r)
+              if (r < p.rows) dst[(size_t)s_roff[r] * D] = __float2bfloat16_rn(o[r] * s_alpha[r]);
+          } else {
+            float* dst = p.part_o + (size_t)slot_idx * p.rows * D + d_mine;
+#pragma unroll
+            for (int r = 0; r < N; ++r)
+              if (r < p.rows) dst[(size_t)r * D] = o[r];
+          }
+        }
+      }
+      tc_fence_before();
+      if (!single) {
+        __threadfence();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (tid == 0) s_ticket = atomicAdd(p.tickets + sg.unit, 1u);
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (s_ticket == sg.nseg - 1) {
+          __threadfence();
+          combine_partials<__nv_bfloat16>(p, sg.b, sg.h, sg.first_cta + sg.unit, sg.nseg, 128);
+          if (tid == 0) p.tickets[sg.unit] = 0u;
+        }
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");    // s_alpha / s_nu reads done
+      x = sg.end;
+      sg = nx;
+    }
+  }
+
+  // ---- teardown: every role is done; wait for the MMAs, free TMEM
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kTokMma) {
+    tc_fence_after();
+    if (lane == 0) mbar_wait_drain(BAR(B_TD), 0, p.status);
+    __syncwarp();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+template <int N, int D>
+cudaError_t launch_tok(const s3r_paged_kv& kv, const AttnParams& p, cudaStream_t st, s3r_status* api) {
+  CUtensorMap mk, mv;
+  if (!make_cache_map(&mk, kv.k_cache, kv) || !make_cache_map(&mv, kv.v_cache, kv)) {
+    *api = S3R_ERR_CUDA;
+    return cudaErrorInvalidValue;
+  }
+  const size_t smem = TokLay<N, D>::kDynBytes + 1024;
+  cudaError_t e = cudaFuncSetAttribute(attn_tok_kernel<N, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  int grid = device_sm_count();
+  if (grid > kMaxPersistentCtas) grid = kMaxPersistentCtas;
+  attn_tok_kernel<N, D><<<grid, kTokThreads, smem, st>>>(mk, mv, p);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_tok_rows(const s3r_paged_kv& kv, const AttnParams& p, cudaStream_t st, s3r_status* api) {
+  if (p.rows <= 16) return launch_tok<16, D>(kv, p, st, api);
+  if (p.rows <= 32) return launch_tok<32, D>(kv, p, st, api);
+  if (p.rows <= 48) return launch_tok<48, D>(kv, p, st, api);
+  return launch_tok<64, D>(kv, p, st, api);
+}
+
+}  // namespace
+
+cudaError_t launch_attention_tok(const s3r_paged_kv& kv, const AttnParams& p, cudaStream_t st, s3r_status* api) {
+  *api = S3R_OK;
+  return kv.head_dim == 64 ? launch_tok_rows<64>(kv, p, st, api) : launch_tok_rows<128>(kv, p, st, api);
+}
+
+}  // namespace s3r

@@ -66,6 +66,8 @@ cudaError_t launch_attention(const s3r_paged_kv& kv, const AttnParams& p, cudaSt
                              s3r_status* api_status);
 cudaError_t launch_attention_tc(const s3r_paged_kv& kv, const AttnParams& p, cudaStream_t st,
                                 s3r_status* api_status);
+cudaError_t launch_attention_tok(const s3r_paged_kv& kv, const AttnParams& p, cudaStream_t st,
+                                s3r_status* api_status);
 bool make_cache_map(CUtensorMap* map, const void* base, const s3r_paged_kv& kv);
 int device_sm_count();
 
