@@ -133,6 +133,20 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- our arm
+def over_ranks(ms, tokens, world, device):
+    """(max over ranks of a device time in ms, sum over ranks of a token count).
+    Every rank must call it at the same point (two collectives)."""
+    if world <= 1:
+        return float(ms), float(tokens)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    k = torch.tensor([float(tokens)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(k, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(k.item())
+
+
 def run_ours(a):
     import torch
     import torch.distributed as dist
@@ -202,15 +216,7 @@ def run_ours(a):
     if bad:
         raise RuntimeError(f"device checks failed: {bad}")
 
-    t = torch.tensor([total_ms, float(tokens)], dtype=torch.float64, device=f"cuda:{local}")
-    if world > 1:
-        tm = t[:1].clone()
-        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
-        tk = t[1:].clone()
-        dist.all_reduce(tk, op=dist.ReduceOp.SUM)
-        total_ms_max, tokens_all = float(tm.item()), float(tk.item())
-    else:
-        total_ms_max, tokens_all = total_ms, float(tokens)
+    total_ms_max, tokens_all = over_ranks(total_ms, tokens, world, f"cuda:{local}")
 
     # ---- end to end: host buffers, H2D of the step's inputs and D2H of the result
     e2e = None
@@ -242,11 +248,7 @@ def run_ours(a):
         barrier()
         e2e_ms = e_s.elapsed_time(e_e)
         e2e_tokens = (int(nacc_h.sum().item()) + ws.num_seqs) * a.steps
-        tt = torch.tensor([e2e_ms, float(e2e_tokens)], dtype=torch.float64, device=f"cuda:{local}")
-        if world > 1:
-            m = tt[:1].clone(); dist.all_reduce(m, op=dist.ReduceOp.MAX)
-            s_ = tt[1:].clone(); dist.all_reduce(s_, op=dist.ReduceOp.SUM)
-            e2e_ms, e2e_tokens = float(m.item()), float(s_.item())
+        e2e_ms, e2e_tokens = over_ranks(e2e_ms, e2e_tokens, world, f"cuda:{local}")
         e2e = {"value": e2e_tokens / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h)}
 
@@ -284,7 +286,7 @@ def run_ours(a):
                    "verify": round(verify_gbs, 1), "verify_frac_of_8tbs": round(verify_gbs / 8000, 4)},
         "acceptance": {"mean_accepted_per_seq": round(n_acc_total / (ws.num_seqs * a.steps), 4),
                        "committed_per_seq": round(tokens / (ws.num_seqs * a.steps), 4)},
-        "gpu_launches": (3 * ws.gamma + 5) * a.steps,
+        "gpu_launches": (3 * ws.gamma + 6) * a.steps,
         "clocks": clk,
     }
     if e2e:
