@@ -133,6 +133,45 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- our arm
+# sources of the verify kernel; the committed ncu summary records their hash
+VERIFY_SOURCES = ("s3r_attn_tok.cu", "s3r_attn_sched.cuh", "s3r_attn_common.cuh", "s3r_device.cuh")
+VERIFY_PROFILE = os.path.join(HERE, "profiles", "verify_attn_tok_qwen3-8b-layer.md")
+
+
+def verify_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    for f in VERIFY_SOURCES:
+        with open(os.path.join(HERE, "self_sparse_speculative_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def verify_traffic():
+    """DRAM bytes (read + write) per verify launch from the committed ncu
+    summary, or None when it was taken on other kernel sources."""
+    try:
+        kv = {}
+        with open(VERIFY_PROFILE) as f:
+            for line in f:
+                if line.startswith("- ") and ":" in line:
+                    k, v = line[2:].split(":", 1)
+                    kv[k.strip()] = v.strip().strip("`")
+        if kv.get("source hash") != verify_source_hash():
+            return None
+        return int(kv["dram bytes per launch"])
+    except Exception:
+        return None
+
+
+def config_of(ws, world, seed):
+    return {"workload": ws.name, "sequences_per_gpu": ws.num_seqs, "context": ws.context,
+            "q_heads": ws.num_q_heads, "kv_heads": ws.num_kv_heads, "head_dim": ws.head_dim,
+            "page": ws.page_size, "budget_pages": ws.budget_pages, "gamma": ws.gamma,
+            "vocab": ws.vocab, "parallelism": f"replicas x{world} (sequence-sharded, no collective)",
+            "l2": "not flushed: inputs larger than L2 (each step reads > 126 MB)", "seed": seed}
+
+
 def over_ranks(ms, tokens, world, device):
     """(max over ranks of a device time in ms, sum over ranks of a token count).
     Every rank must call it at the same point (two collectives)."""
@@ -269,16 +308,11 @@ def run_ours(a):
         "warmup": a.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "impl": "ours",
-        "config": {"workload": ws.name, "sequences_per_gpu": ws.num_seqs, "context": ws.context,
-                   "q_heads": ws.num_q_heads, "kv_heads": ws.num_kv_heads, "head_dim": ws.head_dim,
-                   "page": ws.page_size, "budget_pages": ws.budget_pages, "gamma": ws.gamma,
-                   "vocab": ws.vocab, "parallelism": f"replicas x{world} (sequence-sharded, no collective)",
-                   "l2": "not flushed: each step reads %.2f GB > 126 MB L2" % (nbytes["step"] / 1e9),
-                   "seed": a.seed},
+        "config": config_of(ws, world, a.seed),
         "roofline": {"bound": "hbm", "kernel": "verify attention (s3r_verify_attn)",
                      "achieved": round(verify_gbs, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(verify_gbs / peak, 4), "peak_kind": peak_kind,
-                     "traffic": None,
+                     "traffic": verify_traffic(),
                      "algorithmic_bytes_per_launch": nbytes["verify"]},
         "phases_ms": {"draft_token_draws": round(t_draw, 4), "sparse_draft_per_call": round(t_draft, 4),
                       "verify": round(t_verify, 4), "spec_sample": round(t_sample, 4)},
@@ -286,7 +320,7 @@ def run_ours(a):
                    "verify": round(verify_gbs, 1), "verify_frac_of_8tbs": round(verify_gbs / 8000, 4)},
         "acceptance": {"mean_accepted_per_seq": round(n_acc_total / (ws.num_seqs * a.steps), 4),
                        "committed_per_seq": round(tokens / (ws.num_seqs * a.steps), 4)},
-        "gpu_launches": (3 * ws.gamma + 6) * a.steps,
+        "gpu_launches": (3 * ws.gamma + 5) * a.steps,
         "clocks": clk,
     }
     if e2e:
@@ -305,6 +339,7 @@ def run_ours(a):
 # ---------------------------------------------------------------- reference arm
 def run_reference(a):
     rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return
     from self_sparse_speculative_b200.workloads import spec
@@ -320,10 +355,10 @@ def run_reference(a):
         toks += t
         wall += w
     value = toks / wall
-    line = {"metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": 0, "steps": a.steps,
+    line = {"metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": a.steps,
             "warmup": a.warmup, "ms_per_step": round(wall / a.steps * 1e3, 2), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": ws.name, "sequences_per_step": seqs_per_step},
+            "config": config_of(ws, world, a.seed),
             "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": workers, "kind": "oracle",
                              "sample": f"{seqs_per_step} of {ws.num_seqs} sequences per step, full float64 "
                                        f"round per sequence"},

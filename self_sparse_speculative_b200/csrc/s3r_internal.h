@@ -78,7 +78,7 @@ struct SamplePlan {
   int32_t c2, ch2;      // pass-2 chunks per sequence and elements per chunk
   size_t ws_bytes;
   size_t off_tk_row, off_tk_seq1, off_tk_seq2, off_tk_seq3, off_j;
-  size_t off_part1, off_stats, off_znorm, off_zpart, off_wpart;
+  size_t off_part1, off_stats, off_znorm, off_zpart, off_wpart, off_cmax;
   size_t memset_bytes;  // bytes from the start of the workspace cleared per call
 };
 SamplePlan plan_sampling(int32_t nseq, int32_t gamma, int32_t vocab);
@@ -105,6 +105,7 @@ struct SampleParams {
   double* znorm;           // [nseq, 2] exact float64 Z of the residual's two rows
   double* zpart;           // [nseq, c2, 2] chunk partials of znorm
   double* wpart;           // [nseq, c2, 8] per-warp partial sums of the draw weights
+  float* cmax;             // [nseq, c2] chunk maxima (plain draws)
   int32_t c1, ch1, c2, ch2;
 };
 // Fill the workspace pointers and sizes of `p` from a plan and a workspace base.

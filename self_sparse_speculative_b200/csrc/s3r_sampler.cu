@@ -13,16 +13,18 @@
 // ticket) merges the chunk partials into the row's (max, Z); the last row of
 // a sequence takes the gamma accept/reject tests (one lane each) in float64.
 // Pass 2a (residual sequences only): the exact float64 normalisers of the
-// two rows the residual is drawn from (float64 exponentials).
+// two rows the residual is drawn from.
 // Pass 2b (grid: vocab chunks x sequences): float64 draw weights, summed per
-// warp segment; the last CTA of a sequence finds the chunk, then the warp
-// segment holding u * total, and one warp scans it for the drawn token. Every
-// draw is decided in float64 on both sides, so it is exact up to the order of
-// the float64 sums.
-// The drafter's own draw (s3r_sample_tokens) is pass 1 + pass 2b in "plain"
-// mode: one row per draw, weights exp((x - max)/T).
+// warp segment; the last CTA of a sequence finds, with CTA-wide float64
+// scans, the segment holding u * total and then the token inside it. Every
+// draw is decided in float64 on both sides, so it is exact up to the order
+// of the float64 sums. float64 exponentials are table-driven (exp_tbl).
+// The drafter's own draws (s3r_sample_tokens) are pass 2b alone in "plain"
+// mode: one row per draw, weights exp((x - m_c)/T) with m_c the chunk's own
+// maximum, brought to the row maximum when the chunks are merged.
 #include <cuda_bf16.h>
 
+#include <climits>
 #include <cmath>
 
 #include "s3r_device.cuh"
@@ -92,6 +94,43 @@ __device__ float block_max(float v, float* s_red) {
   for (int w = 1; w < kSmpWarps; ++w) r = fmaxf(r, s_red[w]);
   __syncthreads();
   return r;
+}
+
+// float64 exponential, table-driven (P. T. P. Tang, "Table-driven
+// implementation of the exponential function in IEEE floating-point
+// arithmetic", ACM Trans. Math. Software 15(2), 1989): write
+// x = (32 m + j) ln2/32 + r with |r| <= ln2/64, then
+// exp(x) = 2^m * 2^(j/32) * e^r. Here N = 32 m + j is x * 32/ln2 rounded to
+// an integer by adding 1.5 * 2^52; r = x - N ln2/32 with ln2/32 split into a
+// double and its remainder (two fused multiply-adds); e^r - 1 is its Taylor
+// polynomial to degree 6 (remainder < 4e-18 for |r| <= ln2/64); 2^(j/32) is
+// a 32-entry table `tab`; 2^m goes into the exponent field. The result is
+// within about 2 ulp. Outside (-707, 708) (subnormal results, overflow,
+// infinities, NaN) the CUDA library exp is used.
+__device__ __forceinline__ double exp_tbl(double x, const double* tab) {
+  if (!(x > -707.0 && x < 708.0)) return exp(x);
+  constexpr double kInvStep = 46.16624130844683;           // 32 / ln2
+  constexpr double kStepHi = 0x1.62e42fefa39efp-6;          // ln2 / 32, leading double
+  constexpr double kStepLo = 0x1.abc9e3b39803fp-61;         // ln2 / 32 - kStepHi
+  constexpr double kShifter = 6755399441055744.0;           // 1.5 * 2^52
+  const double t = fma(x, kInvStep, kShifter);
+  const int n = __double2loint(t);
+  const double nd = t - kShifter;
+  double r = fma(-nd, kStepHi, x);
+  r = fma(-nd, kStepLo, r);
+  double q = fma(r, 1.0 / 720.0, 1.0 / 120.0);
+  q = fma(q, r, 1.0 / 24.0);
+  q = fma(q, r, 1.0 / 6.0);
+  q = fma(q, r, 0.5);
+  q = fma(q, r, 1.0);
+  const double tj = tab[n & 31];
+  const double y = fma(tj, q * r, tj);
+  return __hiloint2double(__double2hiint(y) + ((n >> 5) << 20), __double2loint(y));
+}
+
+// 2^(j/32), j = 0..31, into shared memory (threads 0..31; caller syncs).
+__device__ __forceinline__ void fill_exp_tab(double* tab) {
+  if (threadIdx.x < 32) tab[threadIdx.x] = exp2(static_cast<double>(threadIdx.x) * 0.03125);
 }
 
 // Row pointers of the spec layout: rows 0..R-1 target, R..2*gamma draft.
@@ -244,9 +283,9 @@ __device__ DrawRows draw_rows(const SampleParams& p, int s, int j, bool exact_z)
   w.iZq = 1.0;
   w.qrow = nullptr;
   w.Mq = 0.0;
-  if (!SPEC) {
+  if (!SPEC) {                                          // the shift is the chunk's own maximum
     w.prow = static_cast<const T*>(p.target) + (size_t)s * p.vocab;
-    w.Mp = p.stats[2 * (size_t)s];
+    w.Mp = 0.0;
     return w;
   }
   const int per = 2 * p.gamma + 1, R = p.gamma + 1;
@@ -275,7 +314,8 @@ __device__ __forceinline__ void load_vals(const T* row, int e, int n, float* v) 
 }
 
 template <typename T, bool VEC>
-__device__ __forceinline__ void weights(const DrawRows& w, int e, int n, double invT, double* out) {
+__device__ __forceinline__ void weights(const DrawRows& w, int e, int n, double invT, const double* tab,
+                                        double* out) {
   using IO = LogitIO<T>;
   float a[IO::kPerVec], b[IO::kPerVec];
   load_vals<T, VEC>(static_cast<const T*>(w.prow), e, n, a);
@@ -284,9 +324,9 @@ __device__ __forceinline__ void weights(const DrawRows& w, int e, int n, double 
   for (int t = 0; t < IO::kPerVec; ++t) {
     double wt = 0.0;
     if (t < n) {
-      const double pe = exp((static_cast<double>(a[t]) - w.Mp) * invT) * w.iZp;
+      const double pe = exp_tbl((static_cast<double>(a[t]) - w.Mp) * invT, tab) * w.iZp;
       if (w.qrow) {
-        const double qe = exp((static_cast<double>(b[t]) - w.Mq) * invT) * w.iZq;
+        const double qe = exp_tbl((static_cast<double>(b[t]) - w.Mq) * invT, tab) * w.iZq;
         wt = pe > qe ? pe - qe : 0.0;
       } else {
         wt = pe;
@@ -300,11 +340,14 @@ __device__ __forceinline__ void weights(const DrawRows& w, int e, int n, double 
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(kSmpThreads) znorm_kernel(const SampleParams p) {
   __shared__ double s_red[2][kSmpWarps];
+  __shared__ double s_tab[32];
   __shared__ int s_last;
   using IO = LogitIO<T>;
   const int s = blockIdx.y, c = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int j = p.jsel[s];
   if (j >= p.gamma) return;                              // bonus draw: no residual (uniform per sequence)
+  fill_exp_tab(s_tab);
+  __syncthreads();
   DrawRows w = draw_rows<T, true>(p, s, j, false);
   const int beg = c * p.ch2, end = min(p.vocab, beg + p.ch2);
   double zt = 0.0, zd = 0.0;
@@ -316,8 +359,8 @@ __global__ void __launch_bounds__(kSmpThreads) znorm_kernel(const SampleParams p
 #pragma unroll
     for (int t = 0; t < IO::kPerVec; ++t) {
       if (t < n) {
-        zt += exp((static_cast<double>(a[t]) - w.Mp) * p.inv_temp_d);
-        zd += exp((static_cast<double>(b[t]) - w.Mq) * p.inv_temp_d);
+        zt += exp_tbl((static_cast<double>(a[t]) - w.Mp) * p.inv_temp_d, s_tab);
+        zd += exp_tbl((static_cast<double>(b[t]) - w.Mq) * p.inv_temp_d, s_tab);
       }
     }
   }
@@ -350,145 +393,252 @@ __global__ void __launch_bounds__(kSmpThreads) znorm_kernel(const SampleParams p
   }
 }
 
-// One warp scans [beg, end) from running sum `base` for the first k whose
-// running sum exceeds thr. Returns k, or -1 - (last index with weight > 0).
-template <typename T, bool VEC>
-__device__ int warp_scan_find(const DrawRows& w, int beg, int end, double base, double thr, double invT) {
-  using IO = LogitIO<T>;
-  constexpr int PV = IO::kPerVec;
-  const int lane = threadIdx.x & 31;
-  int last_pos = -1;
-  double run = base;
-  for (int e0 = beg; e0 < end; e0 += 32 * PV) {
-    const int e = e0 + lane * PV;
-    double wv[PV];
-    const int n = max(0, min(PV, end - e));
-    if (n > 0) weights<T, VEC>(w, e, n, invT, wv);
-    else
+// Inclusive scan of one float64 per thread over the CTA; *total gets the CTA
+// total. Every thread calls it; it ends with the CTA synchronised.
+__device__ double block_scan_d(double v, double* total, double* s_w) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  double x = v;
 #pragma unroll
-      for (int t = 0; t < PV; ++t) wv[t] = 0.0;
-    double loc = 0.0;
-#pragma unroll
-    for (int t = 0; t < PV; ++t) loc += wv[t];
-    double incl = loc;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const double y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    const double before = run + incl - loc;
-    int hit = -1, lp = -1;
-    double r = before;
-#pragma unroll
-    for (int t = 0; t < PV; ++t) {
-      r += wv[t];
-      if (wv[t] > 0.0) lp = e + t;
-      if (hit < 0 && r > thr) hit = e + t;
-    }
-    const unsigned m = __ballot_sync(0xffffffffu, hit >= 0);
-    if (m) return __shfl_sync(0xffffffffu, hit, __ffs(m) - 1);
-    const unsigned mp = __ballot_sync(0xffffffffu, lp >= 0);
-    if (mp) last_pos = __shfl_sync(0xffffffffu, lp, 31 - __clz(mp));
-    run = __shfl_sync(0xffffffffu, run + incl, 31);
+  for (int o = 1; o < 32; o <<= 1) {
+    const double y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
   }
-  return -1 - last_pos;
+  if (lane == 31) s_w[warp] = x;
+  __syncthreads();
+  double off = 0.0, tot = 0.0;
+#pragma unroll
+  for (int w = 0; w < kSmpWarps; ++w) {
+    const double sw = s_w[w];
+    if (w < warp) off += sw;
+    tot += sw;
+  }
+  __syncthreads();
+  *total = tot;
+  return x + off;
 }
 
-// Pass 2b: the draw.
+// Thread t's contiguous share [e0, e1) of [b0, b1), aligned to the vector width.
+template <int PV>
+__device__ __forceinline__ void thread_range(int b0, int b1, int* e0, int* e1) {
+  int E = (b1 - b0 + kSmpThreads - 1) / kSmpThreads;
+  E = (E + PV - 1) / PV * PV;
+  *e0 = min(b1, b0 + (int)threadIdx.x * E);
+  *e1 = min(b1, *e0 + E);
+}
+
+// Sum of the draw weights over [b0, b1) (every thread calls it).
+template <typename T, bool VEC>
+__device__ double block_total(const DrawRows& w, int b0, int b1, double invT, const double* tab, double* s_w) {
+  constexpr int PV = LogitIO<T>::kPerVec;
+  int e0, e1;
+  thread_range<PV>(b0, b1, &e0, &e1);
+  double loc = 0.0;
+  for (int e = e0; e < e1; e += PV) {
+    double wv[PV];
+    weights<T, VEC>(w, e, min(PV, e1 - e), invT, tab, wv);
+#pragma unroll
+    for (int t = 0; t < PV; ++t) loc += wv[t];
+  }
+  double tot;
+  block_scan_d(loc, &tot, s_w);
+  return tot;
+}
+
+// The first k in [b0, b1) whose running sum (from `base`) exceeds thr, found
+// by the whole CTA: every thread sums its share, a block scan gives each
+// share's starting sum, and the one thread whose share crosses thr walks it.
+// Without a crossing (rounding) the last index with positive weight is
+// returned (-1 if none). Every thread calls it and gets the same k.
+template <typename T, bool VEC>
+__device__ int block_find(const DrawRows& w, int b0, int b1, double base, double thr, double invT,
+                          const double* tab, double* s_w, int* s_i) {
+  constexpr int PV = LogitIO<T>::kPerVec;
+  int e0, e1;
+  thread_range<PV>(b0, b1, &e0, &e1);
+  if (threadIdx.x == 0) { s_i[0] = INT_MAX; s_i[1] = -1; s_i[2] = -1; }
+  double loc = 0.0;
+  int lastpos = -1;
+  for (int e = e0; e < e1; e += PV) {
+    double wv[PV];
+    weights<T, VEC>(w, e, min(PV, e1 - e), invT, tab, wv);
+#pragma unroll
+    for (int t = 0; t < PV; ++t) {
+      loc += wv[t];
+      if (wv[t] > 0.0) lastpos = e + t;
+    }
+  }
+  double tot;
+  const double incl = block_scan_d(loc, &tot, s_w);        // also orders the s_i initialisation
+  const double before = base + (incl - loc);
+  if (loc > 0.0 && before + loc > thr) atomicMin(&s_i[0], (int)threadIdx.x);
+  if (lastpos >= 0) atomicMax(&s_i[1], lastpos);
+  __syncthreads();
+  const int winner = s_i[0];
+  int k;
+  if (winner != INT_MAX) {
+    if ((int)threadIdx.x == winner) {
+      double run = before;
+      int kk = -1, lp = -1;
+      for (int e = e0; e < e1 && kk < 0; e += PV) {
+        double wv[PV];
+        weights<T, VEC>(w, e, min(PV, e1 - e), invT, tab, wv);
+#pragma unroll
+        for (int t = 0; t < PV; ++t) {
+          run += wv[t];
+          if (wv[t] > 0.0) lp = e + t;
+          if (kk < 0 && run > thr) kk = e + t;
+        }
+      }
+      s_i[2] = kk >= 0 ? kk : lp;
+    }
+    __syncthreads();
+    k = s_i[2];
+  } else {
+    k = s_i[1];
+  }
+  __syncthreads();
+  return k;
+}
+
+// Pass 2b: the draw. Spec draws shift by the row statistics of pass 1; plain
+// draws (the drafter's own) shift every chunk by its own maximum and bring
+// the chunk sums to the row maximum with an exact float64 factor when the
+// chunks are merged, so they need no statistics pass.
 template <typename T, bool SPEC, bool VEC>
 __global__ void __launch_bounds__(kSmpThreads) draw_kernel(const SampleParams p) {
   __shared__ double s_w[kSmpWarps];
+  __shared__ double s_tab[32];
+  __shared__ float s_redf[kSmpWarps];
+  __shared__ int s_i[3];
+  __shared__ double s_base;
   __shared__ int s_last;
   using IO = LogitIO<T>;
   constexpr int PV = IO::kPerVec;
   const int s = blockIdx.y, c = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  fill_exp_tab(s_tab);
   const int j = SPEC ? p.jsel[s] : 0;
-  const DrawRows w = draw_rows<T, SPEC>(p, s, j, true);
+  DrawRows w = draw_rows<T, SPEC>(p, s, j, true);
   const int cbeg = c * p.ch2, cend = min(p.vocab, cbeg + p.ch2);
   const int seg = p.ch2 / kWarpSegs;                     // elements per warp segment
   const int sbeg = min(cend, cbeg + warp * seg), send = min(cend, sbeg + seg);
+  float* cmax = p.cmax + (size_t)s * p.c2;
+  if constexpr (!SPEC) {
+    float mx = -INFINITY;
+    for (int e = sbeg + lane * PV; e < send; e += 32 * PV) {
+      float v[PV];
+      const int n = min(PV, send - e);
+      load_vals<T, VEC>(static_cast<const T*>(w.prow), e, n, v);
+#pragma unroll
+      for (int t = 0; t < PV; ++t)
+        if (t < n) mx = fmaxf(mx, v[t]);
+    }
+    const float M = block_max(mx, s_redf);               // synchronises (orders the table too)
+    w.Mp = M == -INFINITY ? 0.0 : static_cast<double>(M);
+    if (tid == 0) cmax[c] = M;
+  } else {
+    __syncthreads();
+  }
   double acc = 0.0;
   for (int e = sbeg + lane * PV; e < send; e += 32 * PV) {
     double wv[PV];
-    weights<T, VEC>(w, e, min(PV, send - e), p.inv_temp_d, wv);
+    weights<T, VEC>(w, e, min(PV, send - e), p.inv_temp_d, s_tab, wv);
 #pragma unroll
     for (int t = 0; t < PV; ++t) acc += wv[t];
   }
   acc = warp_sum_d(acc);
   if (lane == 0) {
     p.wpart[((size_t)s * p.c2 + c) * kWarpSegs + warp] = acc;
-    s_w[warp] = acc;
-  }
-  __syncthreads();
-  if (tid == 0) {
     __threadfence();
-    s_last = atomicAdd(p.tk_seq2 + s, 1u) == (unsigned)(p.c2 - 1);
   }
   __syncthreads();
-  if (!s_last || warp != 0) return;
+  if (tid == 0) s_last = atomicAdd(p.tk_seq2 + s, 1u) == (unsigned)(p.c2 - 1);
+  __syncthreads();
+  if (!s_last) return;
   __threadfence();
+  // ---- last CTA of the sequence (all threads): the draw
   const int R = p.gamma + 1;
   const double u = SPEC ? static_cast<double>(p.u_sample[(size_t)s * R + j]) : static_cast<double>(p.u_sample[s]);
   const double* wp = p.wpart + (size_t)s * p.c2 * kWarpSegs;
   const int nseg = p.c2 * kWarpSegs;
-  // total of all segments, then the first segment whose running sum passes thr
-  double tot = 0.0;
-  for (int i = lane; i < nseg; i += 32) tot += __ldcg(wp + i);
-  tot = warp_sum_d(tot);
+  double Mrow = 0.0;
+  if constexpr (!SPEC) {
+    float m = -INFINITY;
+    for (int i = tid; i < p.c2; i += kSmpThreads) m = fmaxf(m, __ldcg(cmax + i));
+    Mrow = static_cast<double>(block_max(m, s_redf));
+  }
+  // chunk c's factor to the row shift (plain draws), 1 for spec draws
+  auto chunk_scale = [&](int cc, float* mc_out) -> double {
+    if constexpr (SPEC) {
+      *mc_out = 0.f;
+      return 1.0;
+    } else {
+      const float mc = __ldcg(cmax + cc);
+      *mc_out = mc;
+      return mc == -INFINITY ? 0.0 : exp_tbl((static_cast<double>(mc) - Mrow) * p.inv_temp_d, s_tab);
+    }
+  };
+  auto segval = [&](int i) -> double {
+    const double v = __ldcg(wp + i);
+    if constexpr (SPEC) return v;
+    float mc;
+    return v == 0.0 ? 0.0 : v * chunk_scale(i / kWarpSegs, &mc);
+  };
+  double loc = 0.0;
+  for (int i = tid; i < nseg; i += kSmpThreads) loc += segval(i);
+  double total;
+  block_scan_d(loc, &total, s_w);
   int k = -1;
-  if (tot > 0.0) {
-    const double thr = u * tot;
-    double run = 0.0;
-    int sel = -1, lastpos = -1;
-    double sel_base = 0.0;
-    for (int i0 = 0; i0 < nseg && sel < 0; i0 += 32) {
-      const int i = i0 + lane;
-      const double v = i < nseg ? __ldcg(wp + i) : 0.0;
-      double incl = v;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const double y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
+  if (total > 0.0) {
+    const double thr = u * total;
+    // the first segment whose running sum passes thr (rounds of one segment per thread)
+    if (tid == 0) { s_i[0] = INT_MAX; s_i[1] = -1; }
+    double carry = 0.0;
+    for (int i0 = 0; i0 < nseg; i0 += kSmpThreads) {
+      const int i = i0 + tid;
+      const double v = i < nseg ? segval(i) : 0.0;
+      double rt;
+      const double incl = carry + block_scan_d(v, &rt, s_w);
+      if (v > 0.0) {
+        atomicMax(&s_i[1], i);
+        if (incl > thr) atomicMin(&s_i[0], i);
       }
-      const unsigned m = __ballot_sync(0xffffffffu, run + incl > thr && v > 0.0);
-      if (m) {
-        const int src = __ffs(m) - 1;
-        sel = i0 + src;
-        sel_base = __shfl_sync(0xffffffffu, run + incl - v, src);
-      }
-      const unsigned mp = __ballot_sync(0xffffffffu, v > 0.0);
-      if (mp) lastpos = i0 + 31 - __clz(mp);
-      run = __shfl_sync(0xffffffffu, run + incl, 31);
+      __syncthreads();
+      if (i == s_i[0]) s_base = incl - v;
+      __syncthreads();
+      if (s_i[0] != INT_MAX) break;
+      carry += rt;
     }
-    if (sel < 0) {                                       // rounding left no crossing: last segment with weight
-      sel = lastpos;
-      sel_base = 0.0;
-      for (int i = lane; i < sel; i += 32) sel_base += __ldcg(wp + i);
-      sel_base = warp_sum_d(sel_base);
+    int sel = s_i[0];
+    double base;
+    if (sel != INT_MAX) {
+      base = s_base;
+    } else {                                             // rounding left no crossing: last segment with weight
+      sel = s_i[1];
+      double l2 = 0.0;
+      for (int i = tid; i < sel; i += kSmpThreads) l2 += segval(i);
+      block_scan_d(l2, &base, s_w);
     }
+    __syncthreads();
     if (sel >= 0) {
       const int cc = sel / kWarpSegs, ww = sel - cc * kWarpSegs;
       const int b0 = min(p.vocab, cc * p.ch2 + ww * seg), b1 = min(min(p.vocab, cc * p.ch2 + p.ch2), b0 + seg);
-      k = warp_scan_find<T, VEC>(w, b0, b1, sel_base, thr, p.inv_temp_d);
-      if (k < 0) k = -1 - k;                            // last positive weight of the segment
+      DrawRows ws = w;
+      if constexpr (!SPEC) {
+        float mc;
+        ws.iZp = chunk_scale(cc, &mc);
+        ws.Mp = mc == -INFINITY ? 0.0 : static_cast<double>(mc);
+      }
+      k = block_find<T, VEC>(ws, b0, b1, base, thr, p.inv_temp_d, s_tab, s_w, s_i);
     }
   } else if (SPEC && w.qrow) {
     // all-zero residual (p_j == q_j after rounding): draw from p_j instead
     DrawRows wb = w;
     wb.qrow = nullptr;
     wb.iZp = 1.0;
-    double total = 0.0;
-    for (int e = lane * PV; e < p.vocab; e += 32 * PV) {
-      double wv[PV];
-      weights<T, VEC>(wb, e, min(PV, p.vocab - e), p.inv_temp_d, wv);
-#pragma unroll
-      for (int t = 0; t < PV; ++t) total += wv[t];
-    }
-    total = warp_sum_d(total);
-    k = warp_scan_find<T, VEC>(wb, 0, p.vocab, 0.0, u * total, p.inv_temp_d);
-    if (k < 0) k = -1 - k;
+    const double tot = block_total<T, VEC>(wb, 0, p.vocab, p.inv_temp_d, s_tab, s_w);
+    k = block_find<T, VEC>(wb, 0, p.vocab, 0.0, u * tot, p.inv_temp_d, s_tab, s_w, s_i);
   }
-  if (lane == 0) {
+  if (tid == 0) {
     if (k < 0) k = 0;
     if (SPEC) p.out_tokens[(size_t)s * R + j] = k;
     else p.out_tokens[s] = k;
@@ -504,11 +654,12 @@ cudaError_t launch_typed(const SampleParams& p, cudaStream_t st) {
                    (reinterpret_cast<uintptr_t>(p.target) % 16 == 0) &&
                    (!SPEC || reinterpret_cast<uintptr_t>(p.draft) % 16 == 0);
   dim3 g1(p.c1, nrows), g2(p.c2, p.nseq);
-  if (vec) rowstats_kernel<T, SPEC, true><<<g1, kSmpThreads, 0, st>>>(p);
-  else rowstats_kernel<T, SPEC, false><<<g1, kSmpThreads, 0, st>>>(p);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
   if (SPEC) {
+    if (vec) rowstats_kernel<T, SPEC, true><<<g1, kSmpThreads, 0, st>>>(p);
+    else rowstats_kernel<T, SPEC, false><<<g1, kSmpThreads, 0, st>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
     if (vec) znorm_kernel<T, true><<<g2, kSmpThreads, 0, st>>>(p);
     else znorm_kernel<T, false><<<g2, kSmpThreads, 0, st>>>(p);
     e = cudaGetLastError();
@@ -568,6 +719,8 @@ SamplePlan plan_sampling(int32_t nseq, int32_t gamma, int32_t vocab) {
   off = align_up(off + sizeof(double) * 2 * (size_t)nseq * pl.c2, 256);
   pl.off_wpart = off;
   off = align_up(off + sizeof(double) * kWarpSegs * (size_t)nseq * pl.c2, 256);
+  pl.off_cmax = off;
+  off = align_up(off + sizeof(float) * (size_t)nseq * pl.c2, 256);
   pl.ws_bytes = off;
   return pl;
 }
@@ -585,6 +738,7 @@ void bind_sample_workspace(SampleParams* p, const SamplePlan& pl, void* ws) {
   p->znorm = reinterpret_cast<double*>(w + pl.off_znorm);
   p->zpart = reinterpret_cast<double*>(w + pl.off_zpart);
   p->wpart = reinterpret_cast<double*>(w + pl.off_wpart);
+  p->cmax = reinterpret_cast<float*>(w + pl.off_cmax);
   p->c1 = pl.c1;
   p->ch1 = pl.ch1;
   p->c2 = pl.c2;

@@ -17,6 +17,8 @@
 //      and writes them in ascending page order with block-wide prefix sums.
 #include <cuda_bf16.h>
 
+#include <type_traits>
+
 #include "s3r_device.cuh"
 #include "s3r_internal.h"
 
@@ -31,8 +33,6 @@ __device__ __forceinline__ unsigned long long order_key(double x) {
   return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
 }
 
-__device__ __forceinline__ float load_elem(const __nv_bfloat16* p, size_t i) { return __bfloat162float(p[i]); }
-__device__ __forceinline__ float load_elem(const float* p, size_t i) { return p[i]; }
 
 // Exclusive prefix sum over the CTA (kSelThreads threads); also returns the total.
 __device__ int block_exclusive_scan(int v, int* total, int* s_warp) {
@@ -92,26 +92,48 @@ __device__ __forceinline__ void st_cluster_u64(uint32_t local_addr, uint32_t ran
   asm volatile("st.shared::cluster.u64 [%0], %1;" :: "r"(remote), "l"(v) : "memory");
 }
 
-// channels [lane*CPL, lane*CPL+CPL) of one summary row, as floats
-template <typename T, int CPL>
-__device__ __forceinline__ void load_row(const T* row, int lane, float* v) {
-  if constexpr (sizeof(T) == 2) {
-    if constexpr (CPL == 4) {
-      const uint2 u = __ldg(reinterpret_cast<const uint2*>(row) + lane);
-      v[0] = __uint_as_float(u.x << 16); v[1] = __uint_as_float(u.x & 0xFFFF0000u);
-      v[2] = __uint_as_float(u.y << 16); v[3] = __uint_as_float(u.y & 0xFFFF0000u);
-    } else {
-      const uint32_t u = __ldg(reinterpret_cast<const uint32_t*>(row) + lane);
-      v[0] = __uint_as_float(u << 16); v[1] = __uint_as_float(u & 0xFFFF0000u);
-    }
+// A lane's CPL channels of one summary row, as loaded (packed) and unpacked.
+template <typename T, int CPL> struct RawRow;
+template <> struct RawRow<__nv_bfloat16, 4> {
+  using type = uint2;
+  __device__ static void unpack(const uint2& u, float* v) {
+    v[0] = __uint_as_float(u.x << 16); v[1] = __uint_as_float(u.x & 0xFFFF0000u);
+    v[2] = __uint_as_float(u.y << 16); v[3] = __uint_as_float(u.y & 0xFFFF0000u);
+  }
+};
+template <> struct RawRow<__nv_bfloat16, 2> {
+  using type = uint32_t;
+  __device__ static void unpack(const uint32_t& u, float* v) {
+    v[0] = __uint_as_float(u << 16); v[1] = __uint_as_float(u & 0xFFFF0000u);
+  }
+};
+template <> struct RawRow<float, 4> {
+  using type = float4;
+  __device__ static void unpack(const float4& u, float* v) { v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w; }
+};
+template <> struct RawRow<float, 2> {
+  using type = float2;
+  __device__ static void unpack(const float2& u, float* v) { v[0] = u.x; v[1] = u.y; }
+};
+
+__device__ __forceinline__ float load_scalar(const __nv_bfloat16* p, int i) { return __bfloat162float(p[i]); }
+__device__ __forceinline__ float load_scalar(const float* p, int i) { return p[i]; }
+
+// CPL consecutive query values from shared memory as one vector load.
+template <typename Q, int CPL>
+__device__ __forceinline__ void load_qvec(const Q* src, Q* v) {
+  if constexpr (sizeof(Q) == 4 && CPL == 4) {
+    const float4 t = *reinterpret_cast<const float4*>(src);
+    v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+  } else if constexpr (sizeof(Q) == 4) {
+    const float2 t = *reinterpret_cast<const float2*>(src);
+    v[0] = t.x; v[1] = t.y;
+  } else if constexpr (CPL == 4) {
+    const double2 t0 = reinterpret_cast<const double2*>(src)[0], t1 = reinterpret_cast<const double2*>(src)[1];
+    v[0] = t0.x; v[1] = t0.y; v[2] = t1.x; v[3] = t1.y;
   } else {
-    if constexpr (CPL == 4) {
-      const float4 u = __ldg(reinterpret_cast<const float4*>(row) + lane);
-      v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
-    } else {
-      const float2 u = __ldg(reinterpret_cast<const float2*>(row) + lane);
-      v[0] = u.x; v[1] = u.y;
-    }
+    const double2 t = *reinterpret_cast<const double2*>(src);
+    v[0] = t.x; v[1] = t.y;
   }
 }
 
@@ -120,8 +142,7 @@ constexpr int kUnroll = 8;     // pages in flight per warp
 template <typename T, int CPL>
 __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelParams p) {
   extern __shared__ unsigned long long s_keys[];          // [n_b], filled in the first CTA
-  __shared__ float s_q[8 * 128];                          // [G, D] (bf16 path)
-  __shared__ double s_qd[8 * 128];                        // [G, D] (fp32 path)
+  __shared__ __align__(16) double s_qraw[8 * 128];    // [G, D] query rows (float or double)
   __shared__ unsigned int s_hist[256];
   __shared__ unsigned long long s_prefix;
   __shared__ int s_k, s_done, s_shift;
@@ -155,17 +176,19 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelParams p) 
   const int per = (n_b + ncta - 1) / ncta;
   const int beg = min(n_b, (int)rank * per), end = min(n_b, beg + per);
   const T* qp = static_cast<const T*>(p.q) + ((size_t)b * p.Hq + (size_t)h * p.G) * p.D;
-  for (int i = tid; i < p.G * p.D; i += kSelThreads) {
-    if constexpr (sizeof(T) == 2) s_q[i] = load_elem(qp, i);
-    else s_qd[i] = static_cast<double>(load_elem(qp, i));
-  }
-  __syncthreads();
   const T* kmn = static_cast<const T*>(p.kmin);
   const T* kmx = static_cast<const T*>(p.kmax);
+  // the G query rows in shared memory, as float (bf16) or double (fp32); a
+  // lane reads its CPL channels of a row as one vector (conflict-free)
+  using Q = typename std::conditional<sizeof(T) == 2, float, double>::type;
+  Q* s_q = reinterpret_cast<Q*>(s_qraw);
+  for (int i = tid; i < p.G * p.D; i += kSelThreads) s_q[i] = static_cast<Q>(load_scalar(qp, i));
+  __syncthreads();
   for (int pg0 = beg + warp * kUnroll; pg0 < end; pg0 += kSelWarps * kUnroll) {
     int phys_l = -1;
     if (lane < kUnroll && pg0 + lane < end) phys_l = p.block_table[(size_t)b * p.max_pages + pg0 + lane];
-    float lo[kUnroll][CPL], hi[kUnroll][CPL];
+    using Raw = typename RawRow<T, CPL>::type;
+    Raw lo[kUnroll], hi[kUnroll];
     bool ok[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
@@ -173,8 +196,8 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelParams p) 
       ok[u] = pg0 + u < end && phys >= 0 && phys < p.num_pages_total;
       if (ok[u]) {
         const size_t base = ((size_t)phys * p.Hkv + h) * p.D;
-        load_row<T, CPL>(kmn + base, lane, lo[u]);
-        load_row<T, CPL>(kmx + base, lane, hi[u]);
+        lo[u] = __ldg(reinterpret_cast<const Raw*>(kmn + base) + lane);
+        hi[u] = __ldg(reinterpret_cast<const Raw*>(kmx + base) + lane);
       }
     }
 #pragma unroll
@@ -182,16 +205,18 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelParams p) 
       if (pg0 + u >= end) continue;                     // warp-uniform
       double acc = 0.0;
       if (ok[u]) {
+        float l[CPL], r[CPL];
+        RawRow<T, CPL>::unpack(lo[u], l);
+        RawRow<T, CPL>::unpack(hi[u], r);
         for (int g = 0; g < p.G; ++g) {
+          Q qv[CPL];
+          load_qvec<Q, CPL>(s_q + g * p.D + lane * CPL, qv);
 #pragma unroll
           for (int c = 0; c < CPL; ++c) {
-            const int d = lane * CPL + c;
             if constexpr (sizeof(T) == 2) {
-              const float qv = s_q[g * p.D + d];
-              acc += static_cast<double>(fmaxf(qv * lo[u][c], qv * hi[u][c]));   // exact products
+              acc += static_cast<double>(fmaxf(qv[c] * l[c], qv[c] * r[c]));   // exact products
             } else {
-              const double qv = s_qd[g * p.D + d];
-              acc += fmax(qv * static_cast<double>(lo[u][c]), qv * static_cast<double>(hi[u][c]));
+              acc += fmax(qv[c] * static_cast<double>(l[c]), qv[c] * static_cast<double>(r[c]));
             }
           }
         }
@@ -333,11 +358,14 @@ cudaError_t launch_select(const s3r_paged_kv& kv, const void* kmin, const void* 
   p.budget = budget;
   p.status = status;
   const size_t smem = (size_t)kv.max_pages_per_seq * sizeof(unsigned long long);
-  // cluster size: about 64 pages per CTA (one 8-page load round per warp),
-  // at most 4 CTAs (larger clusters cannot all be co-scheduled)
-  int cl = (kv.max_pages_per_seq + 63) / 64;
-  if (cl < 1) cl = 1;
-  if (cl > 4) cl = 4;
+  // cluster size: the largest of 4, 2, 1 CTAs per (sequence, KV head) such
+  // that every CTA of the launch is resident at once (two per SM), and no
+  // more CTAs than 64-page load rounds (larger clusters cannot all be
+  // co-scheduled, and a second wave doubles the time)
+  const long units = (long)kv.num_seqs * kv.num_kv_heads;
+  const long slots = 2L * device_sm_count();
+  int cl = 4;
+  while (cl > 1 && (units * cl > slots || (cl - 1) * 64 >= kv.max_pages_per_seq)) cl >>= 1;
   const bool bf = kv.dtype == S3R_BF16;
   cudaError_t e;
   if (kv.head_dim == 128) e = bf ? launch_typed<__nv_bfloat16, 4>(p, cl, smem, st) : launch_typed<float, 4>(p, cl, smem, st);
