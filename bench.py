@@ -164,6 +164,13 @@ def verify_traffic():
         return None
 
 
+def launches_per_step(ws):
+    """Library kernels per step: the drafter's draws (1), gamma x (tail
+    summaries, select, attention), verify (1), sampling (statistics,
+    normalisers, draw)."""
+    return 1 + 3 * ws.gamma + 1 + 3
+
+
 def config_of(ws, world, seed):
     return {"workload": ws.name, "sequences_per_gpu": ws.num_seqs, "context": ws.context,
             "q_heads": ws.num_q_heads, "kv_heads": ws.num_kv_heads, "head_dim": ws.head_dim,
@@ -320,7 +327,7 @@ def run_ours(a):
                    "verify": round(verify_gbs, 1), "verify_frac_of_8tbs": round(verify_gbs / 8000, 4)},
         "acceptance": {"mean_accepted_per_seq": round(n_acc_total / (ws.num_seqs * a.steps), 4),
                        "committed_per_seq": round(tokens / (ws.num_seqs * a.steps), 4)},
-        "gpu_launches": (3 * ws.gamma + 5) * a.steps,
+        "gpu_launches": launches_per_step(ws) * a.steps,
         "clocks": clk,
     }
     if e2e:

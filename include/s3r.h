@@ -21,6 +21,12 @@
  *   otherwise. The library allocates and frees nothing and keeps no state
  *   between calls; scratch space comes from the caller's workspace (the one
  *   exception, s3r_spec_sample_noalloc, uses a static array of its own).
+ * - A workspace must be zero-filled before its first use. Calls leave it
+ *   ready for the next call (its counters return to zero as each call ends),
+ *   so no call clears it and consecutive kernels of the library overlap
+ *   their launch with the previous kernel's tail (programmatic dependent
+ *   launch). After a call that reported S3R_DEV_WAIT_TIMEOUT, zero the
+ *   workspace again before reusing it.
  * - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *   stream). Work is enqueued asynchronously on it; outputs are ready when the
  *   stream reaches that point.
@@ -226,11 +232,12 @@ size_t s3r_attn_workspace_bytes(const s3r_paged_kv* kv, int32_t rows, int32_t bu
 size_t s3r_sample_workspace_bytes(int32_t num_seqs, int32_t gamma, int32_t vocab);
 
 /*
- * Synchronises `stream`, then reads the status word that the most recent
- * call using `workspace` left there: S3R_OK, or S3R_ERR_DEVICE_CHECK with the
- * S3R_DEV_* bits in *bits (bits may be NULL). Every call clears the word when
- * it starts. s3r_page_summaries has no workspace; its device checks use the
- * status word at `status_word` if given via s3r_page_summaries_checked.
+ * Synchronises `stream`, then reads the status word of `workspace`: S3R_OK,
+ * or S3R_ERR_DEVICE_CHECK with the S3R_DEV_* bits in *bits (bits may be
+ * NULL). The bits accumulate over the calls made with the workspace since the
+ * word was last read; reading it clears it. s3r_page_summaries has no
+ * workspace; its device checks use the status word at `status_word` if given
+ * via s3r_page_summaries_checked.
  */
 s3r_status s3r_device_status(const void* workspace, uint32_t* bits, void* stream);
 

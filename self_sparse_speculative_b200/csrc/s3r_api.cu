@@ -137,8 +137,6 @@ S3R_EXPORT s3r_status s3r_sparse_draft_attn(const s3r_paged_kv* kv, const void* 
   const AttnPlan pl = plan_attention(*kv, 1, budget_pages);
   if (!workspace || workspace_bytes < pl.ws_bytes) return S3R_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  s = from_cuda(cudaMemsetAsync(workspace, 0, pl.off_ml, st));
-  if (s != S3R_OK) return s;
   uint32_t* status = static_cast<uint32_t*>(workspace);
   s = from_cuda(launch_select(*kv, kmin, kmax, q, budget_pages, selected, status, st));
   if (s != S3R_OK) return s;
@@ -157,8 +155,6 @@ S3R_EXPORT s3r_status s3r_verify_attn(const s3r_paged_kv* kv, const void* q, int
   const AttnPlan pl = plan_attention(*kv, rows, 0);
   if (!workspace || workspace_bytes < pl.ws_bytes) return S3R_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  s = from_cuda(cudaMemsetAsync(workspace, 0, pl.off_ml, st));
-  if (s != S3R_OK) return s;
   AttnParams p = make_attn_params(kv, pl, q, out, lse, rows, 0, nullptr, scale, workspace);
   s3r_status api;
   cudaError_t e = launch_attention(*kv, p, st, &api);
@@ -195,8 +191,6 @@ S3R_EXPORT s3r_status s3r_spec_sample(const void* target_logits, const void* dra
   const SamplePlan pl = plan_sampling(num_seqs, gamma, vocab);
   if (!workspace || workspace_bytes < pl.ws_bytes) return S3R_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  s3r_status s = from_cuda(cudaMemsetAsync(workspace, 0, pl.memset_bytes, st));
-  if (s != S3R_OK) return s;
   SampleParams p = make_sample_params(pl, workspace, num_seqs, gamma, vocab, temperature);
   p.target = target_logits;
   p.draft = draft_logits;
@@ -218,8 +212,6 @@ S3R_EXPORT s3r_status s3r_sample_tokens(const void* logits, s3r_dtype logit_dtyp
   const SamplePlan pl = plan_sampling(num_rows, 0, vocab);
   if (!workspace || workspace_bytes < pl.ws_bytes) return S3R_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  s3r_status s = from_cuda(cudaMemsetAsync(workspace, 0, pl.memset_bytes, st));
-  if (s != S3R_OK) return s;
   SampleParams p = make_sample_params(pl, workspace, num_rows, 0, vocab, temperature);
   p.target = logits;
   p.u_sample = u;
@@ -233,6 +225,8 @@ S3R_EXPORT s3r_status s3r_device_status(const void* workspace, uint32_t* bits, v
   if (cudaStreamSynchronize(st) != cudaSuccess) return S3R_ERR_CUDA;
   uint32_t w = 0;
   if (cudaMemcpy(&w, workspace, sizeof(w), cudaMemcpyDeviceToHost) != cudaSuccess) return S3R_ERR_CUDA;
+  // the word is sticky until read: clear it for the calls that follow
+  if (w != 0 && cudaMemset(const_cast<void*>(workspace), 0, sizeof(w)) != cudaSuccess) return S3R_ERR_CUDA;
   if (bits) *bits = w;
   return w == 0 ? S3R_OK : S3R_ERR_DEVICE_CHECK;
 }

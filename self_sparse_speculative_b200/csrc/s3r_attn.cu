@@ -80,6 +80,8 @@ constexpr int kF32Tok = 16;
 
 template <int D>
 __global__ void __launch_bounds__(kF32Threads) attn_f32_kernel(const AttnParams p) {
+  pdl_launch_dependents();
+  pdl_wait();
   extern __shared__ __align__(16) float f32_smem[];
   __shared__ int s_ticket;
   const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -266,8 +268,7 @@ cudaError_t launch_f32(const AttnParams& p, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(attn_f32_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(p.nsplit, p.Hkv, p.S);
-  attn_f32_kernel<D><<<grid, kF32Threads, smem, st>>>(p);
-  return cudaGetLastError();
+  return launch_kernel(attn_f32_kernel<D>, grid, dim3(kF32Threads), smem, st, 1, p);
 }
 
 }  // namespace

@@ -81,6 +81,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
   __shared__ float s_ml[2][2][128];                      // [segment parity][m, l][row] of stream 1
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  pdl_launch_dependents();
 
   // ---- per-sequence prefix of unit pages (warp 0), range of this CTA
   if (warp == 0) {
@@ -102,6 +103,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     if (lane == 31) s_prefix[p.S] = incl;
   }
   __syncthreads();
+  pdl_wait();                                           // earlier kernels' results are visible from here
   if (blockIdx.x == 0) {
     // unusable lengths: flag them, give their rows zero output and lse -inf
     for (int b = 0; b < p.S; ++b) {
@@ -672,8 +674,7 @@ cudaError_t launch_tc(const s3r_paged_kv& kv, const AttnParams& p, cudaStream_t 
   if (e != cudaSuccess) return e;
   int grid = device_sm_count();
   if (grid > kMaxPersistentCtas) grid = kMaxPersistentCtas;
-  attn_tc_kernel<M, D><<<grid, kThreads, smem, st>>>(mk, mv, p);
-  return cudaGetLastError();
+  return launch_kernel(attn_tc_kernel<M, D>, dim3(grid), dim3(kThreads), smem, st, 1, mk, mv, p);
 }
 
 }  // namespace

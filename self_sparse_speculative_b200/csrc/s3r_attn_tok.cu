@@ -24,10 +24,10 @@
 // to finish (atomic ticket, no waiting).
 //
 // Warp roles (192 threads): warps 0-3 softmax and epilogue (thread = token);
-// warp 4 producer (page ids, L2 prefetch of K/V 4 stages ahead, TMA into an
-// NS-stage ring); warp 5 MMA issuer (QK two stages ahead of PV) and TMEM
-// owner. The softmax warps also stage each segment's Q (fetched into
-// registers one segment ahead).
+// warp 4 producer (page ids, TMA into an NS-stage ring; an L2 prefetch ahead
+// of the ring measured slower); warp 5 MMA issuer (QK two stages ahead of
+// PV) and TMEM owner. The softmax warps also stage each segment's Q (fetched
+// into registers one segment ahead).
 #include <cuda_bf16.h>
 
 #include <cmath>
@@ -47,6 +47,7 @@ constexpr int kTok = 128;                    // tokens per stage (MMA M of S^T)
 constexpr float kTau = 8.0f;                 // lazy reference slack, log2 units
 constexpr float kNuInit = 1e30f;             // -(reference) before the first score of a segment
 constexpr int kTokSmemBudget = 232448 - 8192;
+constexpr int kMaxPend = 8;                  // deferred split-unit combines per CTA
 
 template <int N, int D>
 struct TokLay {
@@ -129,6 +130,8 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   __shared__ int s_ticket;
+  __shared__ int4 s_pend[kMaxPend];             // units this CTA combines at its end: (b, h, slot0, nseg)
+  __shared__ int s_npend;
   __shared__ int s_prefix[kMaxSeqs + 1];
   __shared__ int s_stage_lp[NS][8];
   __shared__ int s_roff[64];                    // output row of packed row r relative to (b, h)
@@ -138,6 +141,7 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
   __shared__ __align__(16) float s_alpha[64];   // rescale factor / 1 / l per row
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  pdl_launch_dependents();
 
   // ---- per-sequence prefix of unit pages (warp 0), range of this CTA
   if (warp == 0) {
@@ -160,7 +164,12 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
   }
   if (tid < 64) s_roff[tid] = (tid / p.G) * p.Hq + (tid % p.G);
   __syncthreads();
+  // Earlier kernels' results (page lists) and their use of the outputs and
+  // workspace are ordered by griddepcontrol.wait, taken by each role right
+  // before it needs them: the producer before the page ids, the softmax
+  // warps after fetching their first Q.
   if (blockIdx.x == 0) {
+    pdl_wait();
     // unusable lengths: flag them, give their rows zero output and lse -inf
     for (int b = 0; b < p.S; ++b) {
       if (!bad_context(p, p.context_lens[b])) continue;
@@ -171,7 +180,10 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
   const int total = s_prefix[p.S];
   const int W = (total + gridDim.x - 1) / gridDim.x;
   const int lo = blockIdx.x * W, hi = min(total, lo + W);
-  if (lo >= hi) return;                                 // uniform over the CTA
+  if (lo >= hi) {                                       // uniform over the CTA
+    pdl_wait();
+    return;
+  }
   const int ppt = kTok / p.P;                           // pages per stage
 
   const uint32_t bar0 = smem_addr(&s_bar[0]);
@@ -196,6 +208,7 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
     mbar_init(BAR(B_QFULL), 128);
     mbar_init(BAR(B_TD), 1);
     s_abort = 0;
+    s_npend = 0;
     fence_barrier_init();
   }
   if (warp == kTokProducer && lane == 0) { prefetch_tensormap(&tmK); prefetch_tensormap(&tmV); }
@@ -206,6 +219,7 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
 
   if (warp == kTokProducer) {
     // ======================================================= producer warp
+    pdl_wait();
     const uint64_t pol = l2_policy_evict_first();
     // page-id windows of 32 flattened positions: lane k of a window holds
     // position wbase + k. w0 = in use, w1 = phys loads in flight, w2 = lp
@@ -224,7 +238,6 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
     page_of(p, s_prefix, wbase + 32 + lane, hi, W, &w1_lp, &w1_u);
     w1_ph = phys_load(w1_lp, w1_u);
     page_of(p, s_prefix, wbase + 64 + lane, hi, W, &w2_lp, &w2_u);
-    const int pfd = 4 * ppt;                           // L2 prefetch distance (4 stages, <= 32 positions)
     int g = 0;
     bool ok = true;
     for (int x = lo; x < hi && ok;) {
@@ -236,7 +249,7 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
           ok = false;
           break;
         }
-        int my_lp = -1, my_ph = -1, pf_z = -1;
+        int my_lp = -1, my_ph = -1;
         for (int pp = 0; pp < ppt; ++pp) {
           const int xp = x + j * ppt + pp;
           const bool in = (j * ppt + pp) < sg.npg;
@@ -255,19 +268,6 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             ph = -1;
           }
           if (lane == pp && in) { my_lp = lp; my_ph = ph; }
-          const int s2 = src + pfd;                    // < 64: inside windows w0, w1
-          const int lp2 = __shfl_sync(0xffffffffu, s2 < 32 ? w0_lp : w1_lp, s2 & 31);
-          const int ph2 = __shfl_sync(0xffffffffu, s2 < 32 ? w0_ph : w1_ph, s2 & 31);
-          const int u2 = __shfl_sync(0xffffffffu, s2 < 32 ? w0_u : w1_u, s2 & 31);
-          if (lane == pp && xp + pfd < hi && lp2 >= 0 && ph2 >= 0 && ph2 < p.num_pages_total)
-            pf_z = ph2 * p.Hkv + (u2 % p.Hkv);
-        }
-        if (pf_z >= 0) {
-#pragma unroll
-          for (int hh = 0; hh < L::kHalves; ++hh) {
-            tma_prefetch_3d(&tmK, hh * 64, 0, pf_z);
-            tma_prefetch_3d(&tmV, hh * 64, 0, pf_z);
-          }
         }
         if (lane < 8) s_stage_lp[st][lane] = (lane < ppt && my_ph >= 0) ? my_lp : -1;
         const unsigned real = __ballot_sync(0xffffffffu, my_ph >= 0);
@@ -378,7 +378,8 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
       mbar_arrive(BAR(B_QFULL));
     };
     Seg sg = locate(p, s_prefix, lo, hi, W);
-    q_fetch(sg);
+    q_fetch(sg);                                        // an input: no earlier kernel writes it
+    pdl_wait();
     q_store();
     int g = 0;
     bool ok = true;
@@ -539,14 +540,33 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         if (tid == 0) s_ticket = atomicAdd(p.tickets + sg.unit, 1u);
         asm volatile("bar.sync 1, 128;" ::: "memory");
         if (s_ticket == sg.nseg - 1) {
-          __threadfence();
-          combine_partials<__nv_bfloat16>(p, sg.b, sg.h, sg.first_cta + sg.unit, sg.nseg, 128);
-          if (tid == 0) p.tickets[sg.unit] = 0u;
+          // this CTA finished the unit last: merge its partials after the
+          // CTA's own streaming is done (immediately if the list is full)
+          if (s_npend < kMaxPend) {
+            if (tid == 0) s_pend[s_npend] = make_int4(sg.b, sg.h, sg.first_cta + sg.unit, sg.nseg);
+          } else {
+            __threadfence();
+            combine_partials<__nv_bfloat16>(p, sg.b, sg.h, sg.first_cta + sg.unit, sg.nseg, 128);
+          }
+          asm volatile("bar.sync 1, 128;" ::: "memory");
+          if (tid == 0) {
+            if (s_npend < kMaxPend) ++s_npend;
+            p.tickets[sg.unit] = 0u;
+          }
         }
       }
       asm volatile("bar.sync 1, 128;" ::: "memory");    // s_alpha / s_nu reads done
       x = sg.end;
       sg = nx;
+    }
+    // ---- deferred combines of the units this CTA finished last (skipped,
+    // together, after a failed wait)
+    if (wg_count(!ok) == 0) {
+      __threadfence();
+      for (int k = 0; k < s_npend; ++k) {
+        const int4 u = s_pend[k];
+        combine_partials<__nv_bfloat16>(p, u.x, u.y, u.z, u.w, 128);
+      }
     }
   }
 
@@ -574,8 +594,7 @@ cudaError_t launch_tok(const s3r_paged_kv& kv, const AttnParams& p, cudaStream_t
   if (e != cudaSuccess) return e;
   int grid = device_sm_count();
   if (grid > kMaxPersistentCtas) grid = kMaxPersistentCtas;
-  attn_tok_kernel<N, D><<<grid, kTokThreads, smem, st>>>(mk, mv, p);
-  return cudaGetLastError();
+  return launch_kernel(attn_tok_kernel<N, D>, dim3(grid), dim3(kTokThreads), smem, st, 1, mk, mv, p);
 }
 
 template <int D>

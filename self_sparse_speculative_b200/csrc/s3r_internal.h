@@ -62,6 +62,34 @@ cudaError_t launch_summaries(const s3r_paged_kv& kv, int tail_only, void* kmin, 
 cudaError_t launch_select(const s3r_paged_kv& kv, const void* kmin, const void* kmax,
                           const void* q, int32_t budget, int32_t* selected, uint32_t* status,
                           cudaStream_t st);
+// Launch with programmatic dependent launch allowed (the kernel orders
+// itself after its predecessor with griddepcontrol.wait) and, when
+// cluster_x > 1, thread-block clusters of cluster_x CTAs along x.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                 int cluster_x, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 cudaError_t launch_attention(const s3r_paged_kv& kv, const AttnParams& p, cudaStream_t st,
                              s3r_status* api_status);
 cudaError_t launch_attention_tc(const s3r_paged_kv& kv, const AttnParams& p, cudaStream_t st,

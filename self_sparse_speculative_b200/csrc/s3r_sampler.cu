@@ -7,18 +7,22 @@
 // at the first rejection j draw from norm(max(p_j - q_j, 0)); if all gamma
 // drafts pass, draw a bonus token from p_gamma.
 //
-// Pass 1 (grid: vocab chunks x rows): every CTA holds its chunk of one logits
-// row in registers (one HBM read), reduces its max, then sums exp((x - max)/T)
-// with float32 exponentials into float64. The last CTA of a row (atomic
-// ticket) merges the chunk partials into the row's (max, Z); the last row of
-// a sequence takes the gamma accept/reject tests (one lane each) in float64.
+// Every kernel works on one vocab chunk per CTA, staged into shared memory
+// by a single bulk copy (cp.async.bulk, no multicast) when the rows are
+// 16-byte aligned, so a CTA waits for memory once and runs its passes
+// on-chip (otherwise it reads global memory directly).
+// Pass 1 (one CTA per row chunk): the chunk's max, then the sum of
+// exp((x - max)/T) with float32 exponentials into float64. The last CTA of a
+// row (atomic ticket) merges the chunk partials into the row's (max, Z); the
+// last row of a sequence takes the gamma accept/reject tests (one lane each)
+// in float64.
 // Pass 2a (residual sequences only): the exact float64 normalisers of the
 // two rows the residual is drawn from.
-// Pass 2b (grid: vocab chunks x sequences): float64 draw weights, summed per
-// warp segment; the last CTA of a sequence finds, with CTA-wide float64
-// scans, the segment holding u * total and then the token inside it. Every
-// draw is decided in float64 on both sides, so it is exact up to the order
-// of the float64 sums. float64 exponentials are table-driven (exp_tbl).
+// Pass 2b (one CTA per sequence chunk): float64 draw weights, summed per warp
+// segment; the last CTA of a sequence finds, with CTA-wide float64 scans,
+// the segment holding u * total and then the token inside it. Every draw is
+// decided in float64 on both sides, so it is exact up to the order of the
+// float64 sums. float64 exponentials are table-driven (exp_tbl).
 // The drafter's own draws (s3r_sample_tokens) are pass 2b alone in "plain"
 // mode: one row per draw, weights exp((x - m_c)/T) with m_c the chunk's own
 // maximum, brought to the row maximum when the chunks are merged.
@@ -37,6 +41,7 @@ constexpr int kSmpThreads = 256;
 constexpr int kSmpWarps = kSmpThreads / 32;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kWarpSegs = kSmpWarps;         // pass-2 chunk = 8 contiguous warp segments
+constexpr uint32_t kCopyPiece = 16384;       // bytes per bulk-copy instruction
 
 struct Part1 {
   float m;
@@ -47,7 +52,6 @@ struct Part1 {
 template <typename T> struct LogitIO;
 template <> struct LogitIO<__nv_bfloat16> {
   static constexpr int kPerVec = 8;
-  static constexpr int kVecs = 8;           // 16-byte vectors per thread in pass 1
   __device__ static float at(const __nv_bfloat16* p, size_t i) { return __bfloat162float(p[i]); }
   __device__ static void unpack(const uint4& v, float* x) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -60,7 +64,6 @@ template <> struct LogitIO<__nv_bfloat16> {
 };
 template <> struct LogitIO<float> {
   static constexpr int kPerVec = 4;
-  static constexpr int kVecs = 16;
   __device__ static float at(const float* p, size_t i) { return p[i]; }
   __device__ static void unpack(const uint4& v, float* x) {
     x[0] = __uint_as_float(v.x); x[1] = __uint_as_float(v.y);
@@ -68,11 +71,17 @@ template <> struct LogitIO<float> {
   }
 };
 
-__device__ __forceinline__ uint4 ldg_stream16(const void* p) {
-  uint4 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
-  return r;
+// n (<= kPerVec) consecutive values at ptr as float: one 16-byte load when
+// VEC (ptr 16-byte aligned, in shared or global memory), else scalar loads.
+template <typename T, bool VEC>
+__device__ __forceinline__ void load_vals(const T* ptr, int n, float* v) {
+  using IO = LogitIO<T>;
+  if constexpr (VEC) {
+    IO::unpack(*reinterpret_cast<const uint4*>(ptr), v);
+  } else {
+#pragma unroll
+    for (int t = 0; t < IO::kPerVec; ++t) v[t] = t < n ? IO::at(ptr, t) : 0.f;
+  }
 }
 
 __device__ __forceinline__ double warp_sum_d(double v) {
@@ -95,6 +104,16 @@ __device__ float block_max(float v, float* s_red) {
   __syncthreads();
   return r;
 }
+__device__ double block_sum_d(double v, double* s_red) {
+  v = warp_sum_d(v);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) s_red[warp] = v;
+  __syncthreads();
+  double r = 0.0;
+  for (int w = 0; w < kSmpWarps; ++w) r += s_red[w];
+  __syncthreads();
+  return r;
+}
 
 // float64 exponential, table-driven (P. T. P. Tang, "Table-driven
 // implementation of the exponential function in IEEE floating-point
@@ -105,14 +124,14 @@ __device__ float block_max(float v, float* s_red) {
 // double and its remainder (two fused multiply-adds); e^r - 1 is its Taylor
 // polynomial to degree 6 (remainder < 4e-18 for |r| <= ln2/64); 2^(j/32) is
 // a 32-entry table `tab`; 2^m goes into the exponent field. The result is
-// within about 2 ulp. Outside (-707, 708) (subnormal results, overflow,
-// infinities, NaN) the CUDA library exp is used.
+// within about 2 ulp for -707 < x < 708 (no branch: callers keep x in that
+// range and fix up the rest with exp_fixup).
 __device__ __forceinline__ double exp_tbl(double x, const double* tab) {
-  if (!(x > -707.0 && x < 708.0)) return exp(x);
   constexpr double kInvStep = 46.16624130844683;           // 32 / ln2
   constexpr double kStepHi = 0x1.62e42fefa39efp-6;          // ln2 / 32, leading double
   constexpr double kStepLo = 0x1.abc9e3b39803fp-61;         // ln2 / 32 - kStepHi
   constexpr double kShifter = 6755399441055744.0;           // 1.5 * 2^52
+  x = fmin(fmax(x, -707.0), 708.0);
   const double t = fma(x, kInvStep, kShifter);
   const int n = __double2loint(t);
   const double nd = t - kShifter;
@@ -127,10 +146,49 @@ __device__ __forceinline__ double exp_tbl(double x, const double* tab) {
   const double y = fma(tj, q * r, tj);
   return __hiloint2double(__double2hiint(y) + ((n >> 5) << 20), __double2loint(y));
 }
+// exp(x) given y = exp_tbl(x): outside (-707, 708) the argument is moved
+// into range by 512 ln2 and the result scaled back by an exact power of two
+// (subnormal results round once there), 0 below -746, NaN stays NaN. No
+// library call, so the hot loops carry no call ABI.
+__device__ __forceinline__ double exp_fixup(double x, double y, const double* tab) {
+  if (x > -707.0 && x < 708.0) return y;
+  constexpr double k512ln2 = 354.891356446692;          // 512 ln2 (rounded; shifts an argument only)
+  if (x != x) return x;
+  if (x <= -746.0) return 0.0;
+  if (x < 0.0) return exp_tbl(x + k512ln2, tab) * 0x1p-512;
+  if (x >= 710.0) return INFINITY;
+  return exp_tbl(x - k512ln2, tab) * 0x1p512;
+}
 
 // 2^(j/32), j = 0..31, into shared memory (threads 0..31; caller syncs).
 __device__ __forceinline__ void fill_exp_tab(double* tab) {
   if (threadIdx.x < 32) tab[threadIdx.x] = exp2(static_cast<double>(threadIdx.x) * 0.03125);
+}
+
+// Staging: the CTA's chunk [beg, beg + n) of one or two rows into shared
+// memory with bulk copies (thread 0 issues them; every thread waits on the
+// mbarrier, which thread 0 initialised before a CTA barrier).
+template <typename T>
+__device__ void stage_rows(T* s0, const T* g0, T* s1, const T* g1, int n, uint64_t* bar, volatile int* abort,
+                           uint32_t* status) {
+  const uint32_t bytes = static_cast<uint32_t>(n) * sizeof(T);
+  const uint32_t b = smem_addr(bar);
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(b, g1 ? 2u * bytes : bytes);
+    for (uint32_t off = 0; off < bytes; off += kCopyPiece) {
+      const uint32_t sz = min(kCopyPiece, bytes - off);
+      bulk_load(smem_addr(s0) + off, reinterpret_cast<const char*>(g0) + off, sz, b);
+      if (g1) bulk_load(smem_addr(s1) + off, reinterpret_cast<const char*>(g1) + off, sz, b);
+    }
+  }
+  mbar_wait(b, 0, abort, status);
+}
+__device__ __forceinline__ void init_stage_bar(uint64_t* bar) {
+  if (threadIdx.x == 0) {
+    mbar_init(smem_addr(bar), 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
 }
 
 // Row pointers of the spec layout: rows 0..R-1 target, R..2*gamma draft.
@@ -180,50 +238,58 @@ __device__ void decide(const SampleParams& p, int b) {
 }
 
 // ---------------------------------------------------------------- pass 1
-template <typename T, bool SPEC, bool VEC>
+template <typename T, bool STAGE>
 __global__ void __launch_bounds__(kSmpThreads) rowstats_kernel(const SampleParams p) {
+  pdl_launch_dependents();
+  pdl_wait();
+  extern __shared__ __align__(16) uint8_t s_dyn[];
+  __shared__ uint64_t s_bar;
+  __shared__ int s_abort;
   __shared__ float s_redf[kSmpWarps];
   __shared__ double s_redd[kSmpWarps];
   __shared__ int s_last;
   using IO = LogitIO<T>;
-  constexpr int E = IO::kPerVec * IO::kVecs;     // elements per thread
-  const int row = blockIdx.y, c = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const T* src = row_ptr<T>(p, SPEC, row);
-  const int beg = c * p.ch1;
-  const int end = min(p.vocab, beg + p.ch1);
-  float x[E];
-  if constexpr (VEC) {
+  constexpr int PV = IO::kPerVec;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int row = blockIdx.x / p.c1, c = blockIdx.x - (blockIdx.x / p.c1) * p.c1;
+  const int beg = c * p.ch1, n = min(p.vocab, beg + p.ch1) - beg;
+  const T* src = row_ptr<T>(p, true, row) + beg;
+  if constexpr (STAGE) {
+    if (tid == 0) s_abort = 0;
+    init_stage_bar(&s_bar);
+    T* s_chunk = reinterpret_cast<T*>(s_dyn);
+    stage_rows<T>(s_chunk, src, nullptr, nullptr, n, &s_bar, &s_abort, p.status);
+    src = s_chunk;
+  }
+  float mx = -INFINITY;
+  for (int i = tid * PV; i < n; i += kSmpThreads * PV) {
+    float v[PV];
+    const int m = min(PV, n - i);
+    load_vals<T, STAGE>(src + i, m, v);
 #pragma unroll
-    for (int k = 0; k < IO::kVecs; ++k) {
-      const int e0 = beg + (tid + k * kSmpThreads) * IO::kPerVec;
-      if (e0 < end) {
-        IO::unpack(ldg_stream16(src + e0), x + k * IO::kPerVec);
-      } else {
+    for (int t = 0; t < PV; ++t)
+      if (t < m) mx = fmaxf(mx, v[t]);
+  }
+  const float M = block_max(mx, s_redf);
+  double s = 0.0;
+  if (M != -INFINITY) {
+    const float k2 = kLog2e * p.inv_temp;
+    for (int i = tid * PV; i < n; i += kSmpThreads * PV) {
+      float v[PV];
+      const int m = min(PV, n - i);
+      load_vals<T, STAGE>(src + i, m, v);
+      // a vector's exponentials summed pairwise in float32, then added in float64
 #pragma unroll
-        for (int t = 0; t < IO::kPerVec; ++t) x[k * IO::kPerVec + t] = -INFINITY;
-      }
-    }
-  } else {
+      for (int t = 0; t < PV; ++t) v[t] = t < m ? ex2((v[t] - M) * k2) : 0.f;
 #pragma unroll
-    for (int k = 0; k < E; ++k) {
-      const int e = beg + tid + k * kSmpThreads;
-      x[k] = e < end ? IO::at(src, e) : -INFINITY;
+      for (int w = PV / 2; w > 0; w >>= 1)
+#pragma unroll
+        for (int t = 0; t < w; ++t) v[t] += v[t + w];
+      s += static_cast<double>(v[0]);
     }
   }
-  float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-  for (int k = 0; k < E; ++k) mx[k & 3] = fmaxf(mx[k & 3], x[k]);
-  const float M = block_max(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), s_redf);
-  const float k2 = kLog2e * p.inv_temp;
-  double s4[4] = {0.0, 0.0, 0.0, 0.0};
-#pragma unroll
-  for (int k = 0; k < E; ++k) s4[k & 3] += static_cast<double>(ex2((x[k] - M) * k2));
-  double s = warp_sum_d((s4[0] + s4[1]) + (s4[2] + s4[3]));
-  if (lane == 0) s_redd[warp] = s;
-  __syncthreads();
+  const double S = block_sum_d(s, s_redd);
   if (tid == 0) {
-    double S = 0.0;
-    for (int w = 0; w < kSmpWarps; ++w) S += s_redd[w];
     Part1* part = static_cast<Part1*>(p.part1) + (size_t)row * p.c1 + c;
     part->m = M;
     part->s = S;
@@ -250,20 +316,18 @@ __global__ void __launch_bounds__(kSmpThreads) rowstats_kernel(const SampleParam
     p.stats[2 * (size_t)row + 1] = Z;
     p.tk_row[row] = 0u;
   }
-  if constexpr (SPEC) {
-    const int per = 2 * p.gamma + 1;
-    const int b = row / per;
-    int last = 0;
-    if (lane == 0) {
-      __threadfence();
-      last = atomicAdd(p.tk_seq1 + b, 1u) == (unsigned)(per - 1);
-    }
-    last = __shfl_sync(0xffffffffu, last, 0);
-    if (last) {
-      __threadfence();
-      if (lane == 0) p.tk_seq1[b] = 0u;
-      decide<T>(p, b);
-    }
+  const int per = 2 * p.gamma + 1;
+  const int b = row / per;
+  int last = 0;
+  if (lane == 0) {
+    __threadfence();
+    last = atomicAdd(p.tk_seq1 + b, 1u) == (unsigned)(per - 1);
+  }
+  last = __shfl_sync(0xffffffffu, last, 0);
+  if (last) {
+    __threadfence();
+    if (lane == 0) p.tk_seq1[b] = 0u;
+    decide<T>(p, b);
   }
 }
 
@@ -277,7 +341,7 @@ struct DrawRows {
 };
 
 template <typename T, bool SPEC>
-__device__ DrawRows draw_rows(const SampleParams& p, int s, int j, bool exact_z) {
+__device__ DrawRows draw_rows(const SampleParams& p, int s, int j) {
   DrawRows w;
   w.iZp = 1.0;
   w.iZq = 1.0;
@@ -294,73 +358,110 @@ __device__ DrawRows draw_rows(const SampleParams& p, int s, int j, bool exact_z)
   if (j < p.gamma) {
     w.qrow = static_cast<const T*>(p.draft) + ((size_t)s * p.gamma + j) * p.vocab;
     w.Mq = p.stats[2 * ((size_t)s * per + R + j)];
-    if (exact_z) {
-      w.iZp = 1.0 / __ldcg(p.znorm + 2 * (size_t)s);
-      w.iZq = 1.0 / __ldcg(p.znorm + 2 * (size_t)s + 1);
-    }
+    w.iZp = 1.0 / __ldcg(p.znorm + 2 * (size_t)s);
+    w.iZq = 1.0 / __ldcg(p.znorm + 2 * (size_t)s + 1);
   }
   return w;
 }
 
-// float64 draw weights of n consecutive elements starting at e
+// float64 draw weights of the n (<= kPerVec) elements at pa (and pb for a
+// residual): exp((a - Mp)/T) iZp, or max(that - exp((b - Mq)/T) iZq, 0).
 template <typename T, bool VEC>
-__device__ __forceinline__ void load_vals(const T* row, int e, int n, float* v) {
+__device__ __forceinline__ void weights(const DrawRows& w, const T* pa, const T* pb, int n, double invT,
+                                        const double* tab, double* out) {
   using IO = LogitIO<T>;
-  if constexpr (VEC) {
-    IO::unpack(ldg_stream16(row + e), v);
-  } else {
-    for (int t = 0; t < IO::kPerVec; ++t) v[t] = t < n ? IO::at(row, e + t) : 0.f;
-  }
-}
-
-template <typename T, bool VEC>
-__device__ __forceinline__ void weights(const DrawRows& w, int e, int n, double invT, const double* tab,
-                                        double* out) {
-  using IO = LogitIO<T>;
-  float a[IO::kPerVec], b[IO::kPerVec];
-  load_vals<T, VEC>(static_cast<const T*>(w.prow), e, n, a);
-  if (w.qrow) load_vals<T, VEC>(static_cast<const T*>(w.qrow), e, n, b);
+  constexpr int PV = IO::kPerVec;
+  float a[PV], b[PV];
+  load_vals<T, VEC>(pa, n, a);
+  if (w.qrow) load_vals<T, VEC>(pb, n, b);
+  constexpr int G = 4;                                  // elements interleaved per group
 #pragma unroll
-  for (int t = 0; t < IO::kPerVec; ++t) {
-    double wt = 0.0;
-    if (t < n) {
-      const double pe = exp_tbl((static_cast<double>(a[t]) - w.Mp) * invT, tab) * w.iZp;
+  for (int t0 = 0; t0 < PV; t0 += G) {
+    double xa[G], xb[G], ea[G], eb[G];
+#pragma unroll
+    for (int t = 0; t < G; ++t) {                       // branch-free
+      xa[t] = (static_cast<double>(a[t0 + t]) - w.Mp) * invT;
+      ea[t] = exp_tbl(xa[t], tab);
       if (w.qrow) {
-        const double qe = exp_tbl((static_cast<double>(b[t]) - w.Mq) * invT, tab) * w.iZq;
-        wt = pe > qe ? pe - qe : 0.0;
-      } else {
-        wt = pe;
+        xb[t] = (static_cast<double>(b[t0 + t]) - w.Mq) * invT;
+        eb[t] = exp_tbl(xb[t], tab);
       }
     }
-    out[t] = wt;
+#pragma unroll
+    for (int t = 0; t < G; ++t) {
+      const double pe = exp_fixup(xa[t], ea[t], tab) * w.iZp;
+      double wt = pe;
+      if (w.qrow) {
+        const double qe = exp_fixup(xb[t], eb[t], tab) * w.iZq;
+        wt = pe > qe ? pe - qe : 0.0;
+      }
+      out[t0 + t] = t0 + t < n ? wt : 0.0;
+    }
   }
+}
+template <typename T, bool VEC>
+__device__ __forceinline__ void weights_at(const DrawRows& w, int e, int n, double invT, const double* tab,
+                                           double* out) {
+  weights<T, VEC>(w, static_cast<const T*>(w.prow) + e, w.qrow ? static_cast<const T*>(w.qrow) + e : nullptr, n,
+                  invT, tab, out);
 }
 
 // Pass 2a: exact float64 normalisers of the residual's two rows.
-template <typename T, bool VEC>
+template <typename T, bool STAGE>
 __global__ void __launch_bounds__(kSmpThreads) znorm_kernel(const SampleParams p) {
+  pdl_launch_dependents();
+  pdl_wait();
+  extern __shared__ __align__(16) uint8_t s_dyn[];
+  __shared__ uint64_t s_bar;
+  __shared__ int s_abort;
   __shared__ double s_red[2][kSmpWarps];
   __shared__ double s_tab[32];
   __shared__ int s_last;
   using IO = LogitIO<T>;
-  const int s = blockIdx.y, c = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int PV = IO::kPerVec;
+  const int s = blockIdx.x / p.c2, c = blockIdx.x - (blockIdx.x / p.c2) * p.c2;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int j = p.jsel[s];
   if (j >= p.gamma) return;                              // bonus draw: no residual (uniform per sequence)
+  const int per = 2 * p.gamma + 1, R = p.gamma + 1;
+  const double Mp = p.stats[2 * ((size_t)s * per + j)], Mq = p.stats[2 * ((size_t)s * per + R + j)];
+  const int beg = c * p.ch2, n = min(p.vocab, beg + p.ch2) - beg;
+  const T* pa = static_cast<const T*>(p.target) + ((size_t)s * R + j) * p.vocab + beg;
+  const T* pb = static_cast<const T*>(p.draft) + ((size_t)s * p.gamma + j) * p.vocab + beg;
   fill_exp_tab(s_tab);
-  __syncthreads();
-  DrawRows w = draw_rows<T, true>(p, s, j, false);
-  const int beg = c * p.ch2, end = min(p.vocab, beg + p.ch2);
+  if constexpr (STAGE) {
+    if (tid == 0) s_abort = 0;
+    init_stage_bar(&s_bar);
+    T* s0 = reinterpret_cast<T*>(s_dyn);
+    T* s1 = s0 + p.ch2;
+    stage_rows<T>(s0, pa, s1, pb, n, &s_bar, &s_abort, p.status);
+    pa = s0;
+    pb = s1;
+  } else {
+    __syncthreads();
+  }
   double zt = 0.0, zd = 0.0;
-  for (int e = beg + tid * IO::kPerVec; e < end; e += kSmpThreads * IO::kPerVec) {
-    const int n = min(IO::kPerVec, end - e);
-    float a[IO::kPerVec], b[IO::kPerVec];
-    load_vals<T, VEC>(static_cast<const T*>(w.prow), e, n, a);
-    load_vals<T, VEC>(static_cast<const T*>(w.qrow), e, n, b);
+  for (int i = tid * PV; i < n; i += kSmpThreads * PV) {
+    const int m = min(PV, n - i);
+    float a[PV], b[PV];
+    load_vals<T, STAGE>(pa + i, m, a);
+    load_vals<T, STAGE>(pb + i, m, b);
 #pragma unroll
-    for (int t = 0; t < IO::kPerVec; ++t) {
-      if (t < n) {
-        zt += exp_tbl((static_cast<double>(a[t]) - w.Mp) * p.inv_temp_d, s_tab);
-        zd += exp_tbl((static_cast<double>(b[t]) - w.Mq) * p.inv_temp_d, s_tab);
+    for (int t0 = 0; t0 < PV; t0 += 4) {
+      double xa[4], xb[4], ea[4], eb[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {                     // branch-free
+        xa[t] = (static_cast<double>(a[t0 + t]) - Mp) * p.inv_temp_d;
+        xb[t] = (static_cast<double>(b[t0 + t]) - Mq) * p.inv_temp_d;
+        ea[t] = exp_tbl(xa[t], s_tab);
+        eb[t] = exp_tbl(xb[t], s_tab);
+      }
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        if (t0 + t < m) {
+          zt += exp_fixup(xa[t], ea[t], s_tab);
+          zd += exp_fixup(xb[t], eb[t], s_tab);
+        }
       }
     }
   }
@@ -435,7 +536,7 @@ __device__ double block_total(const DrawRows& w, int b0, int b1, double invT, co
   double loc = 0.0;
   for (int e = e0; e < e1; e += PV) {
     double wv[PV];
-    weights<T, VEC>(w, e, min(PV, e1 - e), invT, tab, wv);
+    weights_at<T, VEC>(w, e, min(PV, e1 - e), invT, tab, wv);
 #pragma unroll
     for (int t = 0; t < PV; ++t) loc += wv[t];
   }
@@ -460,7 +561,7 @@ __device__ int block_find(const DrawRows& w, int b0, int b1, double base, double
   int lastpos = -1;
   for (int e = e0; e < e1; e += PV) {
     double wv[PV];
-    weights<T, VEC>(w, e, min(PV, e1 - e), invT, tab, wv);
+    weights_at<T, VEC>(w, e, min(PV, e1 - e), invT, tab, wv);
 #pragma unroll
     for (int t = 0; t < PV; ++t) {
       loc += wv[t];
@@ -481,7 +582,7 @@ __device__ int block_find(const DrawRows& w, int b0, int b1, double base, double
       int kk = -1, lp = -1;
       for (int e = e0; e < e1 && kk < 0; e += PV) {
         double wv[PV];
-        weights<T, VEC>(w, e, min(PV, e1 - e), invT, tab, wv);
+        weights_at<T, VEC>(w, e, min(PV, e1 - e), invT, tab, wv);
 #pragma unroll
         for (int t = 0; t < PV; ++t) {
           run += wv[t];
@@ -504,8 +605,13 @@ __device__ int block_find(const DrawRows& w, int b0, int b1, double base, double
 // draws (the drafter's own) shift every chunk by its own maximum and bring
 // the chunk sums to the row maximum with an exact float64 factor when the
 // chunks are merged, so they need no statistics pass.
-template <typename T, bool SPEC, bool VEC>
+template <typename T, bool SPEC, bool STAGE>
 __global__ void __launch_bounds__(kSmpThreads) draw_kernel(const SampleParams p) {
+  pdl_launch_dependents();
+  pdl_wait();
+  extern __shared__ __align__(16) uint8_t s_dyn[];
+  __shared__ uint64_t s_bar;
+  __shared__ int s_abort;
   __shared__ double s_w[kSmpWarps];
   __shared__ double s_tab[32];
   __shared__ float s_redf[kSmpWarps];
@@ -514,34 +620,46 @@ __global__ void __launch_bounds__(kSmpThreads) draw_kernel(const SampleParams p)
   __shared__ int s_last;
   using IO = LogitIO<T>;
   constexpr int PV = IO::kPerVec;
-  const int s = blockIdx.y, c = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int s = blockIdx.x / p.c2, c = blockIdx.x - (blockIdx.x / p.c2) * p.c2;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   fill_exp_tab(s_tab);
   const int j = SPEC ? p.jsel[s] : 0;
-  DrawRows w = draw_rows<T, SPEC>(p, s, j, true);
-  const int cbeg = c * p.ch2, cend = min(p.vocab, cbeg + p.ch2);
+  DrawRows w = draw_rows<T, SPEC>(p, s, j);
+  const int cbeg = c * p.ch2, n = min(p.vocab, cbeg + p.ch2) - cbeg;
+  const T* ca = static_cast<const T*>(w.prow) + cbeg;   // this chunk of the rows
+  const T* cb = w.qrow ? static_cast<const T*>(w.qrow) + cbeg : nullptr;
+  if constexpr (STAGE) {
+    if (tid == 0) s_abort = 0;
+    init_stage_bar(&s_bar);                              // also orders the exp table
+    T* s0 = reinterpret_cast<T*>(s_dyn);
+    T* s1 = w.qrow ? s0 + p.ch2 : nullptr;
+    stage_rows<T>(s0, ca, s1, cb, n, &s_bar, &s_abort, p.status);
+    ca = s0;
+    cb = s1;
+  }
   const int seg = p.ch2 / kWarpSegs;                     // elements per warp segment
-  const int sbeg = min(cend, cbeg + warp * seg), send = min(cend, sbeg + seg);
+  const int sb0 = min(n, warp * seg), sb1 = min(n, sb0 + seg);
   float* cmax = p.cmax + (size_t)s * p.c2;
   if constexpr (!SPEC) {
     float mx = -INFINITY;
-    for (int e = sbeg + lane * PV; e < send; e += 32 * PV) {
+    for (int i = sb0 + lane * PV; i < sb1; i += 32 * PV) {
       float v[PV];
-      const int n = min(PV, send - e);
-      load_vals<T, VEC>(static_cast<const T*>(w.prow), e, n, v);
+      const int m = min(PV, sb1 - i);
+      load_vals<T, STAGE>(ca + i, m, v);
 #pragma unroll
       for (int t = 0; t < PV; ++t)
-        if (t < n) mx = fmaxf(mx, v[t]);
+        if (t < m) mx = fmaxf(mx, v[t]);
     }
-    const float M = block_max(mx, s_redf);               // synchronises (orders the table too)
+    const float M = block_max(mx, s_redf);               // synchronises (orders the exp table too)
     w.Mp = M == -INFINITY ? 0.0 : static_cast<double>(M);
     if (tid == 0) cmax[c] = M;
   } else {
     __syncthreads();
   }
   double acc = 0.0;
-  for (int e = sbeg + lane * PV; e < send; e += 32 * PV) {
+  for (int i = sb0 + lane * PV; i < sb1; i += 32 * PV) {
     double wv[PV];
-    weights<T, VEC>(w, e, min(PV, send - e), p.inv_temp_d, s_tab, wv);
+    weights<T, STAGE>(w, ca + i, cb ? cb + i : nullptr, min(PV, sb1 - i), p.inv_temp_d, s_tab, wv);
 #pragma unroll
     for (int t = 0; t < PV; ++t) acc += wv[t];
   }
@@ -574,7 +692,9 @@ __global__ void __launch_bounds__(kSmpThreads) draw_kernel(const SampleParams p)
     } else {
       const float mc = __ldcg(cmax + cc);
       *mc_out = mc;
-      return mc == -INFINITY ? 0.0 : exp_tbl((static_cast<double>(mc) - Mrow) * p.inv_temp_d, s_tab);
+      if (mc == -INFINITY) return 0.0;
+      const double x = (static_cast<double>(mc) - Mrow) * p.inv_temp_d;
+      return exp_fixup(x, exp_tbl(x, s_tab), s_tab);
     }
   };
   auto segval = [&](int i) -> double {
@@ -628,15 +748,15 @@ __global__ void __launch_bounds__(kSmpThreads) draw_kernel(const SampleParams p)
         ws.iZp = chunk_scale(cc, &mc);
         ws.Mp = mc == -INFINITY ? 0.0 : static_cast<double>(mc);
       }
-      k = block_find<T, VEC>(ws, b0, b1, base, thr, p.inv_temp_d, s_tab, s_w, s_i);
+      k = block_find<T, STAGE>(ws, b0, b1, base, thr, p.inv_temp_d, s_tab, s_w, s_i);
     }
   } else if (SPEC && w.qrow) {
     // all-zero residual (p_j == q_j after rounding): draw from p_j instead
     DrawRows wb = w;
     wb.qrow = nullptr;
     wb.iZp = 1.0;
-    const double tot = block_total<T, VEC>(wb, 0, p.vocab, p.inv_temp_d, s_tab, s_w);
-    k = block_find<T, VEC>(wb, 0, p.vocab, 0.0, u * tot, p.inv_temp_d, s_tab, s_w, s_i);
+    const double tot = block_total<T, STAGE>(wb, 0, p.vocab, p.inv_temp_d, s_tab, s_w);
+    k = block_find<T, STAGE>(wb, 0, p.vocab, 0.0, u * tot, p.inv_temp_d, s_tab, s_w, s_i);
   }
   if (tid == 0) {
     if (k < 0) k = 0;
@@ -650,24 +770,36 @@ template <typename T, bool SPEC>
 cudaError_t launch_typed(const SampleParams& p, cudaStream_t st) {
   const int per = SPEC ? 2 * p.gamma + 1 : 1;
   const int nrows = p.nseq * per;
-  const bool vec = (((size_t)p.vocab * sizeof(T)) % 16 == 0) &&
-                   (reinterpret_cast<uintptr_t>(p.target) % 16 == 0) &&
-                   (!SPEC || reinterpret_cast<uintptr_t>(p.draft) % 16 == 0);
-  dim3 g1(p.c1, nrows), g2(p.c2, p.nseq);
+  // bulk staging needs 16-byte aligned rows
+  const bool stage = (((size_t)p.vocab * sizeof(T)) % 16 == 0) &&
+                     (reinterpret_cast<uintptr_t>(p.target) % 16 == 0) &&
+                     (!SPEC || reinterpret_cast<uintptr_t>(p.draft) % 16 == 0);
+  const dim3 blk(kSmpThreads);
+  const size_t sm1 = stage ? (size_t)p.ch1 * sizeof(T) : 0;
+  const size_t sm2 = stage ? (size_t)p.ch2 * sizeof(T) * (SPEC ? 2 : 1) : 0;
   cudaError_t e = cudaSuccess;
   if (SPEC) {
-    if (vec) rowstats_kernel<T, SPEC, true><<<g1, kSmpThreads, 0, st>>>(p);
-    else rowstats_kernel<T, SPEC, false><<<g1, kSmpThreads, 0, st>>>(p);
-    e = cudaGetLastError();
+    if (stage) {
+      e = cudaFuncSetAttribute(rowstats_kernel<T, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1);
+      if (e == cudaSuccess) e = launch_kernel(rowstats_kernel<T, true>, dim3(p.c1 * nrows), blk, sm1, st, 1, p);
+    } else {
+      e = launch_kernel(rowstats_kernel<T, false>, dim3(p.c1 * nrows), blk, 0, st, 1, p);
+    }
     if (e != cudaSuccess) return e;
-    if (vec) znorm_kernel<T, true><<<g2, kSmpThreads, 0, st>>>(p);
-    else znorm_kernel<T, false><<<g2, kSmpThreads, 0, st>>>(p);
-    e = cudaGetLastError();
+    if (stage) {
+      e = cudaFuncSetAttribute(znorm_kernel<T, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
+      if (e == cudaSuccess) e = launch_kernel(znorm_kernel<T, true>, dim3(p.c2 * p.nseq), blk, sm2, st, 1, p);
+    } else {
+      e = launch_kernel(znorm_kernel<T, false>, dim3(p.c2 * p.nseq), blk, 0, st, 1, p);
+    }
     if (e != cudaSuccess) return e;
   }
-  if (vec) draw_kernel<T, SPEC, true><<<g2, kSmpThreads, 0, st>>>(p);
-  else draw_kernel<T, SPEC, false><<<g2, kSmpThreads, 0, st>>>(p);
-  return cudaGetLastError();
+  if (stage) {
+    e = cudaFuncSetAttribute(draw_kernel<T, SPEC, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
+    if (e != cudaSuccess) return e;
+    return launch_kernel(draw_kernel<T, SPEC, true>, dim3(p.c2 * p.nseq), blk, sm2, st, 1, p);
+  }
+  return launch_kernel(draw_kernel<T, SPEC, false>, dim3(p.c2 * p.nseq), blk, 0, st, 1, p);
 }
 
 }  // namespace
@@ -676,7 +808,7 @@ SamplePlan plan_sampling(int32_t nseq, int32_t gamma, int32_t vocab) {
   SamplePlan pl{};
   pl.nseq = nseq;
   pl.nrows = nseq * (gamma > 0 ? 2 * gamma + 1 : 1);
-  // pass 1: at most 64 register-resident elements per thread (16384 per CTA),
+  // pass 1: at most 16384 staged elements per CTA (32 KB bf16, 64 KB fp32),
   // about 4 CTAs per SM overall, at least 256 elements per CTA
   const int max_per_cta = kSmpThreads * 64;
   const int target = 148 * 4;
@@ -689,11 +821,13 @@ SamplePlan plan_sampling(int32_t nseq, int32_t gamma, int32_t vocab) {
   pl.ch1 = (int)align_up((size_t)((vocab + c1 - 1) / c1), 8);
   if (pl.ch1 > max_per_cta) pl.ch1 = max_per_cta;
   pl.c1 = (vocab + pl.ch1 - 1) / pl.ch1;
-  // pass 2: about 4 CTAs per SM, at least 2048 elements per CTA; a chunk is
-  // 8 warp segments whose length is a multiple of 32 lanes x 8 elements
+  // pass 2: about 4 CTAs per SM, 2048 to 8192 elements per CTA (two staged
+  // fp32 rows fit in 64 KB of shared memory); a chunk is 8 warp segments
+  // whose length is a multiple of 32 lanes x 8 elements
   int c2 = (target + nseq - 1) / nseq;
   const int cap2 = (vocab + 2047) / 2048;
   if (c2 > cap2) c2 = cap2;
+  if (c2 < (vocab + 8191) / 8192) c2 = (vocab + 8191) / 8192;
   if (c2 < 1) c2 = 1;
   pl.ch2 = (int)align_up((size_t)((vocab + c2 - 1) / c2), (size_t)kWarpSegs * 32 * 8);
   pl.c2 = (vocab + pl.ch2 - 1) / pl.ch2;

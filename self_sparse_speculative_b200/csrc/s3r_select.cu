@@ -12,7 +12,8 @@
 //      memory);
 //   2. that CTA radix-selects the budget-th largest key (8-bit digits from the
 //      top: shared-memory histogram, one-warp scan of the 256 bins), stopping
-//      as soon as the boundary bin holds exactly the keys still needed;
+//      as soon as the boundary bin holds exactly the keys still needed (a
+//      rank count of every key against all others measured slower);
 //   3. it keeps the keys above the boundary plus the lowest-index pages on it,
 //      and writes them in ascending page order with block-wide prefix sums.
 #include <cuda_bf16.h>
@@ -148,6 +149,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelParams p) 
   __shared__ int s_k, s_done, s_shift;
   __shared__ int s_warp[kSelWarps];
 
+  pdl_launch_dependents();
   const int h = blockIdx.y, b = blockIdx.z;
   const uint32_t rank = cluster_rank();
   const int ncta = gridDim.x;
@@ -156,6 +158,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelParams p) 
   // every decision before the cluster barriers is uniform over the cluster
   const int L = p.context_lens[b];
   if (L < 1 || L > p.max_pages * p.P) {
+    pdl_wait();
     if (rank == 0) {
       if (tid == 0) flag_status(p.status, S3R_DEV_BAD_CONTEXT_LEN);
       for (int k = tid; k < p.budget; k += kSelThreads) out[k] = -1;
@@ -164,6 +167,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelParams p) 
   }
   const int n_b = (L + p.P - 1) / p.P;
   if (n_b <= p.budget) {
+    pdl_wait();
     if (rank == 0)
       for (int k = tid; k < p.budget; k += kSelThreads) out[k] = k < n_b ? k : -1;
     return;
@@ -184,6 +188,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelParams p) 
   Q* s_q = reinterpret_cast<Q*>(s_qraw);
   for (int i = tid; i < p.G * p.D; i += kSelThreads) s_q[i] = static_cast<Q>(load_scalar(qp, i));
   __syncthreads();
+  pdl_wait();                                           // the summaries are the previous kernel's
   for (int pg0 = beg + warp * kUnroll; pg0 < end; pg0 += kSelWarps * kUnroll) {
     int phys_l = -1;
     if (lane < kUnroll && pg0 + lane < end) phys_l = p.block_table[(size_t)b * p.max_pages + pg0 + lane];
@@ -320,19 +325,7 @@ template <typename T, int CPL>
 cudaError_t launch_typed(const SelParams& p, int cl, size_t smem, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(select_kernel<T, CPL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(cl, p.Hkv, p.S);
-  cfg.blockDim = dim3(kSelThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = cl;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, select_kernel<T, CPL>, p);
+  return launch_kernel(select_kernel<T, CPL>, dim3(cl, p.Hkv, p.S), dim3(kSelThreads), smem, st, cl, p);
 }
 
 }  // namespace

@@ -74,17 +74,23 @@ template <typename T>
 __global__ void __launch_bounds__(kSumThreads) summaries_kernel(const SumParams p) {
   __shared__ uint4 s_min[kSumThreads];
   __shared__ uint4 s_max[kSumThreads];
+  pdl_launch_dependents();
   const int h = blockIdx.x, b = blockIdx.z;
   const int L = p.context_lens[b];
   if (L < 1 || L > p.max_pages * p.P) {
+    pdl_wait();
     if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) flag_status(p.status, S3R_DEV_BAD_CONTEXT_LEN);
     return;
   }
   const int n_b = (L + p.P - 1) / p.P;
   const int i = p.tail_only ? n_b - 1 : (int)blockIdx.y;
-  if (i >= n_b) return;
+  if (i >= n_b) {
+    pdl_wait();
+    return;
+  }
   const int phys = p.block_table[(size_t)b * p.max_pages + i];
   if (phys < 0 || phys >= p.num_pages_total) {
+    pdl_wait();
     if (threadIdx.x == 0) flag_status(p.status, S3R_DEV_BAD_PAGE_ID);
     return;
   }
@@ -110,6 +116,7 @@ __global__ void __launch_bounds__(kSumThreads) summaries_kernel(const SumParams 
   s_min[threadIdx.x] = mn;
   s_max[threadIdx.x] = mx;
   __syncthreads();
+  pdl_wait();                                           // earlier kernels may still read the summaries
   if (threadIdx.x < chunks) {
     for (int gi = 1; gi < groups; ++gi) {
       vmin<T>(mn, s_min[gi * chunks + c]);
@@ -140,10 +147,9 @@ cudaError_t launch_summaries(const s3r_paged_kv& kv, int tail_only, void* kmin, 
   p.status = status;
   dim3 grid(kv.num_kv_heads, tail_only ? 1 : kv.max_pages_per_seq, kv.num_seqs);
   if (kv.dtype == S3R_BF16)
-    summaries_kernel<__nv_bfloat16><<<grid, kSumThreads, 0, st>>>(p);
+    return launch_kernel(summaries_kernel<__nv_bfloat16>, grid, dim3(kSumThreads), 0, st, 1, p);
   else
-    summaries_kernel<float><<<grid, kSumThreads, 0, st>>>(p);
-  return cudaGetLastError();
+    return launch_kernel(summaries_kernel<float>, grid, dim3(kSumThreads), 0, st, 1, p);
 }
 
 }  // namespace s3r

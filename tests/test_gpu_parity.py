@@ -200,3 +200,23 @@ def test_device_checks_flag_bad_inputs_without_faulting():
     st.block_table[2, 1] = int(wl.block_table[2, 1])
     st.verify()
     assert s3r.s3r_device_status(st.ws_verify) == (s3r.S3R_OK, 0)
+
+
+def test_status_word_is_sticky_until_read():
+    """A device-check bit survives later clean calls on the same workspace and
+    is cleared by reading it (no call clears the workspace itself)."""
+    ws = custom_spec(1, num_seqs=2, num_q_heads=8, num_kv_heads=2, budget_pages=2, vocab=512)
+    wl = Workload(ws, seed=3, context_lens=[300, 200])
+    st = DecodeStep(wl)
+    st.summaries()
+    torch.cuda.synchronize()
+    st.context_lens[1] = 0
+    st.verify()
+    st.context_lens[1] = 200
+    st.verify()
+    status, bits = s3r.s3r_device_status(st.ws_verify)
+    assert status == s3r.S3R_ERR_DEVICE_CHECK and bits & s3r.S3R_DEV_BAD_CONTEXT_LEN
+    assert s3r.s3r_device_status(st.ws_verify) == (s3r.S3R_OK, 0)
+    # the clean call's results are right
+    ref = RR.oracle_attention_seq(wl, 1, draft_steps=[])
+    RR.assert_close("seq 1 verify", st.verify_out[1].float().cpu().numpy(), ref["verify_out"], "bf16")
