@@ -129,7 +129,11 @@ s3r_status s3r_page_summaries(const s3r_paged_kv* kv, int32_t tail_only,
  * lse: float32 [S, Hq] natural-log log-sum-exp of the scaled scores, or NULL.
  * selected: int32 [S, Hkv, budget_pages], the kept logical page indices in
  *   ascending order, -1 after the first min(n_b, budget_pages) entries.
- * kmin, kmax: as written by s3r_page_summaries for the current cache.
+ * kmin, kmax: as written by s3r_page_summaries, for pages p < n_b - 1. The
+ *   tail page n_b - 1 is the only one whose keys change as a sequence
+ *   decodes; the call summarises it from k_cache itself (min / max over its
+ *   valid tokens), so no summary refresh is needed between draft steps and
+ *   kmin/kmax are only read.
  * workspace: at least s3r_attn_workspace_bytes(kv, 1, budget_pages) bytes.
  */
 s3r_status s3r_sparse_draft_attn(const s3r_paged_kv* kv, const void* kmin, const void* kmax,

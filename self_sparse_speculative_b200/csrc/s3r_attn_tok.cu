@@ -178,7 +178,12 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
     }
   }
   const int total = s_prefix[p.S];
-  const int W = (total + gridDim.x - 1) / gridDim.x;
+  // Sparse draft: when the (sequence, KV head) units nearly fill the grid
+  // (at least 4/5 of it), each CTA takes one whole unit of B pages instead of
+  // an equal share: no unit is split, so no partials, tickets or merges (the
+  // idle CTAs cost less than the split units on the 16 x 16K workload).
+  int W = (total + gridDim.x - 1) / gridDim.x;
+  if (p.page_list && W < p.budget && p.S * p.Hkv * 5 >= (int)gridDim.x * 4) W = p.budget;
   const int lo = blockIdx.x * W, hi = min(total, lo + W);
   if (lo >= hi) {                                       // uniform over the CTA
     pdl_wait();

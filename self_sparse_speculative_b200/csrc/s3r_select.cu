@@ -66,6 +66,7 @@ struct SelParams {
   const void* q;            // [S, Hq, D]
   const void* kmin;
   const void* kmax;         // [num_pages_total, Hkv, D]
+  const void* k_cache;      // [num_pages_total, Hkv, P, D] (the tail page's summary is taken from it)
   const int32_t* block_table;
   const int32_t* context_lens;
   int32_t* selected;        // [S, Hkv, budget]
@@ -117,6 +118,17 @@ template <> struct RawRow<float, 2> {
   __device__ static void unpack(const float2& u, float* v) { v[0] = u.x; v[1] = u.y; }
 };
 
+// A 16-byte vector of K as floats (8 bf16 or 4 fp32 values).
+template <typename T> __device__ __forceinline__ void unpack16(const uint4& u, float* v);
+template <> __device__ __forceinline__ void unpack16<__nv_bfloat16>(const uint4& u, float* v) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) { v[2 * k] = __uint_as_float(w[k] << 16); v[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u); }
+}
+template <> __device__ __forceinline__ void unpack16<float>(const uint4& u, float* v) {
+  v[0] = __uint_as_float(u.x); v[1] = __uint_as_float(u.y); v[2] = __uint_as_float(u.z); v[3] = __uint_as_float(u.w);
+}
+
 __device__ __forceinline__ float load_scalar(const __nv_bfloat16* p, int i) { return __bfloat162float(p[i]); }
 __device__ __forceinline__ float load_scalar(const float* p, int i) { return p[i]; }
 
@@ -144,9 +156,12 @@ template <typename T, int CPL>
 __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelParams p) {
   extern __shared__ unsigned long long s_keys[];          // [n_b], filled in the first CTA
   __shared__ __align__(16) double s_qraw[8 * 128];    // [G, D] query rows (float or double)
+  __shared__ __align__(16) float s_tail[2][128];       // min / max of the tail page (this CTA's, if any)
+  __shared__ float s_tpart[2][kSelWarps][128];          // per-warp partial min / max of the tail page
+  __shared__ unsigned long long s_kred[2][kSelWarps];   // key min / max per warp
   __shared__ unsigned int s_hist[256];
   __shared__ unsigned long long s_prefix;
-  __shared__ int s_k, s_done, s_shift;
+  __shared__ int s_k, s_done, s_shift, s_start;
   __shared__ int s_warp[kSelWarps];
 
   pdl_launch_dependents();
@@ -187,19 +202,71 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelParams p) 
   using Q = typename std::conditional<sizeof(T) == 2, float, double>::type;
   Q* s_q = reinterpret_cast<Q*>(s_qraw);
   for (int i = tid; i < p.G * p.D; i += kSelThreads) s_q[i] = static_cast<Q>(load_scalar(qp, i));
+  // The tail page n_b - 1 is the only one whose summary changes while a
+  // sequence decodes: the CTA that scores it takes its min / max over the
+  // valid tokens straight from K (an input, so before the dependency wait).
+  const int tail = n_b - 1;
+  const bool has_tail = beg <= tail && tail < end;
+  int tail_phys = -1;
+  if (has_tail) {
+    tail_phys = p.block_table[(size_t)b * p.max_pages + tail];
+    if (tail_phys >= 0 && tail_phys < p.num_pages_total) {
+      // thread = (token group, 16-byte chunk of channels); every load in
+      // flight at once, then the groups merge by shuffles and across warps
+      constexpr int VEC = 16 / sizeof(T);
+      const int chunks = p.D / VEC, groups = kSelThreads / chunks;
+      const int c = tid % chunks, grp = tid / chunks;
+      const int valid = L - tail * p.P;
+      const T* kt = static_cast<const T*>(p.k_cache) + ((size_t)tail_phys * p.Hkv + h) * p.P * p.D + c * VEC;
+      constexpr int kMaxPer = 8;                          // tokens per thread: P <= groups * 8
+      uint4 raw[kMaxPer];
+#pragma unroll
+      for (int k = 0; k < kMaxPer; ++k) {
+        const int t = grp + k * groups;
+        if (t < valid) raw[k] = __ldg(reinterpret_cast<const uint4*>(kt + (size_t)t * p.D));
+      }
+      float mn[VEC], mx[VEC];
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) { mn[e] = INFINITY; mx[e] = -INFINITY; }
+#pragma unroll
+      for (int k = 0; k < kMaxPer; ++k) {
+        if (grp + k * groups >= valid) continue;
+        float v[VEC];
+        unpack16<T>(raw[k], v);
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) { mn[e] = fminf(mn[e], v[e]); mx[e] = fmaxf(mx[e], v[e]); }
+      }
+      for (int o = chunks; o < 32; o <<= 1)
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+          mn[e] = fminf(mn[e], __shfl_xor_sync(0xffffffffu, mn[e], o));
+          mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xffffffffu, mx[e], o));
+        }
+      if (lane < chunks)
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) { s_tpart[0][warp][c * VEC + e] = mn[e]; s_tpart[1][warp][c * VEC + e] = mx[e]; }
+      __syncthreads();
+      if (tid < p.D) {
+        float a = INFINITY, z = -INFINITY;
+        for (int w = 0; w < kSelWarps; ++w) { a = fminf(a, s_tpart[0][w][tid]); z = fmaxf(z, s_tpart[1][w][tid]); }
+        s_tail[0][tid] = a;
+        s_tail[1][tid] = z;
+      }
+    }
+  }
   __syncthreads();
-  pdl_wait();                                           // the summaries are the previous kernel's
+  pdl_wait();                                           // earlier kernels may write the summaries
+  using Raw = typename RawRow<T, CPL>::type;
   for (int pg0 = beg + warp * kUnroll; pg0 < end; pg0 += kSelWarps * kUnroll) {
     int phys_l = -1;
     if (lane < kUnroll && pg0 + lane < end) phys_l = p.block_table[(size_t)b * p.max_pages + pg0 + lane];
-    using Raw = typename RawRow<T, CPL>::type;
     Raw lo[kUnroll], hi[kUnroll];
     bool ok[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       const int phys = __shfl_sync(0xffffffffu, phys_l, u);
       ok[u] = pg0 + u < end && phys >= 0 && phys < p.num_pages_total;
-      if (ok[u]) {
+      if (ok[u] && pg0 + u != tail) {
         const size_t base = ((size_t)phys * p.Hkv + h) * p.D;
         lo[u] = __ldg(reinterpret_cast<const Raw*>(kmn + base) + lane);
         hi[u] = __ldg(reinterpret_cast<const Raw*>(kmx + base) + lane);
@@ -211,8 +278,13 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelParams p) 
       double acc = 0.0;
       if (ok[u]) {
         float l[CPL], r[CPL];
-        RawRow<T, CPL>::unpack(lo[u], l);
-        RawRow<T, CPL>::unpack(hi[u], r);
+        if (pg0 + u == tail) {                          // this CTA's own summary of the tail page
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) { l[c] = s_tail[0][lane * CPL + c]; r[c] = s_tail[1][lane * CPL + c]; }
+        } else {
+          RawRow<T, CPL>::unpack(lo[u], l);
+          RawRow<T, CPL>::unpack(hi[u], r);
+        }
         for (int g = 0; g < p.G; ++g) {
           Q qv[CPL];
           load_qvec<Q, CPL>(s_q + g * p.D + lane * CPL, qv);
@@ -244,16 +316,45 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelParams p) 
   cluster_sync_all();                                     // all keys are in the first CTA
   if (rank != 0) return;
 
-  // ---- 2. radix select of the budget-th largest key
-  if (tid == 0) { s_prefix = 0ull; s_k = p.budget; s_done = 0; s_shift = 0; }
+  // ---- 2. radix select of the budget-th largest key, from the first byte
+  // in which the keys differ (all keys share the bits above it)
+  unsigned long long kmin_l = ~0ull, kmax_l = 0ull;
+  for (int pg = tid; pg < n_b; pg += kSelThreads) {
+    const unsigned long long key = s_keys[pg];
+    kmin_l = key < kmin_l ? key : kmin_l;
+    kmax_l = key > kmax_l ? key : kmax_l;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const unsigned long long a = __shfl_xor_sync(0xffffffffu, kmin_l, o), c = __shfl_xor_sync(0xffffffffu, kmax_l, o);
+    kmin_l = a < kmin_l ? a : kmin_l;
+    kmax_l = c > kmax_l ? c : kmax_l;
+  }
+  if (lane == 0) { s_kred[0][warp] = kmin_l; s_kred[1][warp] = kmax_l; }
   __syncthreads();
-  for (int shift = 56; shift >= 0; shift -= 8) {
+  if (tid == 0) {
+    unsigned long long mn = ~0ull, mx = 0ull;
+    for (int w = 0; w < kSelWarps; ++w) {
+      mn = s_kred[0][w] < mn ? s_kred[0][w] : mn;
+      mx = s_kred[1][w] > mx ? s_kred[1][w] : mx;
+    }
+    const unsigned long long diff = mn ^ mx;
+    const int top = diff ? 8 * ((63 - __clzll((long long)diff)) / 8) : 0;   // highest differing byte
+    s_start = top;
+    s_shift = 0;                                        // the stop shift, set when a pass ends it
+    s_prefix = top >= 56 ? 0ull : (mx >> (top + 8)) << (top + 8);
+    s_k = p.budget;
+    s_done = 0;
+  }
+  __syncthreads();
+  const int shift0 = s_start;
+  for (int shift = shift0; shift >= 0; shift -= 8) {
     s_hist[tid] = 0u;                                      // kSelThreads == 256 bins
     __syncthreads();
     const unsigned long long prefix = s_prefix;
     for (int pg = tid; pg < n_b; pg += kSelThreads) {
       const unsigned long long key = s_keys[pg];
-      const bool match = (shift == 56) || (((key ^ prefix) >> (shift + 8)) == 0ull);
+      const bool match = (shift >= 56) || (((key ^ prefix) >> (shift + 8)) == 0ull);
       if (match) atomicAdd(&s_hist[(key >> shift) & 255u], 1u);
     }
     __syncthreads();
@@ -337,6 +438,7 @@ cudaError_t launch_select(const s3r_paged_kv& kv, const void* kmin, const void* 
   p.q = q;
   p.kmin = kmin;
   p.kmax = kmax;
+  p.k_cache = kv.k_cache;
   p.block_table = kv.block_table;
   p.context_lens = kv.context_lens;
   p.selected = selected;

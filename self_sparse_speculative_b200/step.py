@@ -4,10 +4,11 @@ This module owns device buffers (allocated with torch: plumbing only) and
 issues the library calls of one round in order; it performs no arithmetic of
 its own. A round, as the S3R page (weekinpapers.com, Abstract) describes it:
 
-  draft   gamma times: refresh the summary of each sequence's tail page,
-          sparse-attend over the top-B pages per KV head
-          (s3r_page_summaries tail_only + s3r_sparse_draft_attn), and draw the
-          draft token from the draft distribution (s3r_sample_tokens);
+  draft   gamma times: score the pages (the tail page summarised from K
+          inside the call, the others from the page summaries), keep the
+          top-B per KV head and sparse-attend over them
+          (s3r_sparse_draft_attn), and draw the draft token from the draft
+          distribution (s3r_sample_tokens);
   verify  dense causal attention of the gamma+1 rows (s3r_verify_attn);
   commit  exact speculative sampling (s3r_spec_sample).
 
@@ -104,8 +105,9 @@ class DecodeStep:
                               ws.temperature, self.u_draft, self.draft_tokens, self.ws_tokens, stream=stream)
 
     def draft(self, i: int, stream=None):
+        """Draft step i: page scores and top-B (the tail page summarised from K
+        inside the call), then sparse attention."""
         ws = self.wl.spec
-        s3r.s3r_page_summaries(self.kv, 1, self.kmin, self.kmax, stream)
         s3r.s3r_sparse_draft_attn(self.kv, self.kmin, self.kmax, self.q_draft[i], ws.budget_pages, self.scale,
                                   self.selected[i], self.draft_out[i], self.draft_lse[i], self.ws_draft,
                                   stream=stream)
@@ -136,23 +138,32 @@ class DecodeStep:
     # ---------------------------------------------------------------- bytes
     def algorithmic_bytes(self):
         """Bytes each step must move (what the method has to read/write)."""
-        wl, ws = self.wl, self.wl.spec
-        Hkv, D, P, B = ws.num_kv_heads, ws.head_dim, ws.page_size, ws.budget_pages
-        elt = 2 if ws.kv_dtype == "bf16" else 4
-        lelt = 2 if ws.logit_dtype == "bf16" else 4
-        lens = wl.context_lens.astype(np.int64)
-        n_b = wl.pages_per_seq
-        kv_tok = 2 * Hkv * D * elt                                  # K + V per token
-        # sparse draft: page summaries of every page (kmin+kmax) + selected KV
-        sel_tokens = 0
-        for L, n in zip(lens, n_b):
-            k = min(int(n), B)
-            # the selected pages are full except possibly the tail page
-            sel_tokens += min(int(L), k * P)
-        draft = int(n_b.sum()) * Hkv * 2 * D * elt + sel_tokens * kv_tok
-        verify = int(lens.sum()) * kv_tok
-        V, g = ws.vocab, ws.gamma
-        sample = ws.num_seqs * ((2 * g + 1) * V * lelt + 2 * V * lelt)
-        draw = ws.num_seqs * g * V * lelt * 2
-        return {"draft_per_call": draft, "verify": verify, "sample": sample, "draft_tokens": draw,
-                "step": g * draft + verify + sample + draw}
+        return algorithmic_bytes(self.wl)
+
+
+def algorithmic_bytes(wl: Workload):
+    """Bytes one step of workload `wl` must move (what the method has to
+    read/write): per draft call the summaries of every page plus the K/V
+    of the selected pages, verify the K/V of every token, sampling the
+    (2 gamma + 1) rows plus the 2 re-read rows, the drafter's draws
+    gamma rows per sequence."""
+    ws = wl.spec
+    Hkv, D, P, B = ws.num_kv_heads, ws.head_dim, ws.page_size, ws.budget_pages
+    elt = 2 if ws.kv_dtype == "bf16" else 4
+    lelt = 2 if ws.logit_dtype == "bf16" else 4
+    lens = wl.context_lens.astype(np.int64)
+    n_b = wl.pages_per_seq
+    kv_tok = 2 * Hkv * D * elt                                  # K + V per token
+    # sparse draft: page summaries of every page (kmin+kmax) + selected KV
+    sel_tokens = 0
+    for L, n in zip(lens, n_b):
+        k = min(int(n), B)
+        # the selected pages are full except possibly the tail page
+        sel_tokens += min(int(L), k * P)
+    draft = int(n_b.sum()) * Hkv * 2 * D * elt + sel_tokens * kv_tok
+    verify = int(lens.sum()) * kv_tok
+    V, g = ws.vocab, ws.gamma
+    sample = ws.num_seqs * ((2 * g + 1) * V * lelt + 2 * V * lelt)
+    draw = ws.num_seqs * g * V * lelt
+    return {"draft_per_call": draft, "verify": verify, "sample": sample, "draft_tokens": draw,
+            "step": g * draft + verify + sample + draw}

@@ -220,3 +220,29 @@ def test_status_word_is_sticky_until_read():
     # the clean call's results are right
     ref = RR.oracle_attention_seq(wl, 1, draft_steps=[])
     RR.assert_close("seq 1 verify", st.verify_out[1].float().cpu().numpy(), ref["verify_out"], "bf16")
+
+
+def test_draft_summarises_the_tail_page_itself():
+    """The sparse draft call takes the tail page's summary from K, not from
+    kmin/kmax: with the stored tail summaries wiped, the selection and the
+    draft outputs still match the oracle (whose summaries come from K)."""
+    s, lens = CASES["bf16-d128-p64"]
+    wl = Workload(s, seed=1, context_lens=lens)
+    st = DecodeStep(wl)
+    st.summaries(tail_only=False)
+    torch.cuda.synchronize()
+    tails = [int(wl.block_table[b, int(wl.pages_per_seq[b]) - 1]) for b in range(wl.spec.num_seqs)]
+    st.kmin[tails] = -100.0                     # stale values that would make every tail page win
+    st.kmax[tails] = 100.0
+    for i in range(wl.spec.gamma):
+        st.draft(i)
+    torch.cuda.synchronize()
+    sel = st.selected.cpu().numpy()
+    tally = RR.Tally()
+    for b in range(wl.spec.num_seqs):
+        ref = RR.oracle_attention_seq(wl, b)
+        for i, d in ref["draft"].items():
+            ok = RR.compare_selection(f"seq {b} draft {i}", sel[i, b], d["selected"], d["gaps"], tally)
+            if all(ok):
+                RR.assert_close(f"seq {b} draft {i} out", st.draft_out[i, b].float().cpu().numpy(), d["out"], "bf16")
+    assert tally.near_ties <= max(0, int(1e-4 * tally.decisions)), tally.notes
