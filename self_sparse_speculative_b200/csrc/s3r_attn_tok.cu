@@ -57,8 +57,12 @@ struct TokLay {
   static constexpr uint32_t kTileBytes = kTok * D * 2;     // K or V of one stage: [d half][128 tokens][128 B]
   static constexpr int kNSraw = (kTokSmemBudget - (int)kQBytes - (int)kPBytes) / (2 * (int)kTileBytes);
   static constexpr int kNS = kNSraw > 6 ? 6 : kNSraw;
+  // two P buffers (softmax(g) then waits only for PV(g - 2)) when they fit
+  // without losing a stage
+  static constexpr int kPBufs =
+      (kTokSmemBudget - (int)kQBytes - 2 * (int)kPBytes) / (2 * (int)kTileBytes) >= kNS ? 2 : 1;
   static constexpr uint32_t kOffP = kQBytes;
-  static constexpr uint32_t kOffKV = kOffP + kPBytes;
+  static constexpr uint32_t kOffKV = kOffP + kPBufs * kPBytes;
   static constexpr uint32_t kDynBytes = kOffKV + kNS * 2 * kTileBytes;
   static constexpr uint32_t kColS = 0, kColO = 2 * N;      // S^T[2], O^T
   static constexpr int kQChunks = N * D / 8 / 128;         // 16-byte Q chunks per softmax thread
@@ -126,7 +130,7 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
   constexpr int NS = L::kNS;
   extern __shared__ __align__(1024) uint8_t dyn_raw[];
   uint8_t* dyn = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ __align__(8) uint64_t s_bar[2 * NS + 6];
+  __shared__ __align__(8) uint64_t s_bar[2 * NS + 8];
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   __shared__ int s_ticket;
@@ -193,8 +197,14 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
 
   const uint32_t bar0 = smem_addr(&s_bar[0]);
   auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
-  const int B_FULL = 0, B_EMPTY = NS, B_SFULL = 2 * NS, B_PFULL = 2 * NS + 2, B_ODONE = 2 * NS + 3,
-            B_QFULL = 2 * NS + 4, B_TD = 2 * NS + 5;
+  // PFULL[k] / ODONE[k]: completed by softmax(g) / PV(g) for g % 2 == k.
+  // softmax(g + 1) need not wait for PV(g) (two P buffers), so one PFULL
+  // barrier could complete two phases before the MMA thread tests the first;
+  // with one barrier per parity, P(g + 2) waits for PV(g) and no barrier gets
+  // two phases ahead of its waiter.
+  const int B_FULL = 0, B_EMPTY = NS, B_SFULL = 2 * NS, B_PFULL = 2 * NS + 2, B_ODONE = 2 * NS + 4,
+            B_QFULL = 2 * NS + 6, B_TD = 2 * NS + 7;
+  constexpr int PB = L::kPBufs;
   uint8_t* sQ = dyn;
   uint8_t* sP = dyn + L::kOffP;
   uint8_t* sKV = dyn + L::kOffKV;
@@ -209,7 +219,9 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
     mbar_init(BAR(B_SFULL), 1);
     mbar_init(BAR(B_SFULL + 1), 1);
     mbar_init(BAR(B_PFULL), 128);
+    mbar_init(BAR(B_PFULL + 1), 128);
     mbar_init(BAR(B_ODONE), 1);
+    mbar_init(BAR(B_ODONE + 1), 1);
     mbar_init(BAR(B_QFULL), 128);
     mbar_init(BAR(B_TD), 1);
     s_abort = 0;
@@ -250,10 +262,7 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
       const int nst = (sg.npg + ppt - 1) / ppt;
       for (int j = 0; j < nst; ++j, ++g) {
         const int st = g % NS;
-        if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_EMPTY + st), ((g / NS) & 1) ^ 1, &s_abort, p.status))) {
-          ok = false;
-          break;
-        }
+        // the stage's page ids first (they do not need the slot), then the slot
         int my_lp = -1, my_ph = -1;
         for (int pp = 0; pp < ppt; ++pp) {
           const int xp = x + j * ppt + pp;
@@ -273,6 +282,10 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             ph = -1;
           }
           if (lane == pp && in) { my_lp = lp; my_ph = ph; }
+        }
+        if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_EMPTY + st), ((g / NS) & 1) ^ 1, &s_abort, p.status))) {
+          ok = false;
+          break;
         }
         if (lane < 8) s_stage_lp[st][lane] = (lane < ppt && my_ph >= 0) ? my_lp : -1;
         const unsigned real = __ballot_sync(0xffffffffu, my_ph >= 0);
@@ -315,11 +328,14 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
       const uint64_t dP0 = smem_desc_sw128(aP, 16, 1024);
       constexpr uint64_t kQHalf = (N * 128) >> 4, kPHalf = (N * 128) >> 4;
       constexpr uint64_t kStage = (2 * L::kTileBytes) >> 4, kKHalf = (kTok * 128) >> 4, kVStep = (16 * 128) >> 4;
-      auto issue_qk = [&]() -> bool {
-        if (qc.j == 0 && !mbar_wait(BAR(B_QFULL), qc.s & 1, &s_abort, p.status)) return false;
-        const int st = qc.g % NS;
-        if (!mbar_wait(BAR(B_FULL + st), (qc.g / NS) & 1, &s_abort, p.status)) return false;
+      // QK(k) needs its stage's data (first in a segment, also the segment's
+      // Q) and PV(k - 2) issued (softmax(k - 2) has read S buffer k & 1);
+      // PV(k) needs P(k). Each is issued as soon as it is ready, so a PV never
+      // waits for a later stage's data. Bounded: no progress for the wait
+      // limit flags a timeout and stops.
+      auto issue_qk = [&]() {
         tc_fence_after();
+        const int st = qc.g % NS;
         const uint64_t kd = dK0 + (uint64_t)st * kStage;
         const uint32_t dS = tmem + L::kColS + (qc.g & 1) * N;
 #pragma unroll
@@ -329,25 +345,53 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         }
         umma_commit(BAR(B_SFULL + (qc.g & 1)));
         cursor_next(p, s_prefix, hi, W, ppt, qc);
-        return true;
       };
-      for (int k = 0; k < 2 && qc.valid && ok; ++k) ok = issue_qk();
-      while (ok && pc.valid) {
-        if (!mbar_wait(BAR(B_PFULL), pc.g & 1, &s_abort, p.status)) { ok = false; break; }
+      auto issue_pv = [&]() {
         tc_fence_after();
         const int st = pc.g % NS;
         const uint64_t vd = dV0 + (uint64_t)st * kStage;
         const uint32_t tO = tmem + L::kColO;
         const uint32_t acc0 = pc.j > 0 ? 1u : 0u;
+        const uint64_t pd = dP0 + (uint64_t)(pc.g % PB) * (L::kPBytes >> 4);
 #pragma unroll
         for (int kk = 0; kk < kTok / 16; ++kk)
-          umma_f16(tO, vd + (uint64_t)kk * kVStep, dP0 + (kk >> 2) * kPHalf + (uint64_t)(kk & 3) * 2, idPV,
+          umma_f16(tO, vd + (uint64_t)kk * kVStep, pd + (kk >> 2) * kPHalf + (uint64_t)(kk & 3) * 2, idPV,
                    kk > 0 ? 1u : acc0);
         umma_commit(BAR(B_EMPTY + st));
-        umma_commit(BAR(B_ODONE));
+        umma_commit(BAR(B_ODONE + (pc.g & 1)));
         cursor_next(p, s_prefix, hi, W, ppt, pc);
-        if (qc.valid && !issue_qk()) { ok = false; break; }
+      };
+      unsigned long long idle_since = 0;
+      uint32_t spins = 0;
+      while (pc.valid) {
+        bool progress = false;
+        if (mbar_test_wait(BAR(B_PFULL + (pc.g & 1)), (pc.g >> 1) & 1)) {
+          issue_pv();
+          progress = true;
+        }
+        if (qc.valid && qc.g <= pc.g + 1 && (qc.j != 0 || mbar_test_wait(BAR(B_QFULL), qc.s & 1)) &&
+            mbar_test_wait(BAR(B_FULL + qc.g % NS), (qc.g / NS) & 1)) {
+          issue_qk();
+          progress = true;
+        }
+        if (progress) {
+          idle_since = 0;
+          continue;
+        }
+        if ((++spins & 63u) == 0) {
+          if (s_abort) { ok = false; break; }
+          const unsigned long long now = globaltimer_ns();
+          if (idle_since == 0) {
+            idle_since = now;
+          } else if (now - idle_since > kWaitLimitNs) {
+            s_abort = 1;
+            flag_status(p.status, S3R_DEV_WAIT_TIMEOUT);
+            ok = false;
+            break;
+          }
+        }
       }
+      (void)ok;
       umma_commit(BAR(B_TD));
     }
   } else {
@@ -464,8 +508,10 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
           s[r + 3] = ex2(fmaf(s[r + 3], c, v.w));
           l[r] += s[r]; l[r + 1] += s[r + 1]; l[r + 2] += s[r + 2]; l[r + 3] += s[r + 3];
         }
-        // P and O^T were last used by PV(g - 1)
-        if (g > 0) ok &= mbar_wait(BAR(B_ODONE), (g - 1) & 1, &s_abort, p.status);
+        // P buffer g % PB was last read by PV(g - PB); a rescale of O^T also
+        // needs PV(g - 1) done
+        const int gw = g - ((rescale_o || PB == 1) ? 1 : 2);
+        if (gw >= 0) ok &= mbar_wait(BAR(B_ODONE + (gw & 1)), (gw >> 1) & 1, &s_abort, p.status);
         tc_fence_after();
         if (rescale_o) {
           float o[N];
@@ -478,7 +524,7 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         }
         {
           const int half = tid >> 6, tt = tid & 63;
-          uint8_t* pb = sP + half * (N * 128) + (tt & 7) * 2;
+          uint8_t* pb = sP + (g % PB) * L::kPBytes + half * (N * 128) + (tt & 7) * 2;
           const int ck = tt >> 3;
 #pragma unroll
           for (int r = 0; r < N; ++r)
@@ -496,7 +542,7 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(BAR(B_PFULL));
+        mbar_arrive(BAR(B_PFULL + (g & 1)));
       }
       if (abort_all) break;
       // ---- the last QK of this segment is done: stage the next segment's Q
@@ -517,7 +563,7 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         }
         s_alpha[tid] = lt > 0.f ? 1.f / lt : 0.f;
       }
-      ok &= mbar_wait(BAR(B_ODONE), (g - 1) & 1, &s_abort, p.status);     // PV of the last stage
+      ok &= mbar_wait(BAR(B_ODONE + ((g - 1) & 1)), ((g - 1) >> 1) & 1, &s_abort, p.status);   // PV of the last stage
       tc_fence_after();
       asm volatile("bar.sync 1, 128;" ::: "memory");
       {
