@@ -5,11 +5,14 @@
 // One thread-block cluster of CL CTAs per (sequence, KV head):
 //   1. every CTA scores its share of the pages p < n_b with the float64 bound
 //        s(p) = sum_g sum_d max(q[g,d] * kmin[p,d], q[g,d] * kmax[p,d])
-//      over the G query heads of the group (one warp per page, eight pages in
-//      flight per warp; bf16 products are exact in float32, fp32 products are
-//      taken in float64) and copies the pages' order-preserving 64-bit keys
-//      into the shared memory of the cluster's first CTA (distributed shared
-//      memory);
+//      over the G query heads of the group. Per channel the sum over g folds
+//      into two weights (exact in real arithmetic, for any kmin, kmax):
+//        sum_g max(q_g a, q_g b) = A max(a, b) + B min(a, b),
+//        A = sum_g max(q_g, 0),  B = sum_g min(q_g, 0),
+//      so a page costs 2 D float64 multiply-adds whatever G is (one warp per
+//      page, eight pages in flight per warp). The pages' order-preserving
+//      64-bit keys go into the shared memory of the cluster's first CTA
+//      (distributed shared memory);
 //   2. that CTA radix-selects the budget-th largest key (8-bit digits from the
 //      top: shared-memory histogram, one-warp scan of the 256 bins), stopping
 //      as soon as the boundary bin holds exactly the keys still needed (a
@@ -18,7 +21,6 @@
 //      and writes them in ascending page order with block-wide prefix sums.
 #include <cuda_bf16.h>
 
-#include <type_traits>
 
 #include "s3r_device.cuh"
 #include "s3r_internal.h"
@@ -132,30 +134,12 @@ template <> __device__ __forceinline__ void unpack16<float>(const uint4& u, floa
 __device__ __forceinline__ float load_scalar(const __nv_bfloat16* p, int i) { return __bfloat162float(p[i]); }
 __device__ __forceinline__ float load_scalar(const float* p, int i) { return p[i]; }
 
-// CPL consecutive query values from shared memory as one vector load.
-template <typename Q, int CPL>
-__device__ __forceinline__ void load_qvec(const Q* src, Q* v) {
-  if constexpr (sizeof(Q) == 4 && CPL == 4) {
-    const float4 t = *reinterpret_cast<const float4*>(src);
-    v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
-  } else if constexpr (sizeof(Q) == 4) {
-    const float2 t = *reinterpret_cast<const float2*>(src);
-    v[0] = t.x; v[1] = t.y;
-  } else if constexpr (CPL == 4) {
-    const double2 t0 = reinterpret_cast<const double2*>(src)[0], t1 = reinterpret_cast<const double2*>(src)[1];
-    v[0] = t0.x; v[1] = t0.y; v[2] = t1.x; v[3] = t1.y;
-  } else {
-    const double2 t = *reinterpret_cast<const double2*>(src);
-    v[0] = t.x; v[1] = t.y;
-  }
-}
-
 constexpr int kUnroll = 8;     // pages in flight per warp
 
 template <typename T, int CPL>
-__global__ void __launch_bounds__(kSelThreads) select_kernel(const SelParams p) {
-  extern __shared__ unsigned long long s_keys[];          // [n_b], filled in the first CTA
-  __shared__ __align__(16) double s_qraw[8 * 128];    // [G, D] query rows (float or double)
+__global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelParams p) {
+  extern __shared__ unsigned long long s_keys[];          // [max_pages] keys, then [max_pages] page ids
+  __shared__ __align__(16) double s_ab[2][128];         // A, B per channel
   __shared__ __align__(16) float s_tail[2][128];       // min / max of the tail page (this CTA's, if any)
   __shared__ float s_tpart[2][kSelWarps][128];          // per-warp partial min / max of the tail page
   __shared__ unsigned long long s_kred[2][kSelWarps];   // key min / max per warp
@@ -197,11 +181,19 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelParams p) 
   const T* qp = static_cast<const T*>(p.q) + ((size_t)b * p.Hq + (size_t)h * p.G) * p.D;
   const T* kmn = static_cast<const T*>(p.kmin);
   const T* kmx = static_cast<const T*>(p.kmax);
-  // the G query rows in shared memory, as float (bf16) or double (fp32); a
-  // lane reads its CPL channels of a row as one vector (conflict-free)
-  using Q = typename std::conditional<sizeof(T) == 2, float, double>::type;
-  Q* s_q = reinterpret_cast<Q*>(s_qraw);
-  for (int i = tid; i < p.G * p.D; i += kSelThreads) s_q[i] = static_cast<Q>(load_scalar(qp, i));
+  // the weights A, B of every channel, and this CTA's page ids (inputs, so
+  // read before the dependency wait)
+  for (int d = tid; d < p.D; d += kSelThreads) {
+    double a = 0.0, z = 0.0;
+    for (int g = 0; g < p.G; ++g) {
+      const double v = static_cast<double>(load_scalar(qp, g * p.D + d));
+      if (v > 0.0) a += v; else z += v;
+    }
+    s_ab[0][d] = a;
+    s_ab[1][d] = z;
+  }
+  int* s_phys = reinterpret_cast<int*>(s_keys + p.max_pages);
+  for (int pg = beg + tid; pg < end; pg += kSelThreads) s_phys[pg - beg] = p.block_table[(size_t)b * p.max_pages + pg];
   // The tail page n_b - 1 is the only one whose summary changes while a
   // sequence decodes: the CTA that scores it takes its min / max over the
   // valid tokens straight from K (an input, so before the dependency wait).
@@ -257,14 +249,15 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelParams p) 
   __syncthreads();
   pdl_wait();                                           // earlier kernels may write the summaries
   using Raw = typename RawRow<T, CPL>::type;
+  double wa[CPL], wb[CPL];
+#pragma unroll
+  for (int c = 0; c < CPL; ++c) { wa[c] = s_ab[0][lane * CPL + c]; wb[c] = s_ab[1][lane * CPL + c]; }
   for (int pg0 = beg + warp * kUnroll; pg0 < end; pg0 += kSelWarps * kUnroll) {
-    int phys_l = -1;
-    if (lane < kUnroll && pg0 + lane < end) phys_l = p.block_table[(size_t)b * p.max_pages + pg0 + lane];
     Raw lo[kUnroll], hi[kUnroll];
     bool ok[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      const int phys = __shfl_sync(0xffffffffu, phys_l, u);
+      const int phys = pg0 + u < end ? s_phys[pg0 + u - beg] : -1;
       ok[u] = pg0 + u < end && phys >= 0 && phys < p.num_pages_total;
       if (ok[u] && pg0 + u != tail) {
         const size_t base = ((size_t)phys * p.Hkv + h) * p.D;
@@ -285,18 +278,13 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelParams p) 
           RawRow<T, CPL>::unpack(lo[u], l);
           RawRow<T, CPL>::unpack(hi[u], r);
         }
-        for (int g = 0; g < p.G; ++g) {
-          Q qv[CPL];
-          load_qvec<Q, CPL>(s_q + g * p.D + lane * CPL, qv);
+        double acc1 = 0.0;
 #pragma unroll
-          for (int c = 0; c < CPL; ++c) {
-            if constexpr (sizeof(T) == 2) {
-              acc += static_cast<double>(fmaxf(qv[c] * l[c], qv[c] * r[c]));   // exact products
-            } else {
-              acc += fmax(qv[c] * static_cast<double>(l[c]), qv[c] * static_cast<double>(r[c]));
-            }
-          }
+        for (int c = 0; c < CPL; ++c) {
+          acc = fma(wa[c], static_cast<double>(fmaxf(l[c], r[c])), acc);
+          acc1 = fma(wb[c], static_cast<double>(fminf(l[c], r[c])), acc1);
         }
+        acc += acc1;
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
@@ -452,7 +440,7 @@ cudaError_t launch_select(const s3r_paged_kv& kv, const void* kmin, const void* 
   p.num_pages_total = kv.num_pages_total;
   p.budget = budget;
   p.status = status;
-  const size_t smem = (size_t)kv.max_pages_per_seq * sizeof(unsigned long long);
+  const size_t smem = (size_t)kv.max_pages_per_seq * (sizeof(unsigned long long) + sizeof(int));
   // cluster size: the largest of 4, 2, 1 CTAs per (sequence, KV head) such
   // that every CTA of the launch is resident at once (two per SM), and no
   // more CTAs than 64-page load rounds (larger clusters cannot all be
