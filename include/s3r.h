@@ -27,6 +27,11 @@
  *   their launch with the previous kernel's tail (programmatic dependent
  *   launch). After a call that reported S3R_DEV_WAIT_TIMEOUT, zero the
  *   workspace again before reusing it.
+ * - A call may read its inputs (queries, KV cache, block table, context
+ *   lengths) while the previous kernel on the stream is still finishing,
+ *   when that kernel is one of this library's (none writes another call's
+ *   inputs). A kernel of the caller's that writes an input must not signal
+ *   programmatic launch completion before that write.
  * - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *   stream). Work is enqueued asynchronously on it; outputs are ready when the
  *   stream reaches that point.
@@ -134,7 +139,9 @@ s3r_status s3r_page_summaries(const s3r_paged_kv* kv, int32_t tail_only,
  *   decodes; the call summarises it from k_cache itself (min / max over its
  *   valid tokens), so no summary refresh is needed between draft steps and
  *   kmin/kmax are only read.
- * workspace: at least s3r_attn_workspace_bytes(kv, 1, budget_pages) bytes.
+ * workspace: at least s3r_attn_workspace_bytes(kv, 1, budget_pages) bytes;
+ * it also carries the physical ids of the selected pages from the selection
+ * kernel to the attention kernel.
  */
 s3r_status s3r_sparse_draft_attn(const s3r_paged_kv* kv, const void* kmin, const void* kmax,
                                  const void* q, int32_t budget_pages, float scale,

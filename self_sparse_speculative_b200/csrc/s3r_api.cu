@@ -57,6 +57,7 @@ AttnParams make_attn_params(const s3r_paged_kv* kv, const AttnPlan& pl, const vo
   p.block_table = kv->block_table;
   p.context_lens = kv->context_lens;
   p.page_list = page_list;
+  p.page_phys = nullptr;
   p.k_cache = kv->k_cache;
   p.v_cache = kv->v_cache;
   p.S = kv->num_seqs;
@@ -138,9 +139,11 @@ S3R_EXPORT s3r_status s3r_sparse_draft_attn(const s3r_paged_kv* kv, const void* 
   if (!workspace || workspace_bytes < pl.ws_bytes) return S3R_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint32_t* status = static_cast<uint32_t*>(workspace);
-  s = from_cuda(launch_select(*kv, kmin, kmax, q, budget_pages, selected, status, st));
+  int32_t* phys = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + pl.off_phys);
+  s = from_cuda(launch_select(*kv, kmin, kmax, q, budget_pages, selected, phys, status, st));
   if (s != S3R_OK) return s;
   AttnParams p = make_attn_params(kv, pl, q, out, lse, 1, budget_pages, selected, scale, workspace);
+  p.page_phys = phys;
   s3r_status api;
   cudaError_t e = launch_attention(*kv, p, st, &api);
   if (api != S3R_OK) return api;

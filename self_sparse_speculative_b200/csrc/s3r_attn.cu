@@ -308,6 +308,11 @@ AttnPlan plan_attention(const s3r_paged_kv& kv, int32_t rows, int32_t budget_pag
   off = align_up(off + sizeof(float) * 2 * slots * prow, 256);
   pl.off_o = off;
   off = align_up(off + sizeof(float) * slots * prow * kv.head_dim, 256);
+  pl.off_phys = 0;
+  if (budget_pages > 0) {
+    pl.off_phys = off;
+    off = align_up(off + sizeof(int32_t) * units * (size_t)budget_pages, 256);
+  }
   pl.ws_bytes = off;
   return pl;
 }

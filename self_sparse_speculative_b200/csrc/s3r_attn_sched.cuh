@@ -44,15 +44,19 @@ __device__ __forceinline__ Seg locate(const AttnParams& p, const int* s_prefix, 
   return s;
 }
 
-// Logical page and unit (b * Hkv + h) of flattened position x (-1 when out of range).
+// Logical page and unit (b * Hkv + h) of flattened position x (-1 when out
+// of range); with p.page_phys also the physical page id (else -1).
 __device__ __forceinline__ void page_of(const AttnParams& p, const int* s_prefix, int x, int hi, int W,
-                                        int* lp_out, int* u_out) {
+                                        int* lp_out, int* u_out, int* ph_out = nullptr) {
   *lp_out = -1;
   *u_out = 0;
+  if (ph_out) *ph_out = -1;
   if (x >= hi) return;
   const Seg s = locate(p, s_prefix, x, hi, W);
   *u_out = s.unit;
-  *lp_out = p.page_list ? p.page_list[((size_t)s.b * p.Hkv + s.h) * p.budget + s.k0] : s.k0;
+  const size_t i = ((size_t)s.b * p.Hkv + s.h) * p.budget + s.k0;
+  *lp_out = p.page_list ? p.page_list[i] : s.k0;
+  if (ph_out && p.page_phys) *ph_out = p.page_phys[i];
 }
 
 // Walk over the stages of a CTA's range, segment by segment.

@@ -236,25 +236,30 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
 
   if (warp == kTokProducer) {
     // ======================================================= producer warp
-    pdl_wait();
+    // A page list is an earlier kernel's output (wait for it first); the
+    // block table and the K/V cache are inputs, so the dense path resolves
+    // its first page ids before the wait.
+    if (p.page_list) pdl_wait();
     const uint64_t pol = l2_policy_evict_first();
     // page-id windows of 32 flattened positions: lane k of a window holds
     // position wbase + k. w0 = in use, w1 = phys loads in flight, w2 = lp
-    // loads in flight.
-    int w0_lp, w0_ph, w0_u, w1_lp, w1_ph, w1_u, w2_lp, w2_u;
-    auto phys_load = [&](int lp, int u) {
+    // loads in flight (with the selector's physical ids, w2_pp).
+    int w0_lp, w0_ph, w0_u, w1_lp, w1_ph, w1_u, w2_lp, w2_u, w2_pp, pp;
+    auto phys_load = [&](int lp, int u, int ph_sel) {
       if (lp < 0) return -1;
+      if (p.page_phys) return ph_sel;
       const int b = u / p.Hkv;
       const int n_b = (p.context_lens[b] + p.P - 1) / p.P;
       if (lp >= n_b) { flag_status(p.status, S3R_DEV_BAD_PAGE_ID); return -1; }
       return p.block_table[(size_t)b * p.max_pages + lp];
     };
     int wbase = lo;
-    page_of(p, s_prefix, wbase + lane, hi, W, &w0_lp, &w0_u);
-    w0_ph = phys_load(w0_lp, w0_u);
-    page_of(p, s_prefix, wbase + 32 + lane, hi, W, &w1_lp, &w1_u);
-    w1_ph = phys_load(w1_lp, w1_u);
-    page_of(p, s_prefix, wbase + 64 + lane, hi, W, &w2_lp, &w2_u);
+    page_of(p, s_prefix, wbase + lane, hi, W, &w0_lp, &w0_u, &pp);
+    w0_ph = phys_load(w0_lp, w0_u, pp);
+    page_of(p, s_prefix, wbase + 32 + lane, hi, W, &w1_lp, &w1_u, &pp);
+    w1_ph = phys_load(w1_lp, w1_u, pp);
+    page_of(p, s_prefix, wbase + 64 + lane, hi, W, &w2_lp, &w2_u, &w2_pp);
+    if (!p.page_list) pdl_wait();
     int g = 0;
     bool ok = true;
     for (int x = lo; x < hi && ok;) {
@@ -271,8 +276,8 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             wbase += 32;
             w0_lp = w1_lp; w0_ph = w1_ph; w0_u = w1_u;
             w1_lp = w2_lp; w1_u = w2_u;
-            w1_ph = phys_load(w1_lp, w1_u);
-            page_of(p, s_prefix, wbase + 64 + lane, hi, W, &w2_lp, &w2_u);
+            w1_ph = phys_load(w1_lp, w1_u, w2_pp);
+            page_of(p, s_prefix, wbase + 64 + lane, hi, W, &w2_lp, &w2_u, &w2_pp);
           }
           const int src = xp - wbase;
           const int lp = __shfl_sync(0xffffffffu, w0_lp, src & 31);

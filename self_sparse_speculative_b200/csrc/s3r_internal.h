@@ -36,6 +36,7 @@ struct AttnParams {
   const int32_t* block_table;
   const int32_t* context_lens;
   const int32_t* page_list;   // sparse: selected [S, Hkv, budget]; dense: nullptr
+  const int32_t* page_phys;   // sparse: physical ids of page_list's pages (written by the selector); else nullptr
   const void* k_cache;
   const void* v_cache;
   int32_t S, Hq, Hkv, G, D, P, R, rows;
@@ -54,14 +55,15 @@ struct AttnPlan {
   int32_t chunk_pages;
   size_t ws_bytes;
   size_t off_tickets, off_ml, off_o;
+  size_t off_phys;   // sparse: [S, Hkv, budget] physical page ids of the selection (0: none)
 };
 AttnPlan plan_attention(const s3r_paged_kv& kv, int32_t rows, int32_t budget_pages);
 
 cudaError_t launch_summaries(const s3r_paged_kv& kv, int tail_only, void* kmin, void* kmax,
                              uint32_t* status, cudaStream_t st);
 cudaError_t launch_select(const s3r_paged_kv& kv, const void* kmin, const void* kmax,
-                          const void* q, int32_t budget, int32_t* selected, uint32_t* status,
-                          cudaStream_t st);
+                          const void* q, int32_t budget, int32_t* selected, int32_t* selected_phys,
+                          uint32_t* status, cudaStream_t st);
 // Launch with programmatic dependent launch allowed (the kernel orders
 // itself after its predecessor with griddepcontrol.wait) and, when
 // cluster_x > 1, thread-block clusters of cluster_x CTAs along x.

@@ -72,6 +72,7 @@ struct SelParams {
   const int32_t* block_table;
   const int32_t* context_lens;
   int32_t* selected;        // [S, Hkv, budget]
+  int32_t* selected_phys;   // [S, Hkv, budget] physical ids of the selected pages (-1: none)
   int32_t S, Hq, Hkv, G, D, P, max_pages, num_pages_total, budget;
   uint32_t* status;
 };
@@ -89,6 +90,11 @@ __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
   return r;
+}
+__device__ __forceinline__ void st_cluster_u32(uint32_t local_addr, uint32_t rank, uint32_t v) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
+  asm volatile("st.shared::cluster.u32 [%0], %1;" :: "r"(remote), "r"(v) : "memory");
 }
 __device__ __forceinline__ void st_cluster_u64(uint32_t local_addr, uint32_t rank, unsigned long long v) {
   uint32_t remote;
@@ -134,7 +140,14 @@ template <> __device__ __forceinline__ void unpack16<float>(const uint4& u, floa
 __device__ __forceinline__ float load_scalar(const __nv_bfloat16* p, int i) { return __bfloat162float(p[i]); }
 __device__ __forceinline__ float load_scalar(const float* p, int i) { return p[i]; }
 
-constexpr int kUnroll = 8;     // pages in flight per warp
+// Pages per warp and round: 8, or 4 when a page's two summary rows exceed
+// 512 bytes (fp32, D = 128).
+template <typename T, int CPL>
+__host__ __device__ constexpr int sel_unroll() { return sizeof(T) * CPL * 32 * 2 > 512 ? 4 : 8; }
+
+// Dynamic shared memory: keys [max_pages] (u64), then physical page ids
+// [max_pages] (int).
+inline size_t sel_smem_bytes(int max_pages) { return (size_t)max_pages * 12; }
 
 template <typename T, int CPL>
 __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelParams p) {
@@ -154,13 +167,20 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelParams 
   const int ncta = gridDim.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int32_t* out = p.selected + ((size_t)b * p.Hkv + h) * p.budget;
+  int32_t* out_phys = p.selected_phys + ((size_t)b * p.Hkv + h) * p.budget;
+  // the group's query values first (they depend on nothing), so their loads
+  // overlap the context length -> page id -> tail K chain below
+  const T* qp = static_cast<const T*>(p.q) + ((size_t)b * p.Hq + (size_t)h * p.G) * p.D;
+  float qv[8];
+#pragma unroll
+  for (int g = 0; g < 8; ++g) qv[g] = (tid < p.D && g < p.G) ? load_scalar(qp, g * p.D + tid) : 0.f;
   // every decision before the cluster barriers is uniform over the cluster
   const int L = p.context_lens[b];
   if (L < 1 || L > p.max_pages * p.P) {
     pdl_wait();
     if (rank == 0) {
       if (tid == 0) flag_status(p.status, S3R_DEV_BAD_CONTEXT_LEN);
-      for (int k = tid; k < p.budget; k += kSelThreads) out[k] = -1;
+      for (int k = tid; k < p.budget; k += kSelThreads) { out[k] = -1; out_phys[k] = -1; }
     }
     return;
   }
@@ -168,7 +188,10 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelParams 
   if (n_b <= p.budget) {
     pdl_wait();
     if (rank == 0)
-      for (int k = tid; k < p.budget; k += kSelThreads) out[k] = k < n_b ? k : -1;
+      for (int k = tid; k < p.budget; k += kSelThreads) {
+        out[k] = k < n_b ? k : -1;
+        out_phys[k] = k < n_b ? p.block_table[(size_t)b * p.max_pages + k] : -1;
+      }
     return;
   }
   // announce this CTA to the cluster now; wait for the others only before
@@ -178,30 +201,28 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelParams 
   // ---- 1. scores of pages [beg, end) into this CTA's own key array
   const int per = (n_b + ncta - 1) / ncta;
   const int beg = min(n_b, (int)rank * per), end = min(n_b, beg + per);
-  const T* qp = static_cast<const T*>(p.q) + ((size_t)b * p.Hq + (size_t)h * p.G) * p.D;
   const T* kmn = static_cast<const T*>(p.kmin);
   const T* kmx = static_cast<const T*>(p.kmax);
-  // the weights A, B of every channel, and this CTA's page ids (inputs, so
-  // read before the dependency wait)
-  for (int d = tid; d < p.D; d += kSelThreads) {
-    double a = 0.0, z = 0.0;
-    for (int g = 0; g < p.G; ++g) {
-      const double v = static_cast<double>(load_scalar(qp, g * p.D + d));
-      if (v > 0.0) a += v; else z += v;
-    }
-    s_ab[0][d] = a;
-    s_ab[1][d] = z;
-  }
-  int* s_phys = reinterpret_cast<int*>(s_keys + p.max_pages);
-  for (int pg = beg + tid; pg < end; pg += kSelThreads) s_phys[pg - beg] = p.block_table[(size_t)b * p.max_pages + pg];
-  // The tail page n_b - 1 is the only one whose summary changes while a
-  // sequence decodes: the CTA that scores it takes its min / max over the
-  // valid tokens straight from K (an input, so before the dependency wait).
+  // This CTA's page ids and the weights A, B of every channel (inputs, so
+  // read before the dependency wait). The tail page n_b - 1 is the only one
+  // whose summary changes while a sequence decodes: the CTA that scores it
+  // takes its min / max over the valid tokens straight from K.
   const int tail = n_b - 1;
   const bool has_tail = beg <= tail && tail < end;
-  int tail_phys = -1;
+  const int tail_phys = has_tail ? p.block_table[(size_t)b * p.max_pages + tail] : -1;
+  int* s_phys = reinterpret_cast<int*>(s_keys + p.max_pages);
+  for (int pg = beg + tid; pg < end; pg += kSelThreads) s_phys[pg] = p.block_table[(size_t)b * p.max_pages + pg];
+  if (tid < p.D) {
+    double a = 0.0, z = 0.0;
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+      const double v = static_cast<double>(qv[g]);
+      if (v > 0.0) a += v; else z += v;                 // zero padding adds nothing
+    }
+    s_ab[0][tid] = a;
+    s_ab[1][tid] = z;
+  }
   if (has_tail) {
-    tail_phys = p.block_table[(size_t)b * p.max_pages + tail];
     if (tail_phys >= 0 && tail_phys < p.num_pages_total) {
       // thread = (token group, 16-byte chunk of channels); every load in
       // flight at once, then the groups merge by shuffles and across warps
@@ -248,30 +269,41 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelParams 
   }
   __syncthreads();
   pdl_wait();                                           // earlier kernels may write the summaries
+  // Each warp scores kU pages per round, all of a round's summary rows in
+  // flight at once (loading the next round ahead, into a second register
+  // set or by cp.async into shared memory, measured slower).
   using Raw = typename RawRow<T, CPL>::type;
-  double wa[CPL], wb[CPL];
+  constexpr int kU = sel_unroll<T, CPL>();
+  const int span = kSelWarps * kU;
+  auto page_ok = [&](int pg) {
+    const int ph = s_phys[pg];
+    return ph >= 0 && ph < p.num_pages_total;
+  };
+  auto load = [&](int pg0, Raw (&lo)[kU], Raw (&hi)[kU]) {
 #pragma unroll
-  for (int c = 0; c < CPL; ++c) { wa[c] = s_ab[0][lane * CPL + c]; wb[c] = s_ab[1][lane * CPL + c]; }
-  for (int pg0 = beg + warp * kUnroll; pg0 < end; pg0 += kSelWarps * kUnroll) {
-    Raw lo[kUnroll], hi[kUnroll];
-    bool ok[kUnroll];
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int phys = pg0 + u < end ? s_phys[pg0 + u - beg] : -1;
-      ok[u] = pg0 + u < end && phys >= 0 && phys < p.num_pages_total;
-      if (ok[u] && pg0 + u != tail) {
-        const size_t base = ((size_t)phys * p.Hkv + h) * p.D;
+    for (int u = 0; u < kU; ++u) {
+      const int pg = pg0 + u;
+      const int ph = pg < end ? s_phys[pg] : -1;
+      if (pg != tail && ph >= 0 && ph < p.num_pages_total) {
+        const size_t base = ((size_t)ph * p.Hkv + h) * p.D;
         lo[u] = __ldg(reinterpret_cast<const Raw*>(kmn + base) + lane);
         hi[u] = __ldg(reinterpret_cast<const Raw*>(kmx + base) + lane);
       }
     }
+  };
+  double wa[CPL], wb[CPL];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      if (pg0 + u >= end) continue;                     // warp-uniform
+  for (int c = 0; c < CPL; ++c) { wa[c] = s_ab[0][lane * CPL + c]; wb[c] = s_ab[1][lane * CPL + c]; }
+  auto score = [&](int pg0, const Raw (&lo)[kU], const Raw (&hi)[kU]) {
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int pg = pg0 + u;
+      if (pg >= end) continue;                            // warp-uniform
+      const bool ok = page_ok(pg);
       double acc = 0.0;
-      if (ok[u]) {
+      if (ok) {
         float l[CPL], r[CPL];
-        if (pg0 + u == tail) {                          // this CTA's own summary of the tail page
+        if (pg == tail) {                                 // this CTA's own summary of the tail page
 #pragma unroll
           for (int c = 0; c < CPL; ++c) { l[c] = s_tail[0][lane * CPL + c]; r[c] = s_tail[1][lane * CPL + c]; }
         } else {
@@ -289,17 +321,25 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelParams 
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
       if (lane == 0) {
-        if (!ok[u]) flag_status(p.status, S3R_DEV_BAD_PAGE_ID);
-        s_keys[pg0 + u] = ok[u] ? order_key(acc) : 0ull;
+        if (!ok) flag_status(p.status, S3R_DEV_BAD_PAGE_ID);
+        s_keys[pg] = ok ? order_key(acc) : 0ull;
       }
     }
+  };
+  for (int pg0 = beg + warp * kU; pg0 < end; pg0 += span) {
+    Raw lo[kU], hi[kU];
+    load(pg0, lo, hi);
+    score(pg0, lo, hi);
   }
   __syncthreads();
   // ---- copy this CTA's keys into the first CTA (distributed shared memory)
   cluster_wait();                                         // every CTA of the cluster is running
   if (rank != 0) {
-    const uint32_t keys_addr = smem_addr(s_keys);
-    for (int pg = beg + tid; pg < end; pg += kSelThreads) st_cluster_u64(keys_addr + 8u * (uint32_t)pg, 0u, s_keys[pg]);
+    const uint32_t keys_addr = smem_addr(s_keys), phys_addr = smem_addr(s_phys);
+    for (int pg = beg + tid; pg < end; pg += kSelThreads) {
+      st_cluster_u64(keys_addr + 8u * (uint32_t)pg, 0u, s_keys[pg]);
+      st_cluster_u32(phys_addr + 4u * (uint32_t)pg, 0u, s_phys[pg]);
+    }
   }
   cluster_sync_all();                                     // all keys are in the first CTA
   if (rank != 0) return;
@@ -340,10 +380,15 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelParams 
     s_hist[tid] = 0u;                                      // kSelThreads == 256 bins
     __syncthreads();
     const unsigned long long prefix = s_prefix;
-    for (int pg = tid; pg < n_b; pg += kSelThreads) {
-      const unsigned long long key = s_keys[pg];
-      const bool match = (shift >= 56) || (((key ^ prefix) >> (shift + 8)) == 0ull);
-      if (match) atomicAdd(&s_hist[(key >> shift) & 255u], 1u);
+    for (int base = 0; base < n_b; base += kSelThreads) {   // uniform trip count: whole warps
+      const int pg = base + tid;
+      const unsigned long long key = pg < n_b ? s_keys[pg] : 0ull;
+      const bool match = pg < n_b && ((shift >= 56) || (((key ^ prefix) >> (shift + 8)) == 0ull));
+      // lanes with the same bin add once (scores often share their top
+      // digits); a lane without a match groups only with itself
+      const unsigned bin = match ? (unsigned)(key >> shift) & 255u : 256u + (unsigned)lane;
+      const unsigned peers = __match_any_sync(0xffffffffu, bin);
+      if (match && (int)(__ffs(peers) - 1) == lane) atomicAdd(&s_hist[bin], (unsigned)__popc(peers));
     }
     __syncthreads();
     if (warp == 0) {
@@ -405,13 +450,18 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelParams 
       bool take = false;
       if (key > thr) take = true;
       else if (key == thr) { take = e < need_eq; ++e; }
-      if (take && pos < p.budget) out[pos++] = pg;
+      if (take && pos < p.budget) {
+        out[pos] = pg;
+        out_phys[pos] = s_phys[pg];
+        ++pos;
+      }
     }
   }
 }
 
 template <typename T, int CPL>
-cudaError_t launch_typed(const SelParams& p, int cl, size_t smem, cudaStream_t st) {
+cudaError_t launch_typed(const SelParams& p, int cl, cudaStream_t st) {
+  const size_t smem = sel_smem_bytes(p.max_pages);
   cudaError_t e = cudaFuncSetAttribute(select_kernel<T, CPL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   return launch_kernel(select_kernel<T, CPL>, dim3(cl, p.Hkv, p.S), dim3(kSelThreads), smem, st, cl, p);
@@ -420,8 +470,8 @@ cudaError_t launch_typed(const SelParams& p, int cl, size_t smem, cudaStream_t s
 }  // namespace
 
 cudaError_t launch_select(const s3r_paged_kv& kv, const void* kmin, const void* kmax,
-                          const void* q, int32_t budget, int32_t* selected, uint32_t* status,
-                          cudaStream_t st) {
+                          const void* q, int32_t budget, int32_t* selected, int32_t* selected_phys,
+                          uint32_t* status, cudaStream_t st) {
   SelParams p;
   p.q = q;
   p.kmin = kmin;
@@ -430,6 +480,7 @@ cudaError_t launch_select(const s3r_paged_kv& kv, const void* kmin, const void* 
   p.block_table = kv.block_table;
   p.context_lens = kv.context_lens;
   p.selected = selected;
+  p.selected_phys = selected_phys;
   p.S = kv.num_seqs;
   p.Hq = kv.num_q_heads;
   p.Hkv = kv.num_kv_heads;
@@ -440,7 +491,6 @@ cudaError_t launch_select(const s3r_paged_kv& kv, const void* kmin, const void* 
   p.num_pages_total = kv.num_pages_total;
   p.budget = budget;
   p.status = status;
-  const size_t smem = (size_t)kv.max_pages_per_seq * (sizeof(unsigned long long) + sizeof(int));
   // cluster size: the largest of 4, 2, 1 CTAs per (sequence, KV head) such
   // that every CTA of the launch is resident at once (two per SM), and no
   // more CTAs than 64-page load rounds (larger clusters cannot all be
@@ -451,8 +501,8 @@ cudaError_t launch_select(const s3r_paged_kv& kv, const void* kmin, const void* 
   while (cl > 1 && (units * cl > slots || (cl - 1) * 64 >= kv.max_pages_per_seq)) cl >>= 1;
   const bool bf = kv.dtype == S3R_BF16;
   cudaError_t e;
-  if (kv.head_dim == 128) e = bf ? launch_typed<__nv_bfloat16, 4>(p, cl, smem, st) : launch_typed<float, 4>(p, cl, smem, st);
-  else e = bf ? launch_typed<__nv_bfloat16, 2>(p, cl, smem, st) : launch_typed<float, 2>(p, cl, smem, st);
+  if (kv.head_dim == 128) e = bf ? launch_typed<__nv_bfloat16, 4>(p, cl, st) : launch_typed<float, 4>(p, cl, st);
+  else e = bf ? launch_typed<__nv_bfloat16, 2>(p, cl, st) : launch_typed<float, 2>(p, cl, st);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
