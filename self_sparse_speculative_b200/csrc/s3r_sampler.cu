@@ -117,34 +117,32 @@ __device__ double block_sum_d(double v, double* s_red) {
 
 // float64 exponential, table-driven (P. T. P. Tang, "Table-driven
 // implementation of the exponential function in IEEE floating-point
-// arithmetic", ACM Trans. Math. Software 15(2), 1989): write
-// x = (32 m + j) ln2/32 + r with |r| <= ln2/64, then
-// exp(x) = 2^m * 2^(j/32) * e^r. Here N = 32 m + j is x * 32/ln2 rounded to
-// an integer by adding 1.5 * 2^52; r = x - N ln2/32 with ln2/32 split into a
+// arithmetic", ACM Trans. Math. Software 15(2), 1989), with a 256-entry
+// table: write x = (256 m + j) ln2/256 + r with |r| <= ln2/512, then
+// exp(x) = 2^m * 2^(j/256) * e^r. N = 256 m + j is x * 256/ln2 rounded to an
+// integer by adding 1.5 * 2^52; r = x - N ln2/256 with ln2/256 split into a
 // double and its remainder (two fused multiply-adds); e^r - 1 is its Taylor
-// polynomial to degree 6 (remainder < 4e-18 for |r| <= ln2/64); 2^(j/32) is
-// a 32-entry table `tab`; 2^m goes into the exponent field. The result is
-// within about 2 ulp for -707 < x < 708 (no branch: callers keep x in that
-// range and fix up the rest with exp_fixup).
+// polynomial to degree 4 (remainder < 4e-17 for |r| <= ln2/512); 2^(j/256)
+// is the table `tab`; 2^m goes into the exponent field. Within about 2 ulp
+// for -707 < x < 708; outside that range the value is meaningless (callers
+// fix it up with exp_fixup).
+constexpr int kExpTab = 256;
 __device__ __forceinline__ double exp_tbl(double x, const double* tab) {
-  constexpr double kInvStep = 46.16624130844683;           // 32 / ln2
-  constexpr double kStepHi = 0x1.62e42fefa39efp-6;          // ln2 / 32, leading double
-  constexpr double kStepLo = 0x1.abc9e3b39803fp-61;         // ln2 / 32 - kStepHi
+  constexpr double kInvStep = 369.32993046757463;          // 256 / ln2
+  constexpr double kStepHi = 0x1.62e42fefa39efp-9;          // ln2 / 256, leading double
+  constexpr double kStepLo = 0x1.abc9e3b39803fp-64;         // ln2 / 256 - kStepHi
   constexpr double kShifter = 6755399441055744.0;           // 1.5 * 2^52
-  x = fmin(fmax(x, -707.0), 708.0);
   const double t = fma(x, kInvStep, kShifter);
   const int n = __double2loint(t);
   const double nd = t - kShifter;
   double r = fma(-nd, kStepHi, x);
   r = fma(-nd, kStepLo, r);
-  double q = fma(r, 1.0 / 720.0, 1.0 / 120.0);
-  q = fma(q, r, 1.0 / 24.0);
-  q = fma(q, r, 1.0 / 6.0);
+  double q = fma(r, 1.0 / 24.0, 1.0 / 6.0);
   q = fma(q, r, 0.5);
   q = fma(q, r, 1.0);
-  const double tj = tab[n & 31];
+  const double tj = tab[n & (kExpTab - 1)];
   const double y = fma(tj, q * r, tj);
-  return __hiloint2double(__double2hiint(y) + ((n >> 5) << 20), __double2loint(y));
+  return __hiloint2double(__double2hiint(y) + (n >> 8) * (1 << 20), __double2loint(y));
 }
 // exp(x) given y = exp_tbl(x): outside (-707, 708) the argument is moved
 // into range by 512 ln2 and the result scaled back by an exact power of two
@@ -160,9 +158,11 @@ __device__ __forceinline__ double exp_fixup(double x, double y, const double* ta
   return exp_tbl(x - k512ln2, tab) * 0x1p512;
 }
 
-// 2^(j/32), j = 0..31, into shared memory (threads 0..31; caller syncs).
+// 2^(j/256), j = 0..255, into shared memory (one entry per thread of a
+// 256-thread CTA; caller syncs).
 __device__ __forceinline__ void fill_exp_tab(double* tab) {
-  if (threadIdx.x < 32) tab[threadIdx.x] = exp2(static_cast<double>(threadIdx.x) * 0.03125);
+  static_assert(kSmpThreads == kExpTab, "one table entry per thread");
+  tab[threadIdx.x] = exp2(static_cast<double>(threadIdx.x) * (1.0 / kExpTab));
 }
 
 // Staging: the CTA's chunk [beg, beg + n) of one or two rows into shared
@@ -238,57 +238,64 @@ __device__ void decide(const SampleParams& p, int b) {
 }
 
 // ---------------------------------------------------------------- pass 1
-template <typename T, bool STAGE>
-__global__ void __launch_bounds__(kSmpThreads) rowstats_kernel(const SampleParams p) {
+// One streaming pass per chunk: every thread keeps a running maximum m and
+// the float32 sum of 2^((x - m) log2(e)/T), rescaled when m grows (the
+// online normaliser of M. Milakov and N. Gimelshein, "Online normalizer
+// calculation for softmax", 2018); four 16-byte loads in flight per thread.
+// VEC: rows 16-byte aligned with a length that is a multiple of the vector.
+template <typename T, bool VEC>
+__global__ void __launch_bounds__(kSmpThreads, 5) rowstats_kernel(const SampleParams p) {
   pdl_launch_dependents();
   pdl_wait();
-  extern __shared__ __align__(16) uint8_t s_dyn[];
-  __shared__ uint64_t s_bar;
-  __shared__ int s_abort;
   __shared__ float s_redf[kSmpWarps];
   __shared__ double s_redd[kSmpWarps];
   __shared__ int s_last;
   using IO = LogitIO<T>;
   constexpr int PV = IO::kPerVec;
+  constexpr int kB = 4;                                 // vectors in flight per thread
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int row = blockIdx.x / p.c1, c = blockIdx.x - (blockIdx.x / p.c1) * p.c1;
   const int beg = c * p.ch1, n = min(p.vocab, beg + p.ch1) - beg;
   const T* src = row_ptr<T>(p, true, row) + beg;
-  if constexpr (STAGE) {
-    if (tid == 0) s_abort = 0;
-    init_stage_bar(&s_bar);
-    T* s_chunk = reinterpret_cast<T*>(s_dyn);
-    stage_rows<T>(s_chunk, src, nullptr, nullptr, n, &s_bar, &s_abort, p.status);
-    src = s_chunk;
-  }
-  float mx = -INFINITY;
-  for (int i = tid * PV; i < n; i += kSmpThreads * PV) {
-    float v[PV];
-    const int m = min(PV, n - i);
-    load_vals<T, STAGE>(src + i, m, v);
-#pragma unroll
-    for (int t = 0; t < PV; ++t)
-      if (t < m) mx = fmaxf(mx, v[t]);
-  }
-  const float M = block_max(mx, s_redf);
+  const float k2 = kLog2e * p.inv_temp;
+  float m = -INFINITY, nmk = INFINITY;                  // nmk = -m k2
   double s = 0.0;
-  if (M != -INFINITY) {
-    const float k2 = kLog2e * p.inv_temp;
-    for (int i = tid * PV; i < n; i += kSmpThreads * PV) {
-      float v[PV];
-      const int m = min(PV, n - i);
-      load_vals<T, STAGE>(src + i, m, v);
-      // a vector's exponentials summed pairwise in float32, then added in float64
+  for (int i0 = tid * PV; i0 < n; i0 += kB * kSmpThreads * PV) {
+    float v[kB][PV];
+    int cnt[kB];
 #pragma unroll
-      for (int t = 0; t < PV; ++t) v[t] = t < m ? ex2((v[t] - M) * k2) : 0.f;
+    for (int b = 0; b < kB; ++b) {
+      const int i = i0 + b * kSmpThreads * PV;
+      cnt[b] = max(0, min(PV, n - i));
+      if (cnt[b] > 0) load_vals<T, VEC>(src + i, cnt[b], v[b]);
+    }
+#pragma unroll
+    for (int b = 0; b < kB; ++b) {
+      if (cnt[b] <= 0) continue;
+      float vm = -INFINITY;
+#pragma unroll
+      for (int t = 0; t < PV; ++t)
+        if (t < cnt[b]) vm = fmaxf(vm, v[b][t]);
+      if (vm > m) {
+        s *= static_cast<double>(ex2((m - vm) * k2));   // from m = -inf: a factor 0 on s = 0
+        m = vm;
+        nmk = -m * k2;
+      }
+      if (m == -INFINITY) continue;                     // nothing but -inf so far
+      // a vector's exponentials summed pairwise in float32, then added in float64
+      float e[PV];
+#pragma unroll
+      for (int t = 0; t < PV; ++t) e[t] = t < cnt[b] ? ex2(fmaf(v[b][t], k2, nmk)) : 0.f;
 #pragma unroll
       for (int w = PV / 2; w > 0; w >>= 1)
 #pragma unroll
-        for (int t = 0; t < w; ++t) v[t] += v[t + w];
-      s += static_cast<double>(v[0]);
+        for (int t = 0; t < w; ++t) e[t] += e[t + w];
+      s += static_cast<double>(e[0]);
     }
   }
-  const double S = block_sum_d(s, s_redd);
+  const float M = block_max(m, s_redf);
+  const double sc = m == -INFINITY ? 0.0 : s * static_cast<double>(ex2((m - M) * k2));
+  const double S = block_sum_d(sc, s_redd);
   if (tid == 0) {
     Part1* part = static_cast<Part1*>(p.part1) + (size_t)row * p.c1 + c;
     part->m = M;
@@ -375,15 +382,16 @@ __device__ __forceinline__ void weights(const DrawRows& w, const T* pa, const T*
   load_vals<T, VEC>(pa, n, a);
   if (w.qrow) load_vals<T, VEC>(pb, n, b);
   constexpr int G = 4;                                  // elements interleaved per group
+  const double ca = -w.Mp * invT, cb = -w.Mq * invT;    // (x - M)/T as one fused multiply-add
 #pragma unroll
   for (int t0 = 0; t0 < PV; t0 += G) {
     double xa[G], xb[G], ea[G], eb[G];
 #pragma unroll
     for (int t = 0; t < G; ++t) {                       // branch-free
-      xa[t] = (static_cast<double>(a[t0 + t]) - w.Mp) * invT;
+      xa[t] = fma(static_cast<double>(a[t0 + t]), invT, ca);
       ea[t] = exp_tbl(xa[t], tab);
       if (w.qrow) {
-        xb[t] = (static_cast<double>(b[t0 + t]) - w.Mq) * invT;
+        xb[t] = fma(static_cast<double>(b[t0 + t]), invT, cb);
         eb[t] = exp_tbl(xb[t], tab);
       }
     }
@@ -415,7 +423,7 @@ __global__ void __launch_bounds__(kSmpThreads) znorm_kernel(const SampleParams p
   __shared__ uint64_t s_bar;
   __shared__ int s_abort;
   __shared__ double s_red[2][kSmpWarps];
-  __shared__ double s_tab[32];
+  __shared__ double s_tab[kExpTab];
   __shared__ int s_last;
   using IO = LogitIO<T>;
   constexpr int PV = IO::kPerVec;
@@ -441,6 +449,7 @@ __global__ void __launch_bounds__(kSmpThreads) znorm_kernel(const SampleParams p
     __syncthreads();
   }
   double zt = 0.0, zd = 0.0;
+  const double ca = -Mp * p.inv_temp_d, cb = -Mq * p.inv_temp_d;
   for (int i = tid * PV; i < n; i += kSmpThreads * PV) {
     const int m = min(PV, n - i);
     float a[PV], b[PV];
@@ -451,8 +460,8 @@ __global__ void __launch_bounds__(kSmpThreads) znorm_kernel(const SampleParams p
       double xa[4], xb[4], ea[4], eb[4];
 #pragma unroll
       for (int t = 0; t < 4; ++t) {                     // branch-free
-        xa[t] = (static_cast<double>(a[t0 + t]) - Mp) * p.inv_temp_d;
-        xb[t] = (static_cast<double>(b[t0 + t]) - Mq) * p.inv_temp_d;
+        xa[t] = fma(static_cast<double>(a[t0 + t]), p.inv_temp_d, ca);
+        xb[t] = fma(static_cast<double>(b[t0 + t]), p.inv_temp_d, cb);
         ea[t] = exp_tbl(xa[t], s_tab);
         eb[t] = exp_tbl(xb[t], s_tab);
       }
@@ -613,7 +622,7 @@ __global__ void __launch_bounds__(kSmpThreads) draw_kernel(const SampleParams p)
   __shared__ uint64_t s_bar;
   __shared__ int s_abort;
   __shared__ double s_w[kSmpWarps];
-  __shared__ double s_tab[32];
+  __shared__ double s_tab[kExpTab];
   __shared__ float s_redf[kSmpWarps];
   __shared__ int s_i[3];
   __shared__ double s_base;
@@ -775,16 +784,11 @@ cudaError_t launch_typed(const SampleParams& p, cudaStream_t st) {
                      (reinterpret_cast<uintptr_t>(p.target) % 16 == 0) &&
                      (!SPEC || reinterpret_cast<uintptr_t>(p.draft) % 16 == 0);
   const dim3 blk(kSmpThreads);
-  const size_t sm1 = stage ? (size_t)p.ch1 * sizeof(T) : 0;
   const size_t sm2 = stage ? (size_t)p.ch2 * sizeof(T) * (SPEC ? 2 : 1) : 0;
   cudaError_t e = cudaSuccess;
   if (SPEC) {
-    if (stage) {
-      e = cudaFuncSetAttribute(rowstats_kernel<T, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1);
-      if (e == cudaSuccess) e = launch_kernel(rowstats_kernel<T, true>, dim3(p.c1 * nrows), blk, sm1, st, 1, p);
-    } else {
-      e = launch_kernel(rowstats_kernel<T, false>, dim3(p.c1 * nrows), blk, 0, st, 1, p);
-    }
+    if (stage) e = launch_kernel(rowstats_kernel<T, true>, dim3(p.c1 * nrows), blk, 0, st, 1, p);
+    else e = launch_kernel(rowstats_kernel<T, false>, dim3(p.c1 * nrows), blk, 0, st, 1, p);
     if (e != cudaSuccess) return e;
     if (stage) {
       e = cudaFuncSetAttribute(znorm_kernel<T, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
@@ -808,12 +812,13 @@ SamplePlan plan_sampling(int32_t nseq, int32_t gamma, int32_t vocab) {
   SamplePlan pl{};
   pl.nseq = nseq;
   pl.nrows = nseq * (gamma > 0 ? 2 * gamma + 1 : 1);
-  // pass 1: at most 16384 staged elements per CTA (32 KB bf16, 64 KB fp32),
-  // about 4 CTAs per SM overall, at least 256 elements per CTA
-  const int max_per_cta = kSmpThreads * 64;
+  // pass 1 (streamed, no shared memory): at most 32768 elements per CTA, and
+  // no more CTAs than fit at once (5 per SM) unless the rows need them; at
+  // least 256 elements per CTA
+  const int max_per_cta = kSmpThreads * 128;
   const int target = 148 * 4;
   int c1 = (vocab + max_per_cta - 1) / max_per_cta;
-  const int want = (target + pl.nrows - 1) / pl.nrows;
+  const int want = 148 * 5 / pl.nrows;
   if (want > c1) c1 = want;
   const int cap = (vocab + 255) / 256;
   if (c1 > cap) c1 = cap;
