@@ -105,7 +105,10 @@ S3R_EXPORT size_t s3r_attn_workspace_bytes(const s3r_paged_kv* kv, int32_t rows,
 
 S3R_EXPORT size_t s3r_sample_workspace_bytes(int32_t num_seqs, int32_t gamma, int32_t vocab) {
   if (num_seqs < 1 || vocab < 1 || gamma < 0 || gamma > kMaxGamma) return 0;
-  return plan_sampling(num_seqs, gamma, vocab).ws_bytes;
+  // enough for either logit type
+  const size_t a = plan_sampling(num_seqs, gamma, vocab, 2).ws_bytes;
+  const size_t b = plan_sampling(num_seqs, gamma, vocab, 4).ws_bytes;
+  return a > b ? a : b;
 }
 
 S3R_EXPORT s3r_status s3r_page_summaries_checked(const s3r_paged_kv* kv, int32_t tail_only, void* kmin,
@@ -191,7 +194,7 @@ S3R_EXPORT s3r_status s3r_spec_sample(const void* target_logits, const void* dra
   if (num_seqs < 1 || vocab < 1 || gamma < 1) return S3R_ERR_INVALID_ARG;
   if (!(temperature > 0.0f) || !std::isfinite(temperature)) return S3R_ERR_INVALID_ARG;
   if (gamma > kMaxGamma) return S3R_ERR_UNSUPPORTED;
-  const SamplePlan pl = plan_sampling(num_seqs, gamma, vocab);
+  const SamplePlan pl = plan_sampling(num_seqs, gamma, vocab, logit_dtype == S3R_BF16 ? 2 : 4);
   if (!workspace || workspace_bytes < pl.ws_bytes) return S3R_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   SampleParams p = make_sample_params(pl, workspace, num_seqs, gamma, vocab, temperature);
@@ -212,7 +215,7 @@ S3R_EXPORT s3r_status s3r_sample_tokens(const void* logits, s3r_dtype logit_dtyp
   if (logit_dtype != S3R_F32 && logit_dtype != S3R_BF16) return S3R_ERR_INVALID_ARG;
   if (num_rows < 1 || vocab < 1) return S3R_ERR_INVALID_ARG;
   if (!(temperature > 0.0f) || !std::isfinite(temperature)) return S3R_ERR_INVALID_ARG;
-  const SamplePlan pl = plan_sampling(num_rows, 0, vocab);
+  const SamplePlan pl = plan_sampling(num_rows, 0, vocab, logit_dtype == S3R_BF16 ? 2 : 4);
   if (!workspace || workspace_bytes < pl.ws_bytes) return S3R_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   SampleParams p = make_sample_params(pl, workspace, num_rows, 0, vocab, temperature);

@@ -111,7 +111,8 @@ struct SamplePlan {
   size_t off_part1, off_stats, off_znorm, off_zpart, off_wpart, off_cmax;
   size_t memset_bytes;  // bytes from the start of the workspace cleared per call
 };
-SamplePlan plan_sampling(int32_t nseq, int32_t gamma, int32_t vocab);
+// elt: bytes per logit (2 for bf16, 4 for fp32); the chunking depends on it.
+SamplePlan plan_sampling(int32_t nseq, int32_t gamma, int32_t vocab, int32_t elt);
 
 struct SampleParams {
   const void* target;      // spec: [S, R, V]; plain: [N, V]

@@ -60,7 +60,7 @@ S3R_EXPORT s3r_status s3r_spec_sample_noalloc(const void* target_logits, const v
   if (num_seqs < 1 || vocab < 1 || gamma < 1) return S3R_ERR_INVALID_ARG;
   if (!(temperature > 0.0f) || !std::isfinite(temperature)) return S3R_ERR_INVALID_ARG;
   if (gamma > kMaxGamma) return S3R_ERR_UNSUPPORTED;
-  const SamplePlan pl = plan_sampling(num_seqs, gamma, vocab);
+  const SamplePlan pl = plan_sampling(num_seqs, gamma, vocab, logit_dtype == S3R_BF16 ? 2 : 4);
   if (pl.ws_bytes > kStaticScratchBytes) return S3R_ERR_UNSUPPORTED;     // batch too large for the array
   s3r_status s;
   uint8_t* w = static_cast<uint8_t*>(scratch_on_current_device(&s));

@@ -41,6 +41,8 @@ constexpr int kSmpThreads = 256;
 constexpr int kSmpWarps = kSmpThreads / 32;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kWarpSegs = kSmpWarps;         // pass-2 chunk = 8 contiguous warp segments
+constexpr int kDrawCtasPerSm = 3;            // pass-2 CTAs resident per SM (registers, 72 KB staging)
+constexpr int kStatsCtasPerSm = 4;           // pass-1 CTAs resident per SM (registers)
 constexpr uint32_t kCopyPiece = 16384;       // bytes per bulk-copy instruction
 
 struct Part1 {
@@ -244,7 +246,7 @@ __device__ void decide(const SampleParams& p, int b) {
 // calculation for softmax", 2018); four 16-byte loads in flight per thread.
 // VEC: rows 16-byte aligned with a length that is a multiple of the vector.
 template <typename T, bool VEC>
-__global__ void __launch_bounds__(kSmpThreads, 5) rowstats_kernel(const SampleParams p) {
+__global__ void __launch_bounds__(kSmpThreads, kStatsCtasPerSm) rowstats_kernel(const SampleParams p) {
   pdl_launch_dependents();
   pdl_wait();
   __shared__ float s_redf[kSmpWarps];
@@ -272,10 +274,11 @@ __global__ void __launch_bounds__(kSmpThreads, 5) rowstats_kernel(const SamplePa
 #pragma unroll
     for (int b = 0; b < kB; ++b) {
       if (cnt[b] <= 0) continue;
+      const bool full = VEC || cnt[b] == PV;            // VEC: whole vectors only
       float vm = -INFINITY;
 #pragma unroll
       for (int t = 0; t < PV; ++t)
-        if (t < cnt[b]) vm = fmaxf(vm, v[b][t]);
+        if (full || t < cnt[b]) vm = fmaxf(vm, v[b][t]);
       if (vm > m) {
         s *= static_cast<double>(ex2((m - vm) * k2));   // from m = -inf: a factor 0 on s = 0
         m = vm;
@@ -285,7 +288,7 @@ __global__ void __launch_bounds__(kSmpThreads, 5) rowstats_kernel(const SamplePa
       // a vector's exponentials summed pairwise in float32, then added in float64
       float e[PV];
 #pragma unroll
-      for (int t = 0; t < PV; ++t) e[t] = t < cnt[b] ? ex2(fmaf(v[b][t], k2, nmk)) : 0.f;
+      for (int t = 0; t < PV; ++t) e[t] = (full || t < cnt[b]) ? ex2(fmaf(v[b][t], k2, nmk)) : 0.f;
 #pragma unroll
       for (int w = PV / 2; w > 0; w >>= 1)
 #pragma unroll
@@ -373,7 +376,9 @@ __device__ DrawRows draw_rows(const SampleParams& p, int s, int j) {
 
 // float64 draw weights of the n (<= kPerVec) elements at pa (and pb for a
 // residual): exp((a - Mp)/T) iZp, or max(that - exp((b - Mq)/T) iZq, 0).
-template <typename T, bool VEC>
+// G: elements whose exponentials are interleaved (fewer for two rows, to
+// bound the registers).
+template <typename T, bool VEC, int G = 4>
 __device__ __forceinline__ void weights(const DrawRows& w, const T* pa, const T* pb, int n, double invT,
                                         const double* tab, double* out) {
   using IO = LogitIO<T>;
@@ -381,7 +386,6 @@ __device__ __forceinline__ void weights(const DrawRows& w, const T* pa, const T*
   float a[PV], b[PV];
   load_vals<T, VEC>(pa, n, a);
   if (w.qrow) load_vals<T, VEC>(pb, n, b);
-  constexpr int G = 4;                                  // elements interleaved per group
   const double ca = -w.Mp * invT, cb = -w.Mq * invT;    // (x - M)/T as one fused multiply-add
 #pragma unroll
   for (int t0 = 0; t0 < PV; t0 += G) {
@@ -410,13 +414,13 @@ __device__ __forceinline__ void weights(const DrawRows& w, const T* pa, const T*
 template <typename T, bool VEC>
 __device__ __forceinline__ void weights_at(const DrawRows& w, int e, int n, double invT, const double* tab,
                                            double* out) {
-  weights<T, VEC>(w, static_cast<const T*>(w.prow) + e, w.qrow ? static_cast<const T*>(w.qrow) + e : nullptr, n,
+  weights<T, VEC, 2>(w, static_cast<const T*>(w.prow) + e, w.qrow ? static_cast<const T*>(w.qrow) + e : nullptr, n,
                   invT, tab, out);
 }
 
 // Pass 2a: exact float64 normalisers of the residual's two rows.
 template <typename T, bool STAGE>
-__global__ void __launch_bounds__(kSmpThreads) znorm_kernel(const SampleParams p) {
+__global__ void __launch_bounds__(kSmpThreads, kDrawCtasPerSm) znorm_kernel(const SampleParams p) {
   pdl_launch_dependents();
   pdl_wait();
   extern __shared__ __align__(16) uint8_t s_dyn[];
@@ -615,7 +619,7 @@ __device__ int block_find(const DrawRows& w, int b0, int b1, double base, double
 // the chunk sums to the row maximum with an exact float64 factor when the
 // chunks are merged, so they need no statistics pass.
 template <typename T, bool SPEC, bool STAGE>
-__global__ void __launch_bounds__(kSmpThreads) draw_kernel(const SampleParams p) {
+__global__ void __launch_bounds__(kSmpThreads, kDrawCtasPerSm) draw_kernel(const SampleParams p) {
   pdl_launch_dependents();
   pdl_wait();
   extern __shared__ __align__(16) uint8_t s_dyn[];
@@ -668,7 +672,7 @@ __global__ void __launch_bounds__(kSmpThreads) draw_kernel(const SampleParams p)
   double acc = 0.0;
   for (int i = sb0 + lane * PV; i < sb1; i += 32 * PV) {
     double wv[PV];
-    weights<T, STAGE>(w, ca + i, cb ? cb + i : nullptr, min(PV, sb1 - i), p.inv_temp_d, s_tab, wv);
+    weights<T, STAGE, SPEC ? 2 : 4>(w, ca + i, cb ? cb + i : nullptr, min(PV, sb1 - i), p.inv_temp_d, s_tab, wv);
 #pragma unroll
     for (int t = 0; t < PV; ++t) acc += wv[t];
   }
@@ -808,17 +812,16 @@ cudaError_t launch_typed(const SampleParams& p, cudaStream_t st) {
 
 }  // namespace
 
-SamplePlan plan_sampling(int32_t nseq, int32_t gamma, int32_t vocab) {
+SamplePlan plan_sampling(int32_t nseq, int32_t gamma, int32_t vocab, int32_t elt) {
   SamplePlan pl{};
   pl.nseq = nseq;
   pl.nrows = nseq * (gamma > 0 ? 2 * gamma + 1 : 1);
-  // pass 1 (streamed, no shared memory): at most 32768 elements per CTA, and
-  // no more CTAs than fit at once (5 per SM) unless the rows need them; at
-  // least 256 elements per CTA
-  const int max_per_cta = kSmpThreads * 128;
-  const int target = 148 * 4;
+  // pass 1 (streamed, no shared memory): at most 40960 elements per CTA, and
+  // no more CTAs than fit at once unless the rows need them; at least 256
+  // elements per CTA
+  const int max_per_cta = kSmpThreads * 160;
   int c1 = (vocab + max_per_cta - 1) / max_per_cta;
-  const int want = 148 * 5 / pl.nrows;
+  const int want = 148 * kStatsCtasPerSm / pl.nrows;
   if (want > c1) c1 = want;
   const int cap = (vocab + 255) / 256;
   if (c1 > cap) c1 = cap;
@@ -826,13 +829,25 @@ SamplePlan plan_sampling(int32_t nseq, int32_t gamma, int32_t vocab) {
   pl.ch1 = (int)align_up((size_t)((vocab + c1 - 1) / c1), 8);
   if (pl.ch1 > max_per_cta) pl.ch1 = max_per_cta;
   pl.c1 = (vocab + pl.ch1 - 1) / pl.ch1;
-  // pass 2: about 4 CTAs per SM, 2048 to 8192 elements per CTA (two staged
-  // fp32 rows fit in 64 KB of shared memory); a chunk is 8 warp segments
-  // whose length is a multiple of 32 lanes x 8 elements
-  int c2 = (target + nseq - 1) / nseq;
+  // pass 2 (staged): at least 2048 elements per CTA; a chunk is 8 warp
+  // segments whose length is a multiple of 32 lanes x 8 elements.
+  // Speculative draws (two rows per CTA), and plain draws (one row) whose
+  // rows alone fill the GPU: no more CTAs than fit at once (three per SM),
+  // unless a chunk would stage more than 72 KB. Fewer plain rows: about 4
+  // CTAs per SM, at most 8192 elements each (smaller chunks overlap one CTA's
+  // copy with another's arithmetic, which measured faster there).
   const int cap2 = (vocab + 2047) / 2048;
-  if (c2 > cap2) c2 = cap2;
-  if (c2 < (vocab + 8191) / 8192) c2 = (vocab + 8191) / 8192;
+  int c2;
+  if (gamma > 0 || nseq >= 148 * kDrawCtasPerSm) {
+    const int max_chunk = 72 * 1024 / ((gamma > 0 ? 2 : 1) * elt) / 2048 * 2048;
+    c2 = 148 * kDrawCtasPerSm / nseq;
+    if (c2 > cap2) c2 = cap2;
+    if (c2 < (vocab + max_chunk - 1) / max_chunk) c2 = (vocab + max_chunk - 1) / max_chunk;
+  } else {
+    c2 = (148 * 4 + nseq - 1) / nseq;
+    if (c2 > cap2) c2 = cap2;
+    if (c2 < (vocab + 8191) / 8192) c2 = (vocab + 8191) / 8192;
+  }
   if (c2 < 1) c2 = 1;
   pl.ch2 = (int)align_up((size_t)((vocab + c2 - 1) / c2), (size_t)kWarpSegs * 32 * 8);
   pl.c2 = (vocab + pl.ch2 - 1) / pl.ch2;
