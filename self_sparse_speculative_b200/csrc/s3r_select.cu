@@ -69,11 +69,13 @@ struct SelParams {
   const void* kmin;
   const void* kmax;         // [num_pages_total, Hkv, D]
   const void* k_cache;      // [num_pages_total, Hkv, P, D] (the tail page's summary is taken from it)
+  const void* v_cache;      // [num_pages_total, Hkv, P, D] (only prefetched into L2)
   const int32_t* block_table;
   const int32_t* context_lens;
   int32_t* selected;        // [S, Hkv, budget]
   int32_t* selected_phys;   // [S, Hkv, budget] physical ids of the selected pages (-1: none)
   int32_t S, Hq, Hkv, G, D, P, max_pages, num_pages_total, budget;
+  int32_t elt;              // bytes per K/V element
   uint32_t* status;
 };
 
@@ -149,6 +151,18 @@ __host__ __device__ constexpr int sel_unroll() { return sizeof(T) * CPL * 32 * 2
 // [max_pages] (int).
 inline size_t sel_smem_bytes(int max_pages) { return (size_t)max_pages * 12; }
 
+// The attention kernel that follows streams the selected pages in list
+// order; the first kPrefetchPages of them (K and V) are prefetched into L2 as
+// soon as they are known, so its first stages do not wait for DRAM.
+constexpr int kPrefetchPages = 8;
+__device__ __forceinline__ void prefetch_page(const SelParams& p, int phys, int h) {
+  if (phys < 0 || phys >= p.num_pages_total) return;
+  const uint32_t bytes = static_cast<uint32_t>(p.P * p.D) * p.elt;
+  const size_t off = ((size_t)phys * p.Hkv + h) * bytes;
+  bulk_prefetch_l2(static_cast<const char*>(p.k_cache) + off, bytes);
+  bulk_prefetch_l2(static_cast<const char*>(p.v_cache) + off, bytes);
+}
+
 template <typename T, int CPL>
 __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelParams p) {
   extern __shared__ unsigned long long s_keys[];          // [max_pages] keys, then [max_pages] page ids
@@ -189,8 +203,10 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelParams 
     pdl_wait();
     if (rank == 0)
       for (int k = tid; k < p.budget; k += kSelThreads) {
+        const int ph = k < n_b ? p.block_table[(size_t)b * p.max_pages + k] : -1;
         out[k] = k < n_b ? k : -1;
-        out_phys[k] = k < n_b ? p.block_table[(size_t)b * p.max_pages + k] : -1;
+        out_phys[k] = ph;
+        if (k < kPrefetchPages) prefetch_page(p, ph, h);
       }
     return;
   }
@@ -453,6 +469,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelParams 
       if (take && pos < p.budget) {
         out[pos] = pg;
         out_phys[pos] = s_phys[pg];
+        if (pos < kPrefetchPages) prefetch_page(p, s_phys[pg], h);
         ++pos;
       }
     }
@@ -477,6 +494,7 @@ cudaError_t launch_select(const s3r_paged_kv& kv, const void* kmin, const void* 
   p.kmin = kmin;
   p.kmax = kmax;
   p.k_cache = kv.k_cache;
+  p.v_cache = kv.v_cache;
   p.block_table = kv.block_table;
   p.context_lens = kv.context_lens;
   p.selected = selected;
@@ -490,6 +508,7 @@ cudaError_t launch_select(const s3r_paged_kv& kv, const void* kmin, const void* 
   p.max_pages = kv.max_pages_per_seq;
   p.num_pages_total = kv.num_pages_total;
   p.budget = budget;
+  p.elt = kv.dtype == S3R_BF16 ? 2 : 4;
   p.status = status;
   // cluster size: the largest of 4, 2, 1 CTAs per (sequence, KV head) such
   // that every CTA of the launch is resident at once (two per SM), and no
