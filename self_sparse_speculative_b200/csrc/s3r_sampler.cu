@@ -387,6 +387,18 @@ __device__ __forceinline__ void weights(const DrawRows& w, const T* pa, const T*
   load_vals<T, VEC>(pa, n, a);
   if (w.qrow) load_vals<T, VEC>(pb, n, b);
   const double ca = -w.Mp * invT, cb = -w.Mq * invT;    // (x - M)/T as one fused multiply-add
+  // Every argument is <= 0 (shift = a maximum), so exp_tbl needs its fix-up
+  // only below -707: decided once per vector from its smallest value. VEC
+  // vectors are whole (n == PV).
+  float amin = a[0], bmin = w.qrow ? b[0] : 0.f;
+#pragma unroll
+  for (int t = 1; t < PV; ++t)
+    if (VEC || t < n) {
+      amin = fminf(amin, a[t]);
+      if (w.qrow) bmin = fminf(bmin, b[t]);
+    }
+  const bool in_range = fma(static_cast<double>(amin), invT, ca) > -707.0 &&
+                        (!w.qrow || fma(static_cast<double>(bmin), invT, cb) > -707.0);
 #pragma unroll
   for (int t0 = 0; t0 < PV; t0 += G) {
     double xa[G], xb[G], ea[G], eb[G];
@@ -399,15 +411,22 @@ __device__ __forceinline__ void weights(const DrawRows& w, const T* pa, const T*
         eb[t] = exp_tbl(xb[t], tab);
       }
     }
+    if (!in_range) {
+#pragma unroll
+      for (int t = 0; t < G; ++t) {
+        ea[t] = exp_fixup(xa[t], ea[t], tab);
+        if (w.qrow) eb[t] = exp_fixup(xb[t], eb[t], tab);
+      }
+    }
 #pragma unroll
     for (int t = 0; t < G; ++t) {
-      const double pe = exp_fixup(xa[t], ea[t], tab) * w.iZp;
+      const double pe = ea[t] * w.iZp;
       double wt = pe;
       if (w.qrow) {
-        const double qe = exp_fixup(xb[t], eb[t], tab) * w.iZq;
+        const double qe = eb[t] * w.iZq;
         wt = pe > qe ? pe - qe : 0.0;
       }
-      out[t0 + t] = t0 + t < n ? wt : 0.0;
+      out[t0 + t] = (VEC || t0 + t < n) ? wt : 0.0;
     }
   }
 }
@@ -459,6 +478,17 @@ __global__ void __launch_bounds__(kSmpThreads, kDrawCtasPerSm) znorm_kernel(cons
     float a[PV], b[PV];
     load_vals<T, STAGE>(pa + i, m, a);
     load_vals<T, STAGE>(pb + i, m, b);
+    // arguments are <= 0: the exp_tbl fix-up only below -707, decided per
+    // vector (staged vectors are whole)
+    float amin = a[0], bmin = b[0];
+#pragma unroll
+    for (int t = 1; t < PV; ++t)
+      if (STAGE || t < m) {
+        amin = fminf(amin, a[t]);
+        bmin = fminf(bmin, b[t]);
+      }
+    const bool in_range = fma(static_cast<double>(amin), p.inv_temp_d, ca) > -707.0 &&
+                          fma(static_cast<double>(bmin), p.inv_temp_d, cb) > -707.0;
 #pragma unroll
     for (int t0 = 0; t0 < PV; t0 += 4) {
       double xa[4], xb[4], ea[4], eb[4];
@@ -469,11 +499,18 @@ __global__ void __launch_bounds__(kSmpThreads, kDrawCtasPerSm) znorm_kernel(cons
         ea[t] = exp_tbl(xa[t], s_tab);
         eb[t] = exp_tbl(xb[t], s_tab);
       }
+      if (!in_range) {
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          ea[t] = exp_fixup(xa[t], ea[t], s_tab);
+          eb[t] = exp_fixup(xb[t], eb[t], s_tab);
+        }
+      }
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
-        if (t0 + t < m) {
-          zt += exp_fixup(xa[t], ea[t], s_tab);
-          zd += exp_fixup(xb[t], eb[t], s_tab);
+        if (STAGE || t0 + t < m) {
+          zt += ea[t];
+          zd += eb[t];
         }
       }
     }
