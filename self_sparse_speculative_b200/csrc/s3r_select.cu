@@ -93,6 +93,13 @@ __device__ __forceinline__ uint32_t cluster_rank() {
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
   return r;
 }
+// 16-byte global -> shared copy through L2 (cp.async; completion per thread
+// by commit groups)
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void st_cluster_u32(uint32_t local_addr, uint32_t rank, uint32_t v) {
   uint32_t remote;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
@@ -147,9 +154,12 @@ __device__ __forceinline__ float load_scalar(const float* p, int i) { return p[i
 template <typename T, int CPL>
 __host__ __device__ constexpr int sel_unroll() { return sizeof(T) * CPL * 32 * 2 > 512 ? 4 : 8; }
 
-// Dynamic shared memory: keys [max_pages] (u64), then physical page ids
-// [max_pages] (int).
-inline size_t sel_smem_bytes(int max_pages) { return (size_t)max_pages * 12; }
+// Dynamic shared memory: keys [max_pages] (u64), physical page ids
+// [max_pages] (int), then the tail page's K [P, D] (16-byte aligned).
+__host__ __device__ inline size_t sel_off_tailk(int max_pages) { return ((size_t)max_pages * 12 + 15) / 16 * 16; }
+inline size_t sel_smem_bytes(int max_pages, int P, int D, int elt) {
+  return sel_off_tailk(max_pages) + (size_t)P * D * elt;
+}
 
 // The attention kernel that follows streams the selected pages in list
 // order; the first kPrefetchPages of them (K and V) are prefetched into L2 as
@@ -238,50 +248,24 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelParams 
     s_ab[0][tid] = a;
     s_ab[1][tid] = z;
   }
-  if (has_tail) {
-    if (tail_phys >= 0 && tail_phys < p.num_pages_total) {
-      // thread = (token group, 16-byte chunk of channels); every load in
-      // flight at once, then the groups merge by shuffles and across warps
-      constexpr int VEC = 16 / sizeof(T);
-      const int chunks = p.D / VEC, groups = kSelThreads / chunks;
-      const int c = tid % chunks, grp = tid / chunks;
-      const int valid = L - tail * p.P;
-      const T* kt = static_cast<const T*>(p.k_cache) + ((size_t)tail_phys * p.Hkv + h) * p.P * p.D + c * VEC;
-      constexpr int kMaxPer = 8;                          // tokens per thread: P <= groups * 8
-      uint4 raw[kMaxPer];
+  // The tail page's valid tokens of K go to shared memory by cp.async now;
+  // they are reduced to the page's min / max after the other pages are scored.
+  constexpr int VEC = 16 / sizeof(T);
+  const int chunks = p.D / VEC, groups = kSelThreads / chunks;
+  const int tc = tid % chunks, tgrp = tid / chunks;
+  constexpr int kMaxPer = 8;                            // tokens per thread: P <= groups * 8
+  const bool tail_ok = has_tail && tail_phys >= 0 && tail_phys < p.num_pages_total;
+  const int valid = L - tail * p.P;
+  const T* s_tk = reinterpret_cast<const T*>(reinterpret_cast<const uint8_t*>(s_keys) + sel_off_tailk(p.max_pages));
+  if (tail_ok) {
+    const T* kt = static_cast<const T*>(p.k_cache) + ((size_t)tail_phys * p.Hkv + h) * p.P * p.D + tc * VEC;
+    const uint32_t dst = smem_addr(s_tk + tc * VEC);
 #pragma unroll
-      for (int k = 0; k < kMaxPer; ++k) {
-        const int t = grp + k * groups;
-        if (t < valid) raw[k] = __ldg(reinterpret_cast<const uint4*>(kt + (size_t)t * p.D));
-      }
-      float mn[VEC], mx[VEC];
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) { mn[e] = INFINITY; mx[e] = -INFINITY; }
-#pragma unroll
-      for (int k = 0; k < kMaxPer; ++k) {
-        if (grp + k * groups >= valid) continue;
-        float v[VEC];
-        unpack16<T>(raw[k], v);
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) { mn[e] = fminf(mn[e], v[e]); mx[e] = fmaxf(mx[e], v[e]); }
-      }
-      for (int o = chunks; o < 32; o <<= 1)
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) {
-          mn[e] = fminf(mn[e], __shfl_xor_sync(0xffffffffu, mn[e], o));
-          mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xffffffffu, mx[e], o));
-        }
-      if (lane < chunks)
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) { s_tpart[0][warp][c * VEC + e] = mn[e]; s_tpart[1][warp][c * VEC + e] = mx[e]; }
-      __syncthreads();
-      if (tid < p.D) {
-        float a = INFINITY, z = -INFINITY;
-        for (int w = 0; w < kSelWarps; ++w) { a = fminf(a, s_tpart[0][w][tid]); z = fmaxf(z, s_tpart[1][w][tid]); }
-        s_tail[0][tid] = a;
-        s_tail[1][tid] = z;
-      }
+    for (int k = 0; k < kMaxPer; ++k) {
+      const int t = tgrp + k * groups;
+      if (t < valid) cp_async16(dst + (uint32_t)(t * p.D * (int)sizeof(T)), kt + (size_t)t * p.D);
     }
+    cp_async_commit();
   }
   __syncthreads();
   pdl_wait();                                           // earlier kernels may write the summaries
@@ -314,18 +298,13 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelParams 
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
       const int pg = pg0 + u;
-      if (pg >= end) continue;                            // warp-uniform
+      if (pg >= end || pg == tail) continue;              // warp-uniform; the tail page is scored last
       const bool ok = page_ok(pg);
       double acc = 0.0;
       if (ok) {
         float l[CPL], r[CPL];
-        if (pg == tail) {                                 // this CTA's own summary of the tail page
-#pragma unroll
-          for (int c = 0; c < CPL; ++c) { l[c] = s_tail[0][lane * CPL + c]; r[c] = s_tail[1][lane * CPL + c]; }
-        } else {
-          RawRow<T, CPL>::unpack(lo[u], l);
-          RawRow<T, CPL>::unpack(hi[u], r);
-        }
+        RawRow<T, CPL>::unpack(lo[u], l);
+        RawRow<T, CPL>::unpack(hi[u], r);
         double acc1 = 0.0;
 #pragma unroll
         for (int c = 0; c < CPL; ++c) {
@@ -346,6 +325,63 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelParams 
     Raw lo[kU], hi[kU];
     load(pg0, lo, hi);
     score(pg0, lo, hi);
+  }
+  // ---- the tail page: min / max over its valid tokens from the staged K
+  // (thread = token group x 16-byte chunk of channels; the groups merge by
+  // shuffles and across warps), then its score (warp 0)
+  if (has_tail) {
+    if (tail_ok) {
+      cp_async_wait_all();
+      __syncthreads();
+      float mn[VEC], mx[VEC];
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) { mn[e] = INFINITY; mx[e] = -INFINITY; }
+#pragma unroll
+      for (int k = 0; k < kMaxPer; ++k) {
+        const int t = tgrp + k * groups;
+        if (t >= valid) continue;
+        float v[VEC];
+        unpack16<T>(*reinterpret_cast<const uint4*>(s_tk + t * p.D + tc * VEC), v);
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) { mn[e] = fminf(mn[e], v[e]); mx[e] = fmaxf(mx[e], v[e]); }
+      }
+      for (int o = chunks; o < 32; o <<= 1)
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+          mn[e] = fminf(mn[e], __shfl_xor_sync(0xffffffffu, mn[e], o));
+          mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xffffffffu, mx[e], o));
+        }
+      if (lane < chunks)
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) { s_tpart[0][warp][tc * VEC + e] = mn[e]; s_tpart[1][warp][tc * VEC + e] = mx[e]; }
+      __syncthreads();
+      if (tid < p.D) {
+        float a = INFINITY, z = -INFINITY;
+        for (int w = 0; w < kSelWarps; ++w) { a = fminf(a, s_tpart[0][w][tid]); z = fmaxf(z, s_tpart[1][w][tid]); }
+        s_tail[0][tid] = a;
+        s_tail[1][tid] = z;
+      }
+      __syncthreads();
+    }
+    if (warp == 0) {
+      double acc = 0.0;
+      if (tail_ok) {
+        double acc1 = 0.0;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+          const float l = s_tail[0][lane * CPL + c], r = s_tail[1][lane * CPL + c];
+          acc = fma(wa[c], static_cast<double>(fmaxf(l, r)), acc);
+          acc1 = fma(wb[c], static_cast<double>(fminf(l, r)), acc1);
+        }
+        acc += acc1;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (lane == 0) {
+        if (!tail_ok) flag_status(p.status, S3R_DEV_BAD_PAGE_ID);
+        s_keys[tail] = tail_ok ? order_key(acc) : 0ull;
+      }
+    }
   }
   __syncthreads();
   // ---- copy this CTA's keys into the first CTA (distributed shared memory)
@@ -478,7 +514,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelParams 
 
 template <typename T, int CPL>
 cudaError_t launch_typed(const SelParams& p, int cl, cudaStream_t st) {
-  const size_t smem = sel_smem_bytes(p.max_pages);
+  const size_t smem = sel_smem_bytes(p.max_pages, p.P, p.D, (int)sizeof(T));
   cudaError_t e = cudaFuncSetAttribute(select_kernel<T, CPL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   return launch_kernel(select_kernel<T, CPL>, dim3(cl, p.Hkv, p.S), dim3(kSelThreads), smem, st, cl, p);
