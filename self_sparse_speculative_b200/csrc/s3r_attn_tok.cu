@@ -86,9 +86,10 @@ __device__ __forceinline__ float warp_rows_reduce(float* v, int lane) {
     }
   }
   float r = v[0];
-  if constexpr (C == 16) {
-    const float o = __shfl_xor_sync(0xffffffffu, r, 16);
-    r = kMax ? fmaxf(r, o) : r + o;
+#pragma unroll
+  for (int o = C; o < 32; o <<= 1) {                  // lanes that hold the same row
+    const float x = __shfl_xor_sync(0xffffffffu, r, o);
+    r = kMax ? fmaxf(r, x) : r + x;
   }
   return r;
 }
@@ -102,9 +103,16 @@ __device__ __forceinline__ void wg_rows_reduce(float* v, float (*s_red)[64], flo
     if (N - c0 >= 32) {
       const float r = warp_rows_reduce<32, kMax>(v + c0, lane);
       s_red[q4][c0 + lane] = r;
-    } else {
+    } else if (N - c0 >= 16) {
       const float r = warp_rows_reduce<16, kMax>(v + c0, lane);
       if (lane < 16) s_red[q4][c0 + lane] = r;
+      if (N - c0 > 16) {
+        const float r8 = warp_rows_reduce<8, kMax>(v + c0 + 16, lane);
+        if (lane < 8) s_red[q4][c0 + 16 + lane] = r8;
+      }
+    } else {
+      const float r = warp_rows_reduce<8, kMax>(v + c0, lane);
+      if (lane < 8) s_red[q4][c0 + lane] = r;
     }
   }
   asm volatile("bar.sync 1, 128;" ::: "memory");
@@ -122,7 +130,11 @@ __device__ __forceinline__ int wg_count(bool pred) {
   return r;
 }
 
-template <int N, int D>
+// N: packed rows of the MMA (a multiple of 16); NR <= N: rows the softmax
+// handles (the real rows rounded up to 8). Columns NR..N-1 of S^T and O^T
+// belong to padding rows (zero queries): their P is zero and they are never
+// read back.
+template <int N, int NR, int D>
 __global__ void __launch_bounds__(kTokThreads, 1)
 attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                 const AttnParams p) {
@@ -435,6 +447,18 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
     q_fetch(sg);                                        // an input: no earlier kernel writes it
     pdl_wait();
     q_store();
+    if constexpr (NR < N) {
+      // P rows NR..N-1 (padding) are zero in both buffers for the whole run;
+      // the first stage's proxy fence publishes these writes with its P
+      const int half = tid >> 6, tt = tid & 63, ck = tt >> 3;
+#pragma unroll
+      for (int b2 = 0; b2 < PB; ++b2) {
+        uint8_t* pb = sP + b2 * L::kPBytes + half * (N * 128) + (tt & 7) * 2;
+#pragma unroll
+        for (int r = NR; r < N; ++r)
+          *reinterpret_cast<__nv_bfloat16*>(pb + r * 128 + ((ck ^ (r & 7)) << 4)) = __float2bfloat16_rn(0.f);
+      }
+    }
     int g = 0;
     bool ok = true;
     for (int x = lo; x < hi;) {
@@ -447,9 +471,9 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
       const int nst = (sg.npg + ppt - 1) / ppt;
       const int Lb = p.context_lens[sg.b];
       if (tid < N) s_nu[tid] = kNuInit;
-      float l[N];
+      float l[NR];
 #pragma unroll
-      for (int r = 0; r < N; ++r) l[r] = 0.f;
+      for (int r = 0; r < NR; ++r) l[r] = 0.f;
       asm volatile("bar.sync 1, 128;" ::: "memory");
       bool abort_all = false;
       for (int j = 0; j < nst; ++j, ++g) {
@@ -463,20 +487,20 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         const bool valid = lp >= 0 && pos < Lb;
         const int excess = pos - (Lb - p.R);
         const int nm = !valid ? N : (excess > 0 ? min(N, p.G * excess) : 0);
-        float s[N];
+        float s[NR];
         auto load_s = [&]() {
-          tmem_ld_cols<N>(tmem + lane_base + L::kColS + sb * N, s);
+          tmem_ld_cols<NR>(tmem + lane_base + L::kColS + sb * N, s);
           tmem_wait_ld();
           if (nm > 0) {
 #pragma unroll
-            for (int r = 0; r < N; ++r)
+            for (int r = 0; r < NR; ++r)
               if (r < nm) s[r] = -INFINITY;
           }
         };
         load_s();
         float ymax = -INFINITY;
 #pragma unroll
-        for (int r = 0; r < N; r += 4) {
+        for (int r = 0; r < NR; r += 4) {
           const float4 v = *reinterpret_cast<const float4*>(&s_nu[r]);
           ymax = fmaxf(fmaxf(ymax, fmaf(s[r], c, v.x)), fmaf(s[r + 1], c, v.y));
           ymax = fmaxf(fmaxf(ymax, fmaf(s[r + 2], c, v.z)), fmaf(s[r + 3], c, v.w));
@@ -487,8 +511,8 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         if (cnt > 0) {
           if (wg_count(!ok) > 0) { abort_all = true; break; }
           // stage maximum per row (S^T is intact until PFULL), then reload
-          wg_rows_reduce<N, true>(s, s_red, s_mx, q4, lane, tid);
-          if (tid < N) {
+          wg_rows_reduce<NR, true>(s, s_red, s_mx, q4, lane, tid);
+          if (tid < NR) {
             const float m_old = -s_nu[tid];
             const float m_new = fmaxf(m_old, s_mx[tid] * c);
             s_alpha[tid] = ex2(m_old - m_new);
@@ -496,7 +520,7 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
           }
           asm volatile("bar.sync 1, 128;" ::: "memory");
 #pragma unroll
-          for (int r = 0; r < N; r += 4) {
+          for (int r = 0; r < NR; r += 4) {
             const float4 a = *reinterpret_cast<const float4*>(&s_alpha[r]);
             l[r] *= a.x; l[r + 1] *= a.y; l[r + 2] *= a.z; l[r + 3] *= a.w;
           }
@@ -505,7 +529,7 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         }
         // s <- P = 2^(s c - m_ref), row sums
 #pragma unroll
-        for (int r = 0; r < N; r += 4) {
+        for (int r = 0; r < NR; r += 4) {
           const float4 v = *reinterpret_cast<const float4*>(&s_nu[r]);
           s[r] = ex2(fmaf(s[r], c, v.x));
           s[r + 1] = ex2(fmaf(s[r + 1], c, v.y));
@@ -519,12 +543,12 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         if (gw >= 0) ok &= mbar_wait(BAR(B_ODONE + (gw & 1)), (gw >> 1) & 1, &s_abort, p.status);
         tc_fence_after();
         if (rescale_o) {
-          float o[N];
-          tmem_ld_cols<N>(tmem + lane_base + L::kColO, o);
+          float o[NR];
+          tmem_ld_cols<NR>(tmem + lane_base + L::kColO, o);
           tmem_wait_ld();
 #pragma unroll
-          for (int r = 0; r < N; ++r) o[r] *= s_alpha[r];
-          tmem_st_cols<N>(tmem + lane_base + L::kColO, o);
+          for (int r = 0; r < NR; ++r) o[r] *= s_alpha[r];
+          tmem_st_cols<NR>(tmem + lane_base + L::kColO, o);
           tmem_wait_st();
         }
         {
@@ -532,7 +556,7 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
           uint8_t* pb = sP + (g % PB) * L::kPBytes + half * (N * 128) + (tt & 7) * 2;
           const int ck = tt >> 3;
 #pragma unroll
-          for (int r = 0; r < N; ++r)
+          for (int r = 0; r < NR; ++r)
             *reinterpret_cast<__nv_bfloat16*>(pb + r * 128 + ((ck ^ (r & 7)) << 4)) = __float2bfloat16_rn(s[r]);
         }
         if (!valid) {
@@ -553,7 +577,7 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
       // ---- the last QK of this segment is done: stage the next segment's Q
       if (has_next) q_store();
       // ---- segment epilogue: row sums, then O^T / l
-      wg_rows_reduce<N, false>(l, s_red, s_alpha, q4, lane, tid);
+      wg_rows_reduce<NR, false>(l, s_red, s_alpha, q4, lane, tid);
       const bool single = sg.nseg == 1;
       const int slot_idx = sg.unit + blockIdx.x;          // partial slot of (unit, this CTA)
       const size_t rowbase = (size_t)(sg.b * p.R) * p.Hq + (size_t)sg.h * p.G;
@@ -572,19 +596,19 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
       tc_fence_after();
       asm volatile("bar.sync 1, 128;" ::: "memory");
       {
-        float o[N];
-        tmem_ld_cols<N>(tmem + lane_base + L::kColO, o);
+        float o[NR];
+        tmem_ld_cols<NR>(tmem + lane_base + L::kColO, o);
         tmem_wait_ld();
         if (d_mine >= 0) {
           if (single) {
             __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) + rowbase * D + d_mine;
 #pragma unroll
-            for (int r = 0; r < N; ++r)
+            for (int r = 0; r < NR; ++r)
               if (r < p.rows) dst[(size_t)s_roff[r] * D] = __float2bfloat16_rn(o[r] * s_alpha[r]);
           } else {
             float* dst = p.part_o + (size_t)slot_idx * p.rows * D + d_mine;
 #pragma unroll
-            for (int r = 0; r < N; ++r)
+            for (int r = 0; r < NR; ++r)
               if (r < p.rows) dst[(size_t)r * D] = o[r];
           }
         }
@@ -638,7 +662,7 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
   }
 }
 
-template <int N, int D>
+template <int N, int NR, int D>
 cudaError_t launch_tok(const s3r_paged_kv& kv, const AttnParams& p, cudaStream_t st, s3r_status* api) {
   CUtensorMap mk, mv;
   if (!make_cache_map(&mk, kv.k_cache, kv) || !make_cache_map(&mv, kv.v_cache, kv)) {
@@ -646,19 +670,21 @@ cudaError_t launch_tok(const s3r_paged_kv& kv, const AttnParams& p, cudaStream_t
     return cudaErrorInvalidValue;
   }
   const size_t smem = TokLay<N, D>::kDynBytes + 1024;
-  cudaError_t e = cudaFuncSetAttribute(attn_tok_kernel<N, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(attn_tok_kernel<N, NR, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int grid = device_sm_count();
   if (grid > kMaxPersistentCtas) grid = kMaxPersistentCtas;
-  return launch_kernel(attn_tok_kernel<N, D>, dim3(grid), dim3(kTokThreads), smem, st, 1, mk, mv, p);
+  return launch_kernel(attn_tok_kernel<N, NR, D>, dim3(grid), dim3(kTokThreads), smem, st, 1, mk, mv, p);
 }
 
+// MMA rows N: the packed rows rounded up to 16; softmax rows NR: to 8.
 template <int D>
 cudaError_t launch_tok_rows(const s3r_paged_kv& kv, const AttnParams& p, cudaStream_t st, s3r_status* api) {
-  if (p.rows <= 16) return launch_tok<16, D>(kv, p, st, api);
-  if (p.rows <= 32) return launch_tok<32, D>(kv, p, st, api);
-  if (p.rows <= 48) return launch_tok<48, D>(kv, p, st, api);
-  return launch_tok<64, D>(kv, p, st, api);
+  const bool half = (p.rows & 15) != 0 && (p.rows & 15) <= 8;
+  if (p.rows <= 16) return half ? launch_tok<16, 8, D>(kv, p, st, api) : launch_tok<16, 16, D>(kv, p, st, api);
+  if (p.rows <= 32) return half ? launch_tok<32, 24, D>(kv, p, st, api) : launch_tok<32, 32, D>(kv, p, st, api);
+  if (p.rows <= 48) return half ? launch_tok<48, 40, D>(kv, p, st, api) : launch_tok<48, 48, D>(kv, p, st, api);
+  return half ? launch_tok<64, 56, D>(kv, p, st, api) : launch_tok<64, 64, D>(kv, p, st, api);
 }
 
 }  // namespace

@@ -229,18 +229,40 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
          "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
          "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])));
 }
-// N consecutive columns (N a multiple of 16) of this warp's 32 lanes.
+// 32 lanes x 32 bits, 8 consecutive columns.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float* v) {
+  uint32_t r[8];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const float* v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+               :: "r"(taddr),
+                  "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+                  "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+                  "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])));
+}
+// N consecutive columns (N a multiple of 8) of this warp's 32 lanes.
 template <int N>
 __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float* v) {
+  static_assert(N % 8 == 0, "columns in multiples of 8");
 #pragma unroll
   for (int c = 0; c + 32 <= N; c += 32) tmem_ld32(taddr + c, v + c);
-  if constexpr (N % 32 == 16) tmem_ld16(taddr + (N - 16), v + (N - 16));
+  constexpr int c16 = N / 32 * 32;
+  if constexpr (N % 32 >= 16) tmem_ld16(taddr + c16, v + c16);
+  if constexpr (N % 16 == 8) tmem_ld8(taddr + (N - 8), v + (N - 8));
 }
 template <int N>
 __device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const float* v) {
+  static_assert(N % 8 == 0, "columns in multiples of 8");
 #pragma unroll
   for (int c = 0; c + 32 <= N; c += 32) tmem_st32(taddr + c, v + c);
-  if constexpr (N % 32 == 16) tmem_st16(taddr + (N - 16), v + (N - 16));
+  constexpr int c16 = N / 32 * 32;
+  if constexpr (N % 32 >= 16) tmem_st16(taddr + c16, v + c16);
+  if constexpr (N % 16 == 8) tmem_st8(taddr + (N - 8), v + (N - 8));
 }
 
 // 16 lanes x 256 bits, 8 repetitions (64 columns): thread t gets lanes
