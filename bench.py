@@ -149,9 +149,10 @@ def verify_source_hash():
     return h.hexdigest()[:16]
 
 
-def verify_traffic():
+def verify_traffic(workload=None):
     """DRAM bytes (read + write) per verify launch from the committed ncu
-    summary, or None when it was taken on other kernel sources."""
+    summary, or None when it was taken on other kernel sources or (given a
+    workload name) on another workload."""
     try:
         kv = {}
         with open(VERIFY_PROFILE) as f:
@@ -160,6 +161,8 @@ def verify_traffic():
                     k, v = line[2:].split(":", 1)
                     kv[k.strip()] = v.strip().strip("`")
         if kv.get("source hash") != verify_source_hash():
+            return None
+        if workload is not None and kv.get("workload") != workload:
             return None
         return int(kv["dram bytes per launch"])
     except Exception:
@@ -353,7 +356,7 @@ def run_ours(a):
         "roofline": {"bound": "hbm", "kernel": "verify attention (s3r_verify_attn)",
                      "achieved": round(verify_gbs, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(verify_gbs / peak, 4), "peak_kind": peak_kind,
-                     "traffic": verify_traffic(),
+                     "traffic": verify_traffic(ws.name),
                      "algorithmic_bytes_per_launch": nbytes["verify"]},
         "phases_ms": {"draft_token_draws": round(t_draw, 4), "sparse_draft_per_call": round(t_draft, 4),
                       "verify": round(t_verify, 4), "spec_sample": round(t_sample, 4)},

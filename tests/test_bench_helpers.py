@@ -1,0 +1,24 @@
+"""Host-side helpers of bench.py (no GPU)."""
+import pytest
+
+import bench
+from self_sparse_speculative_b200.step import algorithmic_bytes
+from self_sparse_speculative_b200.workloads import Workload, spec
+
+
+def test_profiled_traffic_is_reported_only_for_the_profiled_workload():
+    t = bench.verify_traffic()
+    if t is None:
+        pytest.skip("the committed verify summary was taken on other kernel sources")
+    assert bench.verify_traffic(spec(1).name) == t
+    # workload 3 moves the same verify bytes, but its launch was not profiled
+    assert algorithmic_bytes(Workload(spec(3), seed=0))["verify"] == \
+        algorithmic_bytes(Workload(spec(1), seed=0))["verify"]
+    for w in (0, 2, 3, 4):
+        assert bench.verify_traffic(spec(w).name) is None
+
+
+def test_launch_count_per_step():
+    # drafter draws, gamma x (select, attention), verify, statistics + normalisers + draw
+    assert bench.launches_per_step(spec(1)) == 1 + 2 * 4 + 1 + 3
+    assert bench.launches_per_step(spec(4)) == 1 + 2 * 8 + 1 + 3
