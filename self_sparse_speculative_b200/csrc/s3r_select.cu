@@ -173,8 +173,10 @@ __device__ __forceinline__ void prefetch_page(const SelParams& p, int phys, int 
   bulk_prefetch_l2(static_cast<const char*>(p.v_cache) + off, bytes);
 }
 
-template <typename T, int CPL>
-__global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelParams p) {
+// MINB: CTAs per SM the registers are bounded for (2, or 4 for launches with
+// more units than two per SM hold).
+template <typename T, int CPL, int MINB>
+__global__ void __launch_bounds__(kSelThreads, MINB) select_kernel(const SelParams p) {
   extern __shared__ unsigned long long s_keys[];          // [max_pages] keys, then [max_pages] page ids
   __shared__ __align__(16) double s_ab[2][128];         // A, B per channel
   __shared__ __align__(16) float s_tail[2][128];       // min / max of the tail page (this CTA's, if any)
@@ -512,12 +514,17 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelParams 
   }
 }
 
-template <typename T, int CPL>
-cudaError_t launch_typed(const SelParams& p, int cl, cudaStream_t st) {
+template <typename T, int CPL, int MINB>
+cudaError_t launch_minb(const SelParams& p, int cl, cudaStream_t st) {
   const size_t smem = sel_smem_bytes(p.max_pages, p.P, p.D, (int)sizeof(T));
-  cudaError_t e = cudaFuncSetAttribute(select_kernel<T, CPL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e =
+      cudaFuncSetAttribute(select_kernel<T, CPL, MINB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch_kernel(select_kernel<T, CPL>, dim3(cl, p.Hkv, p.S), dim3(kSelThreads), smem, st, cl, p);
+  return launch_kernel(select_kernel<T, CPL, MINB>, dim3(cl, p.Hkv, p.S), dim3(kSelThreads), smem, st, cl, p);
+}
+template <typename T, int CPL>
+cudaError_t launch_typed(const SelParams& p, int cl, bool four, cudaStream_t st) {
+  return four ? launch_minb<T, CPL, 4>(p, cl, st) : launch_minb<T, CPL, 2>(p, cl, st);
 }
 
 }  // namespace
@@ -547,17 +554,21 @@ cudaError_t launch_select(const s3r_paged_kv& kv, const void* kmin, const void* 
   p.elt = kv.dtype == S3R_BF16 ? 2 : 4;
   p.status = status;
   // cluster size: the largest of 4, 2, 1 CTAs per (sequence, KV head) such
-  // that every CTA of the launch is resident at once (two per SM), and no
-  // more CTAs than 64-page load rounds (larger clusters cannot all be
-  // co-scheduled, and a second wave doubles the time)
+  // that every CTA of the launch is resident at once, and no more CTAs than
+  // 64-page load rounds (larger clusters cannot all be co-scheduled, and a
+  // second wave doubles the time). Two CTAs per SM (registers for a round
+  // of loads without spills); when the units alone exceed that, the build
+  // bounded for four per SM (fewer waves: 299 against 314 us per draft call
+  // on the 256-sequence workload; slower where two per SM suffice).
   const long units = (long)kv.num_seqs * kv.num_kv_heads;
-  const long slots = 2L * device_sm_count();
+  const bool four = units > 2L * device_sm_count();
+  const long slots = (four ? 4L : 2L) * device_sm_count();
   int cl = 4;
   while (cl > 1 && (units * cl > slots || (cl - 1) * 64 >= kv.max_pages_per_seq)) cl >>= 1;
   const bool bf = kv.dtype == S3R_BF16;
   cudaError_t e;
-  if (kv.head_dim == 128) e = bf ? launch_typed<__nv_bfloat16, 4>(p, cl, st) : launch_typed<float, 4>(p, cl, st);
-  else e = bf ? launch_typed<__nv_bfloat16, 2>(p, cl, st) : launch_typed<float, 2>(p, cl, st);
+  if (kv.head_dim == 128) e = bf ? launch_typed<__nv_bfloat16, 4>(p, cl, four, st) : launch_typed<float, 4>(p, cl, four, st);
+  else e = bf ? launch_typed<__nv_bfloat16, 2>(p, cl, four, st) : launch_typed<float, 2>(p, cl, four, st);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
