@@ -140,12 +140,23 @@ VERIFY_SOURCES = ("s3r_attn_tok.cu", "s3r_attn_sched.cuh", "s3r_attn_common.cuh"
 VERIFY_PROFILE = os.path.join(HERE, "profiles", "verify_attn_tok_qwen3-8b-layer.md")
 
 
+def _code_only(text):
+    """Source text without comments, trailing blanks and empty lines, so that
+    the hash identifies the compiled code, not its commentary."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+
+
 def verify_source_hash():
+    """Hash of the verify kernel's sources (code only) that a committed ncu
+    summary names; traffic figures from another build are not reported."""
     import hashlib
     h = hashlib.sha256()
     for f in VERIFY_SOURCES:
-        with open(os.path.join(HERE, "self_sparse_speculative_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(HERE, "self_sparse_speculative_b200", "csrc", f), encoding="utf-8") as fh:
+            h.update(_code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 
@@ -160,7 +171,7 @@ def verify_traffic(workload=None):
                 if line.startswith("- ") and ":" in line:
                     k, v = line[2:].split(":", 1)
                     kv[k.strip()] = v.strip().strip("`")
-        if kv.get("source hash") != verify_source_hash():
+        if kv.get("source hash", "").split("`")[0].strip() != verify_source_hash():
             return None
         if workload is not None and kv.get("workload") != workload:
             return None

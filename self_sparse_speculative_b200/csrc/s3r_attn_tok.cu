@@ -12,11 +12,12 @@
 //   O^T += V^T P^T (M = D, N, K = 128 tokens),
 // both fp32 in TMEM: 16 MMA instructions per 128 tokens at D = 128, where a
 // rows-major M = 64 tile needs 24 and wastes most of its rows. The softmax
-// thread t owns token t of the stage (TMEM lane t of S^T) and all N rows of
-// it, so the per-row sums stay in registers, P^T is written one token per
-// thread, and the row maximum needs a cross-thread reduction only when some
-// score exceeds the row's reference by more than 2^8 (the reference is lazy:
-// O^T columns and the sums always share it, so the result is exact).
+// thread t owns token t of the stage (TMEM lane t of S^T) and the NR real
+// rows (rounded up to 8; N, the MMA's, is a multiple of 16), so the per-row
+// sums stay in registers, P^T is written one token per thread, and the row
+// maximum needs a cross-thread reduction only when some score exceeds the
+// row's reference by more than 2^8 (the reference is lazy: O^T columns and
+// the sums always share it, so the result is exact).
 //
 // Work partition (stream-K): the flattened (sequence, KV head, page) list is
 // split into one contiguous range per CTA (s3r_attn_sched.cuh); a unit split
@@ -25,9 +26,11 @@
 //
 // Warp roles (192 threads): warps 0-3 softmax and epilogue (thread = token);
 // warp 4 producer (page ids, TMA into an NS-stage ring; an L2 prefetch ahead
-// of the ring measured slower); warp 5 MMA issuer (QK two stages ahead of
-// PV) and TMEM owner. The softmax warps also stage each segment's Q (fetched
-// into registers one segment ahead).
+// of the ring measured slower); warp 5 MMA issuer and TMEM owner: it polls its
+// barriers and issues whichever MMA is ready (PV(k) once P(k) is written,
+// QK(k) once stage k has landed and PV(k - 2) is issued). Two P buffers where
+// they fit, so softmax(k) waits only for PV(k - 2). The softmax warps also
+// stage each segment's Q (fetched into registers one segment ahead).
 #include <cuda_bf16.h>
 
 #include <cmath>

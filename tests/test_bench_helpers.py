@@ -22,3 +22,10 @@ def test_launch_count_per_step():
     # drafter draws, gamma x (select, attention), verify, statistics + normalisers + draw
     assert bench.launches_per_step(spec(1)) == 1 + 2 * 4 + 1 + 3
     assert bench.launches_per_step(spec(4)) == 1 + 2 * 8 + 1 + 3
+
+
+def test_source_hash_ignores_comments_and_blank_lines():
+    code = "int a;\nint b;"
+    assert bench._code_only(code) == code
+    assert bench._code_only("int a;   // the first\n\n/* a\n   block */\nint b;  \n") == code
+    assert bench._code_only("int a; int c;") != code
