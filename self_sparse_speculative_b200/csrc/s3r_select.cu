@@ -10,17 +10,21 @@
 //        sum_g max(q_g a, q_g b) = A max(a, b) + B min(a, b),
 //        A = sum_g max(q_g, 0),  B = sum_g min(q_g, 0),
 //      so a page costs 2 D float64 multiply-adds whatever G is (one warp per
-//      page, eight pages in flight per warp). The pages' order-preserving
-//      64-bit keys go into the shared memory of the cluster's first CTA
-//      (distributed shared memory);
+//      page, eight pages in flight per warp). The tail page n_b - 1, whose
+//      summary still changes while the sequence decodes, is summarised from K
+//      (staged by cp.async before the dependency wait) and scored last. The
+//      pages' order-preserving 64-bit keys and physical ids go into the shared
+//      memory of the cluster's first CTA (distributed shared memory);
 //   2. that CTA radix-selects the budget-th largest key (8-bit digits from the
-//      top: shared-memory histogram, one-warp scan of the 256 bins), stopping
-//      as soon as the boundary bin holds exactly the keys still needed (a
-//      rank count of every key against all others measured slower);
+//      first byte in which the keys differ: shared-memory histogram, one-warp
+//      scan of the 256 bins), stopping as soon as the boundary bin holds
+//      exactly the keys still needed (a rank count of every key against all
+//      others measured slower);
 //   3. it keeps the keys above the boundary plus the lowest-index pages on it,
-//      and writes them in ascending page order with block-wide prefix sums.
+//      writes them in ascending page order with block-wide prefix sums (the
+//      logical ids to `selected`, the physical ids for the attention kernel),
+//      and prefetches the first selected pages' K and V into L2.
 #include <cuda_bf16.h>
-
 
 #include "s3r_device.cuh"
 #include "s3r_internal.h"
