@@ -12,6 +12,10 @@ head_dim 128, 64-token pages, B = 32 pages, gamma = 4, vocab 151936, bf16),
 resident in HBM before timing. Metric: verified (committed) tokens per second
 = sum over sequences of (accepted drafts + 1) / step time.
 
+With one process and steps larger than L2, the line also carries "graph":
+the same round captured once into a CUDA graph (DecodeStep.capture_round)
+and replayed K times, device-timed (--no-graph skips it).
+
 Multi-GPU (torchrun, one rank per GPU): sequences are independent, so every
 rank runs its own full batch (weak scaling, no data-path collective); the
 step time is the max over ranks.
@@ -292,6 +296,33 @@ def run_ours(a):
 
     total_ms_max, tokens_all = over_ranks(total_ms, tokens, world, f"cuda:{local}")
 
+    # ---- the same round replayed from one captured CUDA graph (one process,
+    # steps larger than L2, so back-to-back replays read HBM): device time per
+    # replay; reported beside the eager value, which keeps the per-call phases
+    graph_info = None
+    if world == 1 and flush is None and not a.no_graph:
+        try:
+            graph = st.capture_round()
+            for _ in range(3):
+                graph.replay()
+            torch.cuda.synchronize()
+            g_s = torch.cuda.Event(enable_timing=True)
+            g_e = torch.cuda.Event(enable_timing=True)
+            g_s.record(stream)
+            for _ in range(a.steps):
+                graph.replay()
+            g_e.record(stream)
+            torch.cuda.synchronize()
+            g_ms = g_s.elapsed_time(g_e) / a.steps
+            del graph
+            gbad = {k: v for k, v in st.device_checks().items() if v[0] != s3r.S3R_OK}
+            if gbad:
+                raise RuntimeError(f"device checks failed after replays: {gbad}")
+            graph_info = {"ms_per_step": round(g_ms, 4), "value": round(tokens / a.steps / (g_ms / 1e3), 1),
+                          "unit": UNIT}
+        except Exception as exc:                       # reported, never fatal to the eager line
+            graph_info = {"error": f"{type(exc).__name__}: {exc}"[:200]}
+
     # ---- end to end: every step's inputs are copied from pinned host memory
     # and its committed tokens read back, through the public API; the upload
     # of step k+1 (copy stream, second input set) overlaps the compute of step k
@@ -378,6 +409,8 @@ def run_ours(a):
         "gpu_launches": launches_per_step(ws) * a.steps,
         "clocks": clk,
     }
+    if graph_info is not None:
+        line["graph"] = graph_info
     if e2e:
         line["e2e"] = {k: (round(v, 1) if isinstance(v, float) else v) for k, v in e2e.items()}
     if not a.no_cpu_baseline and world == 1:
@@ -435,6 +468,7 @@ def main():
     ap.add_argument("--cpu-seqs", type=int, default=8, help="sequences in the CPU oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay timing")
     a = ap.parse_args()
     if a.impl == "ours":
         a.warmup = max(3, a.warmup)     # at least 3 untimed warm-up steps

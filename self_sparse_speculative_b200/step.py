@@ -130,6 +130,20 @@ class DecodeStep:
         self.verify(stream)
         self.sample(stream)
 
+    def capture_round(self):
+        """One whole round captured into a CUDA graph. The library's kernels
+        chain by programmatic dependent launch, which the capture keeps as
+        programmatic edges; graph.replay() reruns the round on the same
+        buffers (the workspaces need no reset between rounds)."""
+        dev = self.device
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            self.round(side)
+        torch.cuda.current_stream(dev).wait_stream(side)
+        return graph
+
     def device_checks(self):
         """Status words of every workspace (synchronises)."""
         return {name: s3r.s3r_device_status(getattr(self, name))
