@@ -680,14 +680,16 @@ cudaError_t launch_tok(const s3r_paged_kv& kv, const AttnParams& p, cudaStream_t
   return launch_kernel(attn_tok_kernel<N, NR, D>, dim3(grid), dim3(kTokThreads), smem, st, 1, mk, mv, p);
 }
 
-// MMA rows N: the packed rows rounded up to 16; softmax rows NR: to 8.
+// MMA rows N: the packed rows rounded up to 16; softmax rows NR: to 8 for
+// N = 16 and 32 (the draft's G rows, verify's G (gamma + 1) rows of the
+// workloads), N itself for 48 and 64.
 template <int D>
 cudaError_t launch_tok_rows(const s3r_paged_kv& kv, const AttnParams& p, cudaStream_t st, s3r_status* api) {
   const bool half = (p.rows & 15) != 0 && (p.rows & 15) <= 8;
   if (p.rows <= 16) return half ? launch_tok<16, 8, D>(kv, p, st, api) : launch_tok<16, 16, D>(kv, p, st, api);
   if (p.rows <= 32) return half ? launch_tok<32, 24, D>(kv, p, st, api) : launch_tok<32, 32, D>(kv, p, st, api);
-  if (p.rows <= 48) return half ? launch_tok<48, 40, D>(kv, p, st, api) : launch_tok<48, 48, D>(kv, p, st, api);
-  return half ? launch_tok<64, 56, D>(kv, p, st, api) : launch_tok<64, 64, D>(kv, p, st, api);
+  if (p.rows <= 48) return launch_tok<48, 48, D>(kv, p, st, api);
+  return launch_tok<64, 64, D>(kv, p, st, api);
 }
 
 }  // namespace

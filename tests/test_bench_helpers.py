@@ -29,3 +29,12 @@ def test_source_hash_ignores_comments_and_blank_lines():
     assert bench._code_only(code) == code
     assert bench._code_only("int a;   // the first\n\n/* a\n   block */\nint b;  \n") == code
     assert bench._code_only("int a; int c;") != code
+
+
+def test_source_hash_covers_the_attention_device_code():
+    import os
+    path = os.path.join(os.path.dirname(bench.__file__), "self_sparse_speculative_b200", "csrc", "s3r_attn_tok.cu")
+    text = open(path, encoding="utf-8").read()
+    assert bench.HOST_SECTION in text                   # the host launch code follows the kernel
+    h = bench.verify_source_hash()
+    assert len(h) == 16 and int(h, 16) >= 0
