@@ -102,8 +102,12 @@ def test_sampling_argument_checks():
     assert call(T=0.0) == s3r.S3R_ERR_INVALID_ARG
     assert call(T=float("inf")) == s3r.S3R_ERR_INVALID_ARG
     assert call(V=0) == s3r.S3R_ERR_INVALID_ARG
-    assert call(wb=need - 1) == s3r.S3R_ERR_WORKSPACE
+    # a workspace below what either logit type needs (the size query covers both types,
+    # so need - 1 could still suffice for one of them and reach a launch)
+    assert call(wb=16) == s3r.S3R_ERR_WORKSPACE
+    assert call(wb=16, dt=s3r.S3R_F32) == s3r.S3R_ERR_WORKSPACE
     need_t = lib.s3r_sample_workspace_bytes(8, 0, 1000)
-    assert lib.s3r_sample_tokens(FAKE, s3r.S3R_F32, 8, 1000, 1.0, FAKE, FAKE, FAKE, need_t - 1, None) == s3r.S3R_ERR_WORKSPACE
+    assert need_t > 0
+    assert lib.s3r_sample_tokens(FAKE, s3r.S3R_F32, 8, 1000, 1.0, FAKE, FAKE, FAKE, 16, None) == s3r.S3R_ERR_WORKSPACE
     assert lib.s3r_sample_tokens(FAKE, s3r.S3R_F32, 0, 1000, 1.0, FAKE, FAKE, FAKE, need_t, None) == s3r.S3R_ERR_INVALID_ARG
     assert lib.s3r_device_status(None, None, None) == s3r.S3R_ERR_INVALID_ARG
