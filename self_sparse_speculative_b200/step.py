@@ -15,7 +15,8 @@ its own. A round, as the S3R page (weekinpapers.com, Abstract) describes it:
 The synthetic single-layer step has no model between these calls: the
 queries and logits are seeded inputs (workloads.Workload). The gamma draft
 tokens are drawn in one batched call at the start of the round (the same work
-as gamma single-row calls).
+as gamma single-row calls). capture_round() records the whole round into one
+CUDA graph for replay.
 """
 from __future__ import annotations
 
