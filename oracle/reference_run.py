@@ -15,7 +15,14 @@ Comparison rules:
   only the order of the float64 sums differs), or a page boundary whose
   scores differ by at most 1e-12 of the largest score is a near-tie: it is
   counted, and it and every later decision of that sequence are left out of
-  the exact comparison (the GPU's choice there is checked for validity).
+  the exact comparison. The GPU's choices there are still checked for
+  validity: a selection must be a top-B set up to the score band (every kept
+  score at least every dropped one minus the band); after a near-tie in the
+  sampling, the GPU's own draft tokens, accept decisions and drawn token are
+  walked in order, and each must be what the oracle decides for those same
+  tokens, or within the near-tie band of it (an accept needs u < p/q + band,
+  a reject u >= p/q - band, a draw a token of positive weight whose CDF
+  interval holds u up to the band).
 """
 from __future__ import annotations
 
@@ -60,9 +67,10 @@ def oracle_attention_seq(wl, b, draft_steps=None):
     draft = {}
     for i in steps:
         q = to_float64(wl.q_draft[i, b], ws.kv_dtype)[None]            # [1, Hq, D]
-        sel, gaps = O.sparse_draft_select(q, kmin, kmax, bt, lens, P, B, G)
+        sel, gaps, scores = O.sparse_draft_select(q, kmin, kmax, bt, lens, P, B, G, return_scores=True)
         out, lse = O.sparse_draft_attn(q, K, V, bt, lens, sel, scale)
-        draft[i] = {"selected": sel[0], "gaps": gaps[0], "out": out[0], "lse": lse[0], "q": q}
+        draft[i] = {"selected": sel[0], "gaps": gaps[0], "scores": scores[0], "out": out[0], "lse": lse[0],
+                    "q": q}
     qv = to_float64(wl.q_verify[b], ws.kv_dtype)[None]                  # [1, R, Hq, D]
     vout, vlse = O.verify_attn(qv, K, V, bt, lens, scale)
     return {"phys": phys, "kmin": kmin, "kmax": kmax, "draft": draft,
@@ -80,7 +88,27 @@ def oracle_sampling_seq(wl, b):
     out, n_acc, am, sm = O.spec_sample(tl[None], dl[None], x[None], wl.u_accept[b][None],
                                        wl.u_sample[b][None], T)
     return {"x": x, "x_margin": xm, "out_tokens": out[0], "n_acc": int(n_acc[0]),
-            "accept_margin": am[0], "sample_margin": float(sm[0])}
+            "accept_margin": am[0], "sample_margin": float(sm[0]),
+            # for the validity walk after a near-tie
+            "p": O.softmax_t(tl, T), "q": O.softmax_t(dl, T), "u_draft": wl.u_draft[b].astype(np.float64),
+            "u_accept": wl.u_accept[b].astype(np.float64), "u_sample": wl.u_sample[b].astype(np.float64)}
+
+
+def sampling_ref_from_logits(target_logits, draft_logits, u_draft, u_accept, u_sample, temperature):
+    """The same record as oracle_sampling_seq for one sequence's float64
+    logits and uniforms given directly (the draft tokens drawn from q with
+    u_draft)."""
+    T = f32(temperature)
+    tl = np.asarray(target_logits, dtype=np.float64)
+    dl = np.asarray(draft_logits, dtype=np.float64)
+    ud = np.asarray(u_draft, dtype=np.float64)
+    x, xm = O.sample_rows(dl, ud, T)
+    out, n_acc, am, sm = O.spec_sample(tl[None], dl[None], x[None], np.asarray(u_accept)[None],
+                                       np.asarray(u_sample)[None], T)
+    return {"x": x, "x_margin": xm, "out_tokens": out[0], "n_acc": int(n_acc[0]),
+            "accept_margin": am[0], "sample_margin": float(sm[0]),
+            "p": O.softmax_t(tl, T), "q": O.softmax_t(dl, T), "u_draft": ud,
+            "u_accept": np.asarray(u_accept, dtype=np.float64), "u_sample": np.asarray(u_sample, dtype=np.float64)}
 
 
 # ------------------------------------------------------------------ comparisons
@@ -110,8 +138,29 @@ def assert_close(name, gpu, ref, dtype):
                              f"oracle {ref[tuple(idx)]}; max err {np.nanmax(np.where(both_inf, 0, err)):.3e}")
 
 
+def valid_top_set(gpu_set, scores, budget):
+    """Whether gpu_set (ascending logical pages) is a top-`budget` set of
+    `scores` up to the near-tie band: the right size, distinct in-range pages
+    in ascending order, and every kept score >= every dropped score minus
+    NEAR_TIE_SCORE times the largest |score|."""
+    s = np.asarray(scores, dtype=np.float64)
+    n = len(s)
+    g = np.asarray(gpu_set, dtype=np.int64)
+    if len(g) != min(n, budget) or np.any(g < 0) or np.any(g >= n) or np.any(np.diff(g) <= 0):
+        return False
+    if len(g) == n:
+        return True
+    dropped = np.setdiff1d(np.arange(n), g)
+    band = NEAR_TIE_SCORE * float(np.abs(s).max())
+    return float(s[g].min()) >= float(s[dropped].max()) - band
+
+
 def compare_selection(name, gpu_sel, ref_sel, gaps, tally: Tally, scores=None):
-    """gpu_sel [Hkv, B] (-1 padded), ref_sel list of arrays, gaps [Hkv]."""
+    """gpu_sel [Hkv, B] (-1 padded), ref_sel list of arrays, gaps [Hkv],
+    scores [Hkv, n_b] (the oracle's page scores). Exact set equality, except
+    at a near-tie boundary, where the GPU's set must be a valid top-B set up
+    to the band (scores are required there). Returns per head whether the
+    sets are equal (attention outputs are comparable)."""
     ok_heads = []
     for h, rs in enumerate(ref_sel):
         tally.decisions += 1
@@ -120,7 +169,13 @@ def compare_selection(name, gpu_sel, ref_sel, gaps, tally: Tally, scores=None):
         if gaps[h] <= NEAR_TIE_SCORE:
             tally.near_ties += 1
             tally.notes.append(f"{name} head {h}: near-tie page boundary")
-            ok_heads.append(False)
+            if scores is None:
+                raise AssertionError(f"{name} head {h}: near-tie boundary but no scores to check the choice")
+            if not valid_top_set(g, scores[h], len(rs)):
+                raise AssertionError(f"{name} head {h}: gpu selection {g.tolist()} is not a top-B set "
+                                     f"within the near-tie band")
+            eq = np.array_equal(g, np.asarray(rs))
+            ok_heads.append(eq)
             continue
         if not np.array_equal(g, np.asarray(rs)):
             raise AssertionError(f"{name} head {h}: selected pages differ: gpu {g.tolist()} oracle {list(rs)}")
@@ -128,15 +183,65 @@ def compare_selection(name, gpu_sel, ref_sel, gaps, tally: Tally, scores=None):
     return ok_heads
 
 
+def valid_draw(weights, u, k, band=NEAR_TIE_DRAW):
+    """Whether token k is a valid inverse-CDF draw from the unnormalised
+    weights at uniform u, up to the band: positive weight, and
+    C(k-1)/C(V-1) - band <= u < C(k)/C(V-1) + band."""
+    w = np.asarray(weights, dtype=np.float64)
+    k = int(k)
+    if k < 0 or k >= len(w) or not w[k] > 0:
+        return False
+    C = np.cumsum(w)
+    lo = (C[k - 1] if k > 0 else 0.0) / C[-1]
+    hi = C[k] / C[-1]
+    return lo - band <= float(u) < hi + band
+
+
+def validity_walk(name, gpu_x, gpu_out, gpu_nacc, ref):
+    """Check the GPU's sampling of one sequence decision by decision against
+    the oracle's distributions, following the GPU's own choices (used after a
+    near-tie, where the two may legitimately part ways)."""
+    p, q = ref["p"], ref["q"]
+    gamma = q.shape[0]
+    x = np.asarray(gpu_x, dtype=np.int64)
+    out = np.asarray(gpu_out, dtype=np.int64)
+    n = int(gpu_nacc)
+    for i in range(gamma):
+        if not valid_draw(q[i], ref["u_draft"][i], x[i]):
+            raise AssertionError(f"{name}: draft token {i} = {int(x[i])} is not a valid draw from q_{i}")
+    if not 0 <= n <= gamma:
+        raise AssertionError(f"{name}: n_acc {n} outside [0, {gamma}]")
+    for i in range(min(n + 1, gamma)):
+        qx = q[i, x[i]]
+        ratio = p[i, x[i]] / qx if qx > 0 else 0.0
+        u = ref["u_accept"][i]
+        if i < n and not u < ratio + NEAR_TIE_DECISION:
+            raise AssertionError(f"{name}: accept {i} taken with u {u} >= p/q {ratio}")
+        if i == n and not u >= ratio - NEAR_TIE_DECISION:
+            raise AssertionError(f"{name}: reject {i} taken with u {u} < p/q {ratio}")
+    if not np.array_equal(out[:n], x[:n]):
+        raise AssertionError(f"{name}: committed drafts {out[:n].tolist()} differ from the drafts {x[:n].tolist()}")
+    w = p[gamma] if n == gamma else O.residual_weights(p[n], q[n])
+    if not valid_draw(w, ref["u_sample"][n], out[n]):
+        raise AssertionError(f"{name}: drawn token {int(out[n])} at position {n} is not a valid draw")
+    if np.any(out[n + 1:] != -1):
+        raise AssertionError(f"{name}: tokens after the drawn one are not -1: {out.tolist()}")
+
+
 def compare_sampling(name, gpu_x, gpu_out, gpu_nacc, ref, tally: Tally):
     """Exact comparison of one sequence's draft draws, accept decisions and
-    drawn token, leaving out everything downstream of a near-tie."""
+    drawn token. At the first near-tie the exact comparison stops (the
+    decision and everything after it may differ) and the GPU's choices are
+    checked for validity instead (validity_walk)."""
     gamma = len(ref["x"])
     for i in range(gamma):
         tally.decisions += 1
         if ref["x_margin"][i] < NEAR_TIE_DRAW:
             tally.near_ties += 1
             tally.notes.append(f"{name}: near-tie draft draw {i}")
+            if not np.array_equal(np.asarray(gpu_x[:i]), ref["x"][:i]):
+                raise AssertionError(f"{name}: draft tokens before the near-tie differ")
+            validity_walk(name, gpu_x, gpu_out, gpu_nacc, ref)
             return
         if int(gpu_x[i]) != int(ref["x"][i]):
             raise AssertionError(f"{name}: draft token {i} gpu {int(gpu_x[i])} oracle {int(ref['x'][i])}")
@@ -146,6 +251,9 @@ def compare_sampling(name, gpu_x, gpu_out, gpu_nacc, ref, tally: Tally):
         if ref["accept_margin"][i] < NEAR_TIE_DECISION:
             tally.near_ties += 1
             tally.notes.append(f"{name}: near-tie accept test {i}")
+            if int(gpu_nacc) < i:
+                raise AssertionError(f"{name}: n_acc {int(gpu_nacc)} stops before the near-tie test {i}")
+            validity_walk(name, gpu_x, gpu_out, gpu_nacc, ref)
             return
     if int(gpu_nacc) != n_ref:
         raise AssertionError(f"{name}: n_acc gpu {int(gpu_nacc)} oracle {n_ref}")
@@ -153,9 +261,7 @@ def compare_sampling(name, gpu_x, gpu_out, gpu_nacc, ref, tally: Tally):
     if ref["sample_margin"] < NEAR_TIE_DRAW:
         tally.near_ties += 1
         tally.notes.append(f"{name}: near-tie draw")
-        g = np.asarray(gpu_out)
-        if not np.array_equal(g[:n_ref], ref["out_tokens"][:n_ref]) or np.any(g[n_ref + 1:] != -1):
-            raise AssertionError(f"{name}: committed tokens around a near-tie draw differ")
+        validity_walk(name, gpu_x, gpu_out, gpu_nacc, ref)
         return
     if not np.array_equal(np.asarray(gpu_out), ref["out_tokens"]):
         raise AssertionError(f"{name}: out_tokens gpu {np.asarray(gpu_out).tolist()} "

@@ -182,12 +182,15 @@ def dense_decode(q, k_cache, v_cache, block_table, context_lens, scale):
     return o[:, 0], l[:, 0]
 
 
-def sparse_draft_select(q, kmin, kmax, block_table, context_lens, page_size, budget, group):
+def sparse_draft_select(q, kmin, kmax, block_table, context_lens, page_size, budget, group,
+                        return_scores=False):
     """Step (a2) for every sequence: selected [S][Hkv] arrays of logical page ids
-    (ascending) and the boundary score gaps [S, Hkv]."""
+    (ascending) and the boundary score gaps [S, Hkv] relative to the largest
+    |score| of the head. With return_scores, also the page scores [S] of
+    [Hkv, n_b] arrays (for checking a choice at a near-tie boundary)."""
     S = q.shape[0]
     H = kmin.shape[1]
-    sel, gaps = [], np.full((S, H), np.inf)
+    sel, gaps, scores = [], np.full((S, H), np.inf), []
     for b in range(S):
         n_b = -(-int(context_lens[b]) // page_size)
         phys = block_table[b, :n_b]
@@ -198,6 +201,9 @@ def sparse_draft_select(q, kmin, kmax, block_table, context_lens, page_size, bud
             row.append(c)
             gaps[b, h] = gap / max(1e-300, float(np.abs(sc[h]).max()))
         sel.append(row)
+        scores.append(sc)
+    if return_scores:
+        return sel, gaps, scores
     return sel, gaps
 
 
@@ -251,6 +257,16 @@ def sample_rows(logits, u, temperature):
     return inverse_cdf(softmax_t(logits, temperature), u)
 
 
+def residual_weights(p_j, q_j):
+    """The distribution drawn from after a rejection at position j: the
+    residual max(p_j - q_j, 0) (unnormalised; the draw normalises it), or p_j
+    itself where the residual is zero everywhere (reading: p = q makes a
+    rejection a probability-0 event, so any choice keeps the output exact).
+    Works row-wise over the last axis."""
+    resid = np.maximum(p_j - q_j, 0.0)
+    return np.where(resid.sum(axis=-1, keepdims=True) > 0, resid, p_j)
+
+
 def spec_sample(target_logits, draft_logits, draft_tokens, u_accept, u_sample, temperature):
     """Exact speculative sampling of one round, for every sequence.
 
@@ -289,9 +305,7 @@ def spec_sample(target_logits, draft_logits, draft_tokens, u_accept, u_sample, t
     j = n_acc
     p_j = p[np.arange(S), j]                                   # [S, V]
     q_j = q[np.arange(S), np.minimum(j, gamma - 1)]            # unused where j == gamma
-    resid = np.maximum(p_j - q_j, 0.0)
-    resid = np.where(resid.sum(axis=1, keepdims=True) > 0, resid, p_j)
-    w = np.where((j == gamma)[:, None], p_j, resid)
+    w = np.where((j == gamma)[:, None], p_j, residual_weights(p_j, q_j))
     us = np.asarray(u_sample, dtype=np.float64)[np.arange(S), j]
     k, sample_margin = inverse_cdf(w, us)
     out = np.where(gi < j[:, None], x, -1)

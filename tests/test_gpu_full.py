@@ -59,7 +59,8 @@ def test_full_attention_sampled_sequences(full_run):
         assert np.array_equal(kmin[ref["phys"]].astype(np.float64), ref["kmin"]), name
         assert np.array_equal(kmax[ref["phys"]].astype(np.float64), ref["kmax"]), name
         for i, d in ref["draft"].items():
-            ok = RR.compare_selection(f"{name} draft {i}", sel[i, b], d["selected"], d["gaps"], TALLY)
+            ok = RR.compare_selection(f"{name} draft {i}", sel[i, b], d["selected"], d["gaps"], TALLY,
+                                      scores=d["scores"])
             if all(ok):
                 RR.assert_close(f"{name} draft {i} out", st.draft_out[i, b].float().cpu().numpy(), d["out"], dt)
                 RR.assert_close(f"{name} draft {i} lse", st.draft_lse[i, b].cpu().numpy(), d["lse"], dt)

@@ -88,7 +88,8 @@ def test_selection_and_attention(case):
     for b in range(ws.num_seqs):
         ref = RR.oracle_attention_seq(wl, b)
         for i, d in ref["draft"].items():
-            ok = RR.compare_selection(f"{name} seq {b} draft {i}", sel[i, b], d["selected"], d["gaps"], tally)
+            ok = RR.compare_selection(f"{name} seq {b} draft {i}", sel[i, b], d["selected"], d["gaps"], tally,
+                                      scores=d["scores"])
             n_b = int(wl.pages_per_seq[b])
             assert np.all(sel[i, b][:, min(n_b, ws.budget_pages):] == -1)
             if all(ok):
@@ -242,7 +243,8 @@ def test_draft_summarises_the_tail_page_itself():
     for b in range(wl.spec.num_seqs):
         ref = RR.oracle_attention_seq(wl, b)
         for i, d in ref["draft"].items():
-            ok = RR.compare_selection(f"seq {b} draft {i}", sel[i, b], d["selected"], d["gaps"], tally)
+            ok = RR.compare_selection(f"seq {b} draft {i}", sel[i, b], d["selected"], d["gaps"], tally,
+                                      scores=d["scores"])
             if all(ok):
                 RR.assert_close(f"seq {b} draft {i} out", st.draft_out[i, b].float().cpu().numpy(), d["out"], "bf16")
     assert tally.near_ties <= max(0, int(1e-4 * tally.decisions)), tally.notes
