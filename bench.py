@@ -62,34 +62,86 @@ def _peaks():
 
 # ---------------------------------------------------------------- CPU oracle
 def _oracle_seq_worker(args):
+    """One sequence's float64 oracle round in a worker process. Its inputs
+    are generated first, outside the timer; only the oracle's arithmetic
+    (summaries, gamma selections and sparse drafts, verify, draft draws and
+    speculative sampling) is timed. Returns (committed tokens, seconds)."""
     idx, seed, b = args
-    os.environ.setdefault("OMP_NUM_THREADS", "1")
     from self_sparse_speculative_b200.workloads import Workload, spec
     import oracle.reference_run as RR
     wl = Workload(spec(idx), seed=seed)
+    inp = RR.sequence_inputs(wl, b)
     t0 = time.perf_counter()
-    RR.oracle_attention_seq(wl, b)
-    s = RR.oracle_sampling_seq(wl, b)
+    RR.oracle_attention(inp)
+    s = RR.oracle_sampling(inp)
     return s["n_acc"] + 1, time.perf_counter() - t0
 
 
-def oracle_sample(idx, seed, seqs, workers):
-    """Run the oracle round on the listed sequences; returns (tokens, wall s, cores)."""
-    import multiprocessing as mp
-    jobs = [(idx, seed, b) for b in seqs]
-    t0 = time.perf_counter()
-    if workers > 1:
-        ctx = mp.get_context("spawn")
-        with ctx.Pool(workers) as pool:
-            res = pool.map(_oracle_seq_worker, jobs)
-    else:
-        res = [_oracle_seq_worker(j) for j in jobs]
-    wall = time.perf_counter() - t0
-    return sum(r[0] for r in res), wall, workers
+# one BLAS thread per oracle process (the processes already take one core
+# each); set in the environment the spawned processes start with, since the
+# BLAS library reads it when numpy is first imported
+_ONE_THREAD = {"OMP_NUM_THREADS": "1", "OPENBLAS_NUM_THREADS": "1", "MKL_NUM_THREADS": "1"}
+
+
+class OracleRunner:
+    """A pool of `workers` single-threaded processes (spawned, so it is safe
+    whether or not the parent holds a CUDA context) that runs the oracle on
+    one sequence per process. A step's time is the slowest process's
+    arithmetic time: the processes run at once, one per core."""
+
+    def __init__(self, workers):
+        import multiprocessing as mp
+        self.workers = workers
+        self.pool = None
+        if workers > 1:
+            saved = {k: os.environ.get(k) for k in _ONE_THREAD}
+            os.environ.update(_ONE_THREAD)
+            try:
+                self.pool = mp.get_context("spawn").Pool(workers)
+            finally:
+                for k, v in saved.items():
+                    if v is None:
+                        os.environ.pop(k, None)
+                    else:
+                        os.environ[k] = v
+
+    def step(self, idx, seed, seqs):
+        jobs = [(idx, seed, b) for b in seqs]
+        res = self.pool.map(_oracle_seq_worker, jobs, chunksize=1) if self.pool else \
+            [_oracle_seq_worker(j) for j in jobs]
+        if self.pool is None:
+            return sum(r[0] for r in res), sum(r[1] for r in res)
+        # the processes run at once: the slowest one, or the arithmetic spread
+        # over the processes when sequences outnumber them
+        per = [r[1] for r in res]
+        return sum(r[0] for r in res), max(max(per), sum(per) / self.workers)
+
+    def close(self):
+        if self.pool is not None:
+            self.pool.close()
+            self.pool.join()
 
 
 def cpu_cores():
     return len(os.sched_getaffinity(0))
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def oracle_sample_note(ws, seqs, steps, cores):
+    return (f"float64 oracle round (summaries, {ws.gamma} sparse drafts, verify, draft draws, speculative "
+            f"sampling) of {len(seqs)} of {ws.num_seqs} sequences per step, {steps} step(s), one process "
+            f"per sequence on {cores} of {cpu_cores()} host cores ({cpu_model()}); inputs generated "
+            f"before the timer, only the oracle arithmetic timed")
 
 
 # ---------------------------------------------------------------- clocks
@@ -232,7 +284,28 @@ def over_ranks(ms, tokens, world, device):
     return float(t.item()), float(k.item())
 
 
+def cpu_baseline_leg(a, ws):
+    """The oracle timed on the host cores (rank 0 at N = 1 only): a bounded
+    sample of the workload's sequences, the same runner as the reference arm."""
+    seqs = list(range(min(ws.num_seqs, a.cpu_seqs)))
+    workers = max(1, min(len(seqs), cpu_cores()))
+    runner = OracleRunner(workers)
+    try:
+        runner.step(a.workload, a.seed, [0])                      # warm-up: worker start, imports
+        tok, secs = runner.step(a.workload, a.seed, seqs)
+    finally:
+        runner.close()
+    return {"value": round(tok / secs, 3), "unit": UNIT, "cores": workers, "kind": "oracle",
+            "sample": oracle_sample_note(ws, seqs, 1, workers) + f", {secs:.2f} s"}
+
+
 def run_ours(a):
+    world0 = int(os.environ.get("WORLD_SIZE", "1"))
+    # the CPU leg first, before this process touches the GPU
+    cpu_line = None
+    if not a.no_cpu_baseline and world0 == 1:
+        from self_sparse_speculative_b200.workloads import spec as _spec
+        cpu_line = cpu_baseline_leg(a, _spec(a.workload))
     import torch
     import torch.distributed as dist
     from self_sparse_speculative_b200.step import DecodeStep
@@ -437,48 +510,69 @@ def run_ours(a):
         line["graph"] = graph_info
     if e2e:
         line["e2e"] = {k: (round(v, 1) if isinstance(v, float) else v) for k, v in e2e.items()}
-    if not a.no_cpu_baseline and world == 1:
-        seqs = list(range(min(ws.num_seqs, a.cpu_seqs)))
-        workers = max(1, min(len(seqs), cpu_cores()))
-        tok, wall, cores = oracle_sample(a.workload, a.seed, seqs, workers)
-        line["cpu_baseline"] = {"value": round(tok / wall, 3), "unit": UNIT, "cores": cores, "kind": "oracle",
-                                "sample": f"float64 oracle round (summaries, {ws.gamma} sparse drafts, verify, "
-                                          f"sampling) of {len(seqs)} of {ws.num_seqs} sequences, one process "
-                                          f"per sequence, {wall:.1f} s wall"}
+    if cpu_line is not None:
+        line["cpu_baseline"] = cpu_line
     print(json.dumps(line), flush=True)
 
 
 # ---------------------------------------------------------------- reference arm
 def run_reference(a):
+    """The oracle as it stands, on the host cores, in the same metric and
+    configuration as the GPU arm. Imports nothing that loads the CUDA library."""
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return
-    from self_sparse_speculative_b200.workloads import spec
-    from self_sparse_speculative_b200.step import algorithmic_bytes
-    from self_sparse_speculative_b200.workloads import Workload
+    from self_sparse_speculative_b200.workloads import Workload, algorithmic_bytes, spec
     ws = spec(a.workload)
     step_bytes = algorithmic_bytes(Workload(ws, seed=a.seed))["step"]
-    workers = max(1, min(cpu_cores(), a.cpu_seqs))
     seqs_per_step = min(ws.num_seqs, a.cpu_seqs)
-    for _ in range(a.warmup if a.warmup < 1 else 1):
-        oracle_sample(a.workload, a.seed, [0], 1)
-    toks, wall = 0, 0.0
-    for k in range(a.steps):
-        seqs = [(k * seqs_per_step + i) % ws.num_seqs for i in range(seqs_per_step)]
-        t, w, _ = oracle_sample(a.workload, a.seed, seqs, workers)
-        toks += t
-        wall += w
-    value = toks / wall
+    workers = max(1, min(cpu_cores(), seqs_per_step))
+    runner = OracleRunner(workers)
+    try:
+        runner.step(a.workload, a.seed, [0])                      # warm-up: worker start, imports
+        toks, secs = 0, 0.0
+        for k in range(a.steps):
+            seqs = [(k * seqs_per_step + i) % ws.num_seqs for i in range(seqs_per_step)]
+            t, w = runner.step(a.workload, a.seed, seqs)
+            toks += t
+            secs += w
+    finally:
+        runner.close()
+    value = toks / secs
+    seqs = list(range(seqs_per_step))
     line = {"metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": a.steps,
-            "warmup": a.warmup, "ms_per_step": round(wall / a.steps * 1e3, 2), "higher_is_better": True,
+            "warmup": a.warmup, "ms_per_step": round(secs / a.steps * 1e3, 2), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": config_of(ws, world, a.seed, step_bytes),
             "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": workers, "kind": "oracle",
-                             "sample": f"{seqs_per_step} of {ws.num_seqs} sequences per step, full float64 "
-                                       f"round per sequence"},
+                             "sample": oracle_sample_note(ws, seqs, a.steps, workers)},
             "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+def launch_plan(gpus, env, argv, port=None):
+    """How `bench.py --gpus N` runs: None to run in this process (N = 1, or
+    already one rank of an N-rank torchrun launch), else the torchrun command
+    that starts N ranks of this same command line. A WORLD_SIZE that
+    disagrees with N is an error (SystemExit), so no run can report a GPU
+    count it did not use."""
+    world = env.get("WORLD_SIZE")
+    if world is not None:
+        if int(world) != gpus:
+            raise SystemExit(f"bench.py: --gpus {gpus} but WORLD_SIZE={world}")
+        return None
+    if gpus < 1:
+        raise SystemExit(f"bench.py: --gpus must be at least 1, got {gpus}")
+    if gpus == 1:
+        return None
+    if port is None:
+        import socket
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={gpus}",
+            "--master-addr", "127.0.0.1", f"--master-port={port}", os.path.join(HERE, "bench.py")] + list(argv)
 
 
 def main():
@@ -494,6 +588,10 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay timing")
     a = ap.parse_args()
+    cmd = launch_plan(a.gpus, os.environ, sys.argv[1:])
+    if cmd is not None:
+        # one process per GPU: relaunch this command line under torchrun
+        sys.exit(subprocess.call(cmd))
     if a.impl == "ours":
         a.warmup = max(3, a.warmup)     # at least 3 untimed warm-up steps
     if a.impl == "reference":

@@ -54,44 +54,62 @@ def sequence_cache(wl, b):
     return K, V, bt, phys
 
 
-def oracle_attention_seq(wl, b, draft_steps=None):
-    """Oracle summaries, page selection, sparse draft and verify attention of
-    sequence b. draft_steps: which draft queries to run (default: all)."""
+def sequence_inputs(wl, b, draft_steps=None, attention=True, sampling=True):
+    """Every float64 input of sequence b's round, generated from the seeded
+    workload (no arithmetic of the method): the cache of its pages, its draft
+    and verify queries, its logits and uniforms."""
     ws = wl.spec
+    inp = {"b": b, "spec": ws, "scale": f32(wl.scale), "T": f32(ws.temperature),
+           "lens": wl.context_lens[b:b + 1].astype(np.int64)}
+    if attention:
+        inp["K"], inp["V"], inp["bt"], inp["phys"] = sequence_cache(wl, b)
+        steps = range(ws.gamma) if draft_steps is None else draft_steps
+        inp["q_draft"] = {i: to_float64(wl.q_draft[i, b], ws.kv_dtype)[None] for i in steps}   # [1, Hq, D]
+        inp["q_verify"] = to_float64(wl.q_verify[b], ws.kv_dtype)[None]                         # [1, R, Hq, D]
+    if sampling:
+        t, d = wl.logits_for_seq(b)
+        inp["tl"] = to_float64(t, ws.logit_dtype)
+        inp["dl"] = to_float64(d, ws.logit_dtype)
+        inp["u_draft"] = wl.u_draft[b].astype(np.float64)
+        inp["u_accept"] = wl.u_accept[b].astype(np.float64)
+        inp["u_sample"] = wl.u_sample[b].astype(np.float64)
+    return inp
+
+
+def oracle_attention(inp):
+    """Oracle summaries, page selection, sparse draft and verify attention of
+    one sequence's inputs (sequence_inputs)."""
+    ws = inp["spec"]
     P, B, G = ws.page_size, ws.budget_pages, ws.group
-    scale = f32(wl.scale)
-    K, V, bt, phys = sequence_cache(wl, b)
-    lens = wl.context_lens[b:b + 1].astype(np.int64)
+    K, V, bt, lens, scale = inp["K"], inp["V"], inp["bt"], inp["lens"], inp["scale"]
     kmin, kmax = O.page_summaries(K, bt, lens, P)
-    steps = range(ws.gamma) if draft_steps is None else draft_steps
     draft = {}
-    for i in steps:
-        q = to_float64(wl.q_draft[i, b], ws.kv_dtype)[None]            # [1, Hq, D]
+    for i, q in inp["q_draft"].items():
         sel, gaps, scores = O.sparse_draft_select(q, kmin, kmax, bt, lens, P, B, G, return_scores=True)
         out, lse = O.sparse_draft_attn(q, K, V, bt, lens, sel, scale)
         draft[i] = {"selected": sel[0], "gaps": gaps[0], "scores": scores[0], "out": out[0], "lse": lse[0],
                     "q": q}
-    qv = to_float64(wl.q_verify[b], ws.kv_dtype)[None]                  # [1, R, Hq, D]
-    vout, vlse = O.verify_attn(qv, K, V, bt, lens, scale)
-    return {"phys": phys, "kmin": kmin, "kmax": kmax, "draft": draft,
+    vout, vlse = O.verify_attn(inp["q_verify"], K, V, bt, lens, scale)
+    return {"phys": inp["phys"], "kmin": kmin, "kmax": kmax, "draft": draft,
             "verify_out": vout[0], "verify_lse": vlse[0], "K": K, "V": V, "bt": bt, "lens": lens}
+
+
+def oracle_attention_seq(wl, b, draft_steps=None):
+    """Oracle summaries, page selection, sparse draft and verify attention of
+    sequence b. draft_steps: which draft queries to run (default: all)."""
+    return oracle_attention(sequence_inputs(wl, b, draft_steps=draft_steps, sampling=False))
+
+
+def oracle_sampling(inp):
+    """Oracle draft-token draws and speculative sampling of one sequence's
+    inputs (sequence_inputs)."""
+    return sampling_ref_from_logits(inp["tl"], inp["dl"], inp["u_draft"], inp["u_accept"], inp["u_sample"],
+                                    inp["T"])
 
 
 def oracle_sampling_seq(wl, b):
     """Oracle draft-token draws and speculative sampling of sequence b."""
-    ws = wl.spec
-    T = f32(ws.temperature)
-    t, d = wl.logits_for_seq(b)
-    tl = to_float64(t, ws.logit_dtype)
-    dl = to_float64(d, ws.logit_dtype)
-    x, xm = O.sample_rows(dl, wl.u_draft[b].astype(np.float64), T)
-    out, n_acc, am, sm = O.spec_sample(tl[None], dl[None], x[None], wl.u_accept[b][None],
-                                       wl.u_sample[b][None], T)
-    return {"x": x, "x_margin": xm, "out_tokens": out[0], "n_acc": int(n_acc[0]),
-            "accept_margin": am[0], "sample_margin": float(sm[0]),
-            # for the validity walk after a near-tie
-            "p": O.softmax_t(tl, T), "q": O.softmax_t(dl, T), "u_draft": wl.u_draft[b].astype(np.float64),
-            "u_accept": wl.u_accept[b].astype(np.float64), "u_sample": wl.u_sample[b].astype(np.float64)}
+    return oracle_sampling(sequence_inputs(wl, b, attention=False))
 
 
 def sampling_ref_from_logits(target_logits, draft_logits, u_draft, u_accept, u_sample, temperature):

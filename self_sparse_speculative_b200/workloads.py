@@ -270,3 +270,31 @@ class Workload:
         else:
             parts = [self.logits_for_seq(b) for b in seqs]
         return np.stack([p[0] for p in parts]), np.stack([p[1] for p in parts])
+
+
+def algorithmic_bytes(wl: "Workload"):
+    """Bytes one step of workload `wl` must move (what the method has to
+    read/write): per draft call the summaries of every page plus the K/V
+    of the selected pages, verify the K/V of every token, sampling the
+    (2 gamma + 1) rows plus the 2 re-read rows, the drafter's draws
+    gamma rows per sequence."""
+    ws = wl.spec
+    Hkv, D, P, B = ws.num_kv_heads, ws.head_dim, ws.page_size, ws.budget_pages
+    elt = 2 if ws.kv_dtype == "bf16" else 4
+    lelt = 2 if ws.logit_dtype == "bf16" else 4
+    lens = wl.context_lens.astype(np.int64)
+    n_b = wl.pages_per_seq
+    kv_tok = 2 * Hkv * D * elt                                  # K + V per token
+    # sparse draft: page summaries of every page (kmin+kmax) + selected KV
+    sel_tokens = 0
+    for L, n in zip(lens, n_b):
+        k = min(int(n), B)
+        # the selected pages are full except possibly the tail page
+        sel_tokens += min(int(L), k * P)
+    draft = int(n_b.sum()) * Hkv * 2 * D * elt + sel_tokens * kv_tok
+    verify = int(lens.sum()) * kv_tok
+    V, g = ws.vocab, ws.gamma
+    sample = ws.num_seqs * ((2 * g + 1) * V * lelt + 2 * V * lelt)
+    draw = ws.num_seqs * g * V * lelt
+    return {"draft_per_call": draft, "verify": verify, "sample": sample, "draft_tokens": draw,
+            "step": g * draft + verify + sample + draw}

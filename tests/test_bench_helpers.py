@@ -2,7 +2,7 @@
 import pytest
 
 import bench
-from self_sparse_speculative_b200.step import algorithmic_bytes
+from self_sparse_speculative_b200.workloads import algorithmic_bytes
 from self_sparse_speculative_b200.workloads import Workload, spec
 
 

@@ -60,10 +60,41 @@ def test_single_rank_needs_no_process_group():
 def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
     import bench
     called = []
-    monkeypatch.setattr(bench, "oracle_sample", lambda *a, **k: called.append(a) or (1, 1.0, 1))
+
+    class Runner:
+        def __init__(self, workers):
+            called.append(workers)
+    monkeypatch.setattr(bench, "OracleRunner", Runner)
     monkeypatch.setenv("RANK", "1")
 
     class A:
         workload, seed, steps, warmup, cpu_seqs, gpus = 1, 0, 2, 3, 2, 2
     bench.run_reference(A())
     assert called == [] and capsys.readouterr().out == ""
+
+
+def test_launch_plan_runs_n_ranks_or_refuses():
+    import bench
+    # N = 1 without torchrun, or one rank of a matching torchrun launch: run here
+    assert bench.launch_plan(1, {}, ["--gpus", "1"]) is None
+    assert bench.launch_plan(4, {"WORLD_SIZE": "4"}, ["--gpus", "4"]) is None
+    # N > 1 without torchrun: relaunch the same command line as N ranks
+    cmd = bench.launch_plan(2, {}, ["--gpus", "2", "--steps", "3"], port=29511)
+    assert cmd[1:3] == ["-m", "torch.distributed.run"]
+    assert "--nproc-per-node=2" in cmd and "--nnodes=1" in cmd
+    assert cmd[cmd.index("--master-addr") + 1] == "127.0.0.1" and "--master-port=29511" in cmd
+    assert cmd[-4:] == [os.path.join(os.path.dirname(HERE), "bench.py"), "--gpus", "2", "--steps", "3"][-4:]
+    assert cmd[-5].endswith("bench.py")
+    # a rank count that disagrees with --gpus, or no GPU at all, is refused
+    with pytest.raises(SystemExit):
+        bench.launch_plan(2, {"WORLD_SIZE": "4"}, [])
+    with pytest.raises(SystemExit):
+        bench.launch_plan(0, {}, [])
+
+
+def test_bench_refuses_mismatched_world_size():
+    import subprocess
+    env = dict(os.environ, WORLD_SIZE="2", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(os.path.dirname(HERE), "bench.py"), "--gpus", "4",
+                        "--impl", "reference"], env=env, capture_output=True, text=True, timeout=120)
+    assert r.returncode != 0 and "WORLD_SIZE" in r.stderr
