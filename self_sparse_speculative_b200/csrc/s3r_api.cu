@@ -137,15 +137,35 @@ S3R_EXPORT s3r_status s3r_sparse_draft_attn(const s3r_paged_kv* kv, const void* 
   s3r_status s = check_attn(kv, 1, budget_pages, true);
   if (s != S3R_OK) return s;
   if (!kmin || !kmax || !q || !selected || !out) return S3R_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(out) || !std::isfinite(scale)) return S3R_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(kmin) || !aligned16(kmax) || !std::isfinite(scale))
+    return S3R_ERR_INVALID_ARG;
   const AttnPlan pl = plan_attention(*kv, 1, budget_pages);
   if (!workspace || workspace_bytes < pl.ws_bytes) return S3R_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  AttnParams p = make_attn_params(kv, pl, q, out, lse, 1, budget_pages, selected, scale, workspace);
+  if (draft_fused_supported(*kv, budget_pages)) {
+    // one kernel: page scoring, top-B and attention (everything host-side is
+    // prepared before the launch)
+    DraftLaunch dl;
+    s = from_cuda(prepare_draft_fused(*kv, budget_pages, &dl));
+    if (s != S3R_OK) return s;
+    p.page_list = nullptr;
+    p.kmin = kmin;
+    p.kmax = kmax;
+    p.selected_out = selected;
+    p.parts = dl.parts;
+    return from_cuda(launch_draft_fused(*kv, dl, p, st));
+  }
+  // selection kernel, then attention over the selected pages; the tensor maps
+  // the attention needs are checked before anything is enqueued
+  if (kv->dtype == S3R_BF16) {
+    CUtensorMap mk, mv;
+    if (!make_cache_map(&mk, kv->k_cache, *kv) || !make_cache_map(&mv, kv->v_cache, *kv)) return S3R_ERR_CUDA;
+  }
   uint32_t* status = static_cast<uint32_t*>(workspace);
   int32_t* phys = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + pl.off_phys);
   s = from_cuda(launch_select(*kv, kmin, kmax, q, budget_pages, selected, phys, status, st));
   if (s != S3R_OK) return s;
-  AttnParams p = make_attn_params(kv, pl, q, out, lse, 1, budget_pages, selected, scale, workspace);
   p.page_phys = phys;
   s3r_status api;
   cudaError_t e = launch_attention(*kv, p, st, &api);

@@ -47,6 +47,11 @@ struct AttnParams {
   uint32_t* tickets;             // [S * Hkv]
   float* part_ml;                // [slots, rows, 2]  (running max in log2 units, sum)
   float* part_o;                 // [slots, rows, D]  (unnormalised)
+  // fused sparse draft (page selection inside the attention kernel)
+  const void* kmin;              // [num_pages_total, Hkv, D] page summaries
+  const void* kmax;
+  int32_t* selected_out;         // [S, Hkv, budget] logical ids of the kept pages
+  int32_t parts;                 // CTAs sharing one (sequence, KV head) unit
 };
 
 // Split plan shared by the workspace-size query and the launch.
@@ -98,6 +103,20 @@ cudaError_t launch_attention_tc(const s3r_paged_kv& kv, const AttnParams& p, cud
                                 s3r_status* api_status);
 cudaError_t launch_attention_tok(const s3r_paged_kv& kv, const AttnParams& p, cudaStream_t st,
                                 s3r_status* api_status);
+// Whether the fused sparse draft kernel (selection and attention in one
+// launch) serves this cache and budget; else select + attention kernels.
+bool draft_fused_supported(const s3r_paged_kv& kv, int32_t budget_pages);
+// Host-side preparation of the fused draft launch (tensor maps, shared
+// memory size, grid): done before anything is enqueued, so a failure
+// enqueues nothing.
+struct DraftLaunch {
+  CUtensorMap mk, mv;
+  int grid;
+  int parts;
+  size_t smem;
+};
+cudaError_t prepare_draft_fused(const s3r_paged_kv& kv, int32_t budget_pages, DraftLaunch* dl);
+cudaError_t launch_draft_fused(const s3r_paged_kv& kv, const DraftLaunch& dl, const AttnParams& p, cudaStream_t st);
 bool make_cache_map(CUtensorMap* map, const void* base, const s3r_paged_kv& kv);
 int device_sm_count();
 
