@@ -249,11 +249,11 @@ def verify_traffic(workload=None):
         return None
 
 
-def launches_per_step(ws):
-    """Library kernels per step: the drafter's draws (1), gamma x (select with
-    the tail-page summary, attention), verify (1), sampling (statistics,
-    normalisers, draw)."""
-    return 1 + 2 * ws.gamma + 1 + 3
+def launches_per_step(ws, draft_kernels=2):
+    """Library kernels per step: the drafter's draws (1), gamma draft calls of
+    draft_kernels each (one fused kernel, or selection then attention),
+    verify (1), sampling (statistics, normalisers, draw)."""
+    return 1 + draft_kernels * ws.gamma + 1 + 3
 
 
 def l2_note(step_bytes):
@@ -500,7 +500,7 @@ def run_ours(a):
                    "verify": round(verify_gbs, 1), "verify_frac_of_8tbs": round(verify_gbs / 8000, 4)},
         "acceptance": {"mean_accepted_per_seq": round(n_acc_total / (ws.num_seqs * a.steps), 4),
                        "committed_per_seq": round(tokens / (ws.num_seqs * a.steps), 4)},
-        "gpu_launches": launches_per_step(ws) * a.steps,
+        "gpu_launches": launches_per_step(ws, s3r.s3r_sparse_draft_kernels(st.kv, ws.budget_pages)) * a.steps,
         "clocks": clk,
     }
     line["timed"] = "cuda graph replay of the round" if graph_ms_total is not None else "eager launches"

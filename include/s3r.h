@@ -243,6 +243,16 @@ size_t s3r_attn_workspace_bytes(const s3r_paged_kv* kv, int32_t rows, int32_t bu
 size_t s3r_sample_workspace_bytes(int32_t num_seqs, int32_t gamma, int32_t vocab);
 
 /*
+ * Number of kernels one s3r_sparse_draft_attn call with these arguments
+ * launches: 1 when page scoring, top-B and attention run as one kernel (bf16
+ * cache, at most one (sequence, KV head) unit per SM, G <= 8, budget <= 128,
+ * max_pages_per_seq <= 1024), 2 when a selection kernel precedes the
+ * attention kernel; 0 for an invalid or unsupported request. Host-only query
+ * (it reads the current device's SM count).
+ */
+int32_t s3r_sparse_draft_kernels(const s3r_paged_kv* kv, int32_t budget_pages);
+
+/*
  * Synchronises `stream`, then reads the status word of `workspace`: S3R_OK,
  * or S3R_ERR_DEVICE_CHECK with the S3R_DEV_* bits in *bits (bits may be
  * NULL). The bits accumulate over the calls made with the workspace since the

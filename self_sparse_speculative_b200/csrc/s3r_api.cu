@@ -245,6 +245,11 @@ S3R_EXPORT s3r_status s3r_sample_tokens(const void* logits, s3r_dtype logit_dtyp
   return from_cuda(launch_sampling(p, logit_dtype, false, st));
 }
 
+S3R_EXPORT int32_t s3r_sparse_draft_kernels(const s3r_paged_kv* kv, int32_t budget_pages) {
+  if (check_attn(kv, 1, budget_pages, true) != S3R_OK) return 0;
+  return draft_fused_supported(*kv, budget_pages) ? 1 : 2;
+}
+
 S3R_EXPORT s3r_status s3r_device_status(const void* workspace, uint32_t* bits, void* stream) {
   if (!workspace) return S3R_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -20,9 +20,11 @@
 //   accumulated in float64; the tail page n_b - 1 is summarised from K itself
 //   (its keys change while the sequence decodes). The summary rows (and the
 //   tail page's K) are staged by cp.async in the K/V ring, which is still
-//   empty, chunk by chunk. A radix select of the budget-th largest
-//   order-preserving key gives the kept pages, in ascending order with ties
-//   to the lower page, as a list in shared memory.
+//   empty, chunk by chunk, and each quarter of a chunk is scored as soon as
+//   it lands. The kept pages come from the order-preserving keys: for up to
+//   256 pages each page's rank among the keys decides, beyond that a radix
+//   select of the budget-th largest key; they go, in ascending order with
+//   ties to the lower page, into a list in shared memory.
 //
 // Attention over the kept pages is the token-major pipeline of s3r_attn_tok.cu
 // (S^T = K Q^T and O^T += V^T P^T per 128-token stage, fp32 in TMEM):
@@ -31,6 +33,7 @@
 #include <cuda_bf16.h>
 
 #include <cmath>
+#include <type_traits>
 
 #include "s3r_attn_common.cuh"
 #include "s3r_device.cuh"
@@ -66,19 +69,22 @@ struct DfLay {
   static constexpr uint32_t kDynBytes = kOffHist + 4 * 256;
   static_assert(kChunkPages >= 64, "staging chunk");
   static_assert(8 * kDfMaxPages >= kDfThreads * 16, "tail scratch fits in the key array");
+  static_assert(12 * 8 * kDfMaxBudget <= kRing, "candidate arrays fit in the ring");
 };
 
 __device__ __forceinline__ void grp_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
-// 16-byte global -> shared copy (cp.async, through L2); completion per thread
-// by commit groups.
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+// Whether `pred` holds on every thread of the group (a barrier of its own):
+// turns per-thread outcomes of bounded waits into one decision.
+__device__ __forceinline__ bool grp_all(bool pred, int id, int n) {
+  int r;
+  asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, %2, %3, p;\n\t"
+               "selp.u32 %0, 1, 0, q;\n\t}"
+               : "=r"(r) : "r"((int)pred), "r"(id), "r"(n) : "memory");
+  return r != 0;
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 __device__ __forceinline__ unsigned long long order_key(double x) {
   const unsigned long long u = static_cast<unsigned long long>(__double_as_longlong(x));
@@ -164,67 +170,60 @@ __device__ void sel_prepare(const AttnParams& p, const DItem& d, int tg, int nth
   if (d.n_b <= p.budget) return;
   const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(p.q) + ((size_t)d.b * p.Hq + (size_t)d.h * p.G) * D;
   for (int c = tg; c < D; c += nthr) {
+    float v[8];
+#pragma unroll
+    for (int g = 0; g < 8; ++g) v[g] = g < p.G ? __bfloat162float(q[(size_t)g * D + c]) : 0.f;   // all in flight
     double a = 0.0, z = 0.0;
-    for (int g = 0; g < p.G; ++g) {
-      const double v = static_cast<double>(__bfloat162float(q[(size_t)g * D + c]));
-      if (v > 0.0) a += v; else z += v;
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+      const double x = static_cast<double>(v[g]);
+      if (x > 0.0) a += x; else z += x;                  // zero padding adds nothing
     }
     sm.ab[c] = a;
     sm.ab[D + c] = z;
   }
 }
 
-// Scores of pages [c0, c1) (none of them the tail page) into sm.keys. kStaged:
-// the rows sit in `rows` (page c0 first, kRowBytes apart); else in kmin/kmax.
-// Eight pages per warp and round, each lane holding D / 32 channels; the eight
-// page sums are reduced across the warp together (lane l ends with page l % 8).
-template <int D, bool kStaged>
-__device__ void score_pages(const AttnParams& p, const DItem& d, int c0, int c1, const uint8_t* rows, int tg,
-                            int nthr, const SelSmem& sm) {
+// Scores of pages [g0, g1) (none of them the tail page) into sm.keys; the
+// rows of page pg sit at rows + (pg - c0) * kRowBytes (kmin row, then kmax).
+// Sixteen pages per warp and round, each lane holding D / 32 channels of
+// every page; the sixteen page sums are reduced across the warp together
+// (halving exchanges: lane l ends with page l % 16), which keeps sixteen
+// independent chains in flight per lane.
+template <int D>
+__device__ void score_pages(const AttnParams& p, int c0, int g0, int g1, const uint8_t* rows, int tg, int nthr,
+                            const SelSmem& sm) {
   constexpr int CPL = D / 32;
-  constexpr int kU = 8;
+  constexpr int kU = 16;
+  using Raw = typename std::conditional<CPL == 4, uint2, uint32_t>::type;
   const int lane = tg & 31, gw = tg >> 5, nw = nthr >> 5;
   double wa[CPL], wb[CPL];
 #pragma unroll
   for (int c = 0; c < CPL; ++c) { wa[c] = sm.ab[lane * CPL + c]; wb[c] = sm.ab[D + lane * CPL + c]; }
-  const __nv_bfloat16* kmn = static_cast<const __nv_bfloat16*>(p.kmin);
-  const __nv_bfloat16* kmx = static_cast<const __nv_bfloat16*>(p.kmax);
-  for (int pg0 = c0 + gw * kU; pg0 < c1; pg0 += nw * kU) {
-    uint32_t lo[kU][CPL / 2], hi[kU][CPL / 2];
+  for (int pg0 = g0 + gw * kU; pg0 < g1; pg0 += nw * kU) {
+    Raw lo[kU], hi[kU];
     bool ok[kU];
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
       const int pg = pg0 + u;
-      const int ph = pg < c1 ? sm.phys[pg] : -1;
+      const int ph = pg < g1 ? sm.phys[pg] : -1;
       ok[u] = ph >= 0 && ph < p.num_pages_total;
-      if (ok[u]) {
-        const uint32_t* a;
-        const uint32_t* z;
-        if constexpr (kStaged) {
-          a = reinterpret_cast<const uint32_t*>(rows + (size_t)(pg - c0) * DfLay<D>::kRowBytes) + lane * (CPL / 2);
-          z = a + D / 2;
-        } else {
-          const size_t base = ((size_t)ph * p.Hkv + d.h) * D + lane * CPL;
-          a = reinterpret_cast<const uint32_t*>(kmn + base);
-          z = reinterpret_cast<const uint32_t*>(kmx + base);
-        }
-#pragma unroll
-        for (int w = 0; w < CPL / 2; ++w) {
-          if constexpr (kStaged) { lo[u][w] = a[w]; hi[u][w] = z[w]; }
-          else { lo[u][w] = __ldg(a + w); hi[u][w] = __ldg(z + w); }
-        }
-      }
+      const Raw* r = reinterpret_cast<const Raw*>(rows + (size_t)(pg - c0) * DfLay<D>::kRowBytes) + lane;
+      if (ok[u]) { lo[u] = r[0]; hi[u] = r[32]; }      // kmin row, kmax row (2 D bytes apart)
     }
     double acc[kU];
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
       double s0 = 0.0, s1 = 0.0;
       if (ok[u]) {
+        uint32_t lw[CPL / 2], hw[CPL / 2];
+        if constexpr (CPL == 4) { lw[0] = ((uint2&)lo[u]).x; lw[1] = ((uint2&)lo[u]).y; hw[0] = ((uint2&)hi[u]).x; hw[1] = ((uint2&)hi[u]).y; }
+        else { lw[0] = (uint32_t&)lo[u]; hw[0] = (uint32_t&)hi[u]; }
 #pragma unroll
         for (int w = 0; w < CPL / 2; ++w) {
           float l0, l1, r0, r1;
-          bf2(lo[u][w], l0, l1);
-          bf2(hi[u][w], r0, r1);
+          bf2(lw[w], l0, l1);
+          bf2(hw[w], r0, r1);
           s0 = fma(wa[2 * w], static_cast<double>(fmaxf(l0, r0)), s0);
           s1 = fma(wb[2 * w], static_cast<double>(fminf(l0, r0)), s1);
           s0 = fma(wa[2 * w + 1], static_cast<double>(fmaxf(l1, r1)), s0);
@@ -233,8 +232,6 @@ __device__ void score_pages(const AttnParams& p, const DItem& d, int c0, int c1,
       }
       acc[u] = s0 + s1;
     }
-    // transpose-reduce the eight sums: after the halving steps lane l holds a
-    // partial of page l % 8, then the lanes of one page add up
 #pragma unroll
     for (int w = kU / 2; w >= 1; w >>= 1) {
       const bool up = (lane & w) != 0;
@@ -245,11 +242,9 @@ __device__ void score_pages(const AttnParams& p, const DItem& d, int c0, int c1,
         acc[k] = keep + __shfl_xor_sync(0xffffffffu, send, w);
       }
     }
-    double v = acc[0];
-    v += __shfl_xor_sync(0xffffffffu, v, 8);
-    v += __shfl_xor_sync(0xffffffffu, v, 16);
-    const int pg = pg0 + (lane & 7);
-    if (lane < kU && pg < c1) {
+    const double v = acc[0] + __shfl_xor_sync(0xffffffffu, acc[0], 16);
+    const int pg = pg0 + (lane & 15);
+    if (lane < kU && pg < g1) {
       bool okp = false;
 #pragma unroll
       for (int u = 0; u < kU; ++u) okp = (u == lane) ? ok[u] : okp;
@@ -297,32 +292,80 @@ __device__ void tail_minmax(const __nv_bfloat16* src, int valid, int tg, int nth
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-__device__ __forceinline__ void cluster_arrive() {
-  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+// Stores to the same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ void st_cluster_u32(const void* local, uint32_t rank, uint32_t v) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_addr(local)), "r"(rank));
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(remote), "r"(v) : "memory");
 }
-__device__ __forceinline__ void cluster_wait() {
-  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
-}
-// Store to the same shared-memory offset in CTA `rank` of the cluster.
 __device__ __forceinline__ void st_cluster_u64(const void* local, uint32_t rank, unsigned long long v) {
   uint32_t remote;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_addr(local)), "r"(rank));
   asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(remote), "l"(v) : "memory");
 }
 
+// Rank of key kp (page i) among keys[0..n): the keys above it, plus the
+// equal keys of lower pages (ties go to the lower page). keys is 8-byte
+// aligned; one key is taken alone when that puts the rest on a 16-byte
+// boundary, then pairs of keys by 16-byte broadcast reads, four pairs per
+// step with separate counters.
+__device__ __forceinline__ int key_rank(const unsigned long long* keys, int n, unsigned long long kp, int i) {
+  int r0 = 0, r1 = 0, r2 = 0, r3 = 0;
+  int q = 0;
+  if ((reinterpret_cast<uintptr_t>(keys) & 15u) != 0 && n > 0) {
+    r0 += (keys[0] > kp) + (keys[0] == kp && 0 < i);
+    q = 1;
+  }
+  const ulonglong2* k2 = reinterpret_cast<const ulonglong2*>(keys + q);   // 16-byte aligned
+  for (int j = 0; q + 8 <= n; q += 8, j += 4) {
+    const ulonglong2 a = k2[j], b = k2[j + 1], c = k2[j + 2], e = k2[j + 3];
+    r0 += (a.x > kp) + (a.x == kp && q < i) + (a.y > kp) + (a.y == kp && q + 1 < i);
+    r1 += (b.x > kp) + (b.x == kp && q + 2 < i) + (b.y > kp) + (b.y == kp && q + 3 < i);
+    r2 += (c.x > kp) + (c.x == kp && q + 4 < i) + (c.y > kp) + (c.y == kp && q + 5 < i);
+    r3 += (e.x > kp) + (e.x == kp && q + 6 < i) + (e.y > kp) + (e.y == kp && q + 7 < i);
+  }
+  for (; q < n; ++q) r0 += (keys[q] > kp) + (keys[q] == kp && q < i);
+  return (r0 + r1) + (r2 + r3);
+}
+
+// Candidates of one group of at most nthr pages page0.. (keys in page
+// order): the pages whose rank in the group is below `budget`, appended in
+// page order to cand_key / cand_page at `base`. Returns the number appended.
+__device__ int group_candidates(const unsigned long long* keys, int page0, int n, int budget,
+                                unsigned long long* cand_key, int* cand_page, int base, int tg, int nthr,
+                                int barid, SelScratch& sc) {
+  bool keep = false;
+  unsigned long long kp = 0;
+  if (tg < n) {
+    kp = keys[tg];
+    keep = key_rank(keys, n, kp, tg) < budget;
+  }
+  int tot;
+  const int pos = grp_exclusive_scan(keep ? 1 : 0, tg, nthr, barid, sc, &tot);
+  if (keep) {
+    cand_key[base + pos] = kp;
+    cand_page[base + pos] = page0 + tg;
+  }
+  return tot;
+}
+
 // The kept pages of item d's unit, ascending, into `list` (logical,
 // physical) and, for the unit's first piece, into p.selected_out. All
 // threads of the CTA, after sel_prepare and the grid-dependency wait.
 // clustered: the unit is shared by the p.parts CTAs of this cluster (rank =
-// d.k); each scores its share of the pages, the first selects.
+// d.k); each scores its share of the pages and sends its candidates (the
+// pages that are top-B within their group of at most 256) to the first CTA,
+// which ranks the candidates and hands the list back. The global top-B is
+// contained in the union of the groups' top-B, so the result is exact.
 template <int D>
 __device__ void select_unit(const AttnParams& p, const DItem& d, int2* list, const SelSmem& sm, SelScratch& sc,
-                            uint8_t* stage, bool clustered) {
+                            uint8_t* stage, uint32_t bar_g0, uint32_t bar_g1, bool clustered, volatile int* abort) {
   using Lay = DfLay<D>;
   constexpr int nthr = kDfThreads, barid = kBarAll;
-  const int tg = threadIdx.x, lane = tg & 31, gw = tg >> 5, nw = nthr >> 5;
+  const int tg = threadIdx.x, lane = tg & 31, gw = tg >> 5;
   const bool write_out = d.k == 0;
   int32_t* out = p.selected_out + ((size_t)d.b * p.Hkv + d.h) * p.budget;
+  for (int k = tg; k < p.budget; k += nthr) list[k] = make_int2(-1, -1);
   if (d.bad) {
     if (write_out) {
       for (int k = tg; k < p.budget; k += nthr) out[k] = -1;
@@ -348,43 +391,51 @@ __device__ void select_unit(const AttnParams& p, const DItem& d, int2* list, con
   const bool tail_ok = tail_ph >= 0 && tail_ph < p.num_pages_total;
   const __nv_bfloat16* tail_src =
       static_cast<const __nv_bfloat16*>(p.k_cache) + ((size_t)tail_ph * p.Hkv + d.h) * p.P * D;
-  float4* scratch = reinterpret_cast<float4*>(sm.keys);
-  // summary rows of the share's pages through the empty ring, chunk by chunk,
-  // as 16-byte cp.async copies from every thread (all in flight at once); the
-  // tail page's K (when in the share) with the first chunk
-  uint8_t* rows = stage + Lay::kTailBytes;
-  constexpr int kRowPieces = D / 8;                      // 16-byte pieces of one row
   const __nv_bfloat16* kmn = static_cast<const __nv_bfloat16*>(p.kmin);
   const __nv_bfloat16* kmx = static_cast<const __nv_bfloat16*>(p.kmax);
+  float4* scratch = reinterpret_cast<float4*>(sm.keys);
+  uint8_t* rows = stage + Lay::kTailBytes;
+  bool ok = true;
+  // summary rows of the share's pages, bulk-copied into the empty ring chunk
+  // by chunk, each chunk in two halves on two barriers so that the first
+  // half is scored while the second is still landing; the tail page's K
+  // (when in the share) with the first half of the first chunk
   const int e = min(s1, tail);                           // the share's pages other than the tail
-  for (int c0 = s0, first = 1; first || c0 < e; c0 += Lay::kChunkPages, first = 0) {
-    const int c1 = min(e, c0 + Lay::kChunkPages);
-    if (first && has_tail && tail_ok)
-      for (int f = tg; f < valid * kRowPieces; f += nthr)
-        cp_async16(smem_addr(stage + (size_t)f * 16), tail_src + (size_t)f * 8);
-    const int pieces = max(0, c1 - c0) * 2 * kRowPieces;
-    for (int f = tg; f < pieces; f += nthr) {
-      const int pg = c0 + f / (2 * kRowPieces);
-      const int w = f - (pg - c0) * 2 * kRowPieces;      // row (kmin, kmax) x piece
+  int phase = 0;
+  for (int c0 = s0, first = 1; first || c0 < e; c0 += Lay::kChunkPages, first = 0, ++phase) {
+    const int c1 = max(c0, min(e, c0 + Lay::kChunkPages));
+    const int mid = c0 + (c1 - c0 + 1) / 2;
+    if (first && has_tail && tail_ok && tg == 0) {
+      const uint32_t bytes = (uint32_t)valid * D * 2;
+      mbar_expect_tx(bar_g0, bytes);
+      bulk_load(smem_addr(stage), tail_src, bytes, bar_g0);
+    }
+    for (int pg = c0 + tg; pg < c1; pg += nthr) {
       const int ph = sm.phys[pg];
       if (ph < 0 || ph >= p.num_pages_total) continue;
-      const size_t base = ((size_t)ph * p.Hkv + d.h) * D + (size_t)(w % kRowPieces) * 8;
-      cp_async16(smem_addr(rows + (size_t)(pg - c0) * Lay::kRowBytes + (size_t)w * 16),
-                 (w < kRowPieces ? kmn : kmx) + base);
+      const uint32_t bar = pg < mid ? bar_g0 : bar_g1;
+      const size_t base = ((size_t)ph * p.Hkv + d.h) * D;
+      const uint32_t dst = smem_addr(rows + (size_t)(pg - c0) * Lay::kRowBytes);
+      mbar_expect_tx(bar, 4u * D);
+      bulk_load(dst, kmn + base, 2u * D, bar);
+      bulk_load(dst + 2u * D, kmx + base, 2u * D, bar);
     }
-    cp_async_commit();
-    cp_async_wait_all();
-    grp_sync(barid, nthr);                               // every thread's copies have landed
-    if (first && has_tail && tail_ok) {
+    grp_sync(barid, nthr);                               // every expectation is registered
+    if (tg == 0) { mbar_arrive(bar_g0); mbar_arrive(bar_g1); }
+    ok = ok && grp_all(mbar_wait(bar_g0, (uint32_t)(phase & 1), abort, p.status), barid, nthr);
+    if (ok && first && has_tail && tail_ok) {
       tail_minmax<D>(reinterpret_cast<const __nv_bfloat16*>(stage), valid, tg, nthr, barid, sm, scratch);
       grp_sync(barid, nthr);                             // the scratch is the key array
     }
-    if (c1 > c0) score_pages<D, true>(p, d, c0, c1, rows, tg, nthr, sm);
-    fence_proxy_async_smem();                            // reads of the staged rows before TMA reuses them
+    if (ok) score_pages<D>(p, c0, c0, mid, rows, tg, nthr, sm);
+    ok = ok && grp_all(mbar_wait(bar_g1, (uint32_t)(phase & 1), abort, p.status), barid, nthr);
+    if (ok) score_pages<D>(p, c0, mid, c1, rows, tg, nthr, sm);
+    fence_proxy_async_smem();                            // reads of the staged rows before copies reuse them
     grp_sync(barid, nthr);
+    if (!ok) break;
   }
   // the tail page, scored from its fresh min / max (first warp)
-  if (has_tail && gw == 0) {
+  if (ok && has_tail && gw == 0) {
     constexpr int CPL = D / 32;
     double a0 = 0.0, a1 = 0.0;
     if (tail_ok) {
@@ -405,125 +456,52 @@ __device__ void select_unit(const AttnParams& p, const DItem& d, int2* list, con
     }
   }
   grp_sync(barid, nthr);
-  if (clustered) {
-    // the share's keys into the first CTA (every CTA of the cluster has
-    // started: each announced itself before its prologue)
-    cluster_wait();
-    if (rank != 0)
-      for (int pg = s0 + tg; pg < s1; pg += nthr) st_cluster_u64(&sm.keys[pg], 0u, sm.keys[pg]);
-    cluster_sync_all();                                  // all keys are in the first CTA
+  // ---- candidates: the top-B of each group of at most nthr pages of the
+  // share, in page order, at their place in the first CTA's candidate array
+  // (the stage's first bytes: the ring is idle until the list is done)
+  unsigned long long* cand_key = reinterpret_cast<unsigned long long*>(stage);     // [8 * kDfMaxBudget]
+  int* cand_page = reinterpret_cast<int*>(stage + 8 * 8 * kDfMaxBudget);            // [8 * kDfMaxBudget]
+  auto cands_of = [&](int lo, int hi) {                  // candidates of pages [lo, hi), whole groups
+    int c = 0;
+    for (int g = lo; g < hi; g += nthr) c += min(p.budget, min(hi, g + nthr) - g);
+    return c;
+  };
+  if (clustered) cluster_sync_all();                     // every CTA scored: the first one's stage is free
+  int base = 0;
+  for (int r = 0; r < rank; ++r) base += cands_of(r * n_b / parts, (r + 1) * n_b / parts);
+  if (ok) {
+    for (int g = s0; g < s1; g += nthr) {
+      // this group's candidates into this CTA's own array, then (other CTAs
+      // of a cluster) copied to the first CTA's
+      const int n = min(s1, g + nthr) - g;
+      const int got = group_candidates(sm.keys + g, g, n, p.budget, cand_key, cand_page, base, tg, nthr, barid, sc);
+      grp_sync(barid, nthr);
+      if (clustered && rank != 0)
+        for (int k = tg; k < got; k += nthr) {
+          st_cluster_u64(&cand_key[base + k], 0u, cand_key[base + k]);
+          st_cluster_u32(&cand_page[base + k], 0u, (uint32_t)cand_page[base + k]);
+        }
+      base += got;
+    }
   }
-  if (rank == 0) {
-    // ---- radix select of the budget-th largest key, from the first byte in
-    // which the keys differ
-    unsigned long long kmin_l = ~0ull, kmax_l = 0ull;
-    for (int pg = tg; pg < n_b; pg += nthr) {
-      const unsigned long long key = sm.keys[pg];
-      kmin_l = key < kmin_l ? key : kmin_l;
-      kmax_l = key > kmax_l ? key : kmax_l;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const unsigned long long a = __shfl_xor_sync(0xffffffffu, kmin_l, o), c = __shfl_xor_sync(0xffffffffu, kmax_l, o);
-      kmin_l = a < kmin_l ? a : kmin_l;
-      kmax_l = c > kmax_l ? c : kmax_l;
-    }
-    if (lane == 0) { sc.kred[0][gw] = kmin_l; sc.kred[1][gw] = kmax_l; }
-    grp_sync(barid, nthr);
-    if (tg == 0) {
-      unsigned long long mn = ~0ull, mx = 0ull;
-      for (int w = 0; w < nw; ++w) {
-        mn = sc.kred[0][w] < mn ? sc.kred[0][w] : mn;
-        mx = sc.kred[1][w] > mx ? sc.kred[1][w] : mx;
+  if (clustered) cluster_sync_all();                     // all candidates are in the first CTA
+  if (rank == 0 && ok) {
+    // ---- final rank among the candidates (ascending page order already)
+    int nc = 0;                                          // candidates of every share
+    for (int r = 0; r < parts; ++r) nc += cands_of(r * n_b / parts, (r + 1) * n_b / parts);
+    int kept_before = 0;
+    for (int c = 0; c < nc; c += nthr) {
+      const int i = c + tg;
+      bool keep = false;
+      if (i < nc) keep = key_rank(cand_key, nc, cand_key[i], i) < p.budget;
+      int tot;
+      const int pos = kept_before + grp_exclusive_scan(keep ? 1 : 0, tg, nthr, barid, sc, &tot);
+      if (keep && pos < p.budget) {
+        const int pg = cand_page[i];
+        list[pos] = make_int2(pg, sm.phys[pg]);
+        if (write_out) out[pos] = pg;
       }
-      const unsigned long long diff = mn ^ mx;
-      const int top = diff ? 8 * ((63 - __clzll((long long)diff)) / 8) : 0;
-      sc.start = top;
-      sc.shift = 0;
-      sc.prefix = top >= 56 ? 0ull : (mx >> (top + 8)) << (top + 8);
-      sc.k = p.budget;
-      sc.done = 0;
-    }
-    grp_sync(barid, nthr);
-    const int shift0 = sc.start;
-    for (int shift = shift0; shift >= 0; shift -= 8) {
-      for (int bin = tg; bin < 256; bin += nthr) sm.hist[bin] = 0u;
-      grp_sync(barid, nthr);
-      const unsigned long long prefix = sc.prefix;
-      for (int base = 0; base < n_b; base += nthr) {           // uniform trip count: whole warps
-        const int pg = base + tg;
-        const unsigned long long key = pg < n_b ? sm.keys[pg] : 0ull;
-        const bool match = pg < n_b && ((shift >= 56) || (((key ^ prefix) >> (shift + 8)) == 0ull));
-        const unsigned bin = match ? (unsigned)(key >> shift) & 255u : 256u + (unsigned)lane;
-        const unsigned peers = __match_any_sync(0xffffffffu, bin);
-        if (match && (int)(__ffs(peers) - 1) == lane) atomicAdd(&sm.hist[bin], (unsigned)__popc(peers));
-      }
-      grp_sync(barid, nthr);
-      if (gw == 0) {
-        // lane l owns bins 255-8l .. 248-8l, scanned from the top
-        unsigned int c[8];
-        unsigned int sum = 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) { c[i] = sm.hist[255 - 8 * lane - i]; sum += c[i]; }
-        unsigned int incl = sum;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const unsigned int y = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += y;
-        }
-        const int k = sc.k;
-        const unsigned int excl = incl - sum;
-        if (excl < (unsigned)k && incl >= (unsigned)k) {
-          unsigned int run = excl;
-          for (int i = 0; i < 8; ++i) {
-            if (run + c[i] >= (unsigned)k) {
-              const unsigned long long digit = 255u - 8u * lane - i;
-              sc.prefix = prefix | (digit << shift);
-              sc.k = k - (int)run;
-              if (c[i] == (unsigned)(k - (int)run)) { sc.done = 1; sc.shift = shift; }
-              break;
-            }
-            run += c[i];
-          }
-        }
-      }
-      grp_sync(barid, nthr);
-      if (sc.done) break;
-    }
-    const int sh = sc.shift;
-    const unsigned long long thr = sc.prefix >> sh;
-    const int need_eq = sc.k;
-
-    // ---- compaction in ascending page order (keys compared above the stop digit)
-    const int per = (n_b + nthr - 1) / nthr;
-    const int b0 = min(n_b, tg * per), b1 = min(n_b, b0 + per);
-    int n_eq = 0;
-    for (int pg = b0; pg < b1; ++pg) n_eq += ((sm.keys[pg] >> sh) == thr);
-    int tot;
-    const int eq_before = grp_exclusive_scan(n_eq, tg, nthr, barid, sc, &tot);
-    int n_sel = 0;
-    {
-      int e = eq_before;
-      for (int pg = b0; pg < b1; ++pg) {
-        const unsigned long long key = sm.keys[pg] >> sh;
-        if (key > thr) ++n_sel;
-        else if (key == thr) { if (e < need_eq) ++n_sel; ++e; }
-      }
-    }
-    int pos = grp_exclusive_scan(n_sel, tg, nthr, barid, sc, &tot);
-    {
-      int e = eq_before;
-      for (int pg = b0; pg < b1; ++pg) {
-        const unsigned long long key = sm.keys[pg] >> sh;
-        bool take = false;
-        if (key > thr) take = true;
-        else if (key == thr) { take = e < need_eq; ++e; }
-        if (take && pos < p.budget) {
-          list[pos] = make_int2(pg, sm.phys[pg]);
-          if (write_out) out[pos] = pg;
-          ++pos;
-        }
-      }
+      kept_before += tot;
     }
     grp_sync(barid, nthr);
   }
@@ -577,7 +555,7 @@ draft_fused_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
   constexpr int N = kDfN, NR = kDfNR, NS = L::kNS;
   extern __shared__ __align__(1024) uint8_t dyn_raw[];
   uint8_t* dyn = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ __align__(8) uint64_t s_bar[2 * NS + 8];
+  __shared__ __align__(8) uint64_t s_bar[2 * NS + 10];
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   __shared__ int s_ticket;
@@ -599,7 +577,7 @@ draft_fused_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
   const uint32_t bar0 = smem_addr(&s_bar[0]);
   auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
   const int B_FULL = 0, B_EMPTY = NS, B_SFULL = 2 * NS, B_PFULL = 2 * NS + 2, B_ODONE = 2 * NS + 4,
-            B_QFULL = 2 * NS + 6, B_TD = 2 * NS + 7;
+            B_QFULL = 2 * NS + 6, B_TD = 2 * NS + 7, B_G0 = 2 * NS + 8, B_G1 = 2 * NS + 9;
   constexpr int PB = L::kPBufs;
   uint8_t* sQ = dyn;
   uint8_t* sP = dyn + L::kOffP;
@@ -627,6 +605,8 @@ draft_fused_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
     mbar_init(BAR(B_ODONE + 1), 1);
     mbar_init(BAR(B_QFULL), 128);
     mbar_init(BAR(B_TD), 1);
+    mbar_init(BAR(B_G0), 1);
+    mbar_init(BAR(B_G1), 1);
     s_abort = 0;
     fence_barrier_init();
   }
@@ -654,14 +634,13 @@ draft_fused_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
   // ---- the unit's selection, by every thread, staged through the empty ring
   const DItem d0 = draft_item(p, it0);
   const bool clustered = p.parts > 1 && !d0.bad && d0.n_b > p.budget;   // uniform over the cluster
-  if (clustered) cluster_arrive();                       // this CTA is running (for remote writes)
   sel_prepare<D>(p, d0, tid, kDfThreads, sm);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem;
   pdl_wait();                                            // summaries, outputs and workspace from here on
-  select_unit<D>(p, d0, s_list, sm, s_sc, sKV, clustered);
+  select_unit<D>(p, d0, s_list, sm, s_sc, sKV, BAR(B_G0), BAR(B_G1), clustered, &s_abort);
   __syncthreads();
 
   if (warp == kDfProducer) {
@@ -670,7 +649,7 @@ draft_fused_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
     int g = 0;
     bool ok = __all_sync(0xffffffffu, !s_abort);
     for (int it = it0; it < it1 && ok; ++it) {
-      const DItem d = draft_item(p, it);
+      const DItem d = d0;                                  // the CTA's one item
       const int2* list = s_list;
       const int nst = (d.npg + ppt - 1) / ppt;
       for (int j = 0; j < nst; ++j, ++g) {
@@ -821,7 +800,7 @@ draft_fused_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
       return it1;
     };
     for (int it = it0; it < it1; ++it) {
-      const DItem d = draft_item(p, it);
+      const DItem d = d0;                                  // the CTA's one item
       const size_t rowbase = (size_t)d.b * p.Hq + (size_t)d.h * p.G;
       const int slot_idx = d.u * p.parts + d.k;            // partial slot of a piece
       if (d.npg == 0) {

@@ -22,7 +22,7 @@ S3R_DEV_BAD_CONTEXT_LEN, S3R_DEV_BAD_PAGE_ID, S3R_DEV_BAD_TOKEN_ID, S3R_DEV_WAIT
 EXPORTED = [
     "s3r_page_summaries", "s3r_page_summaries_checked", "s3r_sparse_draft_attn", "s3r_verify_attn",
     "s3r_spec_sample", "s3r_spec_sample_noalloc", "s3r_sample_tokens", "s3r_attn_workspace_bytes", "s3r_sample_workspace_bytes",
-    "s3r_device_status", "s3r_status_str", "s3r_version",
+    "s3r_device_status", "s3r_status_str", "s3r_version", "s3r_sparse_draft_kernels",
 ]
 
 
@@ -60,6 +60,7 @@ def _load():
         "s3r_sample_workspace_bytes": ([i32, i32, i32], sz),
         "s3r_device_status": ([vp, ctypes.POINTER(ctypes.c_uint32), vp], i32),
         "s3r_status_str": ([i32], ctypes.c_char_p),
+        "s3r_sparse_draft_kernels": ([kvp, i32], i32),
         "s3r_version": ([], i32),
     }
     for name, (args, res) in sig.items():
@@ -190,6 +191,11 @@ def s3r_device_status(workspace, stream=None):
     bits = ctypes.c_uint32(0)
     st = _lib.s3r_device_status(_ptr(workspace), ctypes.byref(bits), _stream(stream))
     return int(st), int(bits.value)
+
+
+def s3r_sparse_draft_kernels(kv: PagedKV, budget_pages: int) -> int:
+    """Kernels one s3r_sparse_draft_attn call launches (1 fused, 2 select + attention)."""
+    return int(_lib.s3r_sparse_draft_kernels(ctypes.byref(kv), int(budget_pages)))
 
 
 def s3r_version() -> int:

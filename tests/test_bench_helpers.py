@@ -21,6 +21,7 @@ def test_profiled_traffic_is_reported_only_for_the_profiled_workload():
 def test_launch_count_per_step():
     # drafter draws, gamma x (select, attention), verify, statistics + normalisers + draw
     assert bench.launches_per_step(spec(1)) == 1 + 2 * 4 + 1 + 3
+    assert bench.launches_per_step(spec(1), 1) == 1 + 4 + 1 + 3
     assert bench.launches_per_step(spec(4)) == 1 + 2 * 8 + 1 + 3
 
 
