@@ -206,6 +206,40 @@ s3r_status s3r_sample_tokens(const void* logits, s3r_dtype logit_dtype, int32_t 
                              void* stream);
 
 /*
+ * As s3r_sample_tokens, also writing each row's statistics at temperature T:
+ *   row_stats[r] = { M_r, Z_r },  float64 [num_rows, 2],
+ *   M_r = the row's largest logit (-inf for a row of -inf only),
+ *   Z_r = sum over k of exp((logits[r, k] - M_r) / T), accumulated in float64
+ *         from float64 exponentials (the normaliser of q_r = softmax(logits / T)).
+ * row_stats may be NULL (then this is s3r_sample_tokens). It must be 8-byte
+ * aligned. The draw of the round's draft tokens visits every draft logit
+ * once; handing these statistics to s3r_spec_sample_ex spares it a second
+ * pass over the draft rows.
+ */
+s3r_status s3r_sample_tokens_ex(const void* logits, s3r_dtype logit_dtype, int32_t num_rows,
+                                int32_t vocab, float temperature, const float* u,
+                                int32_t* tokens, double* row_stats, void* workspace,
+                                size_t workspace_bytes, void* stream);
+
+/*
+ * As s3r_spec_sample, with the draft rows' statistics given: draft_stats,
+ * float64 [S, gamma, 2], row (b, i) = { M, Z } of draft_logits[b, i] at the
+ * same temperature, as s3r_sample_tokens_ex writes them (NULL: computed here,
+ * which is s3r_spec_sample). With them the call reads the gamma + 1 target
+ * rows for their statistics and, after a rejection at j, only target row j
+ * for its exact normaliser; the draft rows are read at the drafted token and,
+ * after a rejection, draft row j for the residual draw. Results are those of
+ * s3r_spec_sample up to the float64 rounding of the normalisers.
+ */
+s3r_status s3r_spec_sample_ex(const void* target_logits, const void* draft_logits,
+                              s3r_dtype logit_dtype, const int32_t* draft_tokens,
+                              const float* u_accept, const float* u_sample,
+                              const double* draft_stats, int32_t num_seqs, int32_t gamma,
+                              int32_t vocab, float temperature, int32_t* out_tokens,
+                              int32_t* num_accepted, void* workspace, size_t workspace_bytes,
+                              void* stream);
+
+/*
  * s3r_spec_sample without a workspace argument, for callers that cannot
  * allocate device memory themselves (a plug-in inside a host framework whose
  * device memory belongs to the framework's pooling allocator, code that must
@@ -218,8 +252,10 @@ s3r_status s3r_sample_tokens(const void* logits, s3r_dtype logit_dtype, int32_t 
  *   (s3r_sample_workspace_bytes(num_seqs, gamma, vocab) > 4 MiB) return
  *   S3R_ERR_UNSUPPORTED before anything is enqueued.
  * - The first call on a device looks up the array's device address for that
- *   device (with the device current); make that first call before any
- *   stream capture.
+ *   device (with the device current) and keeps it for the device's current
+ *   CUDA context; make that first call before any stream capture. A call made
+ *   in another context (after cudaDeviceReset, say) looks the address up
+ *   again, so make its first call before any capture as well.
  * - The function allocates nothing (no cudaMalloc, cudaFree or allocating
  *   library routine); it clears the part of the array that must start at
  *   zero with cudaMemsetAsync on `stream`.

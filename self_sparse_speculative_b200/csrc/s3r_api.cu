@@ -203,16 +203,18 @@ SampleParams make_sample_params(const SamplePlan& pl, void* ws, int32_t nseq, in
 }
 }  // namespace
 
-S3R_EXPORT s3r_status s3r_spec_sample(const void* target_logits, const void* draft_logits, s3r_dtype logit_dtype,
-                                      const int32_t* draft_tokens, const float* u_accept, const float* u_sample,
-                                      int32_t num_seqs, int32_t gamma, int32_t vocab, float temperature,
-                                      int32_t* out_tokens, int32_t* num_accepted, void* workspace,
-                                      size_t workspace_bytes, void* stream) {
+S3R_EXPORT s3r_status s3r_spec_sample_ex(const void* target_logits, const void* draft_logits,
+                                         s3r_dtype logit_dtype, const int32_t* draft_tokens, const float* u_accept,
+                                         const float* u_sample, const double* draft_stats, int32_t num_seqs,
+                                         int32_t gamma, int32_t vocab, float temperature, int32_t* out_tokens,
+                                         int32_t* num_accepted, void* workspace, size_t workspace_bytes,
+                                         void* stream) {
   if (!target_logits || !draft_logits || !draft_tokens || !u_accept || !u_sample || !out_tokens || !num_accepted)
     return S3R_ERR_INVALID_ARG;
   if (logit_dtype != S3R_F32 && logit_dtype != S3R_BF16) return S3R_ERR_INVALID_ARG;
   if (num_seqs < 1 || vocab < 1 || gamma < 1) return S3R_ERR_INVALID_ARG;
   if (!(temperature > 0.0f) || !std::isfinite(temperature)) return S3R_ERR_INVALID_ARG;
+  if (draft_stats && (reinterpret_cast<uintptr_t>(draft_stats) & 7u)) return S3R_ERR_INVALID_ARG;
   if (gamma > kMaxGamma) return S3R_ERR_UNSUPPORTED;
   const SamplePlan pl = plan_sampling(num_seqs, gamma, vocab, logit_dtype == S3R_BF16 ? 2 : 4);
   if (!workspace || workspace_bytes < pl.ws_bytes) return S3R_ERR_WORKSPACE;
@@ -225,16 +227,29 @@ S3R_EXPORT s3r_status s3r_spec_sample(const void* target_logits, const void* dra
   p.u_sample = u_sample;
   p.out_tokens = out_tokens;
   p.num_accepted = num_accepted;
+  p.draft_stats = draft_stats;
   return from_cuda(launch_sampling(p, logit_dtype, true, st));
 }
 
-S3R_EXPORT s3r_status s3r_sample_tokens(const void* logits, s3r_dtype logit_dtype, int32_t num_rows, int32_t vocab,
-                                        float temperature, const float* u, int32_t* tokens, void* workspace,
-                                        size_t workspace_bytes, void* stream) {
+S3R_EXPORT s3r_status s3r_spec_sample(const void* target_logits, const void* draft_logits, s3r_dtype logit_dtype,
+                                      const int32_t* draft_tokens, const float* u_accept, const float* u_sample,
+                                      int32_t num_seqs, int32_t gamma, int32_t vocab, float temperature,
+                                      int32_t* out_tokens, int32_t* num_accepted, void* workspace,
+                                      size_t workspace_bytes, void* stream) {
+  return s3r_spec_sample_ex(target_logits, draft_logits, logit_dtype, draft_tokens, u_accept, u_sample, nullptr,
+                            num_seqs, gamma, vocab, temperature, out_tokens, num_accepted, workspace,
+                            workspace_bytes, stream);
+}
+
+S3R_EXPORT s3r_status s3r_sample_tokens_ex(const void* logits, s3r_dtype logit_dtype, int32_t num_rows,
+                                           int32_t vocab, float temperature, const float* u, int32_t* tokens,
+                                           double* row_stats, void* workspace, size_t workspace_bytes,
+                                           void* stream) {
   if (!logits || !u || !tokens) return S3R_ERR_INVALID_ARG;
   if (logit_dtype != S3R_F32 && logit_dtype != S3R_BF16) return S3R_ERR_INVALID_ARG;
   if (num_rows < 1 || vocab < 1) return S3R_ERR_INVALID_ARG;
   if (!(temperature > 0.0f) || !std::isfinite(temperature)) return S3R_ERR_INVALID_ARG;
+  if (row_stats && (reinterpret_cast<uintptr_t>(row_stats) & 7u)) return S3R_ERR_INVALID_ARG;
   const SamplePlan pl = plan_sampling(num_rows, 0, vocab, logit_dtype == S3R_BF16 ? 2 : 4);
   if (!workspace || workspace_bytes < pl.ws_bytes) return S3R_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -242,7 +257,15 @@ S3R_EXPORT s3r_status s3r_sample_tokens(const void* logits, s3r_dtype logit_dtyp
   p.target = logits;
   p.u_sample = u;
   p.out_tokens = tokens;
+  p.row_stats_out = row_stats;
   return from_cuda(launch_sampling(p, logit_dtype, false, st));
+}
+
+S3R_EXPORT s3r_status s3r_sample_tokens(const void* logits, s3r_dtype logit_dtype, int32_t num_rows, int32_t vocab,
+                                        float temperature, const float* u, int32_t* tokens, void* workspace,
+                                        size_t workspace_bytes, void* stream) {
+  return s3r_sample_tokens_ex(logits, logit_dtype, num_rows, vocab, temperature, u, tokens, nullptr, workspace,
+                              workspace_bytes, stream);
 }
 
 S3R_EXPORT int32_t s3r_sparse_draft_kernels(const s3r_paged_kv* kv, int32_t budget_pages) {

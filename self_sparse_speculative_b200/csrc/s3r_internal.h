@@ -157,6 +157,8 @@ struct SampleParams {
   double* wpart;           // [nseq, c2, 8] per-warp partial sums of the draw weights
   float* cmax;             // [nseq, c2] chunk maxima (plain draws)
   int32_t c1, ch1, c2, ch2;
+  double* row_stats_out;       // plain: [N, 2] {row max, exact float64 Z} written by the draw, or null
+  const double* draft_stats;   // spec: [S, gamma, 2] the draft rows' {max, exact Z} (from a plain draw), or null
 };
 // Fill the workspace pointers and sizes of `p` from a plan and a workspace base.
 void bind_sample_workspace(SampleParams* p, const SamplePlan& pl, void* ws);

@@ -11,12 +11,14 @@
 //
 // The array is a file-scope __device__ variable, so every GPU that loads the
 // library holds kStaticScratchBytes of it until the process exits. Its
-// device address is looked up once per device (cudaGetSymbolAddress) on the
-// first call made with that device current; the host-side symbol itself is
-// only a stand-in and is never passed to a kernel.
-#include <atomic>
+// device address is looked up (cudaGetSymbolAddress) on the first call made
+// with a device current and kept for that device's current CUDA context; a
+// call from another context (after cudaDeviceReset, for instance, the module
+// is loaded again at a new address) looks it up again. The host-side symbol
+// itself is only a stand-in and is never passed to a kernel.
 #include <cmath>
 #include <cstring>
+#include <mutex>
 
 #include "s3r_internal.h"
 
@@ -31,20 +33,50 @@ constexpr int kMaxDevices = 64;
 
 __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
-std::atomic<void*> g_scratch_addr[kMaxDevices];
+// The array's address in one context (per device; the context it was looked
+// up in, and the address).
+struct ScratchSlot {
+  std::mutex m;
+  CUcontext ctx = nullptr;
+  void* addr = nullptr;
+};
+ScratchSlot g_scratch_slot[kMaxDevices];
 
-// Device address of the scratch array on the current device (nullptr on error).
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+CtxGetCurrentFn get_ctx_fn() {
+  static CtxGetCurrentFn fn = [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      return reinterpret_cast<CtxGetCurrentFn>(ptr);
+    return static_cast<CtxGetCurrentFn>(nullptr);
+  }();
+  return fn;
+}
+
+// Device address of the scratch array in the current device's current
+// context (nullptr on error).
 void* scratch_on_current_device(s3r_status* st) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) { *st = S3R_ERR_CUDA; return nullptr; }
   if (dev < 0 || dev >= kMaxDevices) { *st = S3R_ERR_UNSUPPORTED; return nullptr; }
-  void* p = g_scratch_addr[dev].load(std::memory_order_acquire);
-  if (!p) {
+  CtxGetCurrentFn ctx_fn = get_ctx_fn();
+  if (!ctx_fn) { *st = S3R_ERR_CUDA; return nullptr; }
+  CUcontext ctx = nullptr;
+  if (ctx_fn(&ctx) != CUDA_SUCCESS) { *st = S3R_ERR_CUDA; return nullptr; }   // null before any context exists
+  ScratchSlot& slot = g_scratch_slot[dev];
+  std::lock_guard<std::mutex> lock(slot.m);
+  if (!ctx || slot.ctx != ctx || !slot.addr) {
+    // the lookup also makes the runtime's context current, so read it after
+    void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) { *st = S3R_ERR_CUDA; return nullptr; }
-    g_scratch_addr[dev].store(p, std::memory_order_release);
+    if (ctx_fn(&ctx) != CUDA_SUCCESS || !ctx) { *st = S3R_ERR_CUDA; return nullptr; }
+    slot.ctx = ctx;
+    slot.addr = p;
   }
   *st = S3R_OK;
-  return p;
+  return slot.addr;
 }
 
 }  // namespace

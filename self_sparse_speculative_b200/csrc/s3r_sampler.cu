@@ -216,7 +216,8 @@ __device__ void decide(const SampleParams& p, int b) {
     if (x >= 0 && x < p.vocab) {
       // statistics written by other CTAs of this grid: read through L2
       const double* st = p.stats + 2 * ((size_t)b * per + lane);
-      const double* sd = p.stats + 2 * ((size_t)b * per + R + lane);
+      const double* sd = p.draft_stats ? p.draft_stats + 2 * ((size_t)b * p.gamma + lane)
+                                       : p.stats + 2 * ((size_t)b * per + R + lane);
       const double lt = LogitIO<T>::at(static_cast<const T*>(p.target) + ((size_t)b * R + lane) * p.vocab, x);
       const double ld = LogitIO<T>::at(static_cast<const T*>(p.draft) + ((size_t)b * p.gamma + lane) * p.vocab, x);
       const double px = exp((lt - __ldcg(st)) * p.inv_temp_d) / __ldcg(st + 1);
@@ -256,7 +257,11 @@ __global__ void __launch_bounds__(kSmpThreads, kStatsCtasPerSm) rowstats_kernel(
   constexpr int PV = IO::kPerVec;
   constexpr int kB = 4;                                 // vectors in flight per thread
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int row = blockIdx.x / p.c1, c = blockIdx.x - (blockIdx.x / p.c1) * p.c1;
+  const int per = 2 * p.gamma + 1, R = p.gamma + 1;
+  // with the draft rows' statistics given, only the target rows are visited
+  const int tr = blockIdx.x / p.c1, c = blockIdx.x - (blockIdx.x / p.c1) * p.c1;
+  const int row = p.draft_stats ? (tr / R) * per + (tr - (tr / R) * R) : tr;
+  const int rows_per_seq = p.draft_stats ? R : per;
   const int beg = c * p.ch1, n = min(p.vocab, beg + p.ch1) - beg;
   const T* src = row_ptr<T>(p, true, row) + beg;
   const float k2 = kLog2e * p.inv_temp;
@@ -326,12 +331,11 @@ __global__ void __launch_bounds__(kSmpThreads, kStatsCtasPerSm) rowstats_kernel(
     p.stats[2 * (size_t)row + 1] = Z;
     p.tk_row[row] = 0u;
   }
-  const int per = 2 * p.gamma + 1;
   const int b = row / per;
   int last = 0;
   if (lane == 0) {
     __threadfence();
-    last = atomicAdd(p.tk_seq1 + b, 1u) == (unsigned)(per - 1);
+    last = atomicAdd(p.tk_seq1 + b, 1u) == (unsigned)(rows_per_seq - 1);
   }
   last = __shfl_sync(0xffffffffu, last, 0);
   if (last) {
@@ -367,7 +371,7 @@ __device__ DrawRows draw_rows(const SampleParams& p, int s, int j) {
   w.Mp = p.stats[2 * ((size_t)s * per + j)];
   if (j < p.gamma) {
     w.qrow = static_cast<const T*>(p.draft) + ((size_t)s * p.gamma + j) * p.vocab;
-    w.Mq = p.stats[2 * ((size_t)s * per + R + j)];
+    w.Mq = p.draft_stats ? p.draft_stats[2 * ((size_t)s * p.gamma + j)] : p.stats[2 * ((size_t)s * per + R + j)];
     w.iZp = 1.0 / __ldcg(p.znorm + 2 * (size_t)s);
     w.iZq = 1.0 / __ldcg(p.znorm + 2 * (size_t)s + 1);
   }
@@ -455,7 +459,11 @@ __global__ void __launch_bounds__(kSmpThreads, kDrawCtasPerSm) znorm_kernel(cons
   const int j = p.jsel[s];
   if (j >= p.gamma) return;                              // bonus draw: no residual (uniform per sequence)
   const int per = 2 * p.gamma + 1, R = p.gamma + 1;
-  const double Mp = p.stats[2 * ((size_t)s * per + j)], Mq = p.stats[2 * ((size_t)s * per + R + j)];
+  // with the draft rows' statistics given, the draft row's exact Z is known:
+  // only the target row is summed here
+  const bool two = p.draft_stats == nullptr;
+  const double Mp = p.stats[2 * ((size_t)s * per + j)];
+  const double Mq = two ? p.stats[2 * ((size_t)s * per + R + j)] : 0.0;
   const int beg = c * p.ch2, n = min(p.vocab, beg + p.ch2) - beg;
   const T* pa = static_cast<const T*>(p.target) + ((size_t)s * R + j) * p.vocab + beg;
   const T* pb = static_cast<const T*>(p.draft) + ((size_t)s * p.gamma + j) * p.vocab + beg;
@@ -465,15 +473,44 @@ __global__ void __launch_bounds__(kSmpThreads, kDrawCtasPerSm) znorm_kernel(cons
     init_stage_bar(&s_bar);
     T* s0 = reinterpret_cast<T*>(s_dyn);
     T* s1 = s0 + p.ch2;
-    stage_rows<T>(s0, pa, s1, pb, n, &s_bar, &s_abort, p.status);
+    stage_rows<T>(s0, pa, two ? s1 : nullptr, two ? pb : nullptr, n, &s_bar, &s_abort, p.status);
     pa = s0;
     pb = s1;
   } else {
     __syncthreads();
   }
   double zt = 0.0, zd = 0.0;
+  if (!two) {
+    // the target row alone
+    const double ca = -Mp * p.inv_temp_d;
+    for (int i = tid * PV; i < n; i += kSmpThreads * PV) {
+      const int m = min(PV, n - i);
+      float a[PV];
+      load_vals<T, STAGE>(pa + i, m, a);
+      float amin = a[0];
+#pragma unroll
+      for (int t = 1; t < PV; ++t)
+        if (STAGE || t < m) amin = fminf(amin, a[t]);
+      const bool in_range = fma(static_cast<double>(amin), p.inv_temp_d, ca) > -707.0;
+#pragma unroll
+      for (int t0 = 0; t0 < PV; t0 += 4) {
+        double xa[4], ea[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          xa[t] = fma(static_cast<double>(a[t0 + t]), p.inv_temp_d, ca);
+          ea[t] = exp_tbl(xa[t], s_tab);
+        }
+        if (!in_range)
+#pragma unroll
+          for (int t = 0; t < 4; ++t) ea[t] = exp_fixup(xa[t], ea[t], s_tab);
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+          if (STAGE || t0 + t < m) zt += ea[t];
+      }
+    }
+  }
   const double ca = -Mp * p.inv_temp_d, cb = -Mq * p.inv_temp_d;
-  for (int i = tid * PV; i < n; i += kSmpThreads * PV) {
+  for (int i = tid * PV; two && i < n; i += kSmpThreads * PV) {
     const int m = min(PV, n - i);
     float a[PV], b[PV];
     load_vals<T, STAGE>(pa + i, m, a);
@@ -539,7 +576,7 @@ __global__ void __launch_bounds__(kSmpThreads, kDrawCtasPerSm) znorm_kernel(cons
   b = warp_sum_d(b);
   if (lane == 0) {
     p.znorm[2 * (size_t)s] = a;
-    p.znorm[2 * (size_t)s + 1] = b;
+    p.znorm[2 * (size_t)s + 1] = two ? b : p.draft_stats[2 * ((size_t)s * p.gamma + j) + 1];
     p.tk_seq3[s] = 0u;
   }
 }
@@ -757,6 +794,14 @@ __global__ void __launch_bounds__(kSmpThreads, kDrawCtasPerSm) draw_kernel(const
   for (int i = tid; i < nseg; i += kSmpThreads) loc += segval(i);
   double total;
   block_scan_d(loc, &total, s_w);
+  if constexpr (!SPEC) {
+    // the row's statistics at temperature T: its largest logit and the exact
+    // float64 sum of exp((x - max) / T) (the chunk sums brought to the row max)
+    if (p.row_stats_out && tid == 0) {
+      p.row_stats_out[2 * (size_t)s] = Mrow;
+      p.row_stats_out[2 * (size_t)s + 1] = total;
+    }
+  }
   int k = -1;
   if (total > 0.0) {
     const double thr = u * total;
@@ -819,7 +864,7 @@ __global__ void __launch_bounds__(kSmpThreads, kDrawCtasPerSm) draw_kernel(const
 template <typename T, bool SPEC>
 cudaError_t launch_typed(const SampleParams& p, cudaStream_t st) {
   const int per = SPEC ? 2 * p.gamma + 1 : 1;
-  const int nrows = p.nseq * per;
+  const int nrows = p.nseq * (SPEC && p.draft_stats ? p.gamma + 1 : per);   // rows of the statistics pass
   // bulk staging needs 16-byte aligned rows
   const bool stage = (((size_t)p.vocab * sizeof(T)) % 16 == 0) &&
                      (reinterpret_cast<uintptr_t>(p.target) % 16 == 0) &&

@@ -23,6 +23,7 @@ EXPORTED = [
     "s3r_page_summaries", "s3r_page_summaries_checked", "s3r_sparse_draft_attn", "s3r_verify_attn",
     "s3r_spec_sample", "s3r_spec_sample_noalloc", "s3r_sample_tokens", "s3r_attn_workspace_bytes", "s3r_sample_workspace_bytes",
     "s3r_device_status", "s3r_status_str", "s3r_version", "s3r_sparse_draft_kernels",
+    "s3r_sample_tokens_ex", "s3r_spec_sample_ex",
 ]
 
 
@@ -56,6 +57,8 @@ def _load():
         "s3r_spec_sample": ([vp, vp, i32, vp, vp, vp, i32, i32, i32, f32, vp, vp, vp, sz, vp], i32),
         "s3r_spec_sample_noalloc": ([vp, vp, i32, vp, vp, vp, i32, i32, i32, f32, vp, vp, vp], i32),
         "s3r_sample_tokens": ([vp, i32, i32, i32, f32, vp, vp, vp, sz, vp], i32),
+        "s3r_sample_tokens_ex": ([vp, i32, i32, i32, f32, vp, vp, vp, vp, sz, vp], i32),
+        "s3r_spec_sample_ex": ([vp, vp, i32, vp, vp, vp, vp, i32, i32, i32, f32, vp, vp, vp, sz, vp], i32),
         "s3r_attn_workspace_bytes": ([kvp, i32, i32], sz),
         "s3r_sample_workspace_bytes": ([i32, i32, i32], sz),
         "s3r_device_status": ([vp, ctypes.POINTER(ctypes.c_uint32), vp], i32),
@@ -156,13 +159,22 @@ def s3r_verify_attn(kv: PagedKV, q, rows: int, scale: float, out, lse, workspace
 
 def s3r_spec_sample(target_logits, draft_logits, logit_dtype, draft_tokens, u_accept, u_sample,
                     num_seqs: int, gamma: int, vocab: int, temperature: float, out_tokens, num_accepted,
-                    workspace, workspace_bytes=None, stream=None):
+                    workspace, workspace_bytes=None, stream=None, draft_stats=None):
+    """draft_stats (float64 [S, gamma, 2] from s3r_sample_tokens(..., row_stats=...)) selects
+    s3r_spec_sample_ex."""
     wb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
-    st = _lib.s3r_spec_sample(_ptr(target_logits), _ptr(draft_logits), dtype_code(logit_dtype),
-                              _ptr(draft_tokens), _ptr(u_accept), _ptr(u_sample), int(num_seqs), int(gamma),
-                              int(vocab), float(temperature), _ptr(out_tokens), _ptr(num_accepted),
-                              _ptr(workspace), wb, _stream(stream))
-    _check("s3r_spec_sample", st)
+    if draft_stats is None:
+        st = _lib.s3r_spec_sample(_ptr(target_logits), _ptr(draft_logits), dtype_code(logit_dtype),
+                                  _ptr(draft_tokens), _ptr(u_accept), _ptr(u_sample), int(num_seqs), int(gamma),
+                                  int(vocab), float(temperature), _ptr(out_tokens), _ptr(num_accepted),
+                                  _ptr(workspace), wb, _stream(stream))
+        _check("s3r_spec_sample", st)
+        return
+    st = _lib.s3r_spec_sample_ex(_ptr(target_logits), _ptr(draft_logits), dtype_code(logit_dtype),
+                                 _ptr(draft_tokens), _ptr(u_accept), _ptr(u_sample), _ptr(draft_stats),
+                                 int(num_seqs), int(gamma), int(vocab), float(temperature), _ptr(out_tokens),
+                                 _ptr(num_accepted), _ptr(workspace), wb, _stream(stream))
+    _check("s3r_spec_sample_ex", st)
 
 
 def s3r_spec_sample_noalloc(target_logits, draft_logits, logit_dtype, draft_tokens, u_accept, u_sample,
@@ -178,12 +190,20 @@ def s3r_spec_sample_noalloc(target_logits, draft_logits, logit_dtype, draft_toke
 
 
 def s3r_sample_tokens(logits, logit_dtype, num_rows: int, vocab: int, temperature: float, u, tokens,
-                      workspace, workspace_bytes=None, stream=None):
+                      workspace, workspace_bytes=None, stream=None, row_stats=None):
+    """row_stats (float64 [num_rows, 2]) selects s3r_sample_tokens_ex, which also writes each
+    row's {max, exact Z}."""
     wb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
-    st = _lib.s3r_sample_tokens(_ptr(logits), dtype_code(logit_dtype), int(num_rows), int(vocab),
-                                float(temperature), _ptr(u), _ptr(tokens), _ptr(workspace), wb,
-                                _stream(stream))
-    _check("s3r_sample_tokens", st)
+    if row_stats is None:
+        st = _lib.s3r_sample_tokens(_ptr(logits), dtype_code(logit_dtype), int(num_rows), int(vocab),
+                                    float(temperature), _ptr(u), _ptr(tokens), _ptr(workspace), wb,
+                                    _stream(stream))
+        _check("s3r_sample_tokens", st)
+        return
+    st = _lib.s3r_sample_tokens_ex(_ptr(logits), dtype_code(logit_dtype), int(num_rows), int(vocab),
+                                   float(temperature), _ptr(u), _ptr(tokens), _ptr(row_stats), _ptr(workspace),
+                                   wb, _stream(stream))
+    _check("s3r_sample_tokens_ex", st)
 
 
 def s3r_device_status(workspace, stream=None):

@@ -83,6 +83,7 @@ class DecodeStep:
         self.verify_out = torch.empty((S, R, Hq, D), dtype=kdt, device=dev)
         self.verify_lse = torch.empty((S, R, Hq), dtype=torch.float32, device=dev)
         self.draft_tokens = torch.empty((S, g), dtype=torch.int32, device=dev)
+        self.draft_stats = torch.empty((S, g, 2), dtype=torch.float64, device=dev)   # {max, Z} of each q_i
         self.out_tokens = torch.empty((S, R), dtype=torch.int32, device=dev)
         self.num_accepted = torch.empty((S,), dtype=torch.int32, device=dev)
 
@@ -103,7 +104,8 @@ class DecodeStep:
     def draw_draft_tokens(self, stream=None):
         ws = self.wl.spec
         s3r.s3r_sample_tokens(self.draft_logits, ws.logit_dtype, ws.num_seqs * ws.gamma, ws.vocab,
-                              ws.temperature, self.u_draft, self.draft_tokens, self.ws_tokens, stream=stream)
+                              ws.temperature, self.u_draft, self.draft_tokens, self.ws_tokens, stream=stream,
+                              row_stats=self.draft_stats)
 
     def draft(self, i: int, stream=None):
         """Draft step i: page scores and top-B (the tail page summarised from K
@@ -117,11 +119,14 @@ class DecodeStep:
         s3r.s3r_verify_attn(self.kv, self.q_verify, self.wl.spec.rows, self.scale, self.verify_out,
                             self.verify_lse, self.ws_verify, stream=stream)
 
-    def sample(self, stream=None):
+    def sample(self, stream=None, use_draft_stats=True):
+        """Exact speculative sampling; by default with the draft rows' statistics written by
+        draw_draft_tokens (s3r_spec_sample_ex), else computed inside the call."""
         ws = self.wl.spec
         s3r.s3r_spec_sample(self.target_logits, self.draft_logits, ws.logit_dtype, self.draft_tokens,
                             self.u_accept, self.u_sample, ws.num_seqs, ws.gamma, ws.vocab, ws.temperature,
-                            self.out_tokens, self.num_accepted, self.ws_sample, stream=stream)
+                            self.out_tokens, self.num_accepted, self.ws_sample, stream=stream,
+                            draft_stats=self.draft_stats if use_draft_stats else None)
 
     def round(self, stream=None):
         """One whole decode step: gamma drafts, verify, commit."""
