@@ -312,3 +312,74 @@ def spec_sample(target_logits, draft_logits, draft_tokens, u_accept, u_sample, t
     out = np.concatenate([out, np.full((S, 1), -1, dtype=np.int64)], axis=1)
     out[np.arange(S), j] = k
     return out, n_acc, accept_margin, sample_margin
+
+
+# ----------------------------------------------------------------- KV cache upkeep of a round
+# The S3R page (Abstract) has the drafter and the verifier share the policy's
+# parameters and its KV cache: a draft step adds its token's keys and values
+# to the cache, verification recomputes the round's positions with dense
+# attention (its keys and values replace the drafter's), and speculative
+# sampling commits only the accepted prefix plus one drawn token, so the
+# positions after it leave the cache. Reading: the round's positions are
+# L - R .. L - 1 (verify row r at L - R + r, as above); a write refreshes the
+# summaries of every page it touches (their valid tokens after the write).
+
+def kv_append(k_cache, v_cache, block_table, context_lens, k_new, v_new, overwrite, page_size,
+              kmin=None, kmax=None):
+    """Write n new rows per sequence and refresh the touched pages' summaries.
+
+    For sequence b with length L: the rows go to positions
+    L - overwrite .. L - overwrite + n - 1 (overwrite = 0 appends at the end;
+    overwrite > 0 first replaces the last `overwrite` positions), and the new
+    length is L - overwrite + n. k_new, v_new: [S, n, Hkv, D]. The summaries of
+    every page holding a written position are recomputed over the page's valid
+    tokens under the new length (page_summaries' definition).
+    Returns new k_cache, v_cache, context_lens, kmin, kmax (copies).
+    """
+    K = np.array(k_cache, dtype=np.float64)
+    V = np.array(v_cache, dtype=np.float64)
+    lens = np.array(context_lens, dtype=np.int64)
+    S, n = k_new.shape[0], k_new.shape[1]
+    n_tot, H, P, D = K.shape
+    kmin = np.full((n_tot, H, D), np.nan) if kmin is None else np.array(kmin, dtype=np.float64)
+    kmax = np.full((n_tot, H, D), np.nan) if kmax is None else np.array(kmax, dtype=np.float64)
+    for b in range(S):
+        start = int(lens[b]) - overwrite
+        for t in range(n):
+            pos = start + t
+            phys = int(block_table[b, pos // P])
+            K[phys, :, pos % P, :] = k_new[b, t]
+            V[phys, :, pos % P, :] = v_new[b, t]
+        new_len = start + n
+        lens[b] = new_len
+        for i in range(start // P, (new_len - 1) // P + 1) if n > 0 else ():
+            phys = int(block_table[b, i])
+            valid = min(P, new_len - i * P)
+            kmin[phys] = K[phys, :, :valid, :].min(axis=1)
+            kmax[phys] = K[phys, :, :valid, :].max(axis=1)
+    return K, V, lens, kmin, kmax
+
+
+def kv_rollback(k_cache, block_table, context_lens, num_accepted, rows, page_size, kmin, kmax):
+    """Keep the committed prefix of a round and refresh the new tail page.
+
+    After a round whose R = rows positions end the cache (length L), n_acc
+    drafts accepted: the committed length is L - R + n_acc + 1 (the round's
+    first position, whose token was committed by the previous round, plus the
+    accepted drafts). The summary of the page holding the new last position is
+    recomputed over its valid tokens. Returns new context_lens, kmin, kmax.
+    """
+    K = np.asarray(k_cache, dtype=np.float64)
+    P = page_size
+    lens = np.array(context_lens, dtype=np.int64)
+    kmin = np.array(kmin, dtype=np.float64)
+    kmax = np.array(kmax, dtype=np.float64)
+    for b in range(len(lens)):
+        new_len = int(lens[b]) - rows + int(num_accepted[b]) + 1
+        lens[b] = new_len
+        i = (new_len - 1) // P
+        phys = int(block_table[b, i])
+        valid = new_len - i * P
+        kmin[phys] = K[phys, :, :valid, :].min(axis=1)
+        kmax[phys] = K[phys, :, :valid, :].max(axis=1)
+    return lens, kmin, kmax
