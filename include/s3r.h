@@ -14,6 +14,8 @@
  *   s3r_verify_attn        dense causal attention of the gamma+1 verify rows
  *   s3r_spec_sample        accept/reject, residual or bonus draw
  *   s3r_sample_tokens      the drafter's own draw x ~ softmax(logits / T)
+ *   s3r_kv_append          a round's keys and values into the paged cache
+ *   s3r_kv_rollback        back to the committed prefix after sampling
  *
  * Conventions shared by every call
  * --------------------------------
@@ -29,8 +31,10 @@
  *   workspace again before reusing it.
  * - A call may read its inputs (queries, KV cache, block table, context
  *   lengths) while the previous kernel on the stream is still finishing,
- *   when that kernel is one of this library's (none writes another call's
- *   inputs). A kernel of the caller's that writes an input must not signal
+ *   when that kernel is one of this library's attention or sampling kernels
+ *   (none of them writes another call's inputs; s3r_kv_append and
+ *   s3r_kv_rollback, which do, let the next kernel start only when they are
+ *   done). A kernel of the caller's that writes an input must not signal
  *   programmatic launch completion before that write.
  * - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *   stream). Work is enqueued asynchronously on it; outputs are ready when the
@@ -269,6 +273,59 @@ s3r_status s3r_spec_sample_noalloc(const void* target_logits, const void* draft_
                                    const float* u_accept, const float* u_sample,
                                    int32_t num_seqs, int32_t gamma, int32_t vocab, float temperature,
                                    int32_t* out_tokens, int32_t* num_accepted, void* stream);
+
+/*
+ * KV-cache upkeep of a round (S3R page, Abstract: the drafter and the
+ * verifier share the policy's parameters and its KV cache; speculative
+ * sampling commits the accepted drafts and one drawn token, so the later
+ * positions leave the cache). A round over a cache of committed length C:
+ *   draft step i (i < gamma): s3r_kv_append(n = 1, overwrite = 0) writes the
+ *     step's key and value at position C + i, then s3r_sparse_draft_attn
+ *     attends from that position;
+ *   verification: s3r_kv_append(n = gamma + 1, overwrite = gamma) writes the
+ *     verifier's keys and values over positions C .. C + gamma (the drafter's
+ *     rows and one more), then s3r_verify_attn (rows = gamma + 1);
+ *   commit: s3r_spec_sample, then s3r_kv_rollback(rows = gamma + 1) keeps
+ *     positions up to C + n_acc.
+ * Both calls write the KV cache and the summaries (kv->k_cache, kv->v_cache
+ * are written although the struct holds them as const) and update the
+ * lengths in place: context_lens must be kv->context_lens (else
+ * S3R_ERR_INVALID_ARG). They order themselves after the previous kernel on
+ * the stream and let the next one start only when they are done, so the next
+ * call reads what they wrote.
+ *
+ * s3r_kv_append: for each sequence b with length L_b, the n rows
+ * k_new[b, t], v_new[b, t] go to positions L_b - overwrite + t (t < n), the
+ * length becomes L_b - overwrite + n, and kmin / kmax of every page holding a
+ * written position are recomputed over that page's valid tokens under the new
+ * length (the definition of s3r_page_summaries). k_new, v_new: [S, n, Hkv, D]
+ * in kv->dtype, 16-byte aligned. 0 <= n, overwrite <= 1024; n = 0 with
+ * overwrite = 0 does nothing. Device checks: a sequence with
+ * overwrite > L_b or a new length outside [1, max_pages_per_seq * P] is left
+ * unchanged (S3R_DEV_BAD_CONTEXT_LEN); a row whose page id is out of range is
+ * not written (S3R_DEV_BAD_PAGE_ID). The block-table entries of the new
+ * positions must be set by the caller beforehand (the library allocates no
+ * pages).
+ *
+ * s3r_kv_rollback: after a round of R = rows positions ending the cache,
+ * with num_accepted[b] = n_acc from s3r_spec_sample: L_b becomes
+ * L_b - rows + n_acc + 1, and the summary of the page holding the new last
+ * position is recomputed over its valid tokens. n_acc outside [0, rows - 1],
+ * or a length that would drop below 1, leaves the sequence unchanged
+ * (S3R_DEV_BAD_CONTEXT_LEN). Positions past the new length keep their old
+ * rows (never read again); their pages stay in the block table.
+ *
+ * workspace: at least s3r_kv_workspace_bytes(num_seqs) bytes, zero-filled
+ * before first use (status word and per-sequence counters, which every call
+ * leaves at zero); s3r_device_status() reads its status word.
+ */
+s3r_status s3r_kv_append(const s3r_paged_kv* kv, int32_t* context_lens, const void* k_new,
+                         const void* v_new, int32_t n, int32_t overwrite, void* kmin, void* kmax,
+                         void* workspace, size_t workspace_bytes, void* stream);
+s3r_status s3r_kv_rollback(const s3r_paged_kv* kv, int32_t* context_lens,
+                           const int32_t* num_accepted, int32_t rows, void* kmin, void* kmax,
+                           void* workspace, size_t workspace_bytes, void* stream);
+size_t s3r_kv_workspace_bytes(int32_t num_seqs);
 
 /* Workspace sizes. Return 0 for an invalid or unsupported request.
  * Attention: rows = 1 and budget_pages > 0 for s3r_sparse_draft_attn;

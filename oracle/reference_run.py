@@ -100,6 +100,38 @@ def oracle_attention_seq(wl, b, draft_steps=None):
     return oracle_attention(sequence_inputs(wl, b, draft_steps=draft_steps, sampling=False))
 
 
+def oracle_kv_round_seq(wl, b):
+    """Oracle of sequence b's round with the cache upkept: from committed
+    length C = L - R, each draft step writes its rows at the end of the cache
+    and attends sparsely from that position; verification writes its R rows
+    over the round's positions and attends densely; sampling commits; the
+    cache is rolled back to the committed prefix. Returns the selections,
+    outputs, tokens and the cache state after the round."""
+    ws = wl.spec
+    P, B, G, R, g = ws.page_size, ws.budget_pages, ws.group, ws.rows, ws.gamma
+    dt = ws.kv_dtype
+    scale = f32(wl.scale)
+    K, V, bt, phys = sequence_cache(wl, b)
+    L = int(wl.context_lens[b])
+    lens = np.array([L - R], dtype=np.int64)
+    kmin, kmax = O.page_summaries(K, bt, lens, P)
+    kd, vd, kv_, vv = (to_float64(x, dt) for x in wl.round_kv(b))
+    draft = {}
+    for i in range(g):
+        K, V, lens, kmin, kmax = O.kv_append(K, V, bt, lens, kd[i][None, None], vd[i][None, None], 0, P, kmin, kmax)
+        q = to_float64(wl.q_draft[i, b], dt)[None]
+        sel, gaps, scores = O.sparse_draft_select(q, kmin, kmax, bt, lens, P, B, G, return_scores=True)
+        out, lse = O.sparse_draft_attn(q, K, V, bt, lens, sel, scale)
+        draft[i] = {"selected": sel[0], "gaps": gaps[0], "scores": scores[0], "out": out[0], "lse": lse[0]}
+    K, V, lens, kmin, kmax = O.kv_append(K, V, bt, lens, kv_[None], vv[None], g, P, kmin, kmax)
+    qv = to_float64(wl.q_verify[b], dt)[None]
+    vout, vlse = O.verify_attn(qv, K, V, bt, lens, scale)
+    smp = oracle_sampling_seq(wl, b)
+    lens_c, kmin_c, kmax_c = O.kv_rollback(K, bt, lens, np.array([smp["n_acc"]]), R, P, kmin, kmax)
+    return {"phys": phys, "draft": draft, "verify_out": vout[0], "verify_lse": vlse[0], "sampling": smp,
+            "K": K, "V": V, "len_after": int(lens_c[0]), "kmin": kmin_c, "kmax": kmax_c, "start": L - R}
+
+
 def oracle_sampling(inp):
     """Oracle draft-token draws and speculative sampling of one sequence's
     inputs (sequence_inputs)."""

@@ -268,6 +268,46 @@ S3R_EXPORT s3r_status s3r_sample_tokens(const void* logits, s3r_dtype logit_dtyp
                               workspace_bytes, stream);
 }
 
+S3R_EXPORT size_t s3r_kv_workspace_bytes(int32_t num_seqs) {
+  if (num_seqs < 1) return 0;
+  return kv_workspace_bytes(num_seqs);
+}
+
+namespace {
+s3r_status check_kv_upkeep(const s3r_paged_kv* kv, int32_t* context_lens, void* kmin, void* kmax, void* workspace,
+                           size_t workspace_bytes) {
+  s3r_status s = check_kv(kv);
+  if (s != S3R_OK) return s;
+  if (!context_lens || !kmin || !kmax || !aligned16(kmin) || !aligned16(kmax)) return S3R_ERR_INVALID_ARG;
+  if (reinterpret_cast<const void*>(context_lens) != reinterpret_cast<const void*>(kv->context_lens))
+    return S3R_ERR_INVALID_ARG;                          // the lengths are updated where the cache reads them
+  if (!workspace || workspace_bytes < kv_workspace_bytes(kv->num_seqs)) return S3R_ERR_WORKSPACE;
+  return S3R_OK;
+}
+}  // namespace
+
+S3R_EXPORT s3r_status s3r_kv_append(const s3r_paged_kv* kv, int32_t* context_lens, const void* k_new,
+                                    const void* v_new, int32_t n, int32_t overwrite, void* kmin, void* kmax,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
+  s3r_status s = check_kv_upkeep(kv, context_lens, kmin, kmax, workspace, workspace_bytes);
+  if (s != S3R_OK) return s;
+  if (n < 0 || overwrite < 0 || n > kMaxAppendRows || overwrite > kMaxAppendRows) return S3R_ERR_INVALID_ARG;
+  if (n > 0 && (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new))) return S3R_ERR_INVALID_ARG;
+  if (n == 0 && overwrite == 0) return S3R_OK;
+  return from_cuda(launch_kv_append(*kv, context_lens, k_new, v_new, n, overwrite, kmin, kmax, workspace,
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+S3R_EXPORT s3r_status s3r_kv_rollback(const s3r_paged_kv* kv, int32_t* context_lens, const int32_t* num_accepted,
+                                      int32_t rows, void* kmin, void* kmax, void* workspace, size_t workspace_bytes,
+                                      void* stream) {
+  s3r_status s = check_kv_upkeep(kv, context_lens, kmin, kmax, workspace, workspace_bytes);
+  if (s != S3R_OK) return s;
+  if (!num_accepted || rows < 1 || rows > kMaxGamma + 1) return S3R_ERR_INVALID_ARG;
+  return from_cuda(launch_kv_rollback(*kv, context_lens, num_accepted, rows, kmin, kmax, workspace,
+                                      static_cast<cudaStream_t>(stream)));
+}
+
 S3R_EXPORT int32_t s3r_sparse_draft_kernels(const s3r_paged_kv* kv, int32_t budget_pages) {
   if (check_attn(kv, 1, budget_pages, true) != S3R_OK) return 0;
   return draft_fused_supported(*kv, budget_pages) ? 1 : 2;

@@ -17,6 +17,8 @@ constexpr int kStageTokens = 64;
 constexpr int kMaxSplitPages = 512;
 constexpr int kMaxPagesPerSeq = 8192;
 constexpr int kMaxGamma = 16;
+// Rows one s3r_kv_append call writes (or overwrites) per sequence, at most.
+constexpr int kMaxAppendRows = 1024;
 // Sequences per call (the tensor-core attention keeps a per-sequence prefix
 // of page counts in shared memory).
 constexpr int kMaxSeqs = 1024;
@@ -119,6 +121,13 @@ cudaError_t prepare_draft_fused(const s3r_paged_kv& kv, int32_t budget_pages, Dr
 cudaError_t launch_draft_fused(const s3r_paged_kv& kv, const DraftLaunch& dl, const AttnParams& p, cudaStream_t st);
 bool make_cache_map(CUtensorMap* map, const void* base, const s3r_paged_kv& kv);
 int device_sm_count();
+
+// KV-cache upkeep (s3r_kv.cu): workspace = status word + per-sequence tickets.
+size_t kv_workspace_bytes(int32_t num_seqs);
+cudaError_t launch_kv_append(const s3r_paged_kv& kv, int32_t* lens, const void* k_new, const void* v_new, int32_t n,
+                             int32_t overwrite, void* kmin, void* kmax, void* ws, cudaStream_t st);
+cudaError_t launch_kv_rollback(const s3r_paged_kv& kv, int32_t* lens, const int32_t* num_accepted, int32_t rows,
+                               void* kmin, void* kmax, void* ws, cudaStream_t st);
 
 struct SamplePlan {
   int32_t nrows;        // rows with statistics (2*gamma+1 per sequence, or num_rows)

@@ -23,7 +23,7 @@ EXPORTED = [
     "s3r_page_summaries", "s3r_page_summaries_checked", "s3r_sparse_draft_attn", "s3r_verify_attn",
     "s3r_spec_sample", "s3r_spec_sample_noalloc", "s3r_sample_tokens", "s3r_attn_workspace_bytes", "s3r_sample_workspace_bytes",
     "s3r_device_status", "s3r_status_str", "s3r_version", "s3r_sparse_draft_kernels",
-    "s3r_sample_tokens_ex", "s3r_spec_sample_ex",
+    "s3r_sample_tokens_ex", "s3r_spec_sample_ex", "s3r_kv_append", "s3r_kv_rollback", "s3r_kv_workspace_bytes",
 ]
 
 
@@ -59,6 +59,9 @@ def _load():
         "s3r_sample_tokens": ([vp, i32, i32, i32, f32, vp, vp, vp, sz, vp], i32),
         "s3r_sample_tokens_ex": ([vp, i32, i32, i32, f32, vp, vp, vp, vp, sz, vp], i32),
         "s3r_spec_sample_ex": ([vp, vp, i32, vp, vp, vp, vp, i32, i32, i32, f32, vp, vp, vp, sz, vp], i32),
+        "s3r_kv_append": ([kvp, vp, vp, vp, i32, i32, vp, vp, vp, sz, vp], i32),
+        "s3r_kv_rollback": ([kvp, vp, vp, i32, vp, vp, vp, sz, vp], i32),
+        "s3r_kv_workspace_bytes": ([i32], sz),
         "s3r_attn_workspace_bytes": ([kvp, i32, i32], sz),
         "s3r_sample_workspace_bytes": ([i32, i32, i32], sz),
         "s3r_device_status": ([vp, ctypes.POINTER(ctypes.c_uint32), vp], i32),
@@ -216,6 +219,28 @@ def s3r_device_status(workspace, stream=None):
 def s3r_sparse_draft_kernels(kv: PagedKV, budget_pages: int) -> int:
     """Kernels one s3r_sparse_draft_attn call launches (1 fused, 2 select + attention)."""
     return int(_lib.s3r_sparse_draft_kernels(ctypes.byref(kv), int(budget_pages)))
+
+
+def s3r_kv_workspace_bytes(num_seqs: int) -> int:
+    return int(_lib.s3r_kv_workspace_bytes(int(num_seqs)))
+
+
+def s3r_kv_append(kv: PagedKV, context_lens, k_new, v_new, n: int, overwrite: int, kmin, kmax, workspace,
+                  workspace_bytes=None, stream=None):
+    """Write n rows per sequence at L - overwrite.. (updating L and the touched pages' summaries)."""
+    wb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    st = _lib.s3r_kv_append(ctypes.byref(kv), _ptr(context_lens), _ptr(k_new), _ptr(v_new), int(n),
+                            int(overwrite), _ptr(kmin), _ptr(kmax), _ptr(workspace), wb, _stream(stream))
+    _check("s3r_kv_append", st)
+
+
+def s3r_kv_rollback(kv: PagedKV, context_lens, num_accepted, rows: int, kmin, kmax, workspace,
+                    workspace_bytes=None, stream=None):
+    """L <- L - rows + n_acc + 1, and the new tail page's summary."""
+    wb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    st = _lib.s3r_kv_rollback(ctypes.byref(kv), _ptr(context_lens), _ptr(num_accepted), int(rows), _ptr(kmin),
+                              _ptr(kmax), _ptr(workspace), wb, _stream(stream))
+    _check("s3r_kv_rollback", st)
 
 
 def s3r_version() -> int:

@@ -87,6 +87,16 @@ class DecodeStep:
         self.out_tokens = torch.empty((S, R), dtype=torch.int32, device=dev)
         self.num_accepted = torch.empty((S,), dtype=torch.int32, device=dev)
 
+        # the round's own keys and values (drafter rows per step, verifier rows)
+        kd, vd, kvr, vvr = zip(*(wl.round_kv(b) for b in range(S)))
+        self.k_round_draft = _to_torch(np.stack(kd, axis=1), ws.kv_dtype, dev)[:, :, None]   # [g, S, 1, Hkv, D]
+        self.v_round_draft = _to_torch(np.stack(vd, axis=1), ws.kv_dtype, dev)[:, :, None]
+        self.k_round_verify = _to_torch(np.stack(kvr), ws.kv_dtype, dev)                       # [S, R, Hkv, D]
+        self.v_round_verify = _to_torch(np.stack(vvr), ws.kv_dtype, dev)
+        self.k_round_draft = [self.k_round_draft[i].contiguous() for i in range(g)]
+        self.v_round_draft = [self.v_round_draft[i].contiguous() for i in range(g)]
+        self.lens_committed = self.context_lens - R                                             # C = L - R
+        self.ws_kv = self._ws(s3r.s3r_kv_workspace_bytes(S))
         self.ws_draft = self._ws(s3r.s3r_attn_workspace_bytes(self.kv, 1, B))
         self.ws_verify = self._ws(s3r.s3r_attn_workspace_bytes(self.kv, R, 0))
         self.ws_tokens = self._ws(s3r.s3r_sample_workspace_bytes(S * g, 0, V))
@@ -136,6 +146,31 @@ class DecodeStep:
         self.verify(stream)
         self.sample(stream)
 
+    def round_with_kv(self, stream=None):
+        """One round with the cache kept: from the committed lengths C = L - R,
+        each draft step writes its keys and values at the end of the cache
+        (s3r_kv_append) before its sparse attention; verification writes the
+        verifier's R rows over the round's positions before dense attention;
+        sampling commits and s3r_kv_rollback keeps the committed prefix. The
+        lengths start from C on every call (a copy on the stream), so rounds
+        can be repeated and captured."""
+        ws = self.wl.spec
+        g, R = ws.gamma, ws.rows
+        st = torch.cuda.current_stream(self.device) if stream is None else stream
+        with torch.cuda.stream(st):
+            self.context_lens.copy_(self.lens_committed)
+        self.draw_draft_tokens(stream)
+        for i in range(g):
+            s3r.s3r_kv_append(self.kv, self.context_lens, self.k_round_draft[i], self.v_round_draft[i], 1, 0,
+                              self.kmin, self.kmax, self.ws_kv, stream=stream)
+            self.draft(i, stream)
+        s3r.s3r_kv_append(self.kv, self.context_lens, self.k_round_verify, self.v_round_verify, R, g,
+                          self.kmin, self.kmax, self.ws_kv, stream=stream)
+        self.verify(stream)
+        self.sample(stream)
+        s3r.s3r_kv_rollback(self.kv, self.context_lens, self.num_accepted, R, self.kmin, self.kmax, self.ws_kv,
+                            stream=stream)
+
     def capture_round(self):
         """One whole round captured into a CUDA graph. The library's kernels
         chain by programmatic dependent launch, which the capture keeps as
@@ -153,7 +188,7 @@ class DecodeStep:
     def device_checks(self):
         """Status words of every workspace (synchronises)."""
         return {name: s3r.s3r_device_status(getattr(self, name))
-                for name in ("ws_draft", "ws_verify", "ws_tokens", "ws_sample")}
+                for name in ("ws_draft", "ws_verify", "ws_tokens", "ws_sample", "ws_kv")}
 
     # ---------------------------------------------------------------- bytes
     def algorithmic_bytes(self):

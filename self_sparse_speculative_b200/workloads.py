@@ -44,6 +44,7 @@ import numpy as np
 # stream ids for SeedSequence spawn keys
 _S_K, _S_V, _S_OUT_K, _S_OUT_V = 1, 2, 3, 4
 _S_QDRAFT, _S_QVERIFY, _S_LOGITS, _S_UNIF, _S_PERM, _S_LENS = 5, 6, 7, 8, 9, 10
+_S_ROUND_KV = 11
 
 
 @dataclasses.dataclass(frozen=True)
@@ -243,6 +244,28 @@ class Workload:
     def kv_bytes(self) -> int:
         ws = self.spec
         return 2 * self.num_pages_total * ws.num_kv_heads * ws.page_size * ws.head_dim * storage_itemsize(ws.kv_dtype)
+
+    # -- the keys and values a round writes (a round over the last R positions)
+    def round_kv(self, b: int):
+        """Keys and values of sequence b's round, as the model would produce
+        them: the drafter's rows of the gamma draft steps and the verifier's
+        rows of the R = gamma + 1 round positions, [gamma, Hkv, D] and
+        [R, Hkv, D] each for K and V, drawn like the cache (N(0, 1) plus the
+        workload's outlier component), in the storage dtype."""
+        ws = self.spec
+        H, D, g, R = ws.num_kv_heads, ws.head_dim, ws.gamma, ws.rows
+        out = []
+        for which, sid in (("K", 0), ("V", 1)):
+            rng = self._rng(_S_ROUND_KV, b, sid)
+            x = rng.standard_normal((g + R, H, D), dtype=np.float32)
+            if ws.kv_outliers:
+                ch, w = self._outlier[which]
+                z = 2.0 * rng.standard_normal((g + R, H), dtype=np.float32)
+                for h in range(H):
+                    x[:, h][:, ch[h]] += z[:, h][:, None] * w[h][None, :]
+            out.append(to_storage(x, ws.kv_dtype))
+        k, v = out
+        return k[:g], v[:g], k[g:], v[g:]
 
     # -- logits
     def logits_for_seq(self, b: int):

@@ -111,3 +111,28 @@ def test_sampling_argument_checks():
     assert lib.s3r_sample_tokens(FAKE, s3r.S3R_F32, 8, 1000, 1.0, FAKE, FAKE, FAKE, 16, None) == s3r.S3R_ERR_WORKSPACE
     assert lib.s3r_sample_tokens(FAKE, s3r.S3R_F32, 0, 1000, 1.0, FAKE, FAKE, FAKE, need_t, None) == s3r.S3R_ERR_INVALID_ARG
     assert lib.s3r_device_status(None, None, None) == s3r.S3R_ERR_INVALID_ARG
+
+
+def test_kv_upkeep_rejects_bad_arguments_on_the_host():
+    lib = s3r.lib()
+    kv = _kv()
+    need = s3r.s3r_kv_workspace_bytes(2)
+    assert need > 0 and s3r.s3r_kv_workspace_bytes(0) == 0
+    app = lambda **k: lib.s3r_kv_append(ctypes.byref(k.get("kv", kv)), k.get("lens", FAKE), k.get("kn", FAKE), FAKE,
+                                        k.get("n", 1), k.get("ow", 0), FAKE, FAKE, FAKE, k.get("wb", need), None)
+    # the lengths must be the cache's own (they are updated where the cache reads them)
+    assert app(lens=FAKE + 256) == s3r.S3R_ERR_INVALID_ARG
+    assert app(n=-1) == s3r.S3R_ERR_INVALID_ARG
+    assert app(ow=-2) == s3r.S3R_ERR_INVALID_ARG
+    assert app(n=2000) == s3r.S3R_ERR_INVALID_ARG
+    assert app(kn=FAKE + 8) == s3r.S3R_ERR_INVALID_ARG              # rows not 16-byte aligned
+    assert app(wb=need - 1) == s3r.S3R_ERR_WORKSPACE
+    assert app(kv=_kv(head_dim=96)) == s3r.S3R_ERR_UNSUPPORTED
+    assert app(n=0, ow=0) == s3r.S3R_OK                              # nothing to do, nothing enqueued
+    rb = lambda **k: lib.s3r_kv_rollback(ctypes.byref(kv), k.get("lens", FAKE), k.get("nacc", FAKE), k.get("rows", 5),
+                                         FAKE, FAKE, FAKE, k.get("wb", need), None)
+    assert rb(rows=0) == s3r.S3R_ERR_INVALID_ARG
+    assert rb(rows=18) == s3r.S3R_ERR_INVALID_ARG
+    assert rb(nacc=0) == s3r.S3R_ERR_INVALID_ARG
+    assert rb(lens=FAKE + 4) == s3r.S3R_ERR_INVALID_ARG
+    assert rb(wb=8) == s3r.S3R_ERR_WORKSPACE
