@@ -299,6 +299,35 @@ def cpu_baseline_leg(a, ws):
             "sample": oracle_sample_note(ws, seqs, 1, workers) + f", {secs:.2f} s"}
 
 
+def _tensor_peak():
+    try:
+        with open(os.path.join(HERE, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"])
+    except Exception:
+        return 1590.0
+
+
+def gamma_policy_note(ws, st, hbm_gbs):
+    """The library's draft-length policy on this workload: acceptance
+    measured from the step's counts, round costs from its roofline model at
+    the HBM peak used above and the bf16 tensor peak; the draft length it
+    would choose next (0: drafting off) and the rate gain over plain decoding."""
+    from self_sparse_speculative_b200 import s3r
+    tf = _tensor_peak()
+    L = float(np.mean(st.wl.context_lens))
+    kvb = 2 if ws.kv_dtype == "bf16" else 4
+    lb = 2 if ws.logit_dtype == "bf16" else 4
+    gmax = 8 if ws.gamma <= 8 else ws.gamma
+    cost = [s3r.s3r_round_cost_us(ws.num_seqs, ws.num_q_heads, ws.num_kv_heads, ws.head_dim, ws.page_size, kvb, L,
+                                  ws.budget_pages, ws.vocab, lb, g, hbm_gbs, tf) for g in range(gmax + 1)]
+    pol = s3r.GammaPolicyHandle(gmax, 0.9, 0.5, 1.0, cost)
+    pol.update(st.num_accepted.cpu().tolist(), ws.gamma)
+    g, alpha, rate = pol.choose()
+    return {"acceptance_estimate": round(alpha, 4), "gamma_next": g,
+            "model_rate_gain_vs_plain_decode": round(rate * cost[0], 3),
+            "cost_model": f"roofline at {hbm_gbs:.0f} GB/s and {tf:.0f} TFLOP/s"}
+
+
 def run_ours(a):
     world0 = int(os.environ.get("WORLD_SIZE", "1"))
     # the CPU leg first, before this process touches the GPU
@@ -510,6 +539,7 @@ def run_ours(a):
         line["graph"] = graph_info
     if e2e:
         line["e2e"] = {k: (round(v, 1) if isinstance(v, float) else v) for k, v in e2e.items()}
+    line["gamma_policy"] = gamma_policy_note(ws, st, peak)
     if cpu_line is not None:
         line["cpu_baseline"] = cpu_line
     print(json.dumps(line), flush=True)

@@ -327,6 +327,61 @@ s3r_status s3r_kv_rollback(const s3r_paged_kv* kv, int32_t* context_lens,
                            void* workspace, size_t workspace_bytes, void* stream);
 size_t s3r_kv_workspace_bytes(int32_t num_seqs);
 
+/*
+ * Draft-length policy (host only; every pointer here is a host pointer): the
+ * acceptance-aware draft length with a regime toggle that the researchpod.app
+ * page describes for EfficientRollout (drafting only when it speeds the step
+ * up, which depends on whether the step is compute- or memory-bound; a draft
+ * length that follows how often drafts are accepted).
+ *   alpha    = accepted / tested draft positions (a round tests the accepted
+ *              drafts and the first rejected one), each round's counts
+ *              weighted by decay^age, started from prior_accept with weight
+ *              prior_weight;
+ *   E(g)     = sum_{i=0}^{g} alpha^i committed tokens per sequence and round
+ *              (the speculative-decoding papers on the mlsanity.com list);
+ *   rate(g)  = E(g) / cost_us[g] for g >= 1, rate(0) = 1 / cost_us[0] (a
+ *              plain decode step commits one token);
+ *   choose   = the g in 0..gamma_max with the largest rate (the smaller g on
+ *              ties); 0 switches drafting off.
+ * cost_us[g]: the time of a round with g drafts, measured by the caller or
+ * from s3r_round_cost_us. The struct is plain data owned by the caller.
+ */
+typedef struct {
+  int32_t gamma_max;
+  double decay;
+  double accepted;
+  double tested;
+  double cost_us[17];
+} s3r_gamma_policy;
+
+s3r_status s3r_gamma_policy_init(s3r_gamma_policy* policy, int32_t gamma_max, double decay,
+                                 double prior_accept, double prior_weight, const double* cost_us);
+/* One round's acceptance counts (num_accepted: host int32 [num_seqs], each in
+ * [0, gamma_used]). */
+s3r_status s3r_gamma_policy_update(s3r_gamma_policy* policy, const int32_t* num_accepted,
+                                   int32_t num_seqs, int32_t gamma_used);
+/* The next draft length (0: drafting off) and, if not NULL, the acceptance
+ * estimate and the chosen rate (committed tokens per microsecond). */
+s3r_status s3r_gamma_policy_choose(const s3r_gamma_policy* policy, int32_t* gamma, double* alpha,
+                                   double* rate);
+/*
+ * Roofline times in microseconds (NaN for invalid arguments). Dense attention
+ * of `rows` query rows per sequence over the whole cache: max(bytes of every
+ * key and value / hbm_gbs, 4 Hq rows L D flops / tensor_tflops), so it is
+ * memory-bound at small batch x rows and compute-bound beyond. A round with
+ * gamma >= 1 drafts: gamma sparse draft calls (every page's summary and the
+ * kept pages' keys and values), verification of gamma + 1 rows, the drafter's
+ * draws (gamma rows) and speculative sampling (2 gamma + 1 rows and two
+ * re-read); gamma = 0: one dense decode row and one draw.
+ */
+double s3r_attend_cost_us(int32_t num_seqs, int32_t q_heads, int32_t kv_heads, int32_t head_dim,
+                          int32_t kv_bytes, double mean_context, int32_t rows, double hbm_gbs,
+                          double tensor_tflops);
+double s3r_round_cost_us(int32_t num_seqs, int32_t q_heads, int32_t kv_heads, int32_t head_dim,
+                         int32_t page_size, int32_t kv_bytes, double mean_context, int32_t budget_pages,
+                         int32_t vocab, int32_t logit_bytes, int32_t gamma, double hbm_gbs,
+                         double tensor_tflops);
+
 /* Workspace sizes. Return 0 for an invalid or unsupported request.
  * Attention: rows = 1 and budget_pages > 0 for s3r_sparse_draft_attn;
  * rows = gamma + 1 and budget_pages = 0 for s3r_verify_attn.
@@ -360,6 +415,16 @@ s3r_status s3r_device_status(const void* workspace, uint32_t* bits, void* stream
 s3r_status s3r_page_summaries_checked(const s3r_paged_kv* kv, int32_t tail_only,
                                       void* kmin, void* kmax, uint32_t* status_word,
                                       void* stream);
+
+/*
+ * Diagnostic: the float64 exponential the sampling kernels use for their
+ * draw weights (a table-driven method after P. T. P. Tang, ACM TOMS 15(2),
+ * 1989, with its range fix-up), y_tbl[i] = exp(x[i]), beside CUDA's own
+ * exp(x[i]) in y_ref[i] evaluated on the same device. x, y_tbl, y_ref:
+ * float64 device arrays of n elements. For tests of the sampler's arithmetic;
+ * no part of the decode step calls it.
+ */
+s3r_status s3r_debug_exp64(const double* x, double* y_tbl, double* y_ref, int32_t n, void* stream);
 
 /* Human-readable name of a status code (static storage). */
 const char* s3r_status_str(s3r_status status);

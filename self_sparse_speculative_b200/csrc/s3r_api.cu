@@ -308,6 +308,11 @@ S3R_EXPORT s3r_status s3r_kv_rollback(const s3r_paged_kv* kv, int32_t* context_l
                                       static_cast<cudaStream_t>(stream)));
 }
 
+S3R_EXPORT s3r_status s3r_debug_exp64(const double* x, double* y_tbl, double* y_ref, int32_t n, void* stream) {
+  if (!x || !y_tbl || !y_ref || n < 1) return S3R_ERR_INVALID_ARG;
+  return from_cuda(launch_exp64_probe(x, y_tbl, y_ref, n, static_cast<cudaStream_t>(stream)));
+}
+
 S3R_EXPORT int32_t s3r_sparse_draft_kernels(const s3r_paged_kv* kv, int32_t budget_pages) {
   if (check_attn(kv, 1, budget_pages, true) != S3R_OK) return 0;
   return draft_fused_supported(*kv, budget_pages) ? 1 : 2;

@@ -172,5 +172,6 @@ struct SampleParams {
 // Fill the workspace pointers and sizes of `p` from a plan and a workspace base.
 void bind_sample_workspace(SampleParams* p, const SamplePlan& pl, void* ws);
 cudaError_t launch_sampling(const SampleParams& p, s3r_dtype dt, bool spec, cudaStream_t st);
+cudaError_t launch_exp64_probe(const double* x, double* y_tbl, double* y_ref, int n, cudaStream_t st);
 
 }  // namespace s3r

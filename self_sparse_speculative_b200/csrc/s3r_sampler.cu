@@ -892,7 +892,27 @@ cudaError_t launch_typed(const SampleParams& p, cudaStream_t st) {
   return launch_kernel(draw_kernel<T, SPEC, false>, dim3(p.c2 * p.nseq), blk, 0, st, 1, p);
 }
 
+// Diagnostic: the sampler's float64 exponential (exp_tbl with exp_fixup, as
+// the draw kernels evaluate it) and CUDA's exp() of the same arguments.
+__global__ void __launch_bounds__(kSmpThreads) exp64_probe_kernel(const double* x, double* y_tbl, double* y_ref,
+                                                                  int n) {
+  __shared__ double s_tab[kExpTab];
+  fill_exp_tab(s_tab);
+  __syncthreads();
+  for (int i = blockIdx.x * kSmpThreads + threadIdx.x; i < n; i += gridDim.x * kSmpThreads) {
+    const double v = x[i];
+    y_tbl[i] = exp_fixup(v, exp_tbl(v, s_tab), s_tab);
+    y_ref[i] = exp(v);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_exp64_probe(const double* x, double* y_tbl, double* y_ref, int n, cudaStream_t st) {
+  const int grid = (n + kSmpThreads - 1) / kSmpThreads < 1184 ? (n + kSmpThreads - 1) / kSmpThreads : 1184;
+  exp64_probe_kernel<<<grid, kSmpThreads, 0, st>>>(x, y_tbl, y_ref, n);
+  return cudaGetLastError();
+}
 
 SamplePlan plan_sampling(int32_t nseq, int32_t gamma, int32_t vocab, int32_t elt) {
   SamplePlan pl{};

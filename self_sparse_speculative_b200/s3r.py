@@ -24,6 +24,8 @@ EXPORTED = [
     "s3r_spec_sample", "s3r_spec_sample_noalloc", "s3r_sample_tokens", "s3r_attn_workspace_bytes", "s3r_sample_workspace_bytes",
     "s3r_device_status", "s3r_status_str", "s3r_version", "s3r_sparse_draft_kernels",
     "s3r_sample_tokens_ex", "s3r_spec_sample_ex", "s3r_kv_append", "s3r_kv_rollback", "s3r_kv_workspace_bytes",
+    "s3r_debug_exp64", "s3r_gamma_policy_init", "s3r_gamma_policy_update", "s3r_gamma_policy_choose",
+    "s3r_attend_cost_us", "s3r_round_cost_us",
 ]
 
 
@@ -31,6 +33,11 @@ class S3RError(RuntimeError):
     def __init__(self, fn: str, status: int):
         self.status = status
         super().__init__(f"{fn} failed: {status_str(status)}")
+
+
+class GammaPolicy(ctypes.Structure):
+    _fields_ = [("gamma_max", ctypes.c_int32), ("decay", ctypes.c_double), ("accepted", ctypes.c_double),
+                ("tested", ctypes.c_double), ("cost_us", ctypes.c_double * 17)]
 
 
 class PagedKV(ctypes.Structure):
@@ -47,7 +54,7 @@ def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"libs3r.so is not built ({LIB_PATH}); run python -m self_sparse_speculative_b200.build")
     lib = ctypes.CDLL(LIB_PATH)
-    vp, i32, f32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+    vp, i32, f32, sz, f64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t, ctypes.c_double
     kvp = ctypes.POINTER(PagedKV)
     sig = {
         "s3r_page_summaries": ([kvp, i32, vp, vp, vp], i32),
@@ -62,6 +69,13 @@ def _load():
         "s3r_kv_append": ([kvp, vp, vp, vp, i32, i32, vp, vp, vp, sz, vp], i32),
         "s3r_kv_rollback": ([kvp, vp, vp, i32, vp, vp, vp, sz, vp], i32),
         "s3r_kv_workspace_bytes": ([i32], sz),
+        "s3r_debug_exp64": ([vp, vp, vp, i32, vp], i32),
+        "s3r_gamma_policy_init": ([ctypes.POINTER(GammaPolicy), i32, f64, f64, f64, ctypes.POINTER(f64)], i32),
+        "s3r_gamma_policy_update": ([ctypes.POINTER(GammaPolicy), ctypes.POINTER(i32), i32, i32], i32),
+        "s3r_gamma_policy_choose": ([ctypes.POINTER(GammaPolicy), ctypes.POINTER(i32), ctypes.POINTER(f64),
+                                     ctypes.POINTER(f64)], i32),
+        "s3r_attend_cost_us": ([i32, i32, i32, i32, i32, f64, i32, f64, f64], f64),
+        "s3r_round_cost_us": ([i32, i32, i32, i32, i32, i32, f64, i32, i32, i32, i32, f64, f64], f64),
         "s3r_attn_workspace_bytes": ([kvp, i32, i32], sz),
         "s3r_sample_workspace_bytes": ([i32, i32, i32], sz),
         "s3r_device_status": ([vp, ctypes.POINTER(ctypes.c_uint32), vp], i32),
@@ -241,6 +255,45 @@ def s3r_kv_rollback(kv: PagedKV, context_lens, num_accepted, rows: int, kmin, km
     st = _lib.s3r_kv_rollback(ctypes.byref(kv), _ptr(context_lens), _ptr(num_accepted), int(rows), _ptr(kmin),
                               _ptr(kmax), _ptr(workspace), wb, _stream(stream))
     _check("s3r_kv_rollback", st)
+
+
+def s3r_debug_exp64(x, y_tbl, y_ref, stream=None):
+    """The sampler's float64 exponential of x (y_tbl) and CUDA's exp (y_ref), float64 device tensors."""
+    st = _lib.s3r_debug_exp64(_ptr(x), _ptr(y_tbl), _ptr(y_ref), int(x.numel()), _stream(stream))
+    _check("s3r_debug_exp64", st)
+
+
+class GammaPolicyHandle:
+    """The library's draft-length policy (host code): init, update with a round's
+    acceptance counts, choose the next gamma (0: drafting off)."""
+
+    def __init__(self, gamma_max: int, decay: float, prior_accept: float, prior_weight: float, cost_us):
+        self.p = GammaPolicy()
+        c = (ctypes.c_double * 17)(*[float(x) for x in cost_us])
+        _check("s3r_gamma_policy_init", _lib.s3r_gamma_policy_init(ctypes.byref(self.p), int(gamma_max),
+                                                                   float(decay), float(prior_accept),
+                                                                   float(prior_weight), c))
+
+    def update(self, num_accepted, gamma_used: int):
+        n = [int(x) for x in num_accepted]
+        arr = (ctypes.c_int32 * len(n))(*n)
+        _check("s3r_gamma_policy_update", _lib.s3r_gamma_policy_update(ctypes.byref(self.p), arr, len(n),
+                                                                       int(gamma_used)))
+
+    def choose(self):
+        """(gamma, alpha, rate)."""
+        g, a, r = ctypes.c_int32(0), ctypes.c_double(0), ctypes.c_double(0)
+        _check("s3r_gamma_policy_choose", _lib.s3r_gamma_policy_choose(ctypes.byref(self.p), ctypes.byref(g),
+                                                                       ctypes.byref(a), ctypes.byref(r)))
+        return int(g.value), float(a.value), float(r.value)
+
+
+def s3r_attend_cost_us(*args) -> float:
+    return float(_lib.s3r_attend_cost_us(*args))
+
+
+def s3r_round_cost_us(*args) -> float:
+    return float(_lib.s3r_round_cost_us(*args))
 
 
 def s3r_version() -> int:

@@ -14,7 +14,7 @@ HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))
 
 def _declared():
     text = open(HEADER).read()
-    return sorted(set(re.findall(r"\b(s3r_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(s3r_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_declares_and_library_exports_every_entry_point():
