@@ -383,3 +383,149 @@ def kv_rollback(k_cache, block_table, context_lens, num_accepted, rows, page_siz
         kmin[phys] = K[phys, :, :valid, :].min(axis=1)
         kmax[phys] = K[phys, :, :valid, :].max(axis=1)
     return lens, kmin, kmax
+
+
+# ----------------------------------------------------------------- tree verification
+# The ai.info SpecRoll page (another speculative method for RL rollouts)
+# verifies a sparse tree of proposals instead of a chain: each round gives a
+# response a node budget N_t = clip(floor(C_hw / B_t), N_min, N_max) (C_hw the
+# profiled capacity, B_t the unfinished responses), and exact rejection
+# sampling with the target-residual fallback stays authoritative at every
+# visited node, so the committed tokens still follow the target policy.
+# Readings: a tree of R nodes in topological order (parent[0] = -1 is the
+# round's first position, parent[i] < i), stored in the cache at the round's
+# R positions in node order; node i attends to the committed history and to
+# its ancestors and itself; the children of a node were drawn i.i.d. from
+# that node's draft distribution and are tried in index order (each
+# rejection replaces the target by its normalised residual), the sampling
+# rule the speculative-sampling papers give for several drafts.
+
+def node_budget(capacity, active, n_min, n_max):
+    """N_t = clip(floor(C_hw / B_t), N_min, N_max)."""
+    return int(min(max(capacity // active, n_min), n_max))
+
+
+def tree_ancestor_masks(parents):
+    """Bit j of mask[i] is set iff node j is node i or one of its ancestors."""
+    R = len(parents)
+    masks = [0] * R
+    for i in range(R):
+        m, v = 0, i
+        while v >= 0:
+            m |= 1 << v
+            v = int(parents[v])
+        masks[i] = m
+    return masks
+
+
+def tree_verify_attn(q, k_cache, v_cache, block_table, context_lens, parents, scale):
+    """Dense attention of the R tree nodes of each sequence: node i sits at
+    slot L - R + i and sees every key before L - R and the slots of its
+    ancestors and itself. q [S, R, Hq, D], parents [S, R].
+    Returns out [S, R, Hq, D], lse [S, R, Hq]."""
+    S, R, Hq, D = q.shape
+    H, P = k_cache.shape[1], k_cache.shape[2]
+    G = Hq // H
+    out = np.zeros((S, R, Hq, D))
+    lse = np.zeros((S, R, Hq))
+    for b in range(S):
+        L = int(context_lens[b])
+        n_b = -(-L // P)
+        masks = tree_ancestor_masks(parents[b])
+        for h in range(H):
+            K, pos = _gather_tokens(k_cache, block_table, b, h, range(n_b), L, P)
+            V, _ = _gather_tokens(v_cache, block_table, b, h, range(n_b), L, P)
+            heads = range(h * G, (h + 1) * G)
+            qr = np.stack([q[b, r, hq] for r in range(R) for hq in heads])
+            node = np.array([r for r in range(R) for _ in heads])
+            j = pos[None, :] - (L - R)                                     # tree slot of each key (< 0: history)
+            m = np.array(masks)[node][:, None]
+            valid = (j < 0) | ((m >> np.maximum(j, 0)) & 1).astype(bool)
+            o, s = attend(qr, K, V, valid, scale)
+            i = 0
+            for r in range(R):
+                for hq in heads:
+                    out[b, r, hq] = o[i]
+                    lse[b, r, hq] = s[i]
+                    i += 1
+    return out, lse
+
+
+def tree_spec_sample(target_logits, draft_logits, tokens, parents, u_accept, u_sample, temperature):
+    """Exact speculative sampling over a tree, per sequence.
+
+    p_v = softmax(target_logits[v] / T), q_v = softmax(draft_logits[v] / T)
+    (the distribution node v's children were drawn from). From the root:
+    at node v the children c (ascending index) are tested in turn, accept c iff
+    u_accept[c] < p'(x_c) / q_v(x_c) with p' = p_v at first and, after each
+    rejection, p' = max(p' - q_v, 0) normalised (p' itself where that is all
+    zero); an accepted child commits its token and becomes v. When no child
+    is accepted (or v has none) the token drawn from p' with u_sample[v]
+    (inverse CDF) is committed and the round ends.
+    target_logits, draft_logits [S, R, V]; tokens, parents, u_accept,
+    u_sample [S, R]. Returns out_tokens [S, R] (committed tokens, then -1),
+    n_acc [S] (accepted nodes), path [S, R] (the accepted nodes, then -1), and
+    the margins of every accept test and of the final draw (for near-ties).
+    """
+    S, R, V = target_logits.shape
+    p = softmax_t(target_logits, temperature)
+    q = softmax_t(draft_logits, temperature)
+    out = np.full((S, R), -1, dtype=np.int64)
+    path = np.full((S, R), -1, dtype=np.int64)
+    n_acc = np.zeros(S, dtype=np.int64)
+    accept_margins = [[] for _ in range(S)]
+    draw_margin = np.zeros(S)
+    for b in range(S):
+        v, depth = 0, 0
+        while True:
+            children = [c for c in range(R) if int(parents[b, c]) == v]
+            pr = p[b, v]
+            nxt = None
+            for c in children:
+                x = int(tokens[b, c])
+                qx = q[b, v, x]
+                ratio = pr[x] / qx if qx > 0 else 0.0
+                accept_margins[b].append(abs(float(u_accept[b, c]) - ratio))
+                if float(u_accept[b, c]) < ratio:
+                    nxt = c
+                    break
+                resid = residual_weights(pr, q[b, v])
+                pr = resid / resid.sum()
+            if nxt is None:
+                k, margin = inverse_cdf(pr[None], np.array([float(u_sample[b, v])]))
+                out[b, depth] = int(k[0])
+                draw_margin[b] = float(margin[0])
+                break
+            out[b, depth] = int(tokens[b, nxt])
+            path[b, depth] = nxt
+            depth += 1
+            v = nxt
+        n_acc[b] = depth
+    return out, n_acc, path, accept_margins, draw_margin
+
+
+def chain_parents(R):
+    """The chain tree (ordinary speculative decoding): parent[i] = i - 1."""
+    return np.arange(-1, R - 1)
+
+
+def build_tree(n_nodes, branching):
+    """A tree of n_nodes in breadth-first order: every node of depth d gets
+    branching[d] children (the last entry repeats) until n_nodes exist.
+    Returns parents [n_nodes]. Reading: SpecRoll picks the tree from its
+    heads' candidate probabilities; without those heads the shape is given."""
+    parents = [-1]
+    frontier = [0]
+    d = 0
+    while len(parents) < n_nodes and frontier:
+        k = branching[min(d, len(branching) - 1)]
+        nxt = []
+        for v in frontier:
+            for _ in range(k):
+                if len(parents) >= n_nodes:
+                    break
+                parents.append(v)
+                nxt.append(len(parents) - 1)
+        frontier = nxt
+        d += 1
+    return np.array(parents, dtype=np.int64)
