@@ -439,8 +439,8 @@ def tree_verify_attn(q, k_cache, v_cache, block_table, context_lens, parents, sc
             qr = np.stack([q[b, r, hq] for r in range(R) for hq in heads])
             node = np.array([r for r in range(R) for _ in heads])
             j = pos[None, :] - (L - R)                                     # tree slot of each key (< 0: history)
-            m = np.array(masks)[node][:, None]
-            valid = (j < 0) | ((m >> np.maximum(j, 0)) & 1).astype(bool)
+            m = np.array(masks, dtype=np.uint64)[node][:, None]                # up to 64 nodes: unsigned
+            valid = (j < 0) | ((m >> np.maximum(j, 0).astype(np.uint64)) & np.uint64(1)).astype(bool)
             o, s = attend(qr, K, V, valid, scale)
             i = 0
             for r in range(R):

@@ -65,13 +65,18 @@ def _paged(rng, S, H, P, D, lens):
     return rng.standard_normal((total, H, P, D)), rng.standard_normal((total, H, P, D)), bt, np.array(lens)
 
 
-def test_tree_attention_equals_masked_sdpa_and_chain_equals_verify():
+@pytest.mark.parametrize("R,lens", [(7, [50, 23]), (64, [64, 90])])
+def test_tree_attention_equals_masked_sdpa_and_chain_equals_verify(R, lens):
+    """R = 64: the widest tree, every bit of a 64-bit ancestor mask in use."""
     rng = np.random.default_rng(1)
     P, D, H, G = 16, 32, 2, 3
-    S, R = 2, 7
-    k, v, bt, lens = _paged(rng, S, H, P, D, [50, 23])
+    S = 2
+    k, v, bt, lens = _paged(rng, S, H, P, D, lens)
     q = rng.standard_normal((S, R, G * H, D))
-    par = np.stack([O.build_tree(R, [3, 1]), O.build_tree(R, [1, 2])])
+    if R == 7:
+        par = np.stack([O.build_tree(R, [3, 1]), O.build_tree(R, [1, 2])])
+    else:
+        par = np.stack([O.build_tree(R, [2]), np.array([-1] + [int(rng.integers(0, c)) for c in range(1, R)])])
     out, _ = O.tree_verify_attn(q, k, v, bt, lens, par, 0.2)
     for b in range(S):
         L = int(lens[b])
