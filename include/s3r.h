@@ -16,6 +16,8 @@
  *   s3r_sample_tokens      the drafter's own draw x ~ softmax(logits / T)
  *   s3r_kv_append          a round's keys and values into the paged cache
  *   s3r_kv_rollback        back to the committed prefix after sampling
+ *   s3r_verify_attn_tree   verification of a token tree (ancestor masks)
+ *   s3r_tree_spec_sample   exact speculative sampling walked over the tree
  *
  * Conventions shared by every call
  * --------------------------------
@@ -80,6 +82,7 @@ typedef enum { S3R_F32 = 0, S3R_BF16 = 1 } s3r_dtype;
 #define S3R_DEV_BAD_PAGE_ID      0x2u  /* block-table entry outside [0, num_pages_total)    */
 #define S3R_DEV_BAD_TOKEN_ID     0x4u  /* draft token outside [0, vocab)                    */
 #define S3R_DEV_WAIT_TIMEOUT     0x8u  /* an in-kernel wait ran past its limit              */
+#define S3R_DEV_BAD_TREE         0x10u /* a tree parent entry outside [0, node) (root: -1)  */
 
 /*
  * A paged KV cache (PagedAttention's block tables, cited on the mlsanity.com
@@ -166,6 +169,66 @@ s3r_status s3r_sparse_draft_attn(const s3r_paged_kv* kv, const void* kmin, const
 s3r_status s3r_verify_attn(const s3r_paged_kv* kv, const void* q, int32_t rows, float scale,
                            void* out, float* lse,
                            void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Tree verification attention (the ai.info SpecRoll page: sparse-tree
+ * verification of candidate continuations, exact target verification at every
+ * visited node). The round's R = `nodes` tree nodes of sequence b occupy
+ * positions L_b - R .. L_b - 1 in node order; node i sees every key before
+ * L_b - R and the slots of its ancestors and itself:
+ *   visible(i, L_b - R + j) = j is i or an ancestor of i.
+ * A chain (parents[b, i] = i - 1) gives s3r_verify_attn with rows = R.
+ * parents: int32 [S, R], parents[b, 0] = -1, 0 <= parents[b, i] < i; an
+ *   entry breaking that rule is flagged (S3R_DEV_BAD_TREE) and the node's
+ *   ancestor walk ends there.
+ * q, out: [S, R, Hq, D] in kv->dtype; lse: float32 [S, R, Hq] or NULL.
+ * Supported: R <= 64, G * R <= 64 (bf16) or <= 128 (f32).
+ * workspace: at least s3r_attn_workspace_bytes(kv, R, 0) bytes.
+ */
+s3r_status s3r_verify_attn_tree(const s3r_paged_kv* kv, const void* q, int32_t nodes,
+                                const int32_t* parents, float scale, void* out, float* lse,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Exact speculative sampling over a token tree (the ai.info SpecRoll page:
+ * exact rejection sampling and the target-residual fallback at every visited
+ * node keep the committed tokens on the target distribution).
+ *   p_v = softmax(target_logits[b,v] / T); q_v = softmax(draft_logits[b,v] / T),
+ *   the distribution the children of node v were drawn from.
+ *   From the root v = 0: the children c of v (ascending index) are tested in
+ *   turn, accept c iff u_accept[b,c] < p'(x_c) / q_v(x_c) (q_v(x_c) = 0
+ *   rejects), x_c = tokens[b,c]; p' = p_v at first and after each rejection
+ *   p' <- max(p' - q_v, 0) normalised (p' renormalised where that is zero
+ *   everywhere). An accepted child commits its token and becomes v. When no
+ *   child is accepted, or v is a leaf, the token drawn from p' with
+ *   u_sample[b,v] (the inverse-CDF rule of s3r_spec_sample) is committed.
+ * target_logits, draft_logits: [S, R, V] in logit_dtype (draft rows of leaves
+ *   are not read). tokens, parents: int32 [S, R] (tokens[b,0] unused; parents
+ *   as for s3r_verify_attn_tree; a tree breaking the rule is flagged and the
+ *   walk draws at the root). u_accept, u_sample: float32 [S, R] in [0, 1).
+ * out_tokens: int32 [S, R], the n_acc accepted tokens, the drawn token, then
+ *   -1. num_accepted: int32 [S]. path: int32 [S, R] or NULL, the accepted
+ *   nodes in order, then -1 (which cache rows to keep).
+ * Sums and decisions in float64. Supported: R <= 64.
+ * workspace: at least s3r_tree_sample_workspace_bytes(S, R, V) bytes (the
+ *   status word).
+ */
+size_t s3r_tree_sample_workspace_bytes(int32_t num_seqs, int32_t nodes, int32_t vocab);
+s3r_status s3r_tree_spec_sample(const void* target_logits, const void* draft_logits,
+                                s3r_dtype logit_dtype, const int32_t* tokens, const int32_t* parents,
+                                const float* u_accept, const float* u_sample,
+                                int32_t num_seqs, int32_t nodes, int32_t vocab, float temperature,
+                                int32_t* out_tokens, int32_t* num_accepted, int32_t* path,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Concurrency-aware node budget of the ai.info SpecRoll page (host):
+ *   N_t = clip(floor(capacity / active), n_min, n_max)
+ * with `active` the unfinished responses B_t and `capacity` the profiled
+ * verification capacity C_hw in tree nodes. Returns -1 for active < 1,
+ * n_min < 1, n_max < n_min or capacity < 0.
+ */
+int32_t s3r_tree_node_budget(int64_t capacity, int32_t active, int32_t n_min, int32_t n_max);
 
 /*
  * Exact speculative sampling of one round (S3R page, Abstract: "exact
@@ -384,7 +447,8 @@ double s3r_round_cost_us(int32_t num_seqs, int32_t q_heads, int32_t kv_heads, in
 
 /* Workspace sizes. Return 0 for an invalid or unsupported request.
  * Attention: rows = 1 and budget_pages > 0 for s3r_sparse_draft_attn;
- * rows = gamma + 1 and budget_pages = 0 for s3r_verify_attn.
+ * rows = gamma + 1 and budget_pages = 0 for s3r_verify_attn; rows = nodes
+ * (up to 64) and budget_pages = 0 for s3r_verify_attn_tree.
  * Sampling: (num_seqs, gamma, vocab) for s3r_spec_sample;
  * (num_rows, 0, vocab) for s3r_sample_tokens. */
 size_t s3r_attn_workspace_bytes(const s3r_paged_kv* kv, int32_t rows, int32_t budget_pages);

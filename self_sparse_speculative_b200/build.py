@@ -23,7 +23,7 @@ LIB = os.path.join(HERE, "libs3r.so")
 INCLUDE = os.path.join(ROOT, "include")
 
 SOURCES = ["s3r_api.cu", "s3r_summaries.cu", "s3r_select.cu", "s3r_attn.cu", "s3r_attn_tc.cu", "s3r_attn_tok.cu", "s3r_draft_fused.cu", "s3r_kv.cu", "s3r_sampler.cu",
-           "s3r_noalloc.cu", "s3r_policy.cu"]
+           "s3r_noalloc.cu", "s3r_policy.cu", "s3r_tree.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr",
               "-Xcompiler", "-fPIC,-fvisibility=hidden", "-I" + INCLUDE]

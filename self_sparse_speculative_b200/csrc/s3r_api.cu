@@ -33,14 +33,17 @@ s3r_status check_kv(const s3r_paged_kv* kv) {
   return S3R_OK;
 }
 
-s3r_status check_attn(const s3r_paged_kv* kv, int32_t rows, int32_t budget, bool sparse) {
+// max_dense_rows: rows of a dense call (gamma + 1 for s3r_verify_attn; the
+// workspace query also serves s3r_verify_attn_tree's up to 64 nodes)
+s3r_status check_attn(const s3r_paged_kv* kv, int32_t rows, int32_t budget, bool sparse,
+                      int32_t max_dense_rows = kMaxGamma + 1) {
   s3r_status s = check_kv(kv);
   if (s != S3R_OK) return s;
   if (rows < 1) return S3R_ERR_INVALID_ARG;
   if (sparse && budget < 1) return S3R_ERR_INVALID_ARG;
   const int G = kv->num_q_heads / kv->num_kv_heads;
   if ((int64_t)G * rows > 128) return S3R_ERR_UNSUPPORTED;
-  if (!sparse && rows > kMaxGamma + 1) return S3R_ERR_UNSUPPORTED;
+  if (!sparse && rows > max_dense_rows) return S3R_ERR_UNSUPPORTED;
   if (kv->num_seqs > kMaxSeqs) return S3R_ERR_UNSUPPORTED;
   return S3R_OK;
 }
@@ -99,7 +102,7 @@ S3R_EXPORT const char* s3r_status_str(s3r_status s) {
 S3R_EXPORT int32_t s3r_version(void) { return 100; }
 
 S3R_EXPORT size_t s3r_attn_workspace_bytes(const s3r_paged_kv* kv, int32_t rows, int32_t budget_pages) {
-  if (check_attn(kv, rows, budget_pages, budget_pages > 0) != S3R_OK || budget_pages < 0) return 0;
+  if (check_attn(kv, rows, budget_pages, budget_pages > 0, kMaxTreeNodes) != S3R_OK || budget_pages < 0) return 0;
   return plan_attention(*kv, rows, budget_pages).ws_bytes;
 }
 
@@ -186,6 +189,65 @@ S3R_EXPORT s3r_status s3r_verify_attn(const s3r_paged_kv* kv, const void* q, int
   cudaError_t e = launch_attention(*kv, p, st, &api);
   if (api != S3R_OK) return api;
   return from_cuda(e);
+}
+
+S3R_EXPORT s3r_status s3r_verify_attn_tree(const s3r_paged_kv* kv, const void* q, int32_t nodes,
+                                           const int32_t* parents, float scale, void* out, float* lse,
+                                           void* workspace, size_t workspace_bytes, void* stream) {
+  s3r_status s = check_kv(kv);
+  if (s != S3R_OK) return s;
+  if (nodes < 1 || !parents) return S3R_ERR_INVALID_ARG;
+  const int G = kv->num_q_heads / kv->num_kv_heads;
+  if (nodes > kMaxTreeNodes || kv->num_seqs > kMaxSeqs) return S3R_ERR_UNSUPPORTED;
+  // bf16: the token-major kernel (all packed rows of a unit in one MMA of at
+  // most 64 columns); f32: up to 128 packed rows
+  if ((int64_t)G * nodes > (kv->dtype == S3R_BF16 ? 64 : 128)) return S3R_ERR_UNSUPPORTED;
+  if (!q || !out || !aligned16(q) || !aligned16(out) || !std::isfinite(scale)) return S3R_ERR_INVALID_ARG;
+  const AttnPlan pl = plan_attention(*kv, nodes, 0);
+  if (!workspace || workspace_bytes < pl.ws_bytes) return S3R_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  AttnParams p = make_attn_params(kv, pl, q, out, lse, nodes, 0, nullptr, scale, workspace);
+  p.tree_parent = parents;
+  s3r_status api;
+  cudaError_t e = launch_attention(*kv, p, st, &api);
+  if (api != S3R_OK) return api;
+  return from_cuda(e);
+}
+
+S3R_EXPORT size_t s3r_tree_sample_workspace_bytes(int32_t num_seqs, int32_t nodes, int32_t vocab) {
+  if (num_seqs < 1 || nodes < 1 || nodes > kMaxTreeNodes || vocab < 1) return 0;
+  return kWsHeader;
+}
+
+S3R_EXPORT s3r_status s3r_tree_spec_sample(const void* target_logits, const void* draft_logits,
+                                           s3r_dtype logit_dtype, const int32_t* tokens, const int32_t* parents,
+                                           const float* u_accept, const float* u_sample, int32_t num_seqs,
+                                           int32_t nodes, int32_t vocab, float temperature, int32_t* out_tokens,
+                                           int32_t* num_accepted, int32_t* path, void* workspace,
+                                           size_t workspace_bytes, void* stream) {
+  if (!target_logits || !draft_logits || !tokens || !parents || !u_accept || !u_sample || !out_tokens ||
+      !num_accepted)
+    return S3R_ERR_INVALID_ARG;
+  if (logit_dtype != S3R_F32 && logit_dtype != S3R_BF16) return S3R_ERR_INVALID_ARG;
+  if (num_seqs < 1 || nodes < 1 || vocab < 1 || !(temperature > 0.0f) || !std::isfinite(temperature))
+    return S3R_ERR_INVALID_ARG;
+  if (nodes > kMaxTreeNodes || num_seqs > 65535) return S3R_ERR_UNSUPPORTED;
+  if ((int64_t)num_seqs * nodes * vocab >= (1ll << 40)) return S3R_ERR_UNSUPPORTED;
+  const size_t need = s3r_tree_sample_workspace_bytes(num_seqs, nodes, vocab);
+  if (!workspace || workspace_bytes < need) return S3R_ERR_WORKSPACE;
+  const size_t es = logit_dtype == S3R_BF16 ? 2 : 4;
+  const bool vec = aligned16(target_logits) && aligned16(draft_logits) && ((size_t)vocab * es) % 16 == 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t* status = static_cast<uint32_t*>(workspace);
+  return from_cuda(launch_tree_sample(target_logits, draft_logits, logit_dtype, tokens, parents, u_accept, u_sample,
+                                      num_seqs, nodes, vocab, 1.0 / static_cast<double>(temperature), out_tokens,
+                                      num_accepted, path, status, vec, st));
+}
+
+S3R_EXPORT int32_t s3r_tree_node_budget(int64_t capacity, int32_t active, int32_t n_min, int32_t n_max) {
+  if (active < 1 || n_min < 1 || n_max < n_min || capacity < 0) return -1;
+  const int64_t n = capacity / active;
+  return (int32_t)(n < n_min ? n_min : (n > n_max ? n_max : n));
 }
 
 namespace {

@@ -117,6 +117,20 @@ __global__ void __launch_bounds__(kF32Threads) attn_f32_kernel(const AttnParams 
     sL[i] = 0.f;
     sPos[i] = g.L - p.R + i / p.G;
   }
+  __shared__ unsigned long long s_tmask[64];     // tree: ancestors-or-self of each round node
+  if (p.tree_parent && tid < p.R) {
+    const int32_t* par = p.tree_parent + (size_t)b * p.R;
+    unsigned long long m = 1ull << tid;
+    int v = tid;
+    for (int guard = 0; guard < 64 && v > 0; ++guard) {
+      const int pv = par[v];
+      if (pv < 0 || pv >= v) { flag_status(p.status, S3R_DEV_BAD_TREE); break; }
+      m |= 1ull << pv;
+      v = pv;
+    }
+    if (tid == 0 && par[0] != -1) flag_status(p.status, S3R_DEV_BAD_TREE);
+    s_tmask[tid] = m;
+  }
   __syncthreads();
   const float* kc = static_cast<const float*>(p.k_cache);
   const float* vc = static_cast<const float*>(p.v_cache);
@@ -143,7 +157,10 @@ __global__ void __launch_bounds__(kF32Threads) attn_f32_kernel(const AttnParams 
         const int i = idx / kF32Tok, t = idx - (idx / kF32Tok) * kF32Tok;
         const int pos = lp * p.P + t0 + t;
         float sc = -INFINITY;
-        if (t < ntok && pos <= sPos[i]) {
+        const int slot = pos - (g.L - p.R);             // >= 0: a position of the round
+        const bool seen = t < ntok && (p.tree_parent ? (slot < 0 || (slot < p.R && ((s_tmask[i / p.G] >> slot) & 1ull)))
+                                                      : pos <= sPos[i]);
+        if (seen) {
           const float4* a = reinterpret_cast<const float4*>(sQ + i * D);
           const float4* kk = reinterpret_cast<const float4*>(sK + t * D);
           float acc = 0.f;

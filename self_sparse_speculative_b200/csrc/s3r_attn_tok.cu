@@ -73,6 +73,8 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
   __shared__ float s_mx[64];                    // stage maximum per row (raw score)
   __shared__ __align__(16) float s_nu[64];      // -(reference) per row, log2 units
   __shared__ __align__(16) float s_alpha[64];   // rescale factor / 1 / l per row
+  __shared__ unsigned long long s_tmask[64];    // tree: ancestors-or-self of each round node
+  __shared__ unsigned long long s_pmask[64];    // tree: packed rows that see each round slot
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   pdl_launch_dependents();
@@ -389,6 +391,31 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
       const int nst = (sg.npg + ppt - 1) / ppt;
       const int Lb = p.context_lens[sg.b];
       if (tid < N) s_nu[tid] = kNuInit;
+      if (p.tree_parent) {
+        // the round's nodes: ancestors-or-self of each (parents precede their
+        // children; a bad entry ends the walk and is flagged), then for each
+        // round slot the packed rows allowed to see it
+        if (tid < p.R) {
+          const int32_t* par = p.tree_parent + (size_t)sg.b * p.R;
+          unsigned long long m = 1ull << tid;
+          int v = tid;
+          for (int guard = 0; guard < 64 && v > 0; ++guard) {
+            const int pv = par[v];
+            if (pv < 0 || pv >= v) { flag_status(p.status, S3R_DEV_BAD_TREE); break; }
+            m |= 1ull << pv;
+            v = pv;
+          }
+          if (tid == 0 && par[0] != -1) flag_status(p.status, S3R_DEV_BAD_TREE);
+          s_tmask[tid] = m;
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (tid < p.R) {
+          unsigned long long pm = 0;
+          for (int r = 0; r < p.rows; ++r)
+            if ((s_tmask[r / p.G] >> tid) & 1ull) pm |= 1ull << r;
+          s_pmask[tid] = pm;
+        }
+      }
       float l[NR];
 #pragma unroll
       for (int r = 0; r < NR; ++r) l[r] = 0.f;
@@ -404,15 +431,24 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         const int pos = lp * p.P + (tid & (p.P - 1));
         const bool valid = lp >= 0 && pos < Lb;
         const int excess = pos - (Lb - p.R);
-        const int nm = !valid ? N : (excess > 0 ? min(N, p.G * excess) : 0);
+        // packed rows that may not see this token: a token that does not exist
+        // hides from all; inside the round, the causal chain hides from the
+        // rows of earlier positions, a tree from the rows of non-descendants
+        unsigned long long hide = 0;
+        if (!valid) hide = ~0ull;
+        else if (p.tree_parent) hide = excess >= 0 ? ~s_pmask[excess] : 0ull;
+        else if (excess > 0) {
+          const int nm = min(N, p.G * excess);
+          hide = nm >= 64 ? ~0ull : ((1ull << nm) - 1ull);
+        }
         float s[NR];
         auto load_s = [&]() {
           tmem_ld_cols<NR>(tmem + lane_base + L::kColS + sb * N, s);
           tmem_wait_ld();
-          if (nm > 0) {
+          if (hide) {
 #pragma unroll
             for (int r = 0; r < NR; ++r)
-              if (r < nm) s[r] = -INFINITY;
+              if ((hide >> r) & 1ull) s[r] = -INFINITY;
           }
         };
         load_s();

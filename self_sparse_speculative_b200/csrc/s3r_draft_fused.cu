@@ -288,22 +288,6 @@ __device__ void tail_minmax(const __nv_bfloat16* src, int valid, int tg, int nth
   }
 }
 
-// ---- thread-block cluster: barrier and distributed shared memory
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// Stores to the same shared-memory offset in CTA `rank` of the cluster.
-__device__ __forceinline__ void st_cluster_u32(const void* local, uint32_t rank, uint32_t v) {
-  uint32_t remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_addr(local)), "r"(rank));
-  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(remote), "r"(v) : "memory");
-}
-__device__ __forceinline__ void st_cluster_u64(const void* local, uint32_t rank, unsigned long long v) {
-  uint32_t remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_addr(local)), "r"(rank));
-  asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(remote), "l"(v) : "memory");
-}
-
 // Rank of key kp (page i) among keys[0..n): the keys above it, plus the
 // equal keys of lower pages (ties go to the lower page). keys is 8-byte
 // aligned; one key is taken alone when that puts the rest on a 16-byte

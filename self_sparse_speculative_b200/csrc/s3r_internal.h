@@ -25,6 +25,7 @@ constexpr int kMaxSeqs = 1024;
 // Upper bound on the persistent attention grid (one CTA per SM); sizes the
 // partial-result slots of the workspace.
 constexpr int kMaxPersistentCtas = 160;
+constexpr int kMaxTreeNodes = 64;         // tree verification: nodes per sequence (one 64-bit mask)
 
 // Workspace header: word 0 is the device status word; the rest is reserved.
 constexpr size_t kWsHeader = 256;
@@ -54,6 +55,8 @@ struct AttnParams {
   const void* kmax;
   int32_t* selected_out;         // [S, Hkv, budget] logical ids of the kept pages
   int32_t parts;                 // CTAs sharing one (sequence, KV head) unit
+  // tree verification: parent of each of the R round nodes [S, R] (null: the causal chain)
+  const int32_t* tree_parent;
 };
 
 // Split plan shared by the workspace-size query and the launch.
@@ -172,6 +175,10 @@ struct SampleParams {
 // Fill the workspace pointers and sizes of `p` from a plan and a workspace base.
 void bind_sample_workspace(SampleParams* p, const SamplePlan& pl, void* ws);
 cudaError_t launch_sampling(const SampleParams& p, s3r_dtype dt, bool spec, cudaStream_t st);
+cudaError_t launch_tree_sample(const void* target, const void* draft, s3r_dtype dt, const int32_t* tokens,
+                               const int32_t* parents, const float* u_accept, const float* u_sample, int32_t nseq,
+                               int32_t nodes, int32_t vocab, double inv_temp, int32_t* out_tokens,
+                               int32_t* num_accepted, int32_t* path, uint32_t* status, bool vec, cudaStream_t st);
 cudaError_t launch_exp64_probe(const double* x, double* y_tbl, double* y_ref, int n, cudaStream_t st);
 
 }  // namespace s3r

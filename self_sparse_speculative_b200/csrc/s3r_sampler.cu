@@ -32,6 +32,7 @@
 #include <cmath>
 
 #include "s3r_device.cuh"
+#include "s3r_exp64.cuh"
 #include "s3r_internal.h"
 
 namespace s3r {
@@ -115,56 +116,6 @@ __device__ double block_sum_d(double v, double* s_red) {
   for (int w = 0; w < kSmpWarps; ++w) r += s_red[w];
   __syncthreads();
   return r;
-}
-
-// float64 exponential, table-driven (P. T. P. Tang, "Table-driven
-// implementation of the exponential function in IEEE floating-point
-// arithmetic", ACM Trans. Math. Software 15(2), 1989), with a 256-entry
-// table: write x = (256 m + j) ln2/256 + r with |r| <= ln2/512, then
-// exp(x) = 2^m * 2^(j/256) * e^r. N = 256 m + j is x * 256/ln2 rounded to an
-// integer by adding 1.5 * 2^52; r = x - N ln2/256 with ln2/256 split into a
-// double and its remainder (two fused multiply-adds); e^r - 1 is its Taylor
-// polynomial to degree 4 (remainder < 4e-17 for |r| <= ln2/512); 2^(j/256)
-// is the table `tab`; 2^m goes into the exponent field. Within about 2 ulp
-// for -707 < x < 708; outside that range the value is meaningless (callers
-// fix it up with exp_fixup).
-constexpr int kExpTab = 256;
-__device__ __forceinline__ double exp_tbl(double x, const double* tab) {
-  constexpr double kInvStep = 369.32993046757463;          // 256 / ln2
-  constexpr double kStepHi = 0x1.62e42fefa39efp-9;          // ln2 / 256, leading double
-  constexpr double kStepLo = 0x1.abc9e3b39803fp-64;         // ln2 / 256 - kStepHi
-  constexpr double kShifter = 6755399441055744.0;           // 1.5 * 2^52
-  const double t = fma(x, kInvStep, kShifter);
-  const int n = __double2loint(t);
-  const double nd = t - kShifter;
-  double r = fma(-nd, kStepHi, x);
-  r = fma(-nd, kStepLo, r);
-  double q = fma(r, 1.0 / 24.0, 1.0 / 6.0);
-  q = fma(q, r, 0.5);
-  q = fma(q, r, 1.0);
-  const double tj = tab[n & (kExpTab - 1)];
-  const double y = fma(tj, q * r, tj);
-  return __hiloint2double(__double2hiint(y) + (n >> 8) * (1 << 20), __double2loint(y));
-}
-// exp(x) given y = exp_tbl(x): outside (-707, 708) the argument is moved
-// into range by 512 ln2 and the result scaled back by an exact power of two
-// (subnormal results round once there), 0 below -746, NaN stays NaN. No
-// library call, so the hot loops carry no call ABI.
-__device__ __forceinline__ double exp_fixup(double x, double y, const double* tab) {
-  if (x > -707.0 && x < 708.0) return y;
-  constexpr double k512ln2 = 354.891356446692;          // 512 ln2 (rounded; shifts an argument only)
-  if (x != x) return x;
-  if (x <= -746.0) return 0.0;
-  if (x < 0.0) return exp_tbl(x + k512ln2, tab) * 0x1p-512;
-  if (x >= 710.0) return INFINITY;
-  return exp_tbl(x - k512ln2, tab) * 0x1p512;
-}
-
-// 2^(j/256), j = 0..255, into shared memory (one entry per thread of a
-// 256-thread CTA; caller syncs).
-__device__ __forceinline__ void fill_exp_tab(double* tab) {
-  static_assert(kSmpThreads == kExpTab, "one table entry per thread");
-  tab[threadIdx.x] = exp2(static_cast<double>(threadIdx.x) * (1.0 / kExpTab));
 }
 
 // Staging: the CTA's chunk [beg, beg + n) of one or two rows into shared

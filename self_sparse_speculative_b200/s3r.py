@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libs3r.so")
 S3R_OK, S3R_ERR_INVALID_ARG, S3R_ERR_UNSUPPORTED, S3R_ERR_WORKSPACE, S3R_ERR_CUDA, S3R_ERR_DEVICE_CHECK = range(6)
 S3R_F32, S3R_BF16 = 0, 1
 S3R_DEV_BAD_CONTEXT_LEN, S3R_DEV_BAD_PAGE_ID, S3R_DEV_BAD_TOKEN_ID, S3R_DEV_WAIT_TIMEOUT = 0x1, 0x2, 0x4, 0x8
+S3R_DEV_BAD_TREE = 0x10
 
 EXPORTED = [
     "s3r_page_summaries", "s3r_page_summaries_checked", "s3r_sparse_draft_attn", "s3r_verify_attn",
@@ -25,7 +26,8 @@ EXPORTED = [
     "s3r_device_status", "s3r_status_str", "s3r_version", "s3r_sparse_draft_kernels",
     "s3r_sample_tokens_ex", "s3r_spec_sample_ex", "s3r_kv_append", "s3r_kv_rollback", "s3r_kv_workspace_bytes",
     "s3r_debug_exp64", "s3r_gamma_policy_init", "s3r_gamma_policy_update", "s3r_gamma_policy_choose",
-    "s3r_attend_cost_us", "s3r_round_cost_us",
+    "s3r_attend_cost_us", "s3r_round_cost_us", "s3r_verify_attn_tree", "s3r_tree_spec_sample",
+    "s3r_tree_sample_workspace_bytes", "s3r_tree_node_budget",
 ]
 
 
@@ -82,6 +84,10 @@ def _load():
         "s3r_status_str": ([i32], ctypes.c_char_p),
         "s3r_sparse_draft_kernels": ([kvp, i32], i32),
         "s3r_version": ([], i32),
+        "s3r_verify_attn_tree": ([kvp, vp, i32, vp, f32, vp, vp, vp, sz, vp], i32),
+        "s3r_tree_sample_workspace_bytes": ([i32, i32, i32], sz),
+        "s3r_tree_spec_sample": ([vp, vp, i32, vp, vp, vp, vp, i32, i32, i32, f32, vp, vp, vp, vp, sz, vp], i32),
+        "s3r_tree_node_budget": ([ctypes.c_int64, i32, i32, i32], i32),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -172,6 +178,34 @@ def s3r_verify_attn(kv: PagedKV, q, rows: int, scale: float, out, lse, workspace
     st = _lib.s3r_verify_attn(ctypes.byref(kv), _ptr(q), int(rows), float(scale), _ptr(out), _ptr(lse),
                               _ptr(workspace), wb, _stream(stream))
     _check("s3r_verify_attn", st)
+
+
+def s3r_verify_attn_tree(kv: PagedKV, q, nodes: int, parents, scale: float, out, lse, workspace,
+                         workspace_bytes=None, stream=None):
+    wb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    st = _lib.s3r_verify_attn_tree(ctypes.byref(kv), _ptr(q), int(nodes), _ptr(parents), float(scale), _ptr(out),
+                                   _ptr(lse), _ptr(workspace), wb, _stream(stream))
+    _check("s3r_verify_attn_tree", st)
+
+
+def s3r_tree_sample_workspace_bytes(num_seqs: int, nodes: int, vocab: int) -> int:
+    return int(_lib.s3r_tree_sample_workspace_bytes(num_seqs, nodes, vocab))
+
+
+def s3r_tree_spec_sample(target_logits, draft_logits, logit_dtype, tokens, parents, u_accept, u_sample,
+                         num_seqs: int, nodes: int, vocab: int, temperature: float, out_tokens, num_accepted,
+                         path, workspace, workspace_bytes=None, stream=None):
+    wb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    st = _lib.s3r_tree_spec_sample(_ptr(target_logits), _ptr(draft_logits), dtype_code(logit_dtype), _ptr(tokens),
+                                   _ptr(parents), _ptr(u_accept), _ptr(u_sample), int(num_seqs), int(nodes),
+                                   int(vocab), float(temperature), _ptr(out_tokens), _ptr(num_accepted), _ptr(path),
+                                   _ptr(workspace), wb, _stream(stream))
+    _check("s3r_tree_spec_sample", st)
+
+
+def s3r_tree_node_budget(capacity: int, active: int, n_min: int, n_max: int) -> int:
+    """N_t = clip(floor(capacity / active), n_min, n_max); -1 for bad arguments."""
+    return int(_lib.s3r_tree_node_budget(int(capacity), int(active), int(n_min), int(n_max)))
 
 
 def s3r_spec_sample(target_logits, draft_logits, logit_dtype, draft_tokens, u_accept, u_sample,

@@ -75,3 +75,21 @@ def test_workload_regimes_with_the_native_policy():
         return p.choose()[0]
     assert choose(16, 1500.0, 0.6) > 0
     assert choose(4096, 2.0, 0.6) == 0
+
+
+def test_tree_node_budget_follows_the_oracle():
+    """N_t = clip(floor(C_hw / B_t), N_min, N_max) in libs3r against the
+    oracle's node_budget over random capacities and concurrencies."""
+    import oracle as O
+    rng = np.random.default_rng(7)
+    for _ in range(2000):
+        n_min = int(rng.integers(1, 8))
+        n_max = int(rng.integers(n_min, 65))
+        active = int(rng.integers(1, 513))
+        cap = int(rng.integers(0, 1 << 40)) if rng.random() < 0.1 else int(rng.integers(0, 20000))
+        assert s3r.s3r_tree_node_budget(cap, active, n_min, n_max) == O.node_budget(cap, active, n_min, n_max)
+    # as responses finish (B_t falls) the budget grows up to N_max
+    seq = [s3r.s3r_tree_node_budget(600, b, 2, 32) for b in (256, 64, 32, 16, 8, 1)]
+    assert seq == sorted(seq) and seq[0] == 2 and seq[-1] == 32
+    for bad in ((600, 0, 2, 16), (600, 4, 0, 16), (600, 4, 8, 4), (-1, 4, 2, 16)):
+        assert s3r.s3r_tree_node_budget(*bad) == -1
