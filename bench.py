@@ -328,6 +328,141 @@ def gamma_policy_note(ws, st, hbm_gbs):
             "cost_model": f"roofline at {hbm_gbs:.0f} GB/s and {tf:.0f} TFLOP/s"}
 
 
+def next_rows_measure(st, ws, stream, peak, steps, seed):
+    """The calls beyond the five-part step on the same cache: the KV upkeep
+    of a round (a drafter row appended, the verifier's rows written over the
+    round's positions, the rollback to the committed prefix) and tree
+    verification (a tree of N_t nodes, N_t from the concurrency-aware budget
+    with one node per sequence and head group of capacity, the tree's
+    ancestor-masked attention over the whole cache, and the tree walk of
+    exact speculative sampling). Each: microseconds per call (mean of
+    `steps` calls, CUDA events on the launching stream) and algorithmic
+    bytes over that time against the HBM peak."""
+    import torch
+    from self_sparse_speculative_b200 import s3r
+    from self_sparse_speculative_b200 import workloads as W
+    S, Hq, Hkv, D, P, V = ws.num_seqs, ws.num_q_heads, ws.num_kv_heads, ws.head_dim, ws.page_size, ws.vocab
+    g, R = ws.gamma, ws.rows
+    elt = 2 if ws.kv_dtype == "bf16" else 4
+    lelt = 2 if ws.logit_dtype == "bf16" else 4
+    lens_full = st.context_lens.clone()
+    lens0 = st.lens_committed.cpu().numpy()
+    out = {}
+
+    def timed(fn, n):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        for e0, e1 in evs:
+            fn(e0, e1)
+        torch.cuda.synchronize()
+        return sum(e0.elapsed_time(e1) for e0, e1 in evs) / n * 1e3     # us
+
+    def entry(us, nbytes):
+        gbs = nbytes / (us * 1e-6) / 1e9
+        return {"us_per_call": round(us, 2), "algorithmic_bytes": int(nbytes), "gbs": round(gbs, 1),
+                "frac_of_peak": round(gbs / peak, 4)}
+
+    # ---- KV upkeep: a round's appends and rollback, from the committed lengths
+    t_app, t_ver, t_rb = [], [], []
+
+    def one_round(e0, e1):
+        st.context_lens.copy_(st.lens_committed)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        s3r.s3r_kv_append(st.kv, st.context_lens, st.k_round_draft[0], st.v_round_draft[0], 1, 0, st.kmin, st.kmax,
+                          st.ws_kv, stream=stream)
+        a1.record(stream)
+        t_app.append((a0, a1))
+        for i in range(1, g):
+            s3r.s3r_kv_append(st.kv, st.context_lens, st.k_round_draft[i], st.v_round_draft[i], 1, 0, st.kmin,
+                              st.kmax, st.ws_kv, stream=stream)
+        e0.record(stream)
+        s3r.s3r_kv_append(st.kv, st.context_lens, st.k_round_verify, st.v_round_verify, R, g, st.kmin, st.kmax,
+                          st.ws_kv, stream=stream)
+        e1.record(stream)
+        r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        r0.record(stream)
+        s3r.s3r_kv_rollback(st.kv, st.context_lens, st.num_accepted, R, st.kmin, st.kmax, st.ws_kv, stream=stream)
+        r1.record(stream)
+        t_rb.append((r0, r1))
+
+    for _ in range(3):
+        one_round(torch.cuda.Event(), torch.cuda.Event())
+    t_app.clear(); t_rb.clear()
+    us_ver = timed(one_round, steps)
+    us_app = sum(a.elapsed_time(b) for a, b in t_app) / len(t_app) * 1e3
+    us_rb = sum(a.elapsed_time(b) for a, b in t_rb) / len(t_rb) * 1e3
+    new_lens = lens0 + st.num_accepted.cpu().numpy() + 1
+    out["kv_append_draft_row"] = entry(us_app, W.kv_append_bytes(lens0, 1, 0, P, Hkv, D, elt))
+    out["kv_append_verify_rows"] = entry(us_ver, W.kv_append_bytes(lens0 + g, R, g, P, Hkv, D, elt))
+    out["kv_rollback"] = entry(us_rb, W.kv_rollback_bytes(new_lens, P, Hkv, D, elt))
+    # the cache's lengths and tail summaries as before
+    st.context_lens.copy_(lens_full)
+    st.summaries(tail_only=True)
+    torch.cuda.synchronize()
+
+    # ---- tree verification: node budget, attention, tree walk
+    G = Hq // Hkv
+    n_max = min(64, 64 // G) if ws.kv_dtype == "bf16" else min(64, 128 // G)
+    n_t = s3r.s3r_tree_node_budget(S * n_max, S, 2, n_max)
+    parents = np.broadcast_to(W.breadth_first_tree(n_t, [4, 2, 1]), (S, n_t)).copy()
+    gen = torch.Generator(device=st.device).manual_seed(seed + 1234)
+    dt = st.k_cache.dtype
+    q = torch.randn((S, n_t, Hq, D), generator=gen, device=st.device, dtype=torch.float32).to(dt)
+    par_d = torch.from_numpy(parents.astype(np.int32)).to(st.device)
+    o = torch.empty((S, n_t, Hq, D), dtype=dt, device=st.device)
+    lse = torch.empty((S, n_t, Hq), dtype=torch.float32, device=st.device)
+    wsv = torch.zeros(s3r.s3r_attn_workspace_bytes(st.kv, n_t, 0), dtype=torch.uint8, device=st.device)
+
+    def tree_attn(e0, e1):
+        e0.record(stream)
+        s3r.s3r_verify_attn_tree(st.kv, q, n_t, par_d, st.scale, o, lse, wsv, stream=stream)
+        e1.record(stream)
+
+    for _ in range(3):
+        tree_attn(torch.cuda.Event(), torch.cuda.Event())
+    us_tv = timed(tree_attn, steps)
+    kv_bytes = int(st.wl.context_lens.astype(np.int64).sum()) * 2 * Hkv * D * elt
+    out["tree_verify_attn"] = dict(entry(us_tv, kv_bytes), nodes=n_t, node_budget="N_t = clip(floor(C_hw / B_t), 2, "
+                                   f"{n_max}) with C_hw = {S * n_max}, B_t = {S}")
+    # logits of every node after the workload's recipe (target N(0, s^2), draft
+    # = target + noise); children's tokens drawn from their parent's draft row
+    ldt = st.target_logits.dtype
+    sigma, noise = (1.0, 0.3) if ws.tiny_logits else (ws.target_std, ws.draft_noise_std)
+    tgt = (sigma * torch.randn((S, n_t, V), generator=gen, device=st.device)).to(ldt)
+    drf = (tgt.float() + noise * torch.randn((S, n_t, V), generator=gen, device=st.device)).to(ldt)
+    child_rows = drf[:, torch.from_numpy(np.maximum(parents[0, 1:], 0)).to(st.device)].reshape(S * (n_t - 1), V)
+    u_tok = torch.rand((S * (n_t - 1),), generator=gen, device=st.device)
+    tok = torch.empty((S * (n_t - 1),), dtype=torch.int32, device=st.device)
+    wst = torch.zeros(s3r.s3r_sample_workspace_bytes(S * (n_t - 1), 0, V), dtype=torch.uint8, device=st.device)
+    s3r.s3r_sample_tokens(child_rows.contiguous(), ws.logit_dtype, S * (n_t - 1), V, ws.temperature, u_tok, tok, wst,
+                          stream=stream)
+    tokens = torch.cat([torch.zeros((S, 1), dtype=torch.int32, device=st.device), tok.view(S, n_t - 1)], 1)
+    ua = torch.rand((S, n_t), generator=gen, device=st.device)
+    us = torch.rand((S, n_t), generator=gen, device=st.device)
+    o_tok = torch.empty((S, n_t), dtype=torch.int32, device=st.device)
+    n_acc = torch.empty((S,), dtype=torch.int32, device=st.device)
+    path = torch.empty((S, n_t), dtype=torch.int32, device=st.device)
+    wss = torch.zeros(s3r.s3r_tree_sample_workspace_bytes(S, n_t, V), dtype=torch.uint8, device=st.device)
+
+    def tree_walk(e0, e1):
+        e0.record(stream)
+        s3r.s3r_tree_spec_sample(tgt, drf, ws.logit_dtype, tokens, par_d, ua, us, S, n_t, V, ws.temperature, o_tok,
+                                 n_acc, path, wss, stream=stream)
+        e1.record(stream)
+
+    for _ in range(3):
+        tree_walk(torch.cuda.Event(), torch.cuda.Event())
+    us_ts = timed(tree_walk, steps)
+    na, pa = n_acc.cpu().numpy(), path.cpu().numpy()
+    out["tree_spec_sample"] = dict(entry(us_ts, W.tree_sample_bytes(parents, na, pa, V, lelt)),
+                                   mean_accepted_nodes=round(float(na.mean()), 3))
+    bad = {k: v for k, v in (("tree_attn", s3r.s3r_device_status(wsv)), ("tree_walk", s3r.s3r_device_status(wss)),
+                             ("kv", s3r.s3r_device_status(st.ws_kv))) if v[0] != s3r.S3R_OK}
+    if bad:
+        raise RuntimeError(f"device checks failed in the next-row calls: {bad}")
+    return out
+
+
 def run_ours(a):
     world0 = int(os.environ.get("WORLD_SIZE", "1"))
     # the CPU leg first, before this process touches the GPU
@@ -500,6 +635,11 @@ def run_ours(a):
         e2e = {"value": e2e_tokens / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h)}
 
+    peak, peak_kind = _peaks()
+    next_rows = None
+    if not a.no_next_rows:
+        next_rows = next_rows_measure(st, ws, stream, peak, a.steps, a.seed)
+
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -507,7 +647,6 @@ def run_ours(a):
         return
 
     nbytes = st.algorithmic_bytes()
-    peak, peak_kind = _peaks()
     verify_gbs = nbytes["verify"] / (t_verify * 1e-3) / 1e9
     draft_gbs = nbytes["draft_per_call"] / (t_draft * 1e-3) / 1e9
     ms_per_step = total_ms_max / a.steps
@@ -540,6 +679,8 @@ def run_ours(a):
     if e2e:
         line["e2e"] = {k: (round(v, 1) if isinstance(v, float) else v) for k, v in e2e.items()}
     line["gamma_policy"] = gamma_policy_note(ws, st, peak)
+    if next_rows is not None:
+        line["next_rows"] = next_rows
     if cpu_line is not None:
         line["cpu_baseline"] = cpu_line
     print(json.dumps(line), flush=True)
@@ -617,6 +758,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay timing")
+    ap.add_argument("--no-next-rows", action="store_true",
+                    help="skip the KV-upkeep and tree-verification timings")
     a = ap.parse_args()
     cmd = launch_plan(a.gpus, os.environ, sys.argv[1:])
     if cmd is not None:

@@ -22,9 +22,11 @@
  * Conventions shared by every call
  * --------------------------------
  * - Every pointer argument is a caller-owned DEVICE pointer unless stated
- *   otherwise. The library allocates and frees nothing and keeps no state
+ *   otherwise. The library allocates and frees nothing and keeps no data
  *   between calls; scratch space comes from the caller's workspace (the one
- *   exception, s3r_spec_sample_noalloc, uses a static array of its own).
+ *   exception, s3r_spec_sample_noalloc, uses a static array of its own). Host
+ *   side it remembers only launch choices: the TMA driver entry point, and
+ *   the cluster size s3r_tree_spec_sample picked per device and problem size.
  * - A workspace must be zero-filled before its first use. Calls leave it
  *   ready for the next call (its counters return to zero as each call ends),
  *   so no call clears it and consecutive kernels of the library overlap

@@ -53,21 +53,57 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float
 template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
 
 // kmin / kmax of head h of physical page `phys` over its first `valid` tokens
-// (min and max of stored values are exact in the storage type).
+// (min and max of stored values are exact in the storage type). Each thread
+// owns one 16-byte piece of a key row and a token group (tokens tq, tq + ngrp,
+// ...), eight rows in flight; the groups merge through shared memory.
 template <typename T>
 __device__ void summarise_page(const KvParams& p, int phys, int h, int valid) {
-  const T* kt = static_cast<const T*>(p.k_cache) + ((size_t)phys * p.Hkv + h) * p.P * p.D;
+  constexpr int kPer = 16 / sizeof(T);
+  __shared__ float s_mn[kKvThreads * 8], s_mx[kKvThreads * 8];
+  const int pieces = p.D / kPer;                      // 16-byte pieces per row
+  const int ngrp = kKvThreads / pieces;
+  const int c = threadIdx.x % pieces, tq = threadIdx.x / pieces;
+  const T* kt = static_cast<const T*>(p.k_cache) + ((size_t)phys * p.Hkv + h) * p.P * p.D + (size_t)c * kPer;
+  float mn[kPer], mx[kPer];
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) { mn[k] = INFINITY; mx[k] = -INFINITY; }
+  for (int t0 = tq; t0 < valid; t0 += 8 * ngrp) {
+    uint4 r[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int t = t0 + u * ngrp;
+      r[u] = t < valid ? __ldcg(reinterpret_cast<const uint4*>(kt + (size_t)t * p.D)) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (t0 + u * ngrp >= valid) break;
+      const T* e = reinterpret_cast<const T*>(&r[u]);
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) {
+        const float v = to_f<T>(e[k]);
+        mn[k] = fminf(mn[k], v);
+        mx[k] = fmaxf(mx[k], v);
+      }
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    s_mn[threadIdx.x * kPer + k] = mn[k];
+    s_mx[threadIdx.x * kPer + k] = mx[k];
+  }
+  __syncthreads();
   for (int d = threadIdx.x; d < p.D; d += kKvThreads) {
-    float mn = INFINITY, mx = -INFINITY;
-    for (int t = 0; t < valid; ++t) {
-      const float v = to_f<T>(kt[(size_t)t * p.D + d]);
-      mn = fminf(mn, v);
-      mx = fmaxf(mx, v);
+    const int pc = d / kPer, k = d - (d / kPer) * kPer;
+    float a = INFINITY, b = -INFINITY;
+    for (int g = 0; g < ngrp; ++g) {
+      a = fminf(a, s_mn[(g * pieces + pc) * kPer + k]);
+      b = fmaxf(b, s_mx[(g * pieces + pc) * kPer + k]);
     }
     const size_t o = ((size_t)phys * p.Hkv + h) * p.D + d;
-    static_cast<T*>(p.kmin)[o] = from_f<T>(mn);
-    static_cast<T*>(p.kmax)[o] = from_f<T>(mx);
+    static_cast<T*>(p.kmin)[o] = from_f<T>(a);
+    static_cast<T*>(p.kmax)[o] = from_f<T>(b);
   }
+  __syncthreads();                                   // the arrays are reused by the next page
 }
 
 // The last CTA of sequence b (one per KV head) stores its new length.
@@ -98,6 +134,17 @@ __global__ void __launch_bounds__(kKvThreads) kv_append_kernel(const KvParams p)
   constexpr int kPer = 16 / sizeof(T);
   const int pieces = p.D / kPer;
   const int32_t* bt = p.block_table + (size_t)b * p.max_pages;
+  // the keys of the pages to summarise, towards L2 while the rows are copied
+  if (p.n > 0)
+    for (int pg = start / p.P; pg <= (new_len - 1) / p.P; ++pg) {
+      const int phys = bt[pg];
+      if (phys < 0 || phys >= p.num_pages_total) continue;
+      const char* kp = reinterpret_cast<const char*>(static_cast<const T*>(p.k_cache) +
+                                                     ((size_t)phys * p.Hkv + h) * p.P * p.D);
+      const int lines = (p.P * p.D * (int)sizeof(T)) / 128;
+      for (int l = threadIdx.x; l < lines; l += kKvThreads)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(kp + (size_t)l * 128));
+    }
   for (int f = threadIdx.x; f < p.n * pieces; f += kKvThreads) {
     const int t = f / pieces, c = f - (f / pieces) * pieces;
     const int pos = start + t;

@@ -321,3 +321,61 @@ def algorithmic_bytes(wl: "Workload"):
     draw = ws.num_seqs * g * V * lelt
     return {"draft_per_call": draft, "verify": verify, "sample": sample, "draft_tokens": draw,
             "step": g * draft + verify + sample + draw}
+
+
+def kv_append_bytes(lens, n, overwrite, page_size, kv_heads, head_dim, elt):
+    """Bytes one s3r_kv_append must move: the n new K and V rows read and
+    written per KV head, and for every page holding a written row its valid
+    keys read and its kmin / kmax written. lens: lengths before the call."""
+    P, D = page_size, head_dim
+    total = 0
+    for L in np.asarray(lens, dtype=np.int64):
+        start = int(L) - overwrite
+        new_len = start + n
+        rows = 2 * 2 * n * D * elt                                    # K and V, read and written
+        summ = 0
+        for pg in range(start // P, (new_len - 1) // P + 1):
+            valid = min(P, new_len - pg * P)
+            summ += valid * D * elt + 2 * D * elt
+        total += kv_heads * (rows + summ)
+    return total
+
+
+def kv_rollback_bytes(new_lens, page_size, kv_heads, head_dim, elt):
+    """Bytes one s3r_kv_rollback must move: the new tail page's valid keys
+    read and its kmin / kmax written, per KV head."""
+    P, D = page_size, head_dim
+    total = 0
+    for L in np.asarray(new_lens, dtype=np.int64):
+        pg = (int(L) - 1) // P
+        total += kv_heads * ((int(L) - pg * P) * D * elt + 2 * D * elt)
+    return total
+
+
+def tree_sample_bytes(parents, num_accepted, path, vocab, elt):
+    """Bytes a tree walk must read: the target row of every visited node and
+    the draft row of every visited node that has children (the first pass over
+    a node's rows; the later passes of the walk re-read them from L2)."""
+    total = 0
+    for b in range(parents.shape[0]):
+        visited = [0] + [int(path[b, i]) for i in range(int(num_accepted[b]))]
+        for v in visited:
+            has_child = bool(np.any(parents[b] == v))
+            total += vocab * elt * (2 if has_child else 1)
+    return total
+
+
+def breadth_first_tree(n_nodes, branching):
+    """Parents of an n_nodes tree in breadth-first order, node d-deep getting
+    branching[d] children (the last entry repeats)."""
+    parents, frontier, d = [-1], [0], 0
+    while len(parents) < n_nodes and frontier:
+        k = branching[min(d, len(branching) - 1)]
+        nxt = []
+        for v in frontier:
+            for _ in range(k):
+                if len(parents) < n_nodes:
+                    parents.append(v)
+                    nxt.append(len(parents) - 1)
+        frontier, d = nxt, d + 1
+    return np.array(parents, dtype=np.int64)
