@@ -196,7 +196,7 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- our arm
 # sources of the verify kernel; the committed ncu summary records their hash
-VERIFY_SOURCES = ("s3r_attn_tok.cu", "s3r_attn_sched.cuh", "s3r_attn_common.cuh", "s3r_device.cuh")
+VERIFY_SOURCES = ("s3r_attn_tok.cu", "s3r_tok_common.cuh", "s3r_attn_sched.cuh", "s3r_attn_common.cuh", "s3r_device.cuh")
 VERIFY_PROFILE = os.path.join(HERE, "profiles", "verify_attn_tok_qwen3-8b-layer.md")
 
 

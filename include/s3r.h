@@ -147,7 +147,8 @@ s3r_status s3r_page_summaries(const s3r_paged_kv* kv, int32_t tail_only,
  *   tail page n_b - 1 is the only one whose keys change as a sequence
  *   decodes; the call summarises it from k_cache itself (min / max over its
  *   valid tokens), so no summary refresh is needed between draft steps and
- *   kmin/kmax are only read.
+ *   kmin/kmax are only read. kmin, kmax, q and out must be 16-byte aligned
+ *   (S3R_ERR_INVALID_ARG otherwise): the summary rows are bulk-copied.
  * workspace: at least s3r_attn_workspace_bytes(kv, 1, budget_pages) bytes;
  * it also carries the physical ids of the selected pages from the selection
  * kernel to the attention kernel.

@@ -27,7 +27,13 @@ torch's scaled_dot_product_attention in float64 and hand-derived closed forms;
 summaries bound every key; top-B == exhaustive subset search; q == p accepts
 everything; chi-square of committed tokens against p over 1e6 trials;
 acceptance rate == sum_x min(p, q); exact rational enumeration of the
-committed-sequence distribution.
+committed-sequence distribution. Temperature (tests/test_oracle_temperature.py):
+hand-derived cases at T = 0.5 and 0.7, chi-square and the acceptance rate at
+T = 0.7, planted temperature slips caught. KV upkeep (tests/test_oracle_kv.py):
+a dense per-sequence model over random rounds. Tree verification
+(tests/test_oracle_tree.py): a chain equals ordinary speculative sampling and
+causal verification; tree attention == SDPA with the ancestor mask; the
+multi-draft rule by rational enumeration; chi-square over a two-level tree.
 Parity unpinned (readings fixed by this build, not by the pages): the GQA
 aggregation of the page score (sum over the query heads of a KV group) and
 the absence of forced sink/recent pages in the top-B.

@@ -1,29 +1,22 @@
-// Split-KV paged attention for the S3R draft and verify steps.
+// Paged attention for the S3R draft and verify steps: the fp32 kernel, the
+// workspace plan shared by every attention path, and the dispatcher.
 //
 // S3R ("S3R: Fast and Faithful RL Rollouts via Self-Sparse Speculative
 // Decoding", weekinpapers.com, Abstract) drafts with sparse attention and
 // verifies with full attention over the complete KV history; both read the
-// same paged cache (PagedAttention, mlsanity.com reference list). One kernel
-// serves both: a CTA owns one (sequence, KV head, split) and walks a page
-// list - the selected pages (draft) or every page (verify) - and its partial
-// softmax state is merged across splits by a log-sum-exp combine done by the
-// last CTA of the (sequence, KV head) to finish (atomic ticket, no waiting).
+// same paged cache (PagedAttention, mlsanity.com reference list).
 //
-// bf16 path (tcgen05): all G query heads x R rows of a (sequence, KV head)
-// are packed into the rows of one MMA tile (M = 64, or 128 for more than 64
-// rows), so each K/V page tile fetched from HBM feeds one dense contraction:
-//   S = Q K^T  (M x 64 tokens, K = D), accumulator in tensor memory;
-//   softmax on S by four warps (one TMEM lane = one packed row per thread);
-//   O += P V   (M x D, K = 64 tokens), accumulator in tensor memory.
-// Warp roles: warps 0-3 softmax/epilogue, warp 4 TMA producer, warp 5 MMA
-// issuer + TMEM owner. K/V tiles arrive by TMA (3-D tensor map over the
-// cache, 128-byte swizzle, one box per page and 64-channel half) into a
-// 2-stage ring; S is double-buffered in TMEM so QK(j+1) overlaps softmax(j).
-// The running max is rescaled lazily (only when it grows by more than 2^8),
-// which leaves the result exact: O and l always share one reference.
+// attn_f32_kernel (fp32 caches; fp32 has no exact tensor-core kind): split-KV
+// on CUDA cores. A CTA owns one (sequence, KV head, split) and walks a page
+// list (the selected pages for the draft, every page for verify) in 16-token
+// sub-tiles with 16-byte loads; its partial softmax state is merged across
+// splits by a log-sum-exp combine in the last CTA of the (sequence, KV head)
+// to finish (atomic ticket, no waiting). Rows are masked causally, or by the
+// round's tree (a row sees the slots of its node's ancestors and itself).
 //
-// fp32 path: the same split/combine structure on CUDA cores with 16-byte
-// vector loads (fp32 has no exact tensor-core kind).
+// launch_attention dispatches bf16 work to the tcgen05 kernels: up to 64
+// packed rows (G query heads x R rows) to the token-major kernel
+// (s3r_attn_tok.cu), 65-128 rows to the rows-major kernel (s3r_attn_tc.cu).
 #include <cuda_bf16.h>
 
 #include <cmath>
