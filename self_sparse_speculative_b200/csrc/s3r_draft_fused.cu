@@ -17,14 +17,18 @@
 //   score(p) = sum_g sum_d max(q_g,d kmin_p,d, q_g,d kmax_p,d) for p < n_b,
 //   folded per channel into A max(kmin, kmax) + B min(kmin, kmax) with
 //   A = sum_g max(q_g, 0) and B = sum_g min(q_g, 0) (exact in real arithmetic),
-//   accumulated in float64; the tail page n_b - 1 is summarised from K itself
-//   (its keys change while the sequence decodes). The summary rows (and the
-//   tail page's K) are staged by cp.async in the K/V ring, which is still
-//   empty, chunk by chunk, and each quarter of a chunk is scored as soon as
-//   it lands. The kept pages come from the order-preserving keys: for up to
-//   256 pages each page's rank among the keys decides, beyond that a radix
-//   select of the budget-th largest key; they go, in ascending order with
-//   ties to the lower page, into a list in shared memory.
+//   and the tail page n_b - 1 is summarised from K itself (its keys change
+//   while the sequence decodes). The summary rows are read from global memory
+//   (a unit's rows are 2 D bytes per page, too small for bulk copies to pay);
+//   the tail page's K is bulk-copied into the K/V ring, which is still empty,
+//   while the other pages are scored. Scores are accumulated in float32 with
+//   a rigorous bound E_p on each page's rounding error; a radix select finds
+//   the budget-th largest float32 score s_B. A page with s_p > s_B + 2E (E the
+//   largest bound) is kept for certain, one with s_p < s_B - 2E dropped; the
+//   pages in between are re-scored in float64 and ranked (ties to the lower
+//   page) only when they outnumber the places left, so the kept set is the
+//   float64 top-B. It goes, in ascending page order, into a list in shared
+//   memory.
 //
 // Attention over the kept pages is the token-major pipeline of s3r_attn_tok.cu
 // (S^T = K Q^T and O^T += V^T P^T per 128-token stage, fp32 in TMEM):
@@ -57,9 +61,7 @@ struct DfLay {
   using T = TokLay<kDfN, D>;
   static constexpr int kNS = T::kNS;
   static constexpr uint32_t kRing = kNS * 2 * T::kTileBytes;
-  static constexpr uint32_t kRowBytes = 2 * D * 2;                 // kmin and kmax rows of one page
   static constexpr uint32_t kTailBytes = 64 * D * 2;               // K of one page (P <= 64)
-  static constexpr int kChunkPages = (int)((kRing - kTailBytes) / kRowBytes);
   static constexpr uint32_t kOffKeys = T::kOffKV + kRing;          // u64 [kDfMaxPages]
   static constexpr uint32_t kOffPhys = kOffKeys + 8 * kDfMaxPages; // int [kDfMaxPages]
   static constexpr uint32_t kOffList = kOffPhys + 4 * kDfMaxPages; // int2 [kDfMaxBudget]
@@ -67,9 +69,8 @@ struct DfLay {
   static constexpr uint32_t kOffTail = kOffAB + 2 * 8 * D;         // bf16 [2][D]
   static constexpr uint32_t kOffHist = kOffTail + 2 * 2 * D;       // u32 [256]
   static constexpr uint32_t kDynBytes = kOffHist + 4 * 256;
-  static_assert(kChunkPages >= 64, "staging chunk");
-  static_assert(8 * kDfMaxPages >= kDfThreads * 16, "tail scratch fits in the key array");
-  static_assert(12 * 8 * kDfMaxBudget <= kRing, "candidate arrays fit in the ring");
+  static_assert(4 * kDfMaxPages >= kDfThreads * 16, "tail scratch fits in the key array's upper half");
+  static_assert(kTailBytes + 12 * kDfMaxPages <= kRing, "tail rows and band scratch fit in the ring");
 };
 
 __device__ __forceinline__ void grp_sync(int id, int n) {
@@ -129,6 +130,9 @@ struct SelScratch {
   unsigned long long prefix;
   int k, done, shift, start;
   int wsum[8];
+  float wmax[8];
+  float emax[4];               // per cluster rank: the largest score error bound
+  uint32_t digit, want;
 };
 
 // Exclusive prefix sum over the group's nthr threads (whole warps); *total
@@ -184,22 +188,47 @@ __device__ void sel_prepare(const AttnParams& p, const DItem& d, int tg, int nth
   }
 }
 
-// Scores of pages [g0, g1) (none of them the tail page) into sm.keys; the
-// rows of page pg sit at rows + (pg - c0) * kRowBytes (kmin row, then kmax).
+// Order-preserving 32-bit image of a float score, and back.
+__device__ __forceinline__ uint32_t order_key32(float x) {
+  const uint32_t u = __float_as_uint(x);
+  return (u >> 31) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key32_value(uint32_t k) {
+  return __uint_as_float((k >> 31) ? (k & 0x7fffffffu) : ~k);
+}
+
+// Rounding bound of a float32 score (u = 2^-24): a product meets one
+// rounding of A or B to float32, at most D/32 in its lane's multiply-add
+// chain, one where the lane's two chains are added and five in the warp's
+// reduction: at most 11 at D = 128 (9 at D = 64), the tail page's score
+// likewise. A sum evaluated so is within gamma_11 = 11 u / (1 - 11 u) of the
+// exact value times the sum of the terms' magnitudes (N. Higham, Accuracy
+// and Stability of Numerical Algorithms, 2002, section 3.1); 16 u covers it
+// and the rounding of the magnitude sum itself.
+constexpr float kScoreGamma = 16.0f * 5.9604644775390625e-8f;
+
+// Float32 scores of pages [g0, g1) (none of them the tail page) of KV head
+// h into the 32-bit keys, the summary rows read from global memory (a unit's
+// 2 D bytes of a page are not contiguous with the next page's, so they come
+// as many small pieces; plain loads keep 32 of them in flight per lane).
 // Sixteen pages per warp and round, each lane holding D / 32 channels of
-// every page; the sixteen page sums are reduced across the warp together
-// (halving exchanges: lane l ends with page l % 16), which keeps sixteen
-// independent chains in flight per lane.
+// every page; the sixteen page sums (and their absolute sums for the bound)
+// are reduced across the warp together (halving exchanges: lane l ends with
+// page l % 16). Returns the thread's largest bound.
 template <int D>
-__device__ void score_pages(const AttnParams& p, int c0, int g0, int g1, const uint8_t* rows, int tg, int nthr,
-                            const SelSmem& sm) {
+__device__ float score_pages(const AttnParams& p, int h, int g0, int g1, int tg, int nthr, const SelSmem& sm,
+                             uint32_t* keys32) {
   constexpr int CPL = D / 32;
   constexpr int kU = 16;
   using Raw = typename std::conditional<CPL == 4, uint2, uint32_t>::type;
   const int lane = tg & 31, gw = tg >> 5, nw = nthr >> 5;
-  double wa[CPL], wb[CPL];
+  float wa[CPL], wb[CPL];
 #pragma unroll
-  for (int c = 0; c < CPL; ++c) { wa[c] = sm.ab[lane * CPL + c]; wb[c] = sm.ab[D + lane * CPL + c]; }
+  for (int c = 0; c < CPL; ++c) {
+    wa[c] = static_cast<float>(sm.ab[lane * CPL + c]);
+    wb[c] = static_cast<float>(sm.ab[D + lane * CPL + c]);
+  }
+  float emax = 0.f;
   for (int pg0 = g0 + gw * kU; pg0 < g1; pg0 += nw * kU) {
     Raw lo[kU], hi[kU];
     bool ok[kU];
@@ -208,13 +237,16 @@ __device__ void score_pages(const AttnParams& p, int c0, int g0, int g1, const u
       const int pg = pg0 + u;
       const int ph = pg < g1 ? sm.phys[pg] : -1;
       ok[u] = ph >= 0 && ph < p.num_pages_total;
-      const Raw* r = reinterpret_cast<const Raw*>(rows + (size_t)(pg - c0) * DfLay<D>::kRowBytes) + lane;
-      if (ok[u]) { lo[u] = r[0]; hi[u] = r[32]; }      // kmin row, kmax row (2 D bytes apart)
+      const size_t base = ((size_t)ph * p.Hkv + h) * D;
+      if (ok[u]) {
+        lo[u] = __ldg(reinterpret_cast<const Raw*>(static_cast<const __nv_bfloat16*>(p.kmin) + base) + lane);
+        hi[u] = __ldg(reinterpret_cast<const Raw*>(static_cast<const __nv_bfloat16*>(p.kmax) + base) + lane);
+      }
     }
-    double acc[kU];
+    float acc[kU], mag[kU];
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
-      double s0 = 0.0, s1 = 0.0;
+      float s0 = 0.f, s1 = 0.f, e = 0.f;
       if (ok[u]) {
         uint32_t lw[CPL / 2], hw[CPL / 2];
         if constexpr (CPL == 4) { lw[0] = ((uint2&)lo[u]).x; lw[1] = ((uint2&)lo[u]).y; hw[0] = ((uint2&)hi[u]).x; hw[1] = ((uint2&)hi[u]).y; }
@@ -224,34 +256,184 @@ __device__ void score_pages(const AttnParams& p, int c0, int g0, int g1, const u
           float l0, l1, r0, r1;
           bf2(lw[w], l0, l1);
           bf2(hw[w], r0, r1);
-          s0 = fma(wa[2 * w], static_cast<double>(fmaxf(l0, r0)), s0);
-          s1 = fma(wb[2 * w], static_cast<double>(fminf(l0, r0)), s1);
-          s0 = fma(wa[2 * w + 1], static_cast<double>(fmaxf(l1, r1)), s0);
-          s1 = fma(wb[2 * w + 1], static_cast<double>(fminf(l1, r1)), s1);
+          const float x0 = fmaxf(l0, r0), n0 = fminf(l0, r0), x1 = fmaxf(l1, r1), n1 = fminf(l1, r1);
+          s0 = fmaf(wa[2 * w], x0, s0);
+          s1 = fmaf(wb[2 * w], n0, s1);
+          s0 = fmaf(wa[2 * w + 1], x1, s0);
+          s1 = fmaf(wb[2 * w + 1], n1, s1);
+          e = fmaf(fabsf(wa[2 * w]), fabsf(x0), e);
+          e = fmaf(fabsf(wb[2 * w]), fabsf(n0), e);
+          e = fmaf(fabsf(wa[2 * w + 1]), fabsf(x1), e);
+          e = fmaf(fabsf(wb[2 * w + 1]), fabsf(n1), e);
         }
       }
       acc[u] = s0 + s1;
+      mag[u] = e;
     }
 #pragma unroll
     for (int w = kU / 2; w >= 1; w >>= 1) {
       const bool up = (lane & w) != 0;
 #pragma unroll
       for (int k = 0; k < w; ++k) {
-        const double send = up ? acc[k] : acc[k + w];
-        const double keep = up ? acc[k + w] : acc[k];
+        const float send = up ? acc[k] : acc[k + w];
+        const float keep = up ? acc[k + w] : acc[k];
         acc[k] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+        const float msend = up ? mag[k] : mag[k + w];
+        const float mkeep = up ? mag[k + w] : mag[k];
+        mag[k] = mkeep + __shfl_xor_sync(0xffffffffu, msend, w);
       }
     }
-    const double v = acc[0] + __shfl_xor_sync(0xffffffffu, acc[0], 16);
+    const float v = acc[0] + __shfl_xor_sync(0xffffffffu, acc[0], 16);
+    const float m = mag[0] + __shfl_xor_sync(0xffffffffu, mag[0], 16);
     const int pg = pg0 + (lane & 15);
     if (lane < kU && pg < g1) {
       bool okp = false;
 #pragma unroll
       for (int u = 0; u < kU; ++u) okp = (u == lane) ? ok[u] : okp;
       if (!okp) flag_status(p.status, S3R_DEV_BAD_PAGE_ID);
-      sm.keys[pg] = okp ? order_key(v) : 0ull;
+      keys32[pg] = okp ? order_key32(v) : 0u;
+      if (okp) emax = fmaxf(emax, kScoreGamma * m);
     }
   }
+  return emax;
+}
+
+// Bitonic network over the 32 lanes: descending order (lane 0 the largest).
+// A lane pair (i, i ^ j) keeps the larger value at the lower lane within a
+// descending run of length k.
+__device__ __forceinline__ uint32_t warp_sort_desc(uint32_t v, int lane) {
+#pragma unroll
+  for (int k = 2; k <= 32; k <<= 1)
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      const uint32_t o = __shfl_xor_sync(0xffffffffu, v, j);
+      const bool desc = (lane & k) == 0 || k == 32;
+      const bool lower = (lane & j) == 0;
+      v = (lower == desc) ? max(v, o) : min(v, o);
+    }
+  return v;
+}
+// The 32 largest of two descending 32-lists, descending: the lane-wise
+// maximum of one list and the other reversed is bitonic and holds them;
+// a half-cleaner cascade sorts it.
+__device__ __forceinline__ uint32_t warp_merge_top(uint32_t a, uint32_t b_rev, int lane) {
+  uint32_t v = max(a, b_rev);
+#pragma unroll
+  for (int j = 16; j > 0; j >>= 1) {
+    const uint32_t o = __shfl_xor_sync(0xffffffffu, v, j);
+    v = ((lane & j) == 0) ? max(v, o) : min(v, o);
+  }
+  return v;
+}
+// The B-th largest (B <= 32) of keys[0..n), n <= 256, by the 256 threads:
+// each warp sorts its 32 keys, then a tree of merges keeps the top 32.
+__device__ uint32_t top32_kth(const uint32_t* keys, int n, int B, int tg, int barid, uint32_t* xch) {
+  const int lane = tg & 31, gw = tg >> 5;
+  uint32_t v = warp_sort_desc(tg < n ? keys[tg] : 0u, lane);
+#pragma unroll
+  for (int step = 1; step < 8; step <<= 1) {
+    if ((gw & (2 * step - 1)) == step) xch[(gw - step) * 32 + 31 - lane] = v;   // reversed, for the partner
+    grp_sync(barid, kDfThreads);
+    if ((gw & (2 * step - 1)) == 0) v = warp_merge_top(v, xch[gw * 32 + lane], lane);
+    grp_sync(barid, kDfThreads);
+  }
+  if (gw == 0 && lane == B - 1) xch[0] = v;
+  grp_sync(barid, kDfThreads);
+  const uint32_t k = xch[0];
+  grp_sync(barid, kDfThreads);
+  return k;
+}
+
+// Rank of 32-bit key kp (page i) among keys[0..n): the keys above it plus
+// the equal keys of lower pages. keys 16-byte aligned; four keys per load.
+__device__ __forceinline__ int rank32(const uint32_t* keys, int n, uint32_t kp, int i) {
+  int r0 = 0, r1 = 0;
+  int j = 0;
+  const uint4* k4 = reinterpret_cast<const uint4*>(keys);
+  for (; j + 4 <= n; j += 4) {
+    const uint4 a = k4[j >> 2];
+    r0 += (a.x > kp) + (a.x == kp && j < i) + (a.y > kp) + (a.y == kp && j + 1 < i);
+    r1 += (a.z > kp) + (a.z == kp && j + 2 < i) + (a.w > kp) + (a.w == kp && j + 3 < i);
+  }
+  for (; j < n; ++j) r0 += (keys[j] > kp) + (keys[j] == kp && j < i);
+  return r0 + r1;
+}
+
+// The want-th largest (1-based) of keys[0..n), want <= n: 8-bit digits from
+// the top; per digit a shared-memory histogram of the keys that still match
+// the prefix (one atomic per distinct digit and warp), and warp 0 finds the
+// digit whose bin holds the want-th key. All threads of the group.
+__device__ uint32_t radix_kth_largest(const uint32_t* keys, int n, int want, int tg, int nthr, int barid,
+                                      unsigned* hist, SelScratch& sc) {
+  const int lane = tg & 31, gw = tg >> 5;
+  uint32_t prefix = 0, mask = 0;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = tg; i < 256; i += nthr) hist[i] = 0u;
+    grp_sync(barid, nthr);
+    for (int i0 = 0; i0 < n; i0 += nthr) {
+      const int i = i0 + tg;
+      const uint32_t k = i < n ? keys[i] : 0u;
+      const bool act = i < n && (k & mask) == prefix;
+      const uint32_t dig = act ? (k >> shift) & 255u : 0x100u | (uint32_t)lane;
+      const unsigned peers = __match_any_sync(0xffffffffu, dig);
+      if (act && lane == __ffs(peers) - 1) atomicAdd(&hist[dig], (unsigned)__popc(peers));
+    }
+    grp_sync(barid, nthr);
+    if (gw == 0) {
+      // lane l holds bins 255 - 8 l .. 248 - 8 l (from the top)
+      unsigned cnt[8], tot = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) { cnt[j] = hist[255 - (lane * 8 + j)]; tot += cnt[j]; }
+      unsigned inc = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += y;
+      }
+      const unsigned exc = inc - tot;
+      const unsigned w = (unsigned)want;
+      if (exc < w && w <= inc) {
+        unsigned c = exc;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (c + cnt[j] >= w && c < w) { sc.digit = 255u - (unsigned)(lane * 8 + j); sc.want = w - c; }
+          c += cnt[j];
+        }
+      }
+    }
+    grp_sync(barid, nthr);
+    prefix |= sc.digit << shift;
+    mask |= 255u << shift;
+    want = (int)sc.want;
+    grp_sync(barid, nthr);                             // sc is rewritten by the next digit
+  }
+  return prefix;
+}
+
+// Float64 score of page pg of the unit (warp-wide; every lane gets it): the
+// summaries from global memory, the tail page from sm.tail.
+template <int D>
+__device__ double score_page64(const AttnParams& p, const DItem& d, int pg, const SelSmem& sm, int lane) {
+  constexpr int CPL = D / 32;
+  const int ph = sm.phys[pg];
+  double a0 = 0.0, a1 = 0.0;
+  if (ph >= 0 && ph < p.num_pages_total) {
+    const bool tail = pg == d.n_b - 1;
+    const __nv_bfloat16* mn = static_cast<const __nv_bfloat16*>(p.kmin) + ((size_t)ph * p.Hkv + d.h) * D;
+    const __nv_bfloat16* mx = static_cast<const __nv_bfloat16*>(p.kmax) + ((size_t)ph * p.Hkv + d.h) * D;
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) {
+      const int ch = lane * CPL + c;
+      const float l = tail ? __bfloat162float(sm.tail[ch]) : __bfloat162float(mn[ch]);
+      const float r = tail ? __bfloat162float(sm.tail[D + ch]) : __bfloat162float(mx[ch]);
+      a0 = fma(sm.ab[ch], static_cast<double>(fmaxf(l, r)), a0);
+      a1 = fma(sm.ab[D + ch], static_cast<double>(fminf(l, r)), a1);
+    }
+  }
+  double v = a0 + a1;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
 }
 
 // Min and max of the tail page's valid tokens per channel into sm.tail (bf16,
@@ -312,35 +494,12 @@ __device__ __forceinline__ int key_rank(const unsigned long long* keys, int n, u
   return (r0 + r1) + (r2 + r3);
 }
 
-// Candidates of one group of at most nthr pages page0.. (keys in page
-// order): the pages whose rank in the group is below `budget`, appended in
-// page order to cand_key / cand_page at `base`. Returns the number appended.
-__device__ int group_candidates(const unsigned long long* keys, int page0, int n, int budget,
-                                unsigned long long* cand_key, int* cand_page, int base, int tg, int nthr,
-                                int barid, SelScratch& sc) {
-  bool keep = false;
-  unsigned long long kp = 0;
-  if (tg < n) {
-    kp = keys[tg];
-    keep = key_rank(keys, n, kp, tg) < budget;
-  }
-  int tot;
-  const int pos = grp_exclusive_scan(keep ? 1 : 0, tg, nthr, barid, sc, &tot);
-  if (keep) {
-    cand_key[base + pos] = kp;
-    cand_page[base + pos] = page0 + tg;
-  }
-  return tot;
-}
-
 // The kept pages of item d's unit, ascending, into `list` (logical,
 // physical) and, for the unit's first piece, into p.selected_out. All
 // threads of the CTA, after sel_prepare and the grid-dependency wait.
 // clustered: the unit is shared by the p.parts CTAs of this cluster (rank =
-// d.k); each scores its share of the pages and sends its candidates (the
-// pages that are top-B within their group of at most 256) to the first CTA,
-// which ranks the candidates and hands the list back. The global top-B is
-// contained in the union of the groups' top-B, so the result is exact.
+// d.k); each scores its share of the pages and sends its keys and its bound
+// to the first CTA, which selects and hands the list back.
 template <int D>
 __device__ void select_unit(const AttnParams& p, const DItem& d, int2* list, const SelSmem& sm, SelScratch& sc,
                             uint8_t* stage, uint32_t bar_g0, uint32_t bar_g1, bool clustered, volatile int* abort) {
@@ -351,6 +510,7 @@ __device__ void select_unit(const AttnParams& p, const DItem& d, int2* list, con
   int32_t* out = p.selected_out + ((size_t)d.b * p.Hkv + d.h) * p.budget;
   for (int k = tg; k < p.budget; k += nthr) list[k] = make_int2(-1, -1);
   if (d.bad) {
+    pdl_wait();
     if (write_out) {
       for (int k = tg; k < p.budget; k += nthr) out[k] = -1;
       if (tg == 0) flag_status(p.status, S3R_DEV_BAD_CONTEXT_LEN);
@@ -359,6 +519,7 @@ __device__ void select_unit(const AttnParams& p, const DItem& d, int2* list, con
   }
   const int n_b = d.n_b;
   if (n_b <= p.budget) {
+    pdl_wait();
     for (int k = tg; k < p.budget; k += nthr) {
       if (k < n_b) list[k] = make_int2(k, sm.phys[k]);
       if (write_out) out[k] = k < n_b ? k : -1;
@@ -377,116 +538,160 @@ __device__ void select_unit(const AttnParams& p, const DItem& d, int2* list, con
       static_cast<const __nv_bfloat16*>(p.k_cache) + ((size_t)tail_ph * p.Hkv + d.h) * p.P * D;
   const __nv_bfloat16* kmn = static_cast<const __nv_bfloat16*>(p.kmin);
   const __nv_bfloat16* kmx = static_cast<const __nv_bfloat16*>(p.kmax);
-  float4* scratch = reinterpret_cast<float4*>(sm.keys);
-  uint8_t* rows = stage + Lay::kTailBytes;
+  uint32_t* keys32 = reinterpret_cast<uint32_t*>(sm.keys);   // [kDfMaxPages], the array's lower half
+  float4* scratch = reinterpret_cast<float4*>(sm.keys + kDfMaxPages / 2);   // its upper half
   bool ok = true;
-  // summary rows of the share's pages, bulk-copied into the empty ring chunk
-  // by chunk, each chunk in two halves on two barriers so that the first
-  // half is scored while the second is still landing; the tail page's K
-  // (when in the share) with the first half of the first chunk
+  float emax = 0.f;
+  // the tail page's K (when in the share) bulk-copied into the empty ring
+  // while the other pages are scored from their summaries
+  if (has_tail && tail_ok && tg == 0) {
+    const uint32_t bytes = (uint32_t)valid * D * 2;
+    mbar_arrive_expect_tx(bar_g0, bytes);
+    bulk_load(smem_addr(stage), tail_src, bytes, bar_g0);
+  }
   const int e = min(s1, tail);                           // the share's pages other than the tail
-  int phase = 0;
-  for (int c0 = s0, first = 1; first || c0 < e; c0 += Lay::kChunkPages, first = 0, ++phase) {
-    const int c1 = max(c0, min(e, c0 + Lay::kChunkPages));
-    const int mid = c0 + (c1 - c0 + 1) / 2;
-    if (first && has_tail && tail_ok && tg == 0) {
-      const uint32_t bytes = (uint32_t)valid * D * 2;
-      mbar_expect_tx(bar_g0, bytes);
-      bulk_load(smem_addr(stage), tail_src, bytes, bar_g0);
-    }
-    for (int pg = c0 + tg; pg < c1; pg += nthr) {
-      const int ph = sm.phys[pg];
-      if (ph < 0 || ph >= p.num_pages_total) continue;
-      const uint32_t bar = pg < mid ? bar_g0 : bar_g1;
-      const size_t base = ((size_t)ph * p.Hkv + d.h) * D;
-      const uint32_t dst = smem_addr(rows + (size_t)(pg - c0) * Lay::kRowBytes);
-      mbar_expect_tx(bar, 4u * D);
-      bulk_load(dst, kmn + base, 2u * D, bar);
-      bulk_load(dst + 2u * D, kmx + base, 2u * D, bar);
-    }
-    grp_sync(barid, nthr);                               // every expectation is registered
-    if (tg == 0) { mbar_arrive(bar_g0); mbar_arrive(bar_g1); }
-    ok = ok && grp_all(mbar_wait(bar_g0, (uint32_t)(phase & 1), abort, p.status), barid, nthr);
-    if (ok && first && has_tail && tail_ok) {
+  emax = score_pages<D>(p, d.h, s0, e, tg, nthr, sm, keys32);
+  if (has_tail && tail_ok) {
+    ok = grp_all(mbar_wait(bar_g0, 0u, abort, p.status), barid, nthr);
+    if (ok) {
       tail_minmax<D>(reinterpret_cast<const __nv_bfloat16*>(stage), valid, tg, nthr, barid, sm, scratch);
-      grp_sync(barid, nthr);                             // the scratch is the key array
     }
-    if (ok) score_pages<D>(p, c0, c0, mid, rows, tg, nthr, sm);
-    ok = ok && grp_all(mbar_wait(bar_g1, (uint32_t)(phase & 1), abort, p.status), barid, nthr);
-    if (ok) score_pages<D>(p, c0, mid, c1, rows, tg, nthr, sm);
     fence_proxy_async_smem();                            // reads of the staged rows before copies reuse them
     grp_sync(barid, nthr);
-    if (!ok) break;
   }
   // the tail page, scored from its fresh min / max (first warp)
   if (ok && has_tail && gw == 0) {
     constexpr int CPL = D / 32;
-    double a0 = 0.0, a1 = 0.0;
+    float a0 = 0.f, a1 = 0.f, e = 0.f;
     if (tail_ok) {
 #pragma unroll
       for (int c = 0; c < CPL; ++c) {
         const int ch = lane * CPL + c;
         const float l = __bfloat162float(sm.tail[ch]), r = __bfloat162float(sm.tail[D + ch]);
-        a0 = fma(sm.ab[ch], static_cast<double>(fmaxf(l, r)), a0);
-        a1 = fma(sm.ab[D + ch], static_cast<double>(fminf(l, r)), a1);
+        const float wa = static_cast<float>(sm.ab[ch]), wb = static_cast<float>(sm.ab[D + ch]);
+        a0 = fmaf(wa, fmaxf(l, r), a0);
+        a1 = fmaf(wb, fminf(l, r), a1);
+        e = fmaf(fabsf(wa), fabsf(fmaxf(l, r)), e);
+        e = fmaf(fabsf(wb), fabsf(fminf(l, r)), e);
       }
     }
-    double v = a0 + a1;
+    float v = a0 + a1;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    for (int o = 16; o > 0; o >>= 1) {
+      v += __shfl_xor_sync(0xffffffffu, v, o);
+      e += __shfl_xor_sync(0xffffffffu, e, o);
+    }
     if (lane == 0) {
       if (!tail_ok) flag_status(p.status, S3R_DEV_BAD_PAGE_ID);
-      sm.keys[tail] = tail_ok ? order_key(v) : 0ull;
+      keys32[tail] = tail_ok ? order_key32(v) : 0u;
+      if (tail_ok) emax = fmaxf(emax, kScoreGamma * e);
     }
+  }
+  // the CTA's largest bound
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) emax = fmaxf(emax, __shfl_xor_sync(0xffffffffu, emax, o));
+  if (lane == 0) sc.wmax[gw] = emax;
+  grp_sync(barid, nthr);
+  if (tg == 0) {
+    float m = 0.f;
+    for (int w = 0; w < nthr / 32; ++w) m = fmaxf(m, sc.wmax[w]);
+    sc.emax[rank] = m;
   }
   grp_sync(barid, nthr);
-  // ---- candidates: the top-B of each group of at most nthr pages of the
-  // share, in page order, at their place in the first CTA's candidate array
-  // (the stage's first bytes: the ring is idle until the list is done)
-  unsigned long long* cand_key = reinterpret_cast<unsigned long long*>(stage);     // [8 * kDfMaxBudget]
-  int* cand_page = reinterpret_cast<int*>(stage + 8 * 8 * kDfMaxBudget);            // [8 * kDfMaxBudget]
-  auto cands_of = [&](int lo, int hi) {                  // candidates of pages [lo, hi), whole groups
-    int c = 0;
-    for (int g = lo; g < hi; g += nthr) c += min(p.budget, min(hi, g + nthr) - g);
-    return c;
-  };
-  if (clustered) cluster_sync_all();                     // every CTA scored: the first one's stage is free
-  int base = 0;
-  for (int r = 0; r < rank; ++r) base += cands_of(r * n_b / parts, (r + 1) * n_b / parts);
-  if (ok) {
-    for (int g = s0; g < s1; g += nthr) {
-      // this group's candidates into this CTA's own array, then (other CTAs
-      // of a cluster) copied to the first CTA's
-      const int n = min(s1, g + nthr) - g;
-      const int got = group_candidates(sm.keys + g, g, n, p.budget, cand_key, cand_page, base, tg, nthr, barid, sc);
-      grp_sync(barid, nthr);
-      if (clustered && rank != 0)
-        for (int k = tg; k < got; k += nthr) {
-          st_cluster_u64(&cand_key[base + k], 0u, cand_key[base + k]);
-          st_cluster_u32(&cand_page[base + k], 0u, (uint32_t)cand_page[base + k]);
-        }
-      base += got;
-    }
-  }
-  if (clustered) cluster_sync_all();                     // all candidates are in the first CTA
-  if (rank == 0 && ok) {
-    // ---- final rank among the candidates (ascending page order already)
-    int nc = 0;                                          // candidates of every share
-    for (int r = 0; r < parts; ++r) nc += cands_of(r * n_b / parts, (r + 1) * n_b / parts);
-    int kept_before = 0;
-    for (int c = 0; c < nc; c += nthr) {
-      const int i = c + tg;
-      bool keep = false;
-      if (i < nc) keep = key_rank(cand_key, nc, cand_key[i], i) < p.budget;
-      int tot;
-      const int pos = kept_before + grp_exclusive_scan(keep ? 1 : 0, tg, nthr, barid, sc, &tot);
-      if (keep && pos < p.budget) {
-        const int pg = cand_page[i];
-        list[pos] = make_int2(pg, sm.phys[pg]);
-        if (write_out) out[pos] = pg;
+  if (clustered) {
+    // every share's keys and bound into the first CTA
+    cluster_sync_all();                                  // every CTA has scored
+    if (rank != 0) {
+      for (int pg = s0 + tg; pg < s1; pg += nthr) st_cluster_u32(&keys32[pg], 0u, keys32[pg]);
+      if (tg == 0) st_cluster_u32(&sc.emax[rank], 0u, __float_as_uint(sc.emax[rank]));
+      if (has_tail) {
+        // the tail page's fresh min / max, for a float64 re-score there
+        const uint32_t* t32 = reinterpret_cast<const uint32_t*>(sm.tail);
+        for (int i = tg; i < D; i += nthr) st_cluster_u32(&t32[i], 0u, t32[i]);
       }
-      kept_before += tot;
     }
+    cluster_sync_all();                                  // the first CTA holds every key
+  }
+  pdl_wait();                                            // outputs and the workspace from here on
+  ok = grp_all(ok, barid, nthr);
+  if (rank == 0 && ok) {
+    const int B = p.budget;
+    float E = 0.f;
+    for (int r = 0; r < parts; ++r) E = fmaxf(E, sc.emax[r]);
+    // the B-th largest float32 score, and the band in which float32 cannot
+    // order pages: |s_p - s_B| <= 2E
+    uint32_t kB;
+    if (n_b <= nthr && B <= 32) {
+      kB = top32_kth(keys32, n_b, B, tg, barid, reinterpret_cast<uint32_t*>(stage));   // the ring is idle
+    } else if (n_b <= nthr) {
+      // one key per thread: its rank among all (ties to the lower page)
+      if (tg < n_b && rank32(keys32, n_b, keys32[tg], tg) == B - 1) sc.digit = keys32[tg];
+      grp_sync(barid, nthr);
+      kB = sc.digit;
+      grp_sync(barid, nthr);
+    } else {
+      kB = radix_kth_largest(keys32, n_b, B, tg, nthr, barid, sm.hist, sc);
+    }
+    const double sB = static_cast<double>(key32_value(kB));
+    const double hiB = sB + 2.0 * static_cast<double>(E), loB = sB - 2.0 * static_cast<double>(E);
+    // each thread owns a run of consecutive pages (the list keeps page order)
+    const int per = (n_b + nthr - 1) / nthr;
+    const int q0 = min(n_b, tg * per), q1 = min(n_b, q0 + per);
+    int n_in = 0, n_unc = 0;
+    for (int pg = q0; pg < q1; ++pg) {
+      const double sp = static_cast<double>(key32_value(keys32[pg]));
+      n_in += sp > hiB;
+      n_unc += sp <= hiB && sp >= loB;
+    }
+    int tot_in, tot_unc;
+    grp_exclusive_scan(n_in, tg, nthr, barid, sc, &tot_in);
+    const int unc_before = grp_exclusive_scan(n_unc, tg, nthr, barid, sc, &tot_unc);
+    const int need = B - tot_in;                         // places left for the band's pages
+    // keep flags of the band's pages, one bit per page (the histogram's words)
+    unsigned* keepbits = sm.hist;
+    for (int i = tg; i < 256; i += nthr) keepbits[i] = 0u;
+    grp_sync(barid, nthr);
+    if (tot_unc > need) {
+      // float64 scores of the band's pages, ranked among themselves (ties to
+      // the lower page); the ring is idle until the list is done
+      unsigned long long* ukey = reinterpret_cast<unsigned long long*>(stage);           // [kDfMaxPages]
+      int* upage = reinterpret_cast<int*>(stage + 8 * kDfMaxPages);                     // [kDfMaxPages]
+      int j = unc_before;
+      for (int pg = q0; pg < q1; ++pg) {
+        const double sp = static_cast<double>(key32_value(keys32[pg]));
+        if (sp <= hiB && sp >= loB) upage[j++] = pg;
+      }
+      grp_sync(barid, nthr);
+      for (int u = gw; u < tot_unc; u += nthr / 32) {
+        const double v = score_page64<D>(p, d, upage[u], sm, lane);
+        if (lane == 0) ukey[u] = order_key(v);
+      }
+      grp_sync(barid, nthr);
+      for (int u = tg; u < tot_unc; u += nthr)
+        if (key_rank(ukey, tot_unc, ukey[u], u) < need) atomicOr(&keepbits[upage[u] >> 5], 1u << (upage[u] & 31));
+      grp_sync(barid, nthr);
+    }
+    // the list: certain pages and the band's kept ones, in page order
+    int n_keep = 0;
+    for (int pg = q0; pg < q1; ++pg) {
+      const double sp = static_cast<double>(key32_value(keys32[pg]));
+      const bool band = sp <= hiB && sp >= loB;
+      n_keep += sp > hiB || (band && (tot_unc <= need || ((keepbits[pg >> 5] >> (pg & 31)) & 1u)));
+    }
+    int tot_keep;
+    int pos = grp_exclusive_scan(n_keep, tg, nthr, barid, sc, &tot_keep);
+    for (int pg = q0; pg < q1; ++pg) {
+      const double sp = static_cast<double>(key32_value(keys32[pg]));
+      const bool band = sp <= hiB && sp >= loB;
+      if (sp > hiB || (band && (tot_unc <= need || ((keepbits[pg >> 5] >> (pg & 31)) & 1u)))) {
+        if (pos < B) {
+          list[pos] = make_int2(pg, sm.phys[pg]);
+          if (write_out) out[pos] = pg;
+        }
+        ++pos;
+      }
+    }
+    fence_proxy_async_smem();                            // scratch in the ring before the copies reuse it
     grp_sync(barid, nthr);
   }
   if (clustered) {
@@ -623,7 +828,8 @@ draft_fused_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem;
-  pdl_wait();                                            // summaries, outputs and workspace from here on
+  // the selection reads only inputs (summaries, the tail page's keys) until
+  // its grid-dependency wait, which it executes before any output
   select_unit<D>(p, d0, s_list, sm, s_sc, sKV, BAR(B_G0), BAR(B_G1), clustered, &s_abort);
   __syncthreads();
 

@@ -74,7 +74,8 @@ template <typename T>
 __global__ void __launch_bounds__(kSumThreads) summaries_kernel(const SumParams p) {
   __shared__ uint4 s_min[kSumThreads];
   __shared__ uint4 s_max[kSumThreads];
-  pdl_launch_dependents();
+  // no early release of the next kernel: the summaries written here are
+  // inputs that later calls may read before their grid-dependency wait
   const int h = blockIdx.x, b = blockIdx.z;
   const int L = p.context_lens[b];
   if (L < 1 || L > p.max_pages * p.P) {

@@ -166,3 +166,44 @@ def test_caller_written_tail_keys_and_query_are_seen():
         if all(RR.compare_selection(f"seq {b}", gsel[b], sel[b], gaps[b], tally, scores=scores[b])):
             RR.assert_close(f"seq {b} out", gout[b], out[b], "bf16")
     assert moved > 0                                   # the new keys changed the selection
+
+
+@pytest.mark.parametrize("num_seqs,heads,budget", [(2, 2, 5), (40, 2, 3)], ids=["clusters", "one-cta-per-unit"])
+def test_exact_ties_go_to_the_lower_page(num_seqs, heads, budget):
+    """Every page of a sequence but the tail is a copy of its first page, so
+    their page scores are exactly equal: float32 cannot order them and the
+    float64 re-scoring with ties to the lower page decides. The kept pages
+    are exactly the oracle's (the lowest page ids, plus the tail page when
+    it scores higher); the outputs follow."""
+    s = custom_spec(1, num_seqs=num_seqs, num_q_heads=4 * heads, num_kv_heads=heads, page_size=64, gamma=1,
+                    budget_pages=budget, vocab=512)
+    lens = _ragged(num_seqs, 64 * 6, 64 * 20, 7)
+    wl = Workload(s, seed=12, context_lens=lens)
+    st = DecodeStep(wl)
+    K = wl.kv_cache("K").copy()                       # bf16 bit patterns [pages, H, P, D]
+    V = wl.kv_cache("V")
+    bt = wl.block_table.astype(np.int64)
+    for b in range(num_seqs):
+        n = int(wl.pages_per_seq[b])
+        for j in range(1, n - 1):
+            K[bt[b, j]] = K[bt[b, 0]]
+    st.k_cache.copy_(torch.from_numpy(K.view(np.int16)).view(torch.bfloat16).cuda())
+    st.summaries(tail_only=False)
+    st.draft(0)
+    torch.cuda.synchronize()
+    assert s3r.s3r_device_status(st.ws_draft) == (s3r.S3R_OK, 0)
+    K64, V64 = to_float64(K, "bf16"), to_float64(V, "bf16")
+    q64 = to_float64(wl.q_draft[0], "bf16")
+    cl = np.asarray(lens)
+    kmin, kmax = O.page_summaries(K64, bt, cl, s.page_size)
+    sel, _ = O.sparse_draft_select(q64, kmin, kmax, bt, cl, s.page_size, budget, s.group)
+    out, lse = O.sparse_draft_attn(q64, K64, V64, bt, cl, sel, RR.f32(wl.scale))
+    gsel = st.selected[0].cpu().numpy()
+    gout = st.draft_out[0].float().cpu().numpy()
+    ties = 0
+    for b in range(num_seqs):
+        for h in range(heads):
+            assert gsel[b, h].tolist() == list(sel[b][h]), (b, h, gsel[b, h].tolist(), list(sel[b][h]))
+            ties += int(1 in sel[b][h])
+        RR.assert_close(f"seq {b} out", gout[b], out[b], "bf16")
+    assert ties > 0                                    # the tie rule decided
