@@ -170,7 +170,7 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
     // ======================================================= producer warp
     // A page list is an earlier kernel's output (wait for it first); the
     // block table and the K/V cache are inputs, so the dense path resolves
-    // its first page ids before the wait.
+    // its first page ids and issues its first NS ring stages before the wait.
     if (p.page_list) pdl_wait();
     const uint64_t pol = l2_policy_evict_first();
     // page-id windows of 32 flattened positions: lane k of a window holds
@@ -191,7 +191,7 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
     page_of(p, s_prefix, wbase + 32 + lane, hi, W, &w1_lp, &w1_u, &pp);
     w1_ph = phys_load(w1_lp, w1_u, pp);
     page_of(p, s_prefix, wbase + 64 + lane, hi, W, &w2_lp, &w2_u, &w2_pp);
-    if (!p.page_list) pdl_wait();
+    bool waited = p.page_list != nullptr;
     int g = 0;
     bool ok = true;
     for (int x = lo; x < hi && ok;) {
@@ -199,6 +199,10 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
       const int nst = (sg.npg + ppt - 1) / ppt;
       for (int j = 0; j < nst; ++j, ++g) {
         const int st = g % NS;
+        if (g == NS && !waited) {                        // the ring's first fill went out before it
+          pdl_wait();
+          waited = true;
+        }
         // the stage's page ids first (they do not need the slot), then the slot
         int my_lp = -1, my_ph = -1;
         for (int pp = 0; pp < ppt; ++pp) {
@@ -243,6 +247,7 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
       }
       x = sg.end;
     }
+    if (!waited) pdl_wait();
     // drain: wait until every issued copy has landed
     if (lane == 0)
       for (int k = max(0, g - NS); k < g; ++k) mbar_wait_drain(BAR(B_FULL + k % NS), (k / NS) & 1, p.status);

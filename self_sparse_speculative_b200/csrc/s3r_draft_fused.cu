@@ -495,8 +495,9 @@ __device__ __forceinline__ int key_rank(const unsigned long long* keys, int n, u
 }
 
 // The kept pages of item d's unit, ascending, into `list` (logical,
-// physical) and, for the unit's first piece, into p.selected_out. All
-// threads of the CTA, after sel_prepare and the grid-dependency wait.
+// physical). All threads of the CTA, after sel_prepare. It reads only inputs
+// (summaries, the tail page's keys) and writes only shared memory (and the
+// status word), so it runs before the grid-dependency wait.
 // clustered: the unit is shared by the p.parts CTAs of this cluster (rank =
 // d.k); each scores its share of the pages and sends its keys and its bound
 // to the first CTA, which selects and hands the list back.
@@ -506,24 +507,14 @@ __device__ void select_unit(const AttnParams& p, const DItem& d, int2* list, con
   using Lay = DfLay<D>;
   constexpr int nthr = kDfThreads, barid = kBarAll;
   const int tg = threadIdx.x, lane = tg & 31, gw = tg >> 5;
-  const bool write_out = d.k == 0;
-  int32_t* out = p.selected_out + ((size_t)d.b * p.Hkv + d.h) * p.budget;
   for (int k = tg; k < p.budget; k += nthr) list[k] = make_int2(-1, -1);
   if (d.bad) {
-    pdl_wait();
-    if (write_out) {
-      for (int k = tg; k < p.budget; k += nthr) out[k] = -1;
-      if (tg == 0) flag_status(p.status, S3R_DEV_BAD_CONTEXT_LEN);
-    }
+    if (d.k == 0 && tg == 0) flag_status(p.status, S3R_DEV_BAD_CONTEXT_LEN);
     return;
   }
   const int n_b = d.n_b;
   if (n_b <= p.budget) {
-    pdl_wait();
-    for (int k = tg; k < p.budget; k += nthr) {
-      if (k < n_b) list[k] = make_int2(k, sm.phys[k]);
-      if (write_out) out[k] = k < n_b ? k : -1;
-    }
+    for (int k = tg; k < n_b; k += nthr) list[k] = make_int2(k, sm.phys[k]);
     return;
   }
   // this CTA's share of the pages
@@ -536,8 +527,6 @@ __device__ void select_unit(const AttnParams& p, const DItem& d, int2* list, con
   const bool tail_ok = tail_ph >= 0 && tail_ph < p.num_pages_total;
   const __nv_bfloat16* tail_src =
       static_cast<const __nv_bfloat16*>(p.k_cache) + ((size_t)tail_ph * p.Hkv + d.h) * p.P * D;
-  const __nv_bfloat16* kmn = static_cast<const __nv_bfloat16*>(p.kmin);
-  const __nv_bfloat16* kmx = static_cast<const __nv_bfloat16*>(p.kmax);
   uint32_t* keys32 = reinterpret_cast<uint32_t*>(sm.keys);   // [kDfMaxPages], the array's lower half
   float4* scratch = reinterpret_cast<float4*>(sm.keys + kDfMaxPages / 2);   // its upper half
   bool ok = true;
@@ -612,7 +601,6 @@ __device__ void select_unit(const AttnParams& p, const DItem& d, int2* list, con
     }
     cluster_sync_all();                                  // the first CTA holds every key
   }
-  pdl_wait();                                            // outputs and the workspace from here on
   ok = grp_all(ok, barid, nthr);
   if (rank == 0 && ok) {
     const int B = p.budget;
@@ -684,10 +672,7 @@ __device__ void select_unit(const AttnParams& p, const DItem& d, int2* list, con
       const double sp = static_cast<double>(key32_value(keys32[pg]));
       const bool band = sp <= hiB && sp >= loB;
       if (sp > hiB || (band && (tot_unc <= need || ((keepbits[pg >> 5] >> (pg & 31)) & 1u)))) {
-        if (pos < B) {
-          list[pos] = make_int2(pg, sm.phys[pg]);
-          if (write_out) out[pos] = pg;
-        }
+        if (pos < B) list[pos] = make_int2(pg, sm.phys[pg]);
         ++pos;
       }
     }
@@ -828,8 +813,10 @@ draft_fused_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem;
-  // the selection reads only inputs (summaries, the tail page's keys) until
-  // its grid-dependency wait, which it executes before any output
+  // the selection and the first ring stages read only inputs, so they run
+  // before the grid-dependency wait; every role takes the wait before it
+  // touches an output or the workspace (the producer after its first NS
+  // stages)
   select_unit<D>(p, d0, s_list, sm, s_sc, sKV, BAR(B_G0), BAR(B_G1), clustered, &s_abort);
   __syncthreads();
 
@@ -837,6 +824,7 @@ draft_fused_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
     // ======================================================= producer warp
     const uint64_t pol = l2_policy_evict_first();
     int g = 0;
+    bool waited = false;
     bool ok = __all_sync(0xffffffffu, !s_abort);
     for (int it = it0; it < it1 && ok; ++it) {
       const DItem d = d0;                                  // the CTA's one item
@@ -844,6 +832,10 @@ draft_fused_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
       const int nst = (d.npg + ppt - 1) / ppt;
       for (int j = 0; j < nst; ++j, ++g) {
         const int st = g % NS;
+        if (g == NS && !waited) {                          // the ring's first fill went out before it
+          pdl_wait();
+          waited = true;
+        }
         int my_lp = -1, my_ph = -1;
         if (lane < ppt && j * ppt + lane < d.npg) {
           const int2 e = list[d.k0 + j * ppt + lane];
@@ -876,10 +868,12 @@ draft_fused_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
         }
       }
     }
+    if (!waited) pdl_wait();
     if (lane == 0)
       for (int k = max(0, g - NS); k < g; ++k) mbar_wait_drain(BAR(B_FULL + k % NS), (k / NS) & 1, p.status);
   } else if (warp == kDfMma) {
     // ======================================================= MMA issuer
+    pdl_wait();
     if (lane == 0) {
       constexpr uint32_t idQK = idesc_bf16_f32(kTok, N, false, false);
       constexpr uint32_t idPV = idesc_bf16_f32(D, N, true, false);
@@ -952,6 +946,7 @@ draft_fused_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
     }
   } else if (warp < 4) {
     // ======================================================= softmax warps
+    pdl_wait();
     // Thread t: token t of each stage (TMEM lane t of S^T), and TMEM lane t
     // of O^T in the epilogue (dimension t for D = 128; for D = 64 the M = 64
     // accumulator puts dimension 16q + l in lane 32q + l, l < 16).
@@ -1159,6 +1154,13 @@ draft_fused_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
         }
       }
       asm volatile("bar.sync 1, 128;" ::: "memory");    // s_alpha / s_nu reads done
+    }
+  } else {
+    // ================================== selection helpers: the kept pages
+    pdl_wait();
+    if (d0.k == 0) {
+      int32_t* out = p.selected_out + ((size_t)d0.b * p.Hkv + d0.h) * p.budget;
+      for (int k = tid - 6 * 32; k < p.budget; k += kDfThreads - 6 * 32) out[k] = s_list[k].x;
     }
   }
 
