@@ -167,7 +167,15 @@ S3R_EXPORT s3r_status s3r_sparse_draft_attn(const s3r_paged_kv* kv, const void* 
   }
   uint32_t* status = static_cast<uint32_t*>(workspace);
   int32_t* phys = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + pl.off_phys);
-  s = from_cuda(launch_select(*kv, kmin, kmax, q, budget_pages, selected, phys, status, st));
+  if (select_only_supported(*kv, budget_pages)) {
+    AttnParams ps = p;
+    ps.kmin = kmin;
+    ps.kmax = kmax;
+    ps.selected_out = selected;
+    s = from_cuda(launch_select_only(*kv, ps, phys, st));
+  } else {
+    s = from_cuda(launch_select(*kv, kmin, kmax, q, budget_pages, selected, phys, status, st));
+  }
   if (s != S3R_OK) return s;
   p.page_phys = phys;
   s3r_status api;

@@ -211,15 +211,14 @@ constexpr float kScoreGamma = 16.0f * 5.9604644775390625e-8f;
 // h into the 32-bit keys, the summary rows read from global memory (a unit's
 // 2 D bytes of a page are not contiguous with the next page's, so they come
 // as many small pieces; plain loads keep 32 of them in flight per lane).
-// Sixteen pages per warp and round, each lane holding D / 32 channels of
-// every page; the sixteen page sums (and their absolute sums for the bound)
-// are reduced across the warp together (halving exchanges: lane l ends with
-// page l % 16). Returns the thread's largest bound.
-template <int D>
+// kU pages (16 or 8) per warp and round, each lane holding D / 32 channels
+// of every page; the kU page sums (and their absolute sums for the bound) are
+// reduced across the warp together (halving exchanges: lane l ends with page
+// l % kU). Returns the thread's largest bound.
+template <int D, int kU>
 __device__ float score_pages(const AttnParams& p, int h, int g0, int g1, int tg, int nthr, const SelSmem& sm,
                              uint32_t* keys32) {
   constexpr int CPL = D / 32;
-  constexpr int kU = 16;
   using Raw = typename std::conditional<CPL == 4, uint2, uint32_t>::type;
   const int lane = tg & 31, gw = tg >> 5, nw = nthr >> 5;
   float wa[CPL], wb[CPL];
@@ -283,9 +282,15 @@ __device__ float score_pages(const AttnParams& p, int h, int g0, int g1, int tg,
         mag[k] = mkeep + __shfl_xor_sync(0xffffffffu, msend, w);
       }
     }
-    const float v = acc[0] + __shfl_xor_sync(0xffffffffu, acc[0], 16);
-    const float m = mag[0] + __shfl_xor_sync(0xffffffffu, mag[0], 16);
-    const int pg = pg0 + (lane & 15);
+    // lane l now holds page l % kU summed over its kU-lane group; the groups
+    // combine (five additions on every path whatever kU)
+    float v = acc[0], m = mag[0];
+#pragma unroll
+    for (int o = kU; o < 32; o <<= 1) {
+      v += __shfl_xor_sync(0xffffffffu, v, o);
+      m += __shfl_xor_sync(0xffffffffu, m, o);
+    }
+    const int pg = pg0 + (lane & (kU - 1));
     if (lane < kU && pg < g1) {
       bool okp = false;
 #pragma unroll
@@ -325,11 +330,17 @@ __device__ __forceinline__ uint32_t warp_merge_top(uint32_t a, uint32_t b_rev, i
   }
   return v;
 }
-// The B-th largest (B <= 32) of keys[0..n), n <= 256, by the 256 threads:
-// each warp sorts its 32 keys, then a tree of merges keeps the top 32.
+// The B-th largest (B <= 32) of keys[0..n) by the 256 threads: each warp
+// sorts 32 keys at a time and keeps the top 32 of what it has seen (keys
+// tg, tg + 256, ...), then a tree of merges across the warps keeps the top 32.
 __device__ uint32_t top32_kth(const uint32_t* keys, int n, int B, int tg, int barid, uint32_t* xch) {
   const int lane = tg & 31, gw = tg >> 5;
   uint32_t v = warp_sort_desc(tg < n ? keys[tg] : 0u, lane);
+  for (int base = kDfThreads; base < n; base += kDfThreads) {        // uniform: n is
+    const int i = base + tg;
+    const uint32_t w = warp_sort_desc(i < n ? keys[i] : 0u, lane);
+    v = warp_merge_top(v, __shfl_sync(0xffffffffu, w, 31 - lane), lane);
+  }
 #pragma unroll
   for (int step = 1; step < 8; step <<= 1) {
     if ((gw & (2 * step - 1)) == step) xch[(gw - step) * 32 + 31 - lane] = v;   // reversed, for the partner
@@ -501,7 +512,8 @@ __device__ __forceinline__ int key_rank(const unsigned long long* keys, int n, u
 // clustered: the unit is shared by the p.parts CTAs of this cluster (rank =
 // d.k); each scores its share of the pages and sends its keys and its bound
 // to the first CTA, which selects and hands the list back.
-template <int D>
+// KU: pages per warp and scoring round (registers: two summary pieces each).
+template <int D, int KU = 16>
 __device__ void select_unit(const AttnParams& p, const DItem& d, int2* list, const SelSmem& sm, SelScratch& sc,
                             uint8_t* stage, uint32_t bar_g0, uint32_t bar_g1, bool clustered, volatile int* abort) {
   using Lay = DfLay<D>;
@@ -539,7 +551,7 @@ __device__ void select_unit(const AttnParams& p, const DItem& d, int2* list, con
     bulk_load(smem_addr(stage), tail_src, bytes, bar_g0);
   }
   const int e = min(s1, tail);                           // the share's pages other than the tail
-  emax = score_pages<D>(p, d.h, s0, e, tg, nthr, sm, keys32);
+  emax = score_pages<D, KU>(p, d.h, s0, e, tg, nthr, sm, keys32);
   if (has_tail && tail_ok) {
     ok = grp_all(mbar_wait(bar_g0, 0u, abort, p.status), barid, nthr);
     if (ok) {
@@ -609,7 +621,7 @@ __device__ void select_unit(const AttnParams& p, const DItem& d, int2* list, con
     // the B-th largest float32 score, and the band in which float32 cannot
     // order pages: |s_p - s_B| <= 2E
     uint32_t kB;
-    if (n_b <= nthr && B <= 32) {
+    if (B <= 32) {
       kB = top32_kth(keys32, n_b, B, tg, barid, reinterpret_cast<uint32_t*>(stage));   // the ring is idle
     } else if (n_b <= nthr) {
       // one key per thread: its rank among all (ties to the lower page)
@@ -1176,6 +1188,67 @@ draft_fused_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
   }
 }
 
+// Page selection alone, for launches with more (sequence, KV head) units
+// than SMs: one CTA per unit runs the fused kernel's selection (scoring
+// before the grid-dependency wait), then writes the kept pages' logical ids
+// to selected_out and their physical ids to `phys_out` ([S, Hkv, budget], in
+// the workspace) for the split-KV attention kernel. Small shared memory, so
+// several CTAs share an SM and their summary loads overlap.
+template <int D>
+struct SelOnlyLay {
+  // the tail page's K, then the band scratch (float64 keys and pages)
+  static constexpr uint32_t kStage =
+      DfLay<D>::kTailBytes > 12u * kDfMaxPages ? DfLay<D>::kTailBytes : 12u * kDfMaxPages;
+  static constexpr uint32_t kOffKeys = kStage;                      // u64 [kDfMaxPages]
+  static constexpr uint32_t kOffPhys = kOffKeys + 8 * kDfMaxPages;  // int [kDfMaxPages]
+  static constexpr uint32_t kOffList = kOffPhys + 4 * kDfMaxPages;  // int2 [kDfMaxBudget]
+  static constexpr uint32_t kOffAB = kOffList + 8 * kDfMaxBudget;   // double [2][D]
+  static constexpr uint32_t kOffTail = kOffAB + 2 * 8 * D;          // bf16 [2][D]
+  static constexpr uint32_t kOffHist = kOffTail + 2 * 2 * D;        // u32 [256]
+  static constexpr uint32_t kDynBytes = kOffHist + 4 * 256;
+  static_assert(kStage >= 12 * kDfMaxPages, "band scratch fits in the tail stage");
+};
+
+template <int D>
+__global__ void __launch_bounds__(kDfThreads, 3) select_only_kernel(const AttnParams p, int32_t* phys_out) {
+  using Lay = SelOnlyLay<D>;
+  extern __shared__ __align__(1024) uint8_t dyn_raw[];
+  uint8_t* dyn = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t s_bar[2];
+  __shared__ int s_abort;
+  __shared__ SelScratch s_sc;
+  const int tid = threadIdx.x;
+  SelSmem sm;
+  sm.keys = reinterpret_cast<unsigned long long*>(dyn + Lay::kOffKeys);
+  sm.phys = reinterpret_cast<int*>(dyn + Lay::kOffPhys);
+  sm.ab = reinterpret_cast<double*>(dyn + Lay::kOffAB);
+  sm.tail = reinterpret_cast<__nv_bfloat16*>(dyn + Lay::kOffTail);
+  sm.hist = reinterpret_cast<unsigned*>(dyn + Lay::kOffHist);
+  int2* s_list = reinterpret_cast<int2*>(dyn + Lay::kOffList);
+  if (tid == 0) {
+    mbar_init(smem_addr(&s_bar[0]), 1);
+    mbar_init(smem_addr(&s_bar[1]), 1);
+    s_abort = 0;
+    fence_barrier_init();
+  }
+  const DItem d0 = draft_item(p, blockIdx.x);              // p.parts == 1: one unit per CTA
+  sel_prepare<D>(p, d0, tid, kDfThreads, sm);
+  __syncthreads();
+  select_unit<D, 8>(p, d0, s_list, sm, s_sc, dyn, smem_addr(&s_bar[0]), smem_addr(&s_bar[1]), false, &s_abort);
+  __syncthreads();
+  pdl_wait();                                              // outputs and the workspace from here on
+  const size_t o = ((size_t)d0.b * p.Hkv + d0.h) * p.budget;
+  for (int k = tid; k < p.budget; k += kDfThreads) {
+    const int2 e = s_list[k];
+    p.selected_out[o + k] = e.x;
+    phys_out[o + k] = e.y;
+  }
+  // the attention kernel (persistent, a whole SM per CTA) may launch only
+  // once every selection CTA is done: earlier, it would take SMs from the
+  // selection's later waves
+  pdl_launch_dependents();
+}
+
 }  // namespace
 
 bool draft_fused_supported(const s3r_paged_kv& kv, int32_t budget_pages) {
@@ -1232,6 +1305,30 @@ cudaError_t prepare_draft_fused(const s3r_paged_kv& kv, int32_t budget_pages, Dr
   if (parts < 1) parts = 1;
   dl->parts = parts;
   return kv.head_dim == 64 ? prepare_d<64>(kv, budget_pages, dl) : prepare_d<128>(kv, budget_pages, dl);
+}
+
+bool select_only_supported(const s3r_paged_kv& kv, int32_t budget_pages) {
+  const int G = kv.num_q_heads / kv.num_kv_heads;
+  return kv.dtype == S3R_BF16 && G <= 8 && budget_pages >= 1 && budget_pages <= kDfMaxBudget &&
+         kv.max_pages_per_seq <= kDfMaxPages && (kv.page_size == 16 || kv.page_size == 64) &&
+         (kv.head_dim == 64 || kv.head_dim == 128);
+}
+
+template <int D>
+static cudaError_t launch_select_only_d(const s3r_paged_kv& kv, const AttnParams& p, int32_t* phys_out,
+                                       cudaStream_t st) {
+  const size_t smem = SelOnlyLay<D>::kDynBytes + 1024;
+  cudaError_t e = cudaFuncSetAttribute(select_only_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  AttnParams q = p;
+  q.parts = 1;
+  return launch_kernel(select_only_kernel<D>, dim3(kv.num_seqs * kv.num_kv_heads), dim3(kDfThreads), smem, st, 1, q,
+                       phys_out);
+}
+
+cudaError_t launch_select_only(const s3r_paged_kv& kv, const AttnParams& p, int32_t* phys_out, cudaStream_t st) {
+  return kv.head_dim == 64 ? launch_select_only_d<64>(kv, p, phys_out, st)
+                           : launch_select_only_d<128>(kv, p, phys_out, st);
 }
 
 cudaError_t launch_draft_fused(const s3r_paged_kv& kv, const DraftLaunch& dl, const AttnParams& p, cudaStream_t st) {

@@ -122,6 +122,11 @@ struct DraftLaunch {
 };
 cudaError_t prepare_draft_fused(const s3r_paged_kv& kv, int32_t budget_pages, DraftLaunch* dl);
 cudaError_t launch_draft_fused(const s3r_paged_kv& kv, const DraftLaunch& dl, const AttnParams& p, cudaStream_t st);
+// Selection alone (the fused kernel's selection, one CTA per unit) for the
+// two-kernel sparse draft: kept pages to p.selected_out, their physical ids
+// to phys_out ([S, Hkv, budget]).
+bool select_only_supported(const s3r_paged_kv& kv, int32_t budget_pages);
+cudaError_t launch_select_only(const s3r_paged_kv& kv, const AttnParams& p, int32_t* phys_out, cudaStream_t st);
 bool make_cache_map(CUtensorMap* map, const void* base, const s3r_paged_kv& kv);
 int device_sm_count();
 

@@ -83,12 +83,14 @@ def test_fused_draft_matches_oracle(name):
     _check(name, wl, st, [0])
 
 
-def test_fused_draft_flags_bad_inputs_without_faulting():
+@pytest.mark.parametrize("num_seqs", [3, 100], ids=["fused", "selection-kernel"])
+def test_fused_draft_flags_bad_inputs_without_faulting(num_seqs):
     """A bad context length and an out-of-range block-table entry are recorded
     in the status word; the unusable unit gets zeros, lse -inf and no pages,
-    and the other sequences are unaffected."""
-    s = custom_spec(1, num_seqs=3, num_q_heads=8, num_kv_heads=2, budget_pages=2, vocab=512)
-    wl = Workload(s, seed=2, context_lens=[300, 200, 330])
+    and the other sequences are unaffected (one fused kernel, or with more
+    units than SMs the selection kernel and the split-KV attention)."""
+    s = custom_spec(1, num_seqs=num_seqs, num_q_heads=8, num_kv_heads=2, budget_pages=2, vocab=512)
+    wl = Workload(s, seed=2, context_lens=([300, 200, 330] + [150 + 7 * i for i in range(num_seqs - 3)]))
     st = DecodeStep(wl)
     st.summaries()
     torch.cuda.synchronize()
@@ -168,7 +170,8 @@ def test_caller_written_tail_keys_and_query_are_seen():
     assert moved > 0                                   # the new keys changed the selection
 
 
-@pytest.mark.parametrize("num_seqs,heads,budget", [(2, 2, 5), (40, 2, 3)], ids=["clusters", "one-cta-per-unit"])
+@pytest.mark.parametrize("num_seqs,heads,budget", [(2, 2, 5), (40, 2, 3), (100, 2, 4)],
+                         ids=["clusters", "one-cta-per-unit", "selection-kernel"])
 def test_exact_ties_go_to_the_lower_page(num_seqs, heads, budget):
     """Every page of a sequence but the tail is a copy of its first page, so
     their page scores are exactly equal: float32 cannot order them and the
