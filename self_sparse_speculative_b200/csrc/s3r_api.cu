@@ -172,7 +172,8 @@ S3R_EXPORT s3r_status s3r_sparse_draft_attn(const s3r_paged_kv* kv, const void* 
     ps.kmin = kmin;
     ps.kmax = kmax;
     ps.selected_out = selected;
-    s = from_cuda(launch_select_only(*kv, ps, phys, st));
+    uint32_t* work = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + kWsSelWork);
+    s = from_cuda(launch_select_only(*kv, ps, phys, work, st));
   } else {
     s = from_cuda(launch_select(*kv, kmin, kmax, q, budget_pages, selected, phys, status, st));
   }

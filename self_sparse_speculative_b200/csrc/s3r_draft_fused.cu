@@ -11,7 +11,8 @@
 // distributed shared memory) and hands the list back to the others; each CTA
 // attends over its piece of the list and the last to finish merges the
 // pieces by log-sum-exp. Launches with more units than SMs take the selection
-// kernel and the split-KV attention kernel instead.
+// kernel (persistent CTAs claiming units from a workspace counter) and the
+// split-KV attention kernel instead.
 //
 // Selection of a unit (all 256 threads of the CTA):
 //   score(p) = sum_g sum_d max(q_g,d kmin_p,d, q_g,d kmax_p,d) for p < n_b,
@@ -22,7 +23,8 @@
 //   (a unit's rows are 2 D bytes per page, too small for bulk copies to pay);
 //   the tail page's K is bulk-copied into the K/V ring, which is still empty,
 //   while the other pages are scored. Scores are accumulated in float32 with
-//   a rigorous bound E_p on each page's rounding error; a radix select finds
+//   a rigorous bound E_p on each page's rounding error; warp bitonic sorts
+//   and a merge tree keeping the top 32 or 64 (a radix select past that) find
 //   the budget-th largest float32 score s_B. A page with s_p > s_B + 2E (E the
 //   largest bound) is kept for certain, one with s_p < s_B - 2E dropped; the
 //   pages in between are re-scored in float64 and ranked (ties to the lower
@@ -131,7 +133,7 @@ struct SelScratch {
   int k, done, shift, start;
   int wsum[8];
   float wmax[8];
-  float emax[4];               // per cluster rank: the largest score error bound
+  float emax[4];               // per cluster rank: the largest summary magnitude |kmin|, |kmax|
   uint32_t digit, want;
 };
 
@@ -197,37 +199,75 @@ __device__ __forceinline__ float key32_value(uint32_t k) {
   return __uint_as_float((k >> 31) ? (k & 0x7fffffffu) : ~k);
 }
 
-// Rounding bound of a float32 score (u = 2^-24): a product meets one
-// rounding of A or B to float32, at most D/32 in its lane's multiply-add
-// chain, one where the lane's two chains are added and five in the warp's
-// reduction: at most 11 at D = 128 (9 at D = 64), the tail page's score
-// likewise. A sum evaluated so is within gamma_11 = 11 u / (1 - 11 u) of the
-// exact value times the sum of the terms' magnitudes (N. Higham, Accuracy
-// and Stability of Numerical Algorithms, 2002, section 3.1); 16 u covers it
-// and the rounding of the magnitude sum itself.
-constexpr float kScoreGamma = 16.0f * 5.9604644775390625e-8f;
+// Packed helpers: max / min of two bf16 pairs (exact), the pair as two
+// floats (exact), and two independent fused multiply-adds (each rounded once).
+__device__ __forceinline__ uint32_t bmax2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t bmin2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("min.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ unsigned long long bf2_pair(uint32_t u) {
+  unsigned long long d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "r"(u << 16), "r"(u & 0xFFFF0000u));
+  return d;
+}
+__device__ __forceinline__ unsigned long long ffma2(unsigned long long a, unsigned long long b,
+                                                    unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ unsigned long long f2_pair(float lo, float hi) {
+  unsigned long long d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+  return d;
+}
+__device__ __forceinline__ float f2_sum(unsigned long long v) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  return lo + hi;
+}
+
+// Rounding bound of the float32 scores (u = 2^-24). A product A_c x_c meets
+// one rounding of A_c to float32, at most D/64 in its lane's multiply-add
+// chain (channel pairs: even and odd channels accumulate apart), two where
+// the lane's four chains are added and five in the warp's reduction: at most
+// 10 at D = 128 (9 at D = 64), the tail page's score at most 11. A sum
+// evaluated so is within gamma_11 = 11 u / (1 - 11 u) of the exact value
+// times the sum of the terms' magnitudes (N. Higham, Accuracy and Stability
+// of Numerical Algorithms, 2002, section 3.1), and that sum is at most
+// W M with W = sum_c (A_c + |B_c|) and M the largest |kmin|, |kmax| of the
+// unit's pages; 16 u W M covers it (and the roundings of the product).
+constexpr double kScoreGamma = 16.0 * 5.9604644775390625e-8;
 
 // Float32 scores of pages [g0, g1) (none of them the tail page) of KV head
 // h into the 32-bit keys, the summary rows read from global memory (a unit's
 // 2 D bytes of a page are not contiguous with the next page's, so they come
-// as many small pieces; plain loads keep 32 of them in flight per lane).
+// as many small pieces; plain loads keep 2 kU of them in flight per lane).
 // kU pages (16 or 8) per warp and round, each lane holding D / 32 channels
-// of every page; the kU page sums (and their absolute sums for the bound) are
-// reduced across the warp together (halving exchanges: lane l ends with page
-// l % kU). Returns the thread's largest bound.
+// of every page as bf16 pairs: max / min per pair, then packed multiply-adds;
+// the kU page sums are reduced across the warp together (halving exchanges:
+// lane l ends with page l % kU). Returns the largest |kmin|, |kmax| the
+// thread saw (0 if none), for the rounding bound.
 template <int D, int kU>
 __device__ float score_pages(const AttnParams& p, int h, int g0, int g1, int tg, int nthr, const SelSmem& sm,
                              uint32_t* keys32) {
-  constexpr int CPL = D / 32;
+  constexpr int CPL = D / 32, PPL = CPL / 2;              // channels and channel pairs per lane
   using Raw = typename std::conditional<CPL == 4, uint2, uint32_t>::type;
   const int lane = tg & 31, gw = tg >> 5, nw = nthr >> 5;
-  float wa[CPL], wb[CPL];
+  unsigned long long wa[PPL], wb[PPL];
 #pragma unroll
-  for (int c = 0; c < CPL; ++c) {
-    wa[c] = static_cast<float>(sm.ab[lane * CPL + c]);
-    wb[c] = static_cast<float>(sm.ab[D + lane * CPL + c]);
+  for (int c = 0; c < PPL; ++c) {
+    const int ch = lane * CPL + 2 * c;
+    wa[c] = f2_pair(static_cast<float>(sm.ab[ch]), static_cast<float>(sm.ab[ch + 1]));
+    wb[c] = f2_pair(static_cast<float>(sm.ab[D + ch]), static_cast<float>(sm.ab[D + ch + 1]));
   }
-  float emax = 0.f;
+  uint32_t rmax = 0xFF80FF80u, rmin = 0x7F807F80u;         // bf16 pairs (-inf, -inf), (+inf, +inf)
   for (int pg0 = g0 + gw * kU; pg0 < g1; pg0 += nw * kU) {
     Raw lo[kU], hi[kU];
     bool ok[kU];
@@ -242,32 +282,24 @@ __device__ float score_pages(const AttnParams& p, int h, int g0, int g1, int tg,
         hi[u] = __ldg(reinterpret_cast<const Raw*>(static_cast<const __nv_bfloat16*>(p.kmax) + base) + lane);
       }
     }
-    float acc[kU], mag[kU];
+    float acc[kU];
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
-      float s0 = 0.f, s1 = 0.f, e = 0.f;
+      unsigned long long sx = 0ull, sn = 0ull;            // (+0, +0)
       if (ok[u]) {
-        uint32_t lw[CPL / 2], hw[CPL / 2];
+        uint32_t lw[PPL], hw[PPL];
         if constexpr (CPL == 4) { lw[0] = ((uint2&)lo[u]).x; lw[1] = ((uint2&)lo[u]).y; hw[0] = ((uint2&)hi[u]).x; hw[1] = ((uint2&)hi[u]).y; }
         else { lw[0] = (uint32_t&)lo[u]; hw[0] = (uint32_t&)hi[u]; }
 #pragma unroll
-        for (int w = 0; w < CPL / 2; ++w) {
-          float l0, l1, r0, r1;
-          bf2(lw[w], l0, l1);
-          bf2(hw[w], r0, r1);
-          const float x0 = fmaxf(l0, r0), n0 = fminf(l0, r0), x1 = fmaxf(l1, r1), n1 = fminf(l1, r1);
-          s0 = fmaf(wa[2 * w], x0, s0);
-          s1 = fmaf(wb[2 * w], n0, s1);
-          s0 = fmaf(wa[2 * w + 1], x1, s0);
-          s1 = fmaf(wb[2 * w + 1], n1, s1);
-          e = fmaf(fabsf(wa[2 * w]), fabsf(x0), e);
-          e = fmaf(fabsf(wb[2 * w]), fabsf(n0), e);
-          e = fmaf(fabsf(wa[2 * w + 1]), fabsf(x1), e);
-          e = fmaf(fabsf(wb[2 * w + 1]), fabsf(n1), e);
+        for (int w = 0; w < PPL; ++w) {
+          const uint32_t x = bmax2(lw[w], hw[w]), n = bmin2(lw[w], hw[w]);
+          rmax = bmax2(rmax, x);
+          rmin = bmin2(rmin, n);
+          sx = ffma2(wa[w], bf2_pair(x), sx);
+          sn = ffma2(wb[w], bf2_pair(n), sn);
         }
       }
-      acc[u] = s0 + s1;
-      mag[u] = e;
+      acc[u] = f2_sum(sx) + f2_sum(sn);
     }
 #pragma unroll
     for (int w = kU / 2; w >= 1; w >>= 1) {
@@ -277,19 +309,13 @@ __device__ float score_pages(const AttnParams& p, int h, int g0, int g1, int tg,
         const float send = up ? acc[k] : acc[k + w];
         const float keep = up ? acc[k + w] : acc[k];
         acc[k] = keep + __shfl_xor_sync(0xffffffffu, send, w);
-        const float msend = up ? mag[k] : mag[k + w];
-        const float mkeep = up ? mag[k + w] : mag[k];
-        mag[k] = mkeep + __shfl_xor_sync(0xffffffffu, msend, w);
       }
     }
     // lane l now holds page l % kU summed over its kU-lane group; the groups
     // combine (five additions on every path whatever kU)
-    float v = acc[0], m = mag[0];
+    float v = acc[0];
 #pragma unroll
-    for (int o = kU; o < 32; o <<= 1) {
-      v += __shfl_xor_sync(0xffffffffu, v, o);
-      m += __shfl_xor_sync(0xffffffffu, m, o);
-    }
+    for (int o = kU; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     const int pg = pg0 + (lane & (kU - 1));
     if (lane < kU && pg < g1) {
       bool okp = false;
@@ -297,10 +323,14 @@ __device__ float score_pages(const AttnParams& p, int h, int g0, int g1, int tg,
       for (int u = 0; u < kU; ++u) okp = (u == lane) ? ok[u] : okp;
       if (!okp) flag_status(p.status, S3R_DEV_BAD_PAGE_ID);
       keys32[pg] = okp ? order_key32(v) : 0u;
-      if (okp) emax = fmaxf(emax, kScoreGamma * m);
     }
   }
-  return emax;
+  // the largest magnitude: max over channels of max(x, -n) (every |kmin|,
+  // |kmax| is at most that); NaN summaries are passed over as by the maxima
+  float xa, xb, na, nb;
+  bf2(rmax, xa, xb);
+  bf2(rmin, na, nb);
+  return fmaxf(0.f, fmaxf(fmaxf(xa, xb), -fminf(na, nb)));
 }
 
 // Bitonic network over the 32 lanes: descending order (lane 0 the largest).
@@ -349,6 +379,64 @@ __device__ uint32_t top32_kth(const uint32_t* keys, int n, int B, int tg, int ba
     grp_sync(barid, kDfThreads);
   }
   if (gw == 0 && lane == B - 1) xch[0] = v;
+  grp_sync(barid, kDfThreads);
+  const uint32_t k = xch[0];
+  grp_sync(barid, kDfThreads);
+  return k;
+}
+
+// Descending 64-lists held by a warp as two registers: element e is lane
+// e % 32 of register e / 32 (x0 the larger half). half_clean32 sorts a
+// bitonic 32-list (one register) descending.
+__device__ __forceinline__ uint32_t half_clean32(uint32_t v, int lane) {
+#pragma unroll
+  for (int j = 16; j > 0; j >>= 1) {
+    const uint32_t o = __shfl_xor_sync(0xffffffffu, v, j);
+    v = ((lane & j) == 0) ? max(v, o) : min(v, o);
+  }
+  return v;
+}
+// 64 keys (a, b: one per lane each) sorted descending into (x0, x1): two
+// sorted halves, then the bitonic merge of one with the other reversed.
+__device__ __forceinline__ void warp_sort64_desc(uint32_t a, uint32_t b, int lane, uint32_t& x0, uint32_t& x1) {
+  const uint32_t sa = warp_sort_desc(a, lane);
+  const uint32_t sb = __shfl_sync(0xffffffffu, warp_sort_desc(b, lane), 31 - lane);
+  x0 = half_clean32(max(sa, sb), lane);
+  x1 = half_clean32(min(sa, sb), lane);
+}
+// The 64 largest of descending 64-lists X and Y, descending: element e of
+// max(X, Y reversed) is bitonic and holds them (Y reversed: element e is
+// Y[63 - e]); a distance-32 step in the lane, then each half cleaned.
+__device__ __forceinline__ void warp_merge_top64(uint32_t& x0, uint32_t& x1, uint32_t y0, uint32_t y1, int lane) {
+  const uint32_t z0 = max(x0, __shfl_sync(0xffffffffu, y1, 31 - lane));
+  const uint32_t z1 = max(x1, __shfl_sync(0xffffffffu, y0, 31 - lane));
+  x0 = half_clean32(max(z0, z1), lane);
+  x1 = half_clean32(min(z0, z1), lane);
+}
+// The B-th largest (32 < B <= 64) of keys[0..n) by the 256 threads: each
+// warp sorts 64 keys at a time and keeps the top 64 of what it has seen, then
+// a tree of merges across the warps keeps the top 64. xch: 2 KB.
+__device__ uint32_t top64_kth(const uint32_t* keys, int n, int B, int tg, int barid, uint32_t* xch) {
+  const int lane = tg & 31, gw = tg >> 5;
+  uint32_t x0 = 0u, x1 = 0u;
+  for (int base = 0; base < n; base += 2 * kDfThreads) {           // uniform: n is
+    const int i = base + gw * 64 + lane;
+    uint32_t y0, y1;
+    warp_sort64_desc(i < n ? keys[i] : 0u, i + 32 < n ? keys[i + 32] : 0u, lane, y0, y1);
+    if (base == 0) { x0 = y0; x1 = y1; }
+    else warp_merge_top64(x0, x1, y0, y1, lane);
+  }
+#pragma unroll
+  for (int step = 1; step < 8; step <<= 1) {
+    if ((gw & (2 * step - 1)) == step) {
+      xch[(gw - step) * 64 + lane] = x0;
+      xch[(gw - step) * 64 + 32 + lane] = x1;
+    }
+    grp_sync(barid, kDfThreads);
+    if ((gw & (2 * step - 1)) == 0) warp_merge_top64(x0, x1, xch[gw * 64 + lane], xch[gw * 64 + 32 + lane], lane);
+    grp_sync(barid, kDfThreads);
+  }
+  if (gw == 0 && lane == ((B - 1) & 31)) xch[0] = (B - 1) < 32 ? x0 : x1;
   grp_sync(barid, kDfThreads);
   const uint32_t k = xch[0];
   grp_sync(barid, kDfThreads);
@@ -515,7 +603,7 @@ __device__ __forceinline__ int key_rank(const unsigned long long* keys, int n, u
 // KU: pages per warp and scoring round (registers: two summary pieces each).
 template <int D, int KU = 16>
 __device__ void select_unit(const AttnParams& p, const DItem& d, int2* list, const SelSmem& sm, SelScratch& sc,
-                            uint8_t* stage, uint32_t bar_g0, uint32_t bar_g1, bool clustered, volatile int* abort) {
+                            uint8_t* stage, uint32_t bar_g0, uint32_t* g0_phase, bool clustered, volatile int* abort) {
   using Lay = DfLay<D>;
   constexpr int nthr = kDfThreads, barid = kBarAll;
   const int tg = threadIdx.x, lane = tg & 31, gw = tg >> 5;
@@ -542,7 +630,7 @@ __device__ void select_unit(const AttnParams& p, const DItem& d, int2* list, con
   uint32_t* keys32 = reinterpret_cast<uint32_t*>(sm.keys);   // [kDfMaxPages], the array's lower half
   float4* scratch = reinterpret_cast<float4*>(sm.keys + kDfMaxPages / 2);   // its upper half
   bool ok = true;
-  float emax = 0.f;
+  float mmax = 0.f;                                      // the largest summary magnitude seen
   // the tail page's K (when in the share) bulk-copied into the empty ring
   // while the other pages are scored from their summaries
   if (has_tail && tail_ok && tg == 0) {
@@ -551,9 +639,10 @@ __device__ void select_unit(const AttnParams& p, const DItem& d, int2* list, con
     bulk_load(smem_addr(stage), tail_src, bytes, bar_g0);
   }
   const int e = min(s1, tail);                           // the share's pages other than the tail
-  emax = score_pages<D, KU>(p, d.h, s0, e, tg, nthr, sm, keys32);
+  mmax = score_pages<D, KU>(p, d.h, s0, e, tg, nthr, sm, keys32);
   if (has_tail && tail_ok) {
-    ok = grp_all(mbar_wait(bar_g0, 0u, abort, p.status), barid, nthr);
+    ok = grp_all(mbar_wait(bar_g0, *g0_phase, abort, p.status), barid, nthr);
+    *g0_phase ^= 1u;
     if (ok) {
       tail_minmax<D>(reinterpret_cast<const __nv_bfloat16*>(stage), valid, tg, nthr, barid, sm, scratch);
     }
@@ -563,7 +652,7 @@ __device__ void select_unit(const AttnParams& p, const DItem& d, int2* list, con
   // the tail page, scored from its fresh min / max (first warp)
   if (ok && has_tail && gw == 0) {
     constexpr int CPL = D / 32;
-    float a0 = 0.f, a1 = 0.f, e = 0.f;
+    float a0 = 0.f, a1 = 0.f;
     if (tail_ok) {
 #pragma unroll
       for (int c = 0; c < CPL; ++c) {
@@ -572,26 +661,21 @@ __device__ void select_unit(const AttnParams& p, const DItem& d, int2* list, con
         const float wa = static_cast<float>(sm.ab[ch]), wb = static_cast<float>(sm.ab[D + ch]);
         a0 = fmaf(wa, fmaxf(l, r), a0);
         a1 = fmaf(wb, fminf(l, r), a1);
-        e = fmaf(fabsf(wa), fabsf(fmaxf(l, r)), e);
-        e = fmaf(fabsf(wb), fabsf(fminf(l, r)), e);
+        mmax = fmaxf(mmax, fmaxf(fabsf(l), fabsf(r)));
       }
     }
     float v = a0 + a1;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      v += __shfl_xor_sync(0xffffffffu, v, o);
-      e += __shfl_xor_sync(0xffffffffu, e, o);
-    }
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     if (lane == 0) {
       if (!tail_ok) flag_status(p.status, S3R_DEV_BAD_PAGE_ID);
       keys32[tail] = tail_ok ? order_key32(v) : 0u;
-      if (tail_ok) emax = fmaxf(emax, kScoreGamma * e);
     }
   }
-  // the CTA's largest bound
+  // the CTA's largest summary magnitude
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) emax = fmaxf(emax, __shfl_xor_sync(0xffffffffu, emax, o));
-  if (lane == 0) sc.wmax[gw] = emax;
+  for (int o = 16; o > 0; o >>= 1) mmax = fmaxf(mmax, __shfl_xor_sync(0xffffffffu, mmax, o));
+  if (lane == 0) sc.wmax[gw] = mmax;
   grp_sync(barid, nthr);
   if (tg == 0) {
     float m = 0.f;
@@ -616,13 +700,22 @@ __device__ void select_unit(const AttnParams& p, const DItem& d, int2* list, con
   ok = grp_all(ok, barid, nthr);
   if (rank == 0 && ok) {
     const int B = p.budget;
-    float E = 0.f;
-    for (int r = 0; r < parts; ++r) E = fmaxf(E, sc.emax[r]);
+    // the bound: 16 u W M (W = sum_c A_c + |B_c|, exact in float64; M the
+    // largest magnitude over every share), rounded up to float32
+    float M = 0.f;
+    for (int r = 0; r < parts; ++r) M = fmaxf(M, sc.emax[r]);
+    double W = 0.0;
+    for (int c = lane; c < D; c += 32) W += sm.ab[c] - sm.ab[D + c];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) W += __shfl_xor_sync(0xffffffffu, W, o);
+    const float E = __double2float_ru(kScoreGamma * W * static_cast<double>(M));
     // the B-th largest float32 score, and the band in which float32 cannot
     // order pages: |s_p - s_B| <= 2E
     uint32_t kB;
     if (B <= 32) {
       kB = top32_kth(keys32, n_b, B, tg, barid, reinterpret_cast<uint32_t*>(stage));   // the ring is idle
+    } else if (B <= 64) {
+      kB = top64_kth(keys32, n_b, B, tg, barid, reinterpret_cast<uint32_t*>(stage));
     } else if (n_b <= nthr) {
       // one key per thread: its rank among all (ties to the lower page)
       if (tg < n_b && rank32(keys32, n_b, keys32[tg], tg) == B - 1) sc.digit = keys32[tg];
@@ -632,34 +725,50 @@ __device__ void select_unit(const AttnParams& p, const DItem& d, int2* list, con
     } else {
       kB = radix_kth_largest(keys32, n_b, B, tg, nthr, barid, sm.hist, sc);
     }
+    // the band's edges as keys: a float score s has s > hi iff s > RD(hi)
+    // and s >= lo iff s >= RU(lo) (float32 roundings of the float64 edges);
+    // a zero edge takes the key of the zero that makes both zeros compare as
+    // floats do; keys above +inf's are NaN scores (neither kept nor in band)
     const double sB = static_cast<double>(key32_value(kB));
     const double hiB = sB + 2.0 * static_cast<double>(E), loB = sB - 2.0 * static_cast<double>(E);
-    // each thread owns a run of consecutive pages (the list keeps page order)
+    const float hiF = __double2float_rd(hiB), loF = __double2float_ru(loB);
+    const uint32_t kHi = order_key32(hiF == 0.f ? 0.f : hiF), kLo = order_key32(loF == 0.f ? -0.f : loF);
+    constexpr uint32_t kInf = 0xFF800000u;               // order_key32(+inf)
+    // each thread owns a run of consecutive pages (the list keeps page order);
+    // the pages above the band and those in it, counted together
     const int per = (n_b + nthr - 1) / nthr;
     const int q0 = min(n_b, tg * per), q1 = min(n_b, q0 + per);
-    int n_in = 0, n_unc = 0;
+    int n_cnt = 0;
     for (int pg = q0; pg < q1; ++pg) {
-      const double sp = static_cast<double>(key32_value(keys32[pg]));
-      n_in += sp > hiB;
-      n_unc += sp <= hiB && sp >= loB;
+      const uint32_t k = keys32[pg];
+      n_cnt += (k <= kInf && k > kHi) ? 0x10000 : ((k <= kInf && k >= kLo) ? 1 : 0);
     }
-    int tot_in, tot_unc;
-    grp_exclusive_scan(n_in, tg, nthr, barid, sc, &tot_in);
-    const int unc_before = grp_exclusive_scan(n_unc, tg, nthr, barid, sc, &tot_unc);
+    int tot;
+    const int before = grp_exclusive_scan(n_cnt, tg, nthr, barid, sc, &tot);
+    const int tot_in = tot >> 16, tot_unc = tot & 0xffff;
     const int need = B - tot_in;                         // places left for the band's pages
-    // keep flags of the band's pages, one bit per page (the histogram's words)
-    unsigned* keepbits = sm.hist;
-    for (int i = tg; i < 256; i += nthr) keepbits[i] = 0u;
-    grp_sync(barid, nthr);
-    if (tot_unc > need) {
+    if (tot_unc <= need) {
+      // the whole band is kept (the common case): positions from the scan
+      int pos = (before >> 16) + (before & 0xffff);
+      for (int pg = q0; pg < q1; ++pg) {
+        const uint32_t k = keys32[pg];
+        if (k <= kInf && k >= kLo) {
+          if (pos < B) list[pos] = make_int2(pg, sm.phys[pg]);
+          ++pos;
+        }
+      }
+    } else {
       // float64 scores of the band's pages, ranked among themselves (ties to
-      // the lower page); the ring is idle until the list is done
+      // the lower page); the ring is idle until the list is done. Keep flags
+      // one bit per page (the histogram's words).
+      unsigned* keepbits = sm.hist;
+      for (int i = tg; i < 256; i += nthr) keepbits[i] = 0u;
       unsigned long long* ukey = reinterpret_cast<unsigned long long*>(stage);           // [kDfMaxPages]
       int* upage = reinterpret_cast<int*>(stage + 8 * kDfMaxPages);                     // [kDfMaxPages]
-      int j = unc_before;
+      int j = before & 0xffff;
       for (int pg = q0; pg < q1; ++pg) {
-        const double sp = static_cast<double>(key32_value(keys32[pg]));
-        if (sp <= hiB && sp >= loB) upage[j++] = pg;
+        const uint32_t k = keys32[pg];
+        if (k <= kInf && k >= kLo && k <= kHi) upage[j++] = pg;
       }
       grp_sync(barid, nthr);
       for (int u = gw; u < tot_unc; u += nthr / 32) {
@@ -670,22 +779,20 @@ __device__ void select_unit(const AttnParams& p, const DItem& d, int2* list, con
       for (int u = tg; u < tot_unc; u += nthr)
         if (key_rank(ukey, tot_unc, ukey[u], u) < need) atomicOr(&keepbits[upage[u] >> 5], 1u << (upage[u] & 31));
       grp_sync(barid, nthr);
-    }
-    // the list: certain pages and the band's kept ones, in page order
-    int n_keep = 0;
-    for (int pg = q0; pg < q1; ++pg) {
-      const double sp = static_cast<double>(key32_value(keys32[pg]));
-      const bool band = sp <= hiB && sp >= loB;
-      n_keep += sp > hiB || (band && (tot_unc <= need || ((keepbits[pg >> 5] >> (pg & 31)) & 1u)));
-    }
-    int tot_keep;
-    int pos = grp_exclusive_scan(n_keep, tg, nthr, barid, sc, &tot_keep);
-    for (int pg = q0; pg < q1; ++pg) {
-      const double sp = static_cast<double>(key32_value(keys32[pg]));
-      const bool band = sp <= hiB && sp >= loB;
-      if (sp > hiB || (band && (tot_unc <= need || ((keepbits[pg >> 5] >> (pg & 31)) & 1u)))) {
-        if (pos < B) list[pos] = make_int2(pg, sm.phys[pg]);
-        ++pos;
+      // the list: pages above the band and the band's kept ones, in page order
+      int n_keep = 0;
+      for (int pg = q0; pg < q1; ++pg) {
+        const uint32_t k = keys32[pg];
+        n_keep += k <= kInf && (k > kHi || (k >= kLo && ((keepbits[pg >> 5] >> (pg & 31)) & 1u)));
+      }
+      int tot_keep;
+      int pos = grp_exclusive_scan(n_keep, tg, nthr, barid, sc, &tot_keep);
+      for (int pg = q0; pg < q1; ++pg) {
+        const uint32_t k = keys32[pg];
+        if (k <= kInf && (k > kHi || (k >= kLo && ((keepbits[pg >> 5] >> (pg & 31)) & 1u)))) {
+          if (pos < B) list[pos] = make_int2(pg, sm.phys[pg]);
+          ++pos;
+        }
       }
     }
     fence_proxy_async_smem();                            // scratch in the ring before the copies reuse it
@@ -741,7 +848,7 @@ draft_fused_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
   constexpr int N = kDfN, NR = kDfNR, NS = L::kNS;
   extern __shared__ __align__(1024) uint8_t dyn_raw[];
   uint8_t* dyn = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ __align__(8) uint64_t s_bar[2 * NS + 10];
+  __shared__ __align__(8) uint64_t s_bar[2 * NS + 9];
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   __shared__ int s_ticket;
@@ -763,7 +870,7 @@ draft_fused_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
   const uint32_t bar0 = smem_addr(&s_bar[0]);
   auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
   const int B_FULL = 0, B_EMPTY = NS, B_SFULL = 2 * NS, B_PFULL = 2 * NS + 2, B_ODONE = 2 * NS + 4,
-            B_QFULL = 2 * NS + 6, B_TD = 2 * NS + 7, B_G0 = 2 * NS + 8, B_G1 = 2 * NS + 9;
+            B_QFULL = 2 * NS + 6, B_TD = 2 * NS + 7, B_G0 = 2 * NS + 8;
   constexpr int PB = L::kPBufs;
   uint8_t* sQ = dyn;
   uint8_t* sP = dyn + L::kOffP;
@@ -792,7 +899,6 @@ draft_fused_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
     mbar_init(BAR(B_QFULL), 128);
     mbar_init(BAR(B_TD), 1);
     mbar_init(BAR(B_G0), 1);
-    mbar_init(BAR(B_G1), 1);
     s_abort = 0;
     fence_barrier_init();
   }
@@ -829,7 +935,8 @@ draft_fused_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
   // before the grid-dependency wait; every role takes the wait before it
   // touches an output or the workspace (the producer after its first NS
   // stages)
-  select_unit<D>(p, d0, s_list, sm, s_sc, sKV, BAR(B_G0), BAR(B_G1), clustered, &s_abort);
+  uint32_t g0_phase = 0;
+  select_unit<D>(p, d0, s_list, sm, s_sc, sKV, BAR(B_G0), &g0_phase, clustered, &s_abort);
   __syncthreads();
 
   if (warp == kDfProducer) {
@@ -1189,11 +1296,16 @@ draft_fused_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
 }
 
 // Page selection alone, for launches with more (sequence, KV head) units
-// than SMs: one CTA per unit runs the fused kernel's selection (scoring
-// before the grid-dependency wait), then writes the kept pages' logical ids
-// to selected_out and their physical ids to `phys_out` ([S, Hkv, budget], in
-// the workspace) for the split-KV attention kernel. Small shared memory, so
-// several CTAs share an SM and their summary loads overlap.
+// than SMs: persistent CTAs run the fused kernel's selection one unit after
+// another, then write the kept pages' logical ids to selected_out and their
+// physical ids to `phys_out` ([S, Hkv, budget], in the workspace) for the
+// split-KV attention kernel. Small shared memory, so several CTAs share an
+// SM and their summary loads overlap. CTA c takes unit c first (scored before
+// the grid-dependency wait), then claims units from the workspace counter
+// work[0] (after the wait: the previous call's selection resets it as it
+// ends); the last CTA to finish (work[1]) returns both counters to zero, so
+// ragged units (contexts of different lengths) balance over the CTAs instead
+// of leaving a second wave.
 template <int D>
 struct SelOnlyLay {
   // the tail page's K, then the band scratch (float64 keys and pages)
@@ -1208,14 +1320,17 @@ struct SelOnlyLay {
   static constexpr uint32_t kDynBytes = kOffHist + 4 * 256;
   static_assert(kStage >= 12 * kDfMaxPages, "band scratch fits in the tail stage");
 };
+constexpr int kSelOnlyCtasPerSm = 3;
 
 template <int D>
-__global__ void __launch_bounds__(kDfThreads, 3) select_only_kernel(const AttnParams p, int32_t* phys_out) {
+__global__ void __launch_bounds__(kDfThreads, kSelOnlyCtasPerSm)
+    select_only_kernel(const AttnParams p, int32_t* phys_out, uint32_t* work) {
   using Lay = SelOnlyLay<D>;
   extern __shared__ __align__(1024) uint8_t dyn_raw[];
   uint8_t* dyn = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ __align__(8) uint64_t s_bar[2];
+  __shared__ __align__(8) uint64_t s_bar[1];
   __shared__ int s_abort;
+  __shared__ int s_unit;
   __shared__ SelScratch s_sc;
   const int tid = threadIdx.x;
   SelSmem sm;
@@ -1227,25 +1342,44 @@ __global__ void __launch_bounds__(kDfThreads, 3) select_only_kernel(const AttnPa
   int2* s_list = reinterpret_cast<int2*>(dyn + Lay::kOffList);
   if (tid == 0) {
     mbar_init(smem_addr(&s_bar[0]), 1);
-    mbar_init(smem_addr(&s_bar[1]), 1);
     s_abort = 0;
     fence_barrier_init();
   }
-  const DItem d0 = draft_item(p, blockIdx.x);              // p.parts == 1: one unit per CTA
-  sel_prepare<D>(p, d0, tid, kDfThreads, sm);
-  __syncthreads();
-  select_unit<D, 8>(p, d0, s_list, sm, s_sc, dyn, smem_addr(&s_bar[0]), smem_addr(&s_bar[1]), false, &s_abort);
-  __syncthreads();
-  pdl_wait();                                              // outputs and the workspace from here on
-  const size_t o = ((size_t)d0.b * p.Hkv + d0.h) * p.budget;
-  for (int k = tid; k < p.budget; k += kDfThreads) {
-    const int2 e = s_list[k];
-    p.selected_out[o + k] = e.x;
-    phys_out[o + k] = e.y;
+  const int units = p.S * p.Hkv;
+  uint32_t g0_phase = 0;
+  bool waited = false;
+  for (int u = blockIdx.x; u < units;) {
+    const DItem d = draft_item(p, u);                      // p.parts == 1: item = unit
+    sel_prepare<D>(p, d, tid, kDfThreads, sm);
+    __syncthreads();
+    select_unit<D, 8>(p, d, s_list, sm, s_sc, dyn, smem_addr(&s_bar[0]), &g0_phase, false, &s_abort);
+    __syncthreads();
+    if (!waited) {
+      pdl_wait();                                          // outputs and the workspace from here on
+      waited = true;
+    }
+    const size_t o = ((size_t)d.b * p.Hkv + d.h) * p.budget;
+    for (int k = tid; k < p.budget; k += kDfThreads) {
+      const int2 e = s_list[k];
+      p.selected_out[o + k] = e.x;
+      phys_out[o + k] = e.y;
+    }
+    // after a timed-out wait the tail stage may still be filling: claim no more
+    if (tid == 0) s_unit = s_abort ? units : (int)(gridDim.x + atomicAdd(work, 1u));
+    __syncthreads();                                       // s_unit; s_list and the stage are free again
+    u = s_unit;
+  }
+  if (!waited) pdl_wait();
+  if (tid == 0) {
+    __threadfence();
+    if (atomicAdd(work + 1, 1u) == gridDim.x - 1) {        // every CTA has claimed its last unit
+      atomicExch(work, 0u);
+      atomicExch(work + 1, 0u);
+    }
   }
   // the attention kernel (persistent, a whole SM per CTA) may launch only
-  // once every selection CTA is done: earlier, it would take SMs from the
-  // selection's later waves
+  // once every selection CTA is done: earlier, it would take SMs the
+  // selection still needs
   pdl_launch_dependents();
 }
 
@@ -1316,19 +1450,31 @@ bool select_only_supported(const s3r_paged_kv& kv, int32_t budget_pages) {
 
 template <int D>
 static cudaError_t launch_select_only_d(const s3r_paged_kv& kv, const AttnParams& p, int32_t* phys_out,
-                                       cudaStream_t st) {
+                                       uint32_t* work, cudaStream_t st) {
   const size_t smem = SelOnlyLay<D>::kDynBytes + 1024;
   cudaError_t e = cudaFuncSetAttribute(select_only_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  // resident CTAs (once per process and head size; the kernel's resources do
+  // not change)
+  static int per_sm = 0;
+  if (per_sm == 0) {
+    int n = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, select_only_kernel<D>, kDfThreads, smem);
+    if (e != cudaSuccess) return e;
+    per_sm = n < 1 ? 1 : n;
+  }
+  const int units = kv.num_seqs * kv.num_kv_heads;
+  int grid = device_sm_count() * per_sm;
+  if (grid > units) grid = units;
   AttnParams q = p;
   q.parts = 1;
-  return launch_kernel(select_only_kernel<D>, dim3(kv.num_seqs * kv.num_kv_heads), dim3(kDfThreads), smem, st, 1, q,
-                       phys_out);
+  return launch_kernel(select_only_kernel<D>, dim3(grid), dim3(kDfThreads), smem, st, 1, q, phys_out, work);
 }
 
-cudaError_t launch_select_only(const s3r_paged_kv& kv, const AttnParams& p, int32_t* phys_out, cudaStream_t st) {
-  return kv.head_dim == 64 ? launch_select_only_d<64>(kv, p, phys_out, st)
-                           : launch_select_only_d<128>(kv, p, phys_out, st);
+cudaError_t launch_select_only(const s3r_paged_kv& kv, const AttnParams& p, int32_t* phys_out, uint32_t* work,
+                               cudaStream_t st) {
+  return kv.head_dim == 64 ? launch_select_only_d<64>(kv, p, phys_out, work, st)
+                           : launch_select_only_d<128>(kv, p, phys_out, work, st);
 }
 
 cudaError_t launch_draft_fused(const s3r_paged_kv& kv, const DraftLaunch& dl, const AttnParams& p, cudaStream_t st) {

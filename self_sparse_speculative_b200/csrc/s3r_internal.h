@@ -27,8 +27,11 @@ constexpr int kMaxSeqs = 1024;
 constexpr int kMaxPersistentCtas = 160;
 constexpr int kMaxTreeNodes = 64;         // tree verification: nodes per sequence (one 64-bit mask)
 
-// Workspace header: word 0 is the device status word; the rest is reserved.
+// Workspace header: word 0 is the device status word; words 32 and 33 are
+// the two-kernel sparse draft's selection counters (next unit, CTAs done);
+// the rest is reserved.
 constexpr size_t kWsHeader = 256;
+constexpr size_t kWsSelWork = 128;        // byte offset of the selection counters
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -122,11 +125,13 @@ struct DraftLaunch {
 };
 cudaError_t prepare_draft_fused(const s3r_paged_kv& kv, int32_t budget_pages, DraftLaunch* dl);
 cudaError_t launch_draft_fused(const s3r_paged_kv& kv, const DraftLaunch& dl, const AttnParams& p, cudaStream_t st);
-// Selection alone (the fused kernel's selection, one CTA per unit) for the
-// two-kernel sparse draft: kept pages to p.selected_out, their physical ids
-// to phys_out ([S, Hkv, budget]).
+// Selection alone (the fused kernel's selection, persistent CTAs taking units
+// from the counters `work` [2] of the workspace header) for the two-kernel
+// sparse draft: kept pages to p.selected_out, their physical ids to phys_out
+// ([S, Hkv, budget]).
 bool select_only_supported(const s3r_paged_kv& kv, int32_t budget_pages);
-cudaError_t launch_select_only(const s3r_paged_kv& kv, const AttnParams& p, int32_t* phys_out, cudaStream_t st);
+cudaError_t launch_select_only(const s3r_paged_kv& kv, const AttnParams& p, int32_t* phys_out, uint32_t* work,
+                               cudaStream_t st);
 bool make_cache_map(CUtensorMap* map, const void* base, const s3r_paged_kv& kv);
 int device_sm_count();
 

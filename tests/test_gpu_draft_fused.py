@@ -1,10 +1,11 @@
 """The sparse draft call against the float64 oracle, on shapes that reach each
 path of the fused kernel (page scoring, top-B and attention in one launch):
-units cut into pieces over clusters of two and four CTAs, a sequence whose
-page summaries take several staging chunks, pieces that keep no page, bad
+units cut into pieces over clusters of two and four CTAs, budgets on both
+sides of 32 pages, pieces that keep no page, bad
 lengths and page ids, and queries and tail-page keys written by the caller's
-own kernels right before the call; plus a launch with more units than SMs,
-which takes the selection kernel and the split-KV attention kernel. Every GPU
+own kernels right before the call; plus launches with more units than SMs,
+which take the selection kernel (persistent CTAs claiming units from a
+workspace counter) and the split-KV attention kernel. Every GPU
 result comes from the C ABI (libs3r.so)."""
 import numpy as np
 import pytest
@@ -34,13 +35,23 @@ CASES = {
     # attention kernel; 16-token pages (eight pages per stage)
     "many-units-p16": (custom_spec(1, num_seqs=200, num_q_heads=8, num_kv_heads=2, page_size=16, gamma=2,
                                    budget_pages=5, vocab=512), _ragged(200, 40, 700, 1)),
-    # one unit: cut into four pieces; 800 pages of summaries pass through the
-    # ring in three chunks (352 pages per chunk at D = 128)
+    # one unit: cut into four pieces of 200 pages each
     "long-chunks": (custom_spec(1, num_seqs=1, num_q_heads=4, num_kv_heads=1, page_size=16, gamma=1,
                                 budget_pages=9, vocab=512), [800 * 16 - 5]),
     # split units whose kept-page list is shorter than the number of pieces
     "empty-pieces": (custom_spec(1, num_seqs=2, num_q_heads=8, num_kv_heads=2, page_size=64, gamma=1,
                                  budget_pages=4, vocab=512), [100, 64 * 9 + 3]),
+    # budgets between 32 and 64 pages (the 64-key bitonic selection): units
+    # cut into four pieces with up to ~940 pages each, some below the budget
+    "top64-clusters": (custom_spec(1, num_seqs=3, num_q_heads=8, num_kv_heads=4, page_size=16, gamma=1,
+                                   budget_pages=48, vocab=512), [1000, 9000, 15000]),
+    # the same budgets through the selection kernel (160 units)
+    "top64-selection-kernel": (custom_spec(1, num_seqs=80, num_q_heads=4, num_kv_heads=2, page_size=16, gamma=1,
+                                           budget_pages=64, vocab=512), _ragged(80, 700, 9000, 3)),
+    # 640 units, more than the selection kernel's resident CTAs: CTAs claim
+    # further units from the workspace counter (ragged lengths)
+    "selection-claims": (custom_spec(1, num_seqs=320, num_q_heads=4, num_kv_heads=2, page_size=16, gamma=2,
+                                     budget_pages=6, vocab=512), _ragged(320, 50, 3000, 5)),
     # D = 64, G = 8: 60 units, each cut into two pieces (clusters of two CTAs)
     "d64-g8-pairs": (custom_spec(1, num_seqs=30, num_q_heads=16, num_kv_heads=2, head_dim=64, page_size=64,
                                  gamma=1, budget_pages=3, vocab=512), _ragged(30, 130, 2000, 2)),
