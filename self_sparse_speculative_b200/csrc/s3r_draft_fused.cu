@@ -167,13 +167,13 @@ __device__ int grp_exclusive_scan(int v, int tg, int nthr, int barid, SelScratch
 
 // Inputs of a unit's selection that no kernel of the library writes (so they
 // may be read before the grid-dependency wait): the physical ids of its pages
-// and the folded query weights of its KV head.
+// and the folded query weights of its KV head. The whole block-table row and
+// the query are loaded whatever the length, so these loads do not wait for
+// the context length's (entries past the last page are never used).
 template <int D>
 __device__ void sel_prepare(const AttnParams& p, const DItem& d, int tg, int nthr, const SelSmem& sm) {
-  if (d.bad) return;
   const int32_t* bt = p.block_table + (size_t)d.b * p.max_pages;
-  for (int i = tg; i < d.n_b; i += nthr) sm.phys[i] = __ldg(bt + i);
-  if (d.n_b <= p.budget) return;
+  for (int i = tg; i < p.max_pages; i += nthr) sm.phys[i] = __ldg(bt + i);
   const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(p.q) + ((size_t)d.b * p.Hq + (size_t)d.h * p.G) * D;
   for (int c = tg; c < D; c += nthr) {
     float v[8];
@@ -1300,12 +1300,13 @@ draft_fused_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constan
 // another, then write the kept pages' logical ids to selected_out and their
 // physical ids to `phys_out` ([S, Hkv, budget], in the workspace) for the
 // split-KV attention kernel. Small shared memory, so several CTAs share an
-// SM and their summary loads overlap. CTA c takes unit c first (scored before
-// the grid-dependency wait), then claims units from the workspace counter
+// SM and their summary loads overlap. Units are taken longest sequence first
+// (every CTA ranks the context lengths, ties to the lower sequence, when
+// there are at most kSelOrderMax sequences of unequal lengths), so the last
+// claims are short units: CTA c takes position c first (scored before the
+// grid-dependency wait), then claims positions from the workspace counter
 // work[0] (after the wait: the previous call's selection resets it as it
-// ends); the last CTA to finish (work[1]) returns both counters to zero, so
-// ragged units (contexts of different lengths) balance over the CTAs instead
-// of leaving a second wave.
+// ends); the last CTA to finish (work[1]) returns both counters to zero.
 template <int D>
 struct SelOnlyLay {
   // the tail page's K, then the band scratch (float64 keys and pages)
@@ -1321,6 +1322,7 @@ struct SelOnlyLay {
   static_assert(kStage >= 12 * kDfMaxPages, "band scratch fits in the tail stage");
 };
 constexpr int kSelOnlyCtasPerSm = 3;
+constexpr int kSelOrderMax = 256;
 
 template <int D>
 __global__ void __launch_bounds__(kDfThreads, kSelOnlyCtasPerSm)
@@ -1332,6 +1334,8 @@ __global__ void __launch_bounds__(kDfThreads, kSelOnlyCtasPerSm)
   __shared__ int s_abort;
   __shared__ int s_unit;
   __shared__ SelScratch s_sc;
+  __shared__ int s_len[kSelOrderMax];
+  __shared__ int s_order[kSelOrderMax];                   // sequences, longest first
   const int tid = threadIdx.x;
   SelSmem sm;
   sm.keys = reinterpret_cast<unsigned long long*>(dyn + Lay::kOffKeys);
@@ -1346,10 +1350,33 @@ __global__ void __launch_bounds__(kDfThreads, kSelOnlyCtasPerSm)
     fence_barrier_init();
   }
   const int units = p.S * p.Hkv;
+  bool lpt = p.S <= kSelOrderMax;
+  if (lpt) {
+    int differs = 0;
+    for (int b = tid; b < p.S; b += kDfThreads) {
+      s_len[b] = __ldg(p.context_lens + b);
+      differs |= s_len[b] != __ldg(p.context_lens);
+    }
+    lpt = __syncthreads_or(differs) != 0;                  // equal lengths: index order is as good
+  }
+  if (lpt) {
+    for (int b = tid; b < p.S; b += kDfThreads) {
+      const int L = s_len[b];
+      int r = 0;
+      for (int c = 0; c < p.S; ++c) r += s_len[c] > L || (s_len[c] == L && c < b);
+      s_order[r] = b;
+    }
+    __syncthreads();
+  }
+  auto unit_at = [&](int k) {                              // claim position -> unit
+    if (!lpt) return k;
+    const int i = k / p.Hkv;
+    return s_order[i] * p.Hkv + (k - i * p.Hkv);
+  };
   uint32_t g0_phase = 0;
   bool waited = false;
-  for (int u = blockIdx.x; u < units;) {
-    const DItem d = draft_item(p, u);                      // p.parts == 1: item = unit
+  for (int k = blockIdx.x; k < units;) {
+    const DItem d = draft_item(p, unit_at(k));             // p.parts == 1: item = unit
     sel_prepare<D>(p, d, tid, kDfThreads, sm);
     __syncthreads();
     select_unit<D, 8>(p, d, s_list, sm, s_sc, dyn, smem_addr(&s_bar[0]), &g0_phase, false, &s_abort);
@@ -1367,7 +1394,7 @@ __global__ void __launch_bounds__(kDfThreads, kSelOnlyCtasPerSm)
     // after a timed-out wait the tail stage may still be filling: claim no more
     if (tid == 0) s_unit = s_abort ? units : (int)(gridDim.x + atomicAdd(work, 1u));
     __syncthreads();                                       // s_unit; s_list and the stage are free again
-    u = s_unit;
+    k = s_unit;
   }
   if (!waited) pdl_wait();
   if (tid == 0) {
@@ -1377,9 +1404,8 @@ __global__ void __launch_bounds__(kDfThreads, kSelOnlyCtasPerSm)
       atomicExch(work + 1, 0u);
     }
   }
-  // the attention kernel (persistent, a whole SM per CTA) may launch only
-  // once every selection CTA is done: earlier, it would take SMs the
-  // selection still needs
+  // the attention kernel is released only now: released at the start, it
+  // measured slower with many units per CTA (2048 units: 9 us per call)
   pdl_launch_dependents();
 }
 
