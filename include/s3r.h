@@ -34,9 +34,9 @@
  *   launch). After a call that reported S3R_DEV_WAIT_TIMEOUT, zero the
  *   workspace again before reusing it.
  * - A call may read its inputs (queries, KV cache, page summaries, block
- *   table, context lengths) while the previous kernel on the stream is still
- *   finishing, when that kernel is one of this library's attention or
- *   sampling kernels (none of them writes another call's inputs;
+ *   table, context lengths, logits) while the previous kernel on the stream
+ *   is still finishing, when that kernel is one of this library's attention
+ *   or sampling kernels (none of them writes another call's inputs;
  *   s3r_page_summaries, s3r_kv_append and s3r_kv_rollback, which do, let the
  *   next kernel start only when they are done). A kernel of the caller's
  *   that writes an input must not signal programmatic launch completion

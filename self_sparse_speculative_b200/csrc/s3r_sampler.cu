@@ -26,6 +26,11 @@
 // The drafter's own draws (s3r_sample_tokens) are pass 2b alone in "plain"
 // mode: one row per draw, weights exp((x - m_c)/T) with m_c the chunk's own
 // maximum, brought to the row maximum when the chunks are merged.
+// Dependent launches: every kernel releases the next one at its start; pass 1
+// and plain draws read their logits (inputs) before the grid-dependency wait,
+// so they work while the previous kernel finishes (the wait comes before
+// their first workspace write). Released only once every CTA had done its
+// chunk instead, the step measured slower on every workload.
 #include <cuda_bf16.h>
 
 #include <climits>
@@ -200,7 +205,6 @@ __device__ void decide(const SampleParams& p, int b) {
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(kSmpThreads, kStatsCtasPerSm) rowstats_kernel(const SampleParams p) {
   pdl_launch_dependents();
-  pdl_wait();
   __shared__ float s_redf[kSmpWarps];
   __shared__ double s_redd[kSmpWarps];
   __shared__ int s_last;
@@ -255,6 +259,8 @@ __global__ void __launch_bounds__(kSmpThreads, kStatsCtasPerSm) rowstats_kernel(
   const float M = block_max(m, s_redf);
   const double sc = m == -INFINITY ? 0.0 : s * static_cast<double>(ex2((m - M) * k2));
   const double S = block_sum_d(sc, s_redd);
+  // the logits are inputs: only the workspace waits for the previous kernel
+  pdl_wait();
   if (tid == 0) {
     Part1* part = static_cast<Part1*>(p.part1) + (size_t)row * p.c1 + c;
     part->m = M;
@@ -646,7 +652,9 @@ __device__ int block_find(const DrawRows& w, int b0, int b1, double base, double
 template <typename T, bool SPEC, bool STAGE>
 __global__ void __launch_bounds__(kSmpThreads, kDrawCtasPerSm) draw_kernel(const SampleParams p) {
   pdl_launch_dependents();
-  pdl_wait();
+  // speculative draws start from the earlier passes' results; plain draws
+  // read only inputs (the logits) until their first workspace write
+  if constexpr (SPEC) pdl_wait();
   extern __shared__ __align__(16) uint8_t s_dyn[];
   __shared__ uint64_t s_bar;
   __shared__ int s_abort;
@@ -678,6 +686,7 @@ __global__ void __launch_bounds__(kSmpThreads, kDrawCtasPerSm) draw_kernel(const
   const int seg = p.ch2 / kWarpSegs;                     // elements per warp segment
   const int sb0 = min(n, warp * seg), sb1 = min(n, sb0 + seg);
   float* cmax = p.cmax + (size_t)s * p.c2;
+  float Mc = -INFINITY;
   if constexpr (!SPEC) {
     float mx = -INFINITY;
     for (int i = sb0 + lane * PV; i < sb1; i += 32 * PV) {
@@ -688,9 +697,8 @@ __global__ void __launch_bounds__(kSmpThreads, kDrawCtasPerSm) draw_kernel(const
       for (int t = 0; t < PV; ++t)
         if (t < m) mx = fmaxf(mx, v[t]);
     }
-    const float M = block_max(mx, s_redf);               // synchronises (orders the exp table too)
-    w.Mp = M == -INFINITY ? 0.0 : static_cast<double>(M);
-    if (tid == 0) cmax[c] = M;
+    Mc = block_max(mx, s_redf);                          // synchronises (orders the exp table too)
+    w.Mp = Mc == -INFINITY ? 0.0 : static_cast<double>(Mc);
   } else {
     __syncthreads();
   }
@@ -702,6 +710,10 @@ __global__ void __launch_bounds__(kSmpThreads, kDrawCtasPerSm) draw_kernel(const
     for (int t = 0; t < PV; ++t) acc += wv[t];
   }
   acc = warp_sum_d(acc);
+  if constexpr (!SPEC) {
+    pdl_wait();                                          // outputs and the workspace from here on
+    if (tid == 0) cmax[c] = Mc;
+  }
   if (lane == 0) {
     p.wpart[((size_t)s * p.c2 + c) * kWarpSegs + warp] = acc;
     __threadfence();
