@@ -221,3 +221,61 @@ def test_exact_ties_go_to_the_lower_page(num_seqs, heads, budget):
             ties += int(1 in sel[b][h])
         RR.assert_close(f"seq {b} out", gout[b], out[b], "bf16")
     assert ties > 0                                    # the tie rule decided
+
+
+@pytest.mark.parametrize("num_seqs,heads,budget", [(2, 2, 5), (40, 2, 3), (100, 2, 4)],
+                         ids=["clusters", "one-cta-per-unit", "selection-kernel"])
+def test_near_ties_inside_the_float32_band_follow_float64(num_seqs, heads, budget):
+    """Pages that float32 cannot order but float64 can: every page but the
+    tail copies the first page, then page j raises the largest key of one
+    channel by j bf16 ulps, and every query head weighs that channel by 2^-16.
+    The page scores then differ by ~1e-9 of their size: well inside the
+    float32 rounding band (so the float64 re-scoring decides) and far above
+    the comparison's near-tie threshold (1e-12), so the kept pages must be
+    exactly the oracle's: the highest raises (and the tail page when it
+    scores higher)."""
+    s = custom_spec(1, num_seqs=num_seqs, num_q_heads=4 * heads, num_kv_heads=heads, page_size=64, gamma=1,
+                    budget_pages=budget, vocab=512)
+    lens = _ragged(num_seqs, 64 * 6, 64 * 20, 9)
+    wl = Workload(s, seed=13, context_lens=lens)
+    st = DecodeStep(wl)
+    c0 = 5                                            # the raised channel
+    K = wl.kv_cache("K").copy()                       # bf16 bit patterns [pages, H, P, D]
+    V = wl.kv_cache("V")
+    bt = wl.block_table.astype(np.int64)
+    Kf = to_float64(K, "bf16")
+    for b in range(num_seqs):
+        n = int(wl.pages_per_seq[b])
+        p0 = bt[b, 0]
+        for j in range(1, n - 1):
+            K[bt[b, j]] = K[p0]
+            for h in range(heads):
+                t = int(np.argmax(Kf[p0, h, :, c0]))
+                x = int(K[p0, h, t, c0])
+                assert x < 0x8000                      # a positive largest key: its bits grow with it
+                K[bt[b, j], h, t, c0] = np.uint16(x + j)
+    q = wl.q_draft[0].copy()                          # [S, Hq, D] bf16 bits
+    q[:, :, c0] = np.uint16(0x3780)                   # 2^-16
+    st.k_cache.copy_(torch.from_numpy(K.view(np.int16)).view(torch.bfloat16).cuda())
+    st.q_draft[0].copy_(torch.from_numpy(q.view(np.int16)).view(torch.bfloat16).cuda())
+    st.summaries(tail_only=False)
+    st.draft(0)
+    torch.cuda.synchronize()
+    assert s3r.s3r_device_status(st.ws_draft) == (s3r.S3R_OK, 0)
+    K64, V64 = to_float64(K, "bf16"), to_float64(V, "bf16")
+    q64 = to_float64(q, "bf16")
+    cl = np.asarray(lens)
+    kmin, kmax = O.page_summaries(K64, bt, cl, s.page_size)
+    sel, gaps = O.sparse_draft_select(q64, kmin, kmax, bt, cl, s.page_size, budget, s.group)
+    out, lse = O.sparse_draft_attn(q64, K64, V64, bt, cl, sel, RR.f32(wl.scale))
+    gsel = st.selected[0].cpu().numpy()
+    gout = st.draft_out[0].float().cpu().numpy()
+    decided = 0
+    for b in range(num_seqs):
+        n = int(wl.pages_per_seq[b])
+        for h in range(heads):
+            assert gaps[b][h] > RR.NEAR_TIE_SCORE      # not a near-tie: an exact comparison
+            assert gsel[b, h].tolist() == list(sel[b][h]), (b, h, gsel[b, h].tolist(), list(sel[b][h]))
+            decided += int(n > budget and (n - 2) in set(int(x) for x in sel[b][h]))
+        RR.assert_close(f"seq {b} out", gout[b], out[b], "bf16")
+    assert decided > 0                                # the raises decided
