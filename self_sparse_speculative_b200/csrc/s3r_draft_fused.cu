@@ -22,15 +22,15 @@
 //   while the sequence decodes). The summary rows are read from global memory
 //   (a unit's rows are 2 D bytes per page, too small for bulk copies to pay);
 //   the tail page's K is bulk-copied into the K/V ring, which is still empty,
-//   while the other pages are scored. Scores are accumulated in float32 with
-//   a rigorous bound E_p on each page's rounding error; warp bitonic sorts
-//   and a merge tree keeping the top 32 or 64 (a radix select past that) find
-//   the budget-th largest float32 score s_B. A page with s_p > s_B + 2E (E the
-//   largest bound) is kept for certain, one with s_p < s_B - 2E dropped; the
-//   pages in between are re-scored in float64 and ranked (ties to the lower
-//   page) only when they outnumber the places left, so the kept set is the
-//   float64 top-B. It goes, in ascending page order, into a list in shared
-//   memory.
+//   while the other pages are scored. Scores are accumulated in float32
+//   (packed bf16x2 max / min, f32x2 multiply-adds) with one rigorous bound E
+//   on the rounding error of every score of the unit; warp bitonic sorts and a
+//   merge tree keeping the top 32 or 64 (a radix select past that) find the
+//   budget-th largest float32 score s_B. A page with s_p > s_B + 2E is kept
+//   for certain, one with s_p < s_B - 2E dropped; the pages in between are
+//   re-scored in float64 and ranked (ties to the lower page) only when they
+//   outnumber the places left, so the kept set is the float64 top-B. It goes,
+//   in ascending page order, into a list in shared memory.
 //
 // Attention over the kept pages is the token-major pipeline of s3r_attn_tok.cu
 // (S^T = K Q^T and O^T += V^T P^T per 128-token stage, fp32 in TMEM):
