@@ -28,7 +28,8 @@
 // warp 4 producer (page ids, TMA into an NS-stage ring; an L2 prefetch ahead
 // of the ring measured slower); warp 5 MMA issuer and TMEM owner: it polls its
 // barriers and issues whichever MMA is ready (PV(k) once P(k) is written,
-// QK(k) once stage k has landed and PV(k - 2) is issued). Two P buffers where
+// QK(k) once stage k's K has landed and PV(k - 2) is issued; K and V land on
+// separate barriers, so V's transfer overlaps QK(k) and softmax(k)). Two P buffers where
 // they fit, so softmax(k) waits only for PV(k - 2). The softmax warps also
 // stage each segment's Q (fetched into registers one segment ahead).
 #include <cuda_bf16.h>
@@ -60,7 +61,7 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
   constexpr int NS = L::kNS;
   extern __shared__ __align__(1024) uint8_t dyn_raw[];
   uint8_t* dyn = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ __align__(8) uint64_t s_bar[2 * NS + 8];
+  __shared__ __align__(8) uint64_t s_bar[3 * NS + 8];
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   __shared__ int s_ticket;
@@ -134,8 +135,9 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
   // barrier could complete two phases before the MMA thread tests the first;
   // with one barrier per parity, P(g + 2) waits for PV(g) and no barrier gets
   // two phases ahead of its waiter.
+  // FULL[st]: the stage's K landed (and its page ids written); FULLV[st]: its V
   const int B_FULL = 0, B_EMPTY = NS, B_SFULL = 2 * NS, B_PFULL = 2 * NS + 2, B_ODONE = 2 * NS + 4,
-            B_QFULL = 2 * NS + 6, B_TD = 2 * NS + 7;
+            B_QFULL = 2 * NS + 6, B_TD = 2 * NS + 7, B_FULLV = 2 * NS + 8;
   constexpr int PB = L::kPBufs;
   uint8_t* sQ = dyn;
   uint8_t* sP = dyn + L::kOffP;
@@ -147,7 +149,11 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
     tmem_relinquish();
   }
   if (tid == 0) {
-    for (int i = 0; i < NS; ++i) { mbar_init(BAR(B_FULL + i), 1); mbar_init(BAR(B_EMPTY + i), 1); }
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(BAR(B_FULL + i), 1);
+      mbar_init(BAR(B_FULLV + i), 1);
+      mbar_init(BAR(B_EMPTY + i), 1);
+    }
     mbar_init(BAR(B_SFULL), 1);
     mbar_init(BAR(B_SFULL + 1), 1);
     mbar_init(BAR(B_PFULL), 128);
@@ -231,18 +237,23 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         if (lane < 8) s_stage_lp[st][lane] = (lane < ppt && my_ph >= 0) ? my_lp : -1;
         const unsigned real = __ballot_sync(0xffffffffu, my_ph >= 0);
         __syncwarp();
-        if (lane == 0)
-          mbar_arrive_expect_tx(BAR(B_FULL + st), (uint32_t)__popc(real) * L::kHalves * 2u * (uint32_t)p.P * 128u);
+        if (lane == 0) {
+          // K and V land on separate barriers: QK(g) needs only K, so V's
+          // transfer is no longer between the stage's arrival and its QK
+          const uint32_t half = (uint32_t)__popc(real) * L::kHalves * (uint32_t)p.P * 128u;
+          mbar_arrive_expect_tx(BAR(B_FULL + st), half);
+          mbar_arrive_expect_tx(BAR(B_FULLV + st), half);
+        }
         __syncwarp();
         if (my_ph >= 0) {
           const uint32_t dK = aKV + st * 2 * L::kTileBytes, dV = dK + L::kTileBytes;
           const int z = my_ph * p.Hkv + sg.h;
 #pragma unroll
-          for (int hh = 0; hh < L::kHalves; ++hh) {
-            const uint32_t off = hh * (kTok * 128) + lane * (p.P * 128);
-            tma_load_3d(dK + off, &tmK, BAR(B_FULL + st), hh * 64, 0, z, pol);
-            tma_load_3d(dV + off, &tmV, BAR(B_FULL + st), hh * 64, 0, z, pol);
-          }
+          for (int hh = 0; hh < L::kHalves; ++hh)
+            tma_load_3d(dK + hh * (kTok * 128) + lane * (p.P * 128), &tmK, BAR(B_FULL + st), hh * 64, 0, z, pol);
+#pragma unroll
+          for (int hh = 0; hh < L::kHalves; ++hh)
+            tma_load_3d(dV + hh * (kTok * 128) + lane * (p.P * 128), &tmV, BAR(B_FULLV + st), hh * 64, 0, z, pol);
         }
       }
       x = sg.end;
@@ -250,7 +261,10 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
     if (!waited) pdl_wait();
     // drain: wait until every issued copy has landed
     if (lane == 0)
-      for (int k = max(0, g - NS); k < g; ++k) mbar_wait_drain(BAR(B_FULL + k % NS), (k / NS) & 1, p.status);
+      for (int k = max(0, g - NS); k < g; ++k) {
+        mbar_wait_drain(BAR(B_FULL + k % NS), (k / NS) & 1, p.status);
+        mbar_wait_drain(BAR(B_FULLV + k % NS), (k / NS) & 1, p.status);
+      }
   } else if (warp == kTokMma) {
     // ======================================================= MMA issuer
     if (lane == 0) {
@@ -307,7 +321,8 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
       uint32_t spins = 0;
       while (pc.valid) {
         bool progress = false;
-        if (mbar_test_wait(BAR(B_PFULL + (pc.g & 1)), (pc.g >> 1) & 1)) {
+        if (mbar_test_wait(BAR(B_PFULL + (pc.g & 1)), (pc.g >> 1) & 1) &&
+            mbar_test_wait(BAR(B_FULLV + pc.g % NS), (pc.g / NS) & 1)) {
           issue_pv();
           progress = true;
         }
@@ -520,7 +535,9 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         }
         if (!valid) {
           // a token that does not exist (beyond L, or a missing page): zero
-          // its V row so that 0 * stale data cannot reach O
+          // its V row so that 0 * stale data cannot reach O (once the
+          // stage's V has landed, so that the copy cannot overwrite it)
+          ok &= mbar_wait(BAR(B_FULLV + st), (g / NS) & 1, &s_abort, p.status);
           uint8_t* sV = sKV + st * 2 * L::kTileBytes + L::kTileBytes + tid * 128;
 #pragma unroll
           for (int hh = 0; hh < L::kHalves; ++hh)
