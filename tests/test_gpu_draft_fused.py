@@ -52,6 +52,9 @@ CASES = {
     # further units from the workspace counter (ragged lengths)
     "selection-claims": (custom_spec(1, num_seqs=320, num_q_heads=4, num_kv_heads=2, page_size=16, gamma=2,
                                      budget_pages=6, vocab=512), _ragged(320, 50, 3000, 5)),
+    # D = 64 through the selection kernel (200 units), budget 40 (the 64-key select)
+    "d64-selection-top64": (custom_spec(1, num_seqs=100, num_q_heads=16, num_kv_heads=2, head_dim=64, page_size=64,
+                                        gamma=1, budget_pages=40, vocab=512), _ragged(100, 1500, 6400, 6)),
     # D = 64, G = 8: 60 units, each cut into two pieces (clusters of two CTAs)
     "d64-g8-pairs": (custom_spec(1, num_seqs=30, num_q_heads=16, num_kv_heads=2, head_dim=64, page_size=64,
                                  gamma=1, budget_pages=3, vocab=512), _ragged(30, 130, 2000, 2)),
