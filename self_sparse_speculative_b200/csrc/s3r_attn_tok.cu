@@ -212,8 +212,10 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         // the stage's page ids first (they do not need the slot), then the slot
         int my_lp = -1, my_ph = -1;
         for (int pp = 0; pp < ppt; ++pp) {
+          // positions past the segment belong to the next one: the windows
+          // must not move past its first page (warp-uniform)
+          if (j * ppt + pp >= sg.npg) break;
           const int xp = x + j * ppt + pp;
-          const bool in = (j * ppt + pp) < sg.npg;
           while (xp >= wbase + 32) {                   // advance the windows (warp-uniform)
             wbase += 32;
             w0_lp = w1_lp; w0_ph = w1_ph; w0_u = w1_u;
@@ -224,11 +226,11 @@ attn_tok_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
           const int src = xp - wbase;
           const int lp = __shfl_sync(0xffffffffu, w0_lp, src & 31);
           int ph = __shfl_sync(0xffffffffu, w0_ph, src & 31);
-          if (in && lp >= 0 && (ph < 0 || ph >= p.num_pages_total)) {
+          if (lp >= 0 && (ph < 0 || ph >= p.num_pages_total)) {
             if (lane == 0) flag_status(p.status, S3R_DEV_BAD_PAGE_ID);
             ph = -1;
           }
-          if (lane == pp && in) { my_lp = lp; my_ph = ph; }
+          if (lane == pp) { my_lp = lp; my_ph = ph; }
         }
         if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_EMPTY + st), ((g / NS) & 1) ^ 1, &s_abort, p.status))) {
           ok = false;

@@ -52,6 +52,10 @@ CASES = {
     # further units from the workspace counter (ragged lengths)
     "selection-claims": (custom_spec(1, num_seqs=320, num_q_heads=4, num_kv_heads=2, page_size=16, gamma=2,
                                      budget_pages=6, vocab=512), _ragged(320, 50, 3000, 5)),
+    # the selection kernel, 16-token pages and a 34-page budget: units end
+    # mid-stage inside the split-KV attention's 41-page CTA ranges
+    "selection-p16-budget34": (custom_spec(1, num_seqs=100, num_q_heads=8, num_kv_heads=2, page_size=16, gamma=1,
+                                           budget_pages=34, vocab=512), _ragged(100, 16 * 6, 16 * 60, 11)),
     # D = 64 through the selection kernel (200 units), budget 40 (the 64-key select)
     "d64-selection-top64": (custom_spec(1, num_seqs=100, num_q_heads=16, num_kv_heads=2, head_dim=64, page_size=64,
                                         gamma=1, budget_pages=40, vocab=512), _ragged(100, 1500, 6400, 6)),
@@ -282,3 +286,37 @@ def test_near_ties_inside_the_float32_band_follow_float64(num_seqs, heads, budge
             decided += int(n > budget and (n - 2) in set(int(x) for x in sel[b][h]))
         RR.assert_close(f"seq {b} out", gout[b], out[b], "bf16")
     assert decided > 0                                # the raises decided
+
+
+@pytest.mark.parametrize("num_seqs,heads,budget", [(2, 2, 5), (40, 2, 3), (100, 2, 34)],
+                         ids=["clusters", "one-cta-per-unit", "selection-kernel-top64"])
+def test_zero_queries_keep_the_lowest_pages(num_seqs, heads, budget):
+    """All-zero queries: every page scores exactly 0 (the rounding bound is 0
+    too, and the band's edges are the two zeros), so the float64 tie rule
+    keeps the lowest pages; attention over them gives the mean of their
+    values (uniform weights)."""
+    s = custom_spec(1, num_seqs=num_seqs, num_q_heads=4 * heads, num_kv_heads=heads, page_size=16, gamma=1,
+                    budget_pages=budget, vocab=512)
+    lens = _ragged(num_seqs, 16 * 6, 16 * 60, 11)
+    wl = Workload(s, seed=14, context_lens=lens)
+    st = DecodeStep(wl)
+    st.q_draft[0].zero_()
+    st.summaries(tail_only=False)
+    st.draft(0)
+    torch.cuda.synchronize()
+    assert s3r.s3r_device_status(st.ws_draft) == (s3r.S3R_OK, 0)
+    K64, V64 = to_float64(wl.kv_cache("K"), "bf16"), to_float64(wl.kv_cache("V"), "bf16")
+    q64 = np.zeros_like(to_float64(wl.q_draft[0], "bf16"))
+    bt = wl.block_table.astype(np.int64)
+    cl = np.asarray(lens)
+    kmin, kmax = O.page_summaries(K64, bt, cl, s.page_size)
+    sel, _ = O.sparse_draft_select(q64, kmin, kmax, bt, cl, s.page_size, budget, s.group)
+    out, lse = O.sparse_draft_attn(q64, K64, V64, bt, cl, sel, RR.f32(wl.scale))
+    gsel = st.selected[0].cpu().numpy()
+    gout = st.draft_out[0].float().cpu().numpy()
+    for b in range(num_seqs):
+        n = int(wl.pages_per_seq[b])
+        for h in range(heads):
+            assert list(sel[b][h]) == list(range(min(n, budget)))
+            assert gsel[b, h].tolist()[:min(n, budget)] == list(range(min(n, budget))), (b, h, gsel[b, h].tolist())
+        RR.assert_close(f"seq {b} out", gout[b], out[b], "bf16")

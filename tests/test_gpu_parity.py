@@ -31,6 +31,16 @@ CASES = {
     # D64 with 16-token pages (four pages per 64-token stage)
     "bf16-d64-p16": (custom_spec(1, num_seqs=3, num_q_heads=8, num_kv_heads=2, head_dim=64, page_size=16,
                                  gamma=3, budget_pages=6, vocab=999), [500, 33, 16 * 40 + 5]),
+    # 16-token pages (eight per 128-token stage), many short ragged units:
+    # a CTA's range of more than 32 pages holds three or more units, and a
+    # unit ending mid-stage inside it must not move the page-id windows past
+    # the next unit's first page (20 rows, then 72 rows)
+    "bf16-p16-wide": (custom_spec(1, num_seqs=200, num_q_heads=8, num_kv_heads=2, page_size=16, gamma=4,
+                                  budget_pages=13, vocab=512),
+                      np.random.default_rng(21).integers(96, 600, size=200).tolist()),
+    "bf16-p16-wide-r9": (custom_spec(1, num_seqs=160, num_q_heads=16, num_kv_heads=2, page_size=16, gamma=8,
+                                     budget_pages=5, vocab=512),
+                         np.random.default_rng(22).integers(150, 700, size=160).tolist()),
     # fp32 with D128, P64 and fp32 logits
     "f32-d128-p64": (custom_spec(0, num_seqs=2, num_q_heads=6, num_kv_heads=2, head_dim=128, page_size=64,
                                  budget_pages=2, vocab=777), [200, 4 * 64 + 1]),
